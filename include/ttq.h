@@ -1,0 +1,155 @@
+/*
+ * ttq.h - C ABI of the TTQ hot path on NVIDIA B200 (sm_100a).
+ *
+ * TTQ, activation-aware test-time quantization, quantizes the weights of a linear
+ * layer on the fly for every prompt, from that prompt's own activations.
+ * Definitions come from the pages on "TTQ: Activation-Aware Test-Time Quantization to
+ * Accelerate LLM Inference On The Fly":
+ *   [DR]  paper-daily.com deep reading, section 2 (method) and section 6 (deployment);
+ *   [NR]  nubint.ai review, section "proposed method";
+ *   [GDE] gist.science German technical summary, section 2 (Methodik);
+ *   [GFR] gist.science French technical summary, sections 2A and 2B.
+ *
+ * Conventions for every entry point
+ *   - Layouts: X is [T, d] bf16 row-major (tokens by input channels); W is [d_out, d]
+ *     bf16 row-major (the usual linear-layer layout); s is fp32 [d]; codes are uint32
+ *     [d_out, d*q/32]; scale and zero are fp16 [d_out, d/g]; Y is [T, d_out] bf16.
+ *   - Packed codes: groups run along d. q = 2 or 4: 32/q codes per word, code k of the
+ *     word at bits [q*k, q*k+q). q = 3: every 32 consecutive codes occupy 3 words, word
+ *     b holding bit b of each code (code k at bit k). Always exactly q/8 bytes a weight.
+ *   - Ownership: the caller allocates and owns every buffer (device memory); the library
+ *     allocates nothing, keeps no state between calls beyond one device error word, and
+ *     never writes to its inputs.
+ *   - Asynchrony: every compute call enqueues work on `stream` and returns. Argument
+ *     errors are returned synchronously and nothing is launched. A failed launch returns
+ *     TTQ_ERR_CUDA. A kernel that gives up on a bounded wait records TTQ_ERR_TIMEOUT in
+ *     the device error word, which ttq_device_status() reports.
+ *   - Alignment: every pointer must be 16-byte aligned (TTQ_ERR_MISALIGNED otherwise).
+ *   - Supported settings: q in {2,3,4}; g in {32,64,128}; d % g == 0; p in {1,2};
+ *     alpha >= 0; lambda > 0 when alpha > 0; 0 <= r <= 64 with A and B non-NULL
+ *     exactly when r > 0.
+ *   - Numerics: the quantizer runs in pinned IEEE fp32 and is reproducible bit for bit
+ *     given the same s; statistics accumulate in fp32; the projection multiplies bf16
+ *     operands on the tensor cores with fp32 accumulation and rounds Y to bf16.
+ */
+#ifndef TTQ_H_
+#define TTQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TTQ_OK = 0,
+  TTQ_ERR_INVALID_ARG = -1,  /* a size, pointer or setting is out of range          */
+  TTQ_ERR_UNSUPPORTED = -2,  /* q, g, p or r outside the supported set               */
+  TTQ_ERR_MISALIGNED = -3,   /* a pointer (or leading dimension) is not 16-byte aligned */
+  TTQ_ERR_WORKSPACE = -4,    /* ws is NULL or smaller than ttq_workspace_size()       */
+  TTQ_ERR_CUDA = -5,         /* a CUDA runtime call or kernel launch failed            */
+  TTQ_ERR_TIMEOUT = -6       /* a kernel gave up on a bounded wait (device error word) */
+} ttq_status;
+
+/* TTQ settings. q: bits per weight; g: group size along d; alpha, lambda, p: the
+ * statistic s_j = (mean_t |x_tj|^p + lambda)^(alpha/p) (p = 2 gives D^(1/2) with
+ * D = diag[X X^T / T + lambda I]^alpha, [DR] section 2); r: rank of the static low-rank
+ * factors B [d_out, r] and A [r, d] ([DR] section 2, [GFR] section 2B; 0 = none). */
+typedef struct {
+  int32_t q;
+  int32_t g;
+  float alpha;
+  float lambda;
+  int32_t p;
+  int32_t r;
+} ttq_config;
+
+/* Number of uint32 words of packed codes for a [d_out, d] weight at q bits
+ * (d_out * d * q / 32). Returns 0 when d is not a multiple of 32 or q is unsupported. */
+size_t ttq_codes_words(int64_t d_out, int64_t d, int32_t q);
+
+/* Bytes of scratch workspace that ttq_linear_prefill (and ttq_act_stats, and
+ * ttq_linear_decode with T = b rows) needs for these sizes. The workspace holds the
+ * partial column sums of the statistics, the folded activations X diag(1/s) in bf16,
+ * the low-rank projection X A^T and split-K partial products. Contents need not be
+ * initialised and are not preserved. */
+ttq_status ttq_workspace_size(int64_t T, int64_t d, int64_t d_out, const ttq_config* cfg,
+                              size_t* bytes);
+
+/* Online activation statistics ([DR] section 2 online diagonal D of each prompt;
+ * [GDE] section 2 D_ii from the norms of the input rows).
+ *   X      device bf16 [T, ld_x] (first d columns used), ld_x >= d, ld_x % 8 == 0
+ *   s      device fp32 [d] output: s_j = (mean_t |x_tj|^p + lambda)^(alpha/p)
+ *   ws     device scratch of at least ttq_workspace_size(T, d, 0, ...) bytes
+ * The column sums accumulate in fp32 in a fixed order, so results are deterministic. */
+ttq_status ttq_act_stats(const void* X_bf16, int64_t T, int64_t d, int64_t ld_x, float alpha,
+                         float lambda, int32_t p, float* s, void* ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/* Re-quantization of W diag(s) ([DR] section 2 W_hat = Q[W D^(1/2)] D^(-1/2); [NR]
+ * group-wise round-to-nearest quantize-dequantize). For each output row i and each
+ * group G of g consecutive input channels: v = fl32(w * s), sigma = smallest fp16 >=
+ * fl32((max v - min v) / (2^q - 1)), z = rint(fl32(-min v / sigma)) clamped to
+ * [-2048, 2048], c = clamp(rint(fl32(v / sigma)) + z, 0, 2^q - 1); a zero range is
+ * replaced by |min v| (or 1). rint rounds halves to even.
+ *   W      device bf16 [d_out, d] (pass the residual R = W - B A when r > 0)
+ *   s      device fp32 [d]
+ *   codes  device uint32 [ttq_codes_words(d_out, d, q)] output
+ *   scale  device fp16 [d_out, d/g] output (sigma)
+ *   zero   device fp16 [d_out, d/g] output (z, an integer held in fp16)
+ * Needs no workspace. Bit-exact and deterministic for given (W, s). */
+ttq_status ttq_requant(const void* W_bf16, int64_t d_out, int64_t d, const float* s, int32_t q,
+                       int32_t g, uint32_t* codes, void* scale_f16, void* zero_f16,
+                       cudaStream_t stream);
+
+/* One prompt through a TTQ linear layer ([DR] section 2 and section 6: statistics and
+ * scale-quantize-rescale at prefill): s = stats(X); (codes, scale, zero) = requant(W, s);
+ * Y = (X diag(1/s)) deq(codes)^T + (X A^T) B^T, where deq(c) = (c - z) * sigma is the
+ * quantized weight in the scaled domain. diag(1/s) is folded into X (bf16) instead of
+ * into the weight, so the tensor cores multiply bf16 X diag(1/s) by bf16 deq(codes)
+ * with fp32 accumulation.
+ *   X      device bf16 [T, d], contiguous
+ *   W      device bf16 [d_out, d] (the residual R = W - B A when r > 0)
+ *   A, B   device bf16 [r, d] and [d_out, r] when cfg->r > 0, else NULL
+ *   s, codes, scale, zero   outputs as in ttq_act_stats / ttq_requant, kept by the
+ *          caller for the decode steps that follow
+ *   Y      device bf16 [T, d_out] output
+ *   ws     device scratch of at least ttq_workspace_size(T, d, d_out, cfg) bytes */
+ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const void* W_bf16,
+                              int64_t d_out, const void* A_bf16, const void* B_bf16,
+                              const ttq_config* cfg, float* s, uint32_t* codes, void* scale_f16,
+                              void* zero_f16, void* Y_bf16, void* ws, size_t ws_bytes,
+                              cudaStream_t stream);
+
+/* Decode steps reuse the prefill's quantized weight ([DR] section 6: parameters computed
+ * at prefill are reused at decode): Y = (X diag(1/s)) deq(codes)^T + (X A^T) B^T for b
+ * new token rows, with s, codes, scale and zero from ttq_linear_prefill (or from
+ * ttq_act_stats + ttq_requant). Any b >= 1 is accepted.
+ *   X      device bf16 [b, d], contiguous;  Y  device bf16 [b, d_out] output
+ *   ws     device scratch of at least ttq_workspace_size(b, d, d_out, cfg) bytes */
+ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d_out,
+                             const float* s, const uint32_t* codes, const void* scale_f16,
+                             const void* zero_f16, const void* A_bf16, const void* B_bf16,
+                             const ttq_config* cfg, void* Y_bf16, void* ws, size_t ws_bytes,
+                             cudaStream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word: TTQ_OK, or
+ * TTQ_ERR_TIMEOUT when a kernel gave up on a bounded wait since the last call, or
+ * TTQ_ERR_CUDA when the synchronisation itself failed. */
+ttq_status ttq_device_status(cudaStream_t stream);
+
+/* Sets the limit, in nanoseconds, after which a kernel waiting on an mbarrier gives up
+ * and records TTQ_ERR_TIMEOUT (default 2e9, i.e. two seconds). Applies to launches made
+ * after the call. A limit of 0 restores the default. */
+ttq_status ttq_set_wait_limit_ns(uint64_t ns);
+
+/* A static string naming a status code. */
+const char* ttq_status_string(ttq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTQ_H_ */
