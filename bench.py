@@ -1,0 +1,545 @@
+#!/usr/bin/env python
+"""Benchmark of the TTQ linear layer on B200: statistics + re-quantization + tensor-core
+projection for each prompt (one "step" = one prompt through the layer), on the Qwen3-32B
+query projection 5120 -> 8192 with 4-bit codes, group 128 (the runtime table of the
+paper-daily.com deep reading of TTQ, section 4, measures this module).
+
+Prints ONE JSON line (rank 0). ``value`` is whole-job prefill throughput in k tokens/s
+with inputs resident in HBM; ``e2e`` is the same metric through the public Python API
+with the prompt copied in from pinned host memory and Y copied back every step.
+Per-stage times come from CUDA events the library records between its launches.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from online_activation_aware_b200 import dist as D  # noqa: E402
+from online_activation_aware_b200 import synthetic  # noqa: E402
+
+METRIC = "TTQ linear k tokens/s (stats+requant+GEMM), 5120→8192 4-bit; requant GB/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen3_32b_qproj")
+    ap.add_argument("--T", type=int, default=None, help="prompt length (default: the workload's)")
+    ap.add_argument("--r", type=int, default=None, help="low-rank r (default: the workload's)")
+    ap.add_argument("--no-extras", action="store_true", help="skip the T sweep, decode and e2e legs")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def requant_bytes(d, d_out, q, g):
+    # read bf16 W and fp32 s; write packed codes and fp16 scale + zero
+    return d_out * d * 2 + d * 4 + d_out * d * q // 8 + d_out * (d // g) * 4
+
+
+def stats_bytes(T, d):
+    return T * d * 2 + d * 4
+
+
+def fold_bytes(T, d):
+    return T * d * 4 + d * 4
+
+
+def gemm_flops(T, d, d_out, r):
+    return 2.0 * T * d * d_out + (2.0 * T * r * d_out if r else 0.0)
+
+
+def decode_bytes(b, d, d_out, q, g):
+    return d_out * d * q // 8 + d_out * (d // g) * 4 + b * d * 2 + b * d_out * 2 + d * 4
+
+
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.perf_counter(), line.strip()))
+
+    def window(self, t0, t1):
+        self.t0, self.t1 = t0, t1
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self._t.join(timeout=2)
+        sm, mx, reasons, pw = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        t0, t1 = getattr(self, "t0", -1e30), getattr(self, "t1", 1e30)
+        for ts, ln in self.lines:
+            if ts < t0 or ts > t1:
+                continue
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+                pw.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_uuid(torch, dev):
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return str(dev)
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for name in ("gemm.cu", "ttq_common.cuh"):
+        with open(os.path.join(ROOT, "online_activation_aware_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload_key: str):
+    """DRAM bytes per launch recorded from an ncu capture in profiles/ (null when the
+    kernel source changed since the capture, or no capture exists)."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(path):
+        return None
+    cur = kernel_hash()
+    with open(path) as f:
+        for line in f:
+            parts = [p.strip() for p in line.strip().strip("|").split("|")]
+            if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload_key and parts[3] == cur:
+                try:
+                    return float(parts[2])
+                except ValueError:
+                    return None
+    return None
+
+
+# ------------------------------------------------------------------ CPU oracle legs
+
+
+def oracle_sample(X, W, wl, T_tok: int, rows: int, seed: int = 0):
+    """Times the oracle on a slice (T_tok tokens, `rows` output rows) and extrapolates
+    the whole prompt (T tokens, all rows). Returns (seconds for the whole layer, info)."""
+    import numpy as np
+
+    from oracle import ttq_oracle as O
+
+    T, d = X.shape
+    d_out = W.shape[0]
+    rng = np.random.default_rng(seed)
+    t0 = rng.integers(0, max(1, T - T_tok + 1))
+    r0 = rng.integers(0, max(1, d_out - rows + 1))
+    Xs = X[t0:t0 + T_tok]
+    Ws = W[r0:r0 + rows]
+    a = time.perf_counter()
+    s64, s32 = O.act_stats(Xs, wl.alpha, wl.lam, wl.p)
+    b = time.perf_counter()
+    codes, scale, zero = O.requant(Ws, s32, wl.q, wl.g)
+    c = time.perf_counter()
+    O.linear(Xs, s32, codes, scale, zero, wl.g)
+    e = time.perf_counter()
+    full = (b - a) * (T / T_tok) + (c - b) * (d_out / rows) + (e - c) * (T / T_tok) * (d_out / rows)
+    return full, {"stats_s": b - a, "requant_s": c - b, "linear_s": e - c}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def host_inputs(wl, T, seed):
+    lin = wl.layers[0]
+    X, W = synthetic.draw_layer(T, lin.d, lin.d_out, seed)
+    Xb, Wb = synthetic.as_bf16(X), synthetic.as_bf16(W)
+    return Xb, Wb
+
+
+def cpu_baseline(Xv, Wv, wl, budget_s):
+    """The oracle, as it stands, on a bounded sample of the workload: 512 tokens x 256
+    rows per sample, repeated on fresh slices until the budget is spent."""
+    T = Xv.shape[0]
+    T_tok = min(T, 512)
+    rows = min(Wv.shape[0], 256)
+    ests = []
+    t_start = time.perf_counter()
+    n = 0
+    while time.perf_counter() - t_start < budget_s or n == 0:
+        full, _ = oracle_sample(Xv, Wv, wl, T_tok, rows, seed=n)
+        ests.append(full)
+        n += 1
+        if n >= 64:
+            break
+    full = statistics.median(ests)
+    return {"value": round(T / full / 1e3, 6), "unit": "k tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} samples of {T_tok} tokens x {rows} output rows, each extrapolated to the full "
+                      f"{T}-token prompt and {Wv.shape[0]} rows; median",
+            "seconds": round(time.perf_counter() - t_start, 2)}
+
+
+def run_reference(args, wl, T):
+    rank, world, _ = D.env()
+    if rank != 0:
+        return 0
+    import numpy as np
+
+    Xb, Wb = host_inputs(wl, T, wl.seed)
+    Xv, Wv = synthetic.bf16_values(Xb), synthetic.bf16_values(Wb)
+    # size each step so the whole run stays within about two minutes
+    nsteps = args.steps + args.warmup
+    per_step = max(0.01, 120.0 / max(1, nsteps))
+    T_tok, rows = 256, 64
+    if per_step > 1.0:
+        T_tok, rows = 512, 256
+    times = []
+    for i in range(nsteps):
+        full, _ = oracle_sample(Xv, Wv, wl, T_tok, rows, seed=i)
+        if i >= args.warmup:
+            times.append(full)
+    t = statistics.median(times)
+    value = T / t / 1e3
+    lin = wl.layers[0]
+    cores = blas_threads()
+    out = {"metric": METRIC, "value": round(value, 6), "unit": "k tokens/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "impl": "reference",
+           "config": {"workload": f"{wl.name} {lin.d}->{lin.d_out} q={wl.q} g={wl.g} T={T}", "T": T,
+                      "d": lin.d, "d_out": lin.d_out, "q": wl.q, "g": wl.g, "alpha": wl.alpha, "lambda": wl.lam,
+                      "r": 0},
+           "cpu_baseline": {"value": round(value, 6), "unit": "k tokens/s", "cores": cores, "kind": "oracle",
+                            "sample": f"each step: {T_tok} tokens x {rows} output rows, extrapolated to "
+                                      f"{T} tokens x {lin.d_out} rows; median over {args.steps} steps"},
+           "e2e": {"value": round(value, 6), "unit": "k tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU legs
+
+
+def main():
+    args = parse()
+    wl = synthetic.WORKLOADS[args.workload]
+    T = args.T or wl.T
+    r = wl.r if args.r is None else args.r
+    if args.impl == "reference":
+        return run_reference(args, wl, T)
+
+    import numpy as np
+    import torch
+
+    import online_activation_aware_b200 as ttq
+
+    rank, world, local_rank = D.env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    D.init("nccl")
+    ttq.load_library()
+    hbm_peak, tc_peak, tc_sust, peak_src = peaks()
+    lin = wl.layers[0]
+    d, d_out, q, g = lin.d, lin.d_out, wl.q, wl.g
+    cfg = ttq.make_config(q, g, wl.alpha, wl.lam, wl.p, r)
+
+    # inputs: this rank's own prompt and weight, copied into several buffer sets so that
+    # consecutive steps never find their operands in the 126 MB L2
+    Xb, Wb = host_inputs(wl, T, D.rank_seed(wl.seed, rank))
+    A = B = None
+    if r > 0:
+        Bh, Ah, Rh = ttq.lowrank_factors(Wb, r)
+        A, B = Ah.to(dev), Bh.to(dev)
+        Wb = Rh
+    set_bytes = (T * d + d_out * d) * 2
+    nsets = max(2, int(np.ceil(3 * 126e6 / set_bytes)) + 1)
+    nsets = min(nsets, 6)
+    Xs = [Xb.to(dev) for _ in range(nsets)]
+    Ws = [Wb.to(dev) for _ in range(nsets)]
+    outs = [{"s": torch.empty(d, dtype=torch.float32, device=dev),
+             "codes": torch.empty(ttq.codes_words(d_out, d, q), dtype=torch.int32, device=dev),
+             "scale": torch.empty(d_out, d // g, dtype=torch.float16, device=dev),
+             "zero": torch.empty(d_out, d // g, dtype=torch.float16, device=dev),
+             "Y": torch.empty(T, d_out, dtype=torch.bfloat16, device=dev)} for _ in range(nsets)]
+    ws = ttq.alloc_workspace(T, d, d_out, cfg, dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        k = i % nsets
+        ttq.linear_prefill(Xs[k], Ws[k], cfg, A, B, out=outs[k], ws=ws, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert ttq.device_status() == 0
+
+    # timed region: K prefill steps back to back, stage events recorded by the library
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    for e6 in evs:
+        for e in e6:
+            e.record()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_uuid(torch, dev))
+    sampler.start()
+    time.sleep(0.3)
+    D.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    wall0 = time.perf_counter()
+    start.record()
+    for i in range(K):
+        ttq.set_trace_events(evs[i])
+        step(i)
+    end.record()
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    sampler.window(wall0, wall0 + wall)
+    ttq.set_trace_events(None)
+    D.barrier()
+    clocks = sampler.stop()
+    assert ttq.device_status() == 0
+    t_ms = start.elapsed_time(end)
+    t_max_ms = D.max_over_ranks(t_ms, dev)
+    stage_names = ["stats", "fold", "requant", "gemm", "reduce"]
+    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
+                for j, n in enumerate(stage_names)}
+    tokens = T * K * world
+    value = tokens / (t_max_ms / 1e3) / 1e3
+
+    plan_split = stage_ms["reduce"] > 0.002
+    launches_per_step = 4 + (1 if r > 0 else 0) + (1 if plan_split else 0)
+
+    kern = {
+        "stats": {"ms": stage_ms["stats"], "bound": "hbm", "bytes": stats_bytes(T, d)},
+        "fold": {"ms": stage_ms["fold"], "bound": "hbm", "bytes": fold_bytes(T, d) + (T * d * 2 if r else 0)},
+        "requant": {"ms": stage_ms["requant"], "bound": "hbm", "bytes": requant_bytes(d, d_out, q, g)},
+        "gemm": {"ms": stage_ms["gemm"] + stage_ms["reduce"], "bound": "tensor", "flops": gemm_flops(T, d, d_out, r)},
+    }
+    for k_, v in kern.items():
+        sec = v["ms"] / 1e3
+        if v["bound"] == "hbm":
+            v["GBps"] = round(v["bytes"] / sec / 1e9, 1)
+            v["frac"] = round(v["GBps"] / hbm_peak, 4)
+        else:
+            v["TFLOPs"] = round(v["flops"] / sec / 1e12, 1)
+            v["frac"] = round(v["TFLOPs"] / tc_peak, 4)
+        v["ms"] = round(v["ms"], 5)
+    dom = max(kern, key=lambda k_: kern[k_]["ms"])
+    dk = kern[dom]
+    wkey = f"{wl.name}_T{T}_r{r}"
+    if dk["bound"] == "tensor":
+        roof = {"kernel": "ttq_gemm_kernel", "bound": "tensor", "achieved": dk["TFLOPs"], "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": dk["frac"],
+                "traffic": profiled_traffic("ttq_gemm_kernel", wkey),
+                "algorithmic": f"2*T*d*d_out flops per launch = {dk['flops']:.4g}",
+                "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"}
+    else:
+        roof = {"kernel": {"requant": "requant_kernel", "stats": "act_stats_kernel", "fold": "fold_kernel"}[dom],
+                "bound": "hbm", "achieved": dk["GBps"], "peak": hbm_peak, "unit": "GB/s", "frac": dk["frac"],
+                "traffic": profiled_traffic(dom, wkey), "algorithmic": f"{dk['bytes']} bytes per launch",
+                "peak_source": f"{peak_src} HBM copy (MEASURED_PEAKS.json)"}
+
+    result = {
+        "metric": METRIC, "value": round(value, 3), "unit": "k tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(t_max_ms / K, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{wl.name} {d}->{d_out} q={q} g={g} T={T}", "T": T, "d": d, "d_out": d_out,
+                   "q": q, "g": g, "alpha": wl.alpha, "lambda": wl.lam, "r": r, "parallelism": f"replicas{world}",
+                   "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.0f} MB (> 126 MB L2)"},
+        "requant_gbs": kern["requant"]["GBps"],
+        "roofline": roof,
+        "kernels": kern,
+        "rho_measured": round((stage_ms["stats"] + stage_ms["requant"]) / (stage_ms["gemm"] + stage_ms["reduce"]), 4),
+        "gpu_launches": K * launches_per_step,
+        "clocks": clocks,
+        "wall_s_timed": round(wall, 3),
+    }
+
+    # ---- end to end through the public API: pinned host X in, Y back out, every step
+    if not args.no_extras:
+        Xh = Xb.pin_memory()
+        Yh = torch.empty(T, d_out, dtype=torch.bfloat16).pin_memory()
+        layer_ = ttq.TTQLinear(Ws[0], q, g, wl.alpha, wl.lam, wl.p, r, A, B)
+        Xd = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+        Yd = torch.empty(T, d_out, dtype=torch.bfloat16, device=dev)
+        Ke = max(3, min(K, 50))
+        for _ in range(3):
+            Xd.copy_(Xh, non_blocking=True)
+            layer_.prefill(Xd, Y=Yd)
+            Yh.copy_(Yd, non_blocking=True)
+        torch.cuda.synchronize()
+        D.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(Ke):
+            Xd.copy_(Xh, non_blocking=True)
+            layer_.prefill(Xd, Y=Yd)
+            Yh.copy_(Yd, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        te = D.max_over_ranks(e0.elapsed_time(e1), dev)
+        result["e2e"] = {"value": round(T * Ke * world / (te / 1e3) / 1e3, 3), "unit": "k tokens/s",
+                         "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d_out * 2,
+                         "steps": Ke, "api": "TTQLinear.prefill"}
+    else:
+        result["e2e"] = None
+
+    # ---- rank 0 extras: oracle baseline, decode steps, prompt-length sweep
+    if world == 1 and not args.no_extras:
+        Xv, Wv = synthetic.bf16_values(Xb), synthetic.bf16_values(Wb)
+        result["cpu_baseline"] = cpu_baseline(Xv, Wv, wl, args.cpu_seconds)
+        result["decode"] = decode_leg(torch, ttq, wl, cfg, Xs[0], Ws[0], A, B, dev, hbm_peak)
+        result["sweep"] = sweep_leg(torch, ttq, wl, cfg, Wb, A, B, dev, r)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    D.barrier()
+    D.finalize()
+    return 0
+
+
+def decode_leg(torch, ttq, wl, cfg, X, W, A, B, dev, hbm_peak):
+    """Decode steps reusing one prefill's codes, b tokens per step, each step a CUDA
+    graph replay timed with events; L2 is flushed between steps (outside the events)."""
+    lin = wl.layers[0]
+    d, d_out = lin.d, lin.d_out
+    layer_ = ttq.TTQLinear(W, cfg.q, cfg.g, cfg.alpha, cfg.lambda_, cfg.p, cfg.r, A, B)
+    layer_.prefill(X)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    out = {}
+    for b in wl.decode_batches or (1,):
+        xt = synthetic.as_bf16(synthetic.draw_tokens(b, d, seed=1234 + b)).to(dev)
+        Y = torch.empty(b, d_out, dtype=torch.bfloat16, device=dev)
+        layer_.workspace(b)
+        for _ in range(3):
+            layer_.decode(xt, Y=Y)
+        torch.cuda.synchronize()
+        g_ = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g_, stream=s):
+                layer_.decode(xt, Y=Y, stream=s)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        times = []
+        n = 64
+        for i in range(n + 4):
+            flush.fill_(i & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g_.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 4:
+                times.append(e0.elapsed_time(e1))
+        del g_
+        t = statistics.median(times) / 1e3
+        by = decode_bytes(b, d, d_out, cfg.q, cfg.g)
+        out[f"b{b}"] = {"us_per_step": round(t * 1e6, 2), "k_tokens_per_s": round(b / t / 1e3, 2),
+                        "GBps": round(by / t / 1e9, 1), "frac_hbm": round(by / t / 1e9 / hbm_peak, 4)}
+    assert ttq.device_status() == 0
+    return out
+
+
+def sweep_leg(torch, ttq, wl, cfg, Wb, A, B, dev, r):
+    """Prefill throughput across prompt lengths (k tokens/s), rotating buffer sets."""
+    import numpy as np
+
+    lin = wl.layers[0]
+    d, d_out = lin.d, lin.d_out
+    res = {}
+    for T in (wl.T_sweep or ()):
+        Xb = synthetic.as_bf16(synthetic.draw_layer(T, d, 8, seed=500 + T)[0])
+        nsets = 3 if T <= 4096 else 2
+        Xs = [Xb.to(dev) for _ in range(nsets)]
+        Ws = [Wb.to(dev) for _ in range(nsets)]
+        ws = ttq.alloc_workspace(T, d, d_out, cfg, dev)
+        outs = [None] * nsets
+        for i in range(3):
+            outs[i % nsets] = ttq.linear_prefill(Xs[i % nsets], Ws[i % nsets], cfg, A, B, ws=ws)
+        torch.cuda.synchronize()
+        K = 30 if T <= 4096 else 8
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(K):
+            k = i % nsets
+            ttq.linear_prefill(Xs[k], Ws[k], cfg, A, B, out=outs[k], ws=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) / 1e3 / K
+        res[f"T{T}"] = {"k_tokens_per_s": round(T / t / 1e3, 2), "us_per_prompt": round(t * 1e6, 1)}
+        del Xs, Ws, outs, ws
+        torch.cuda.empty_cache()
+    assert ttq.device_status() == 0
+    return res
+
+
+if __name__ == "__main__":
+    sys.exit(main())

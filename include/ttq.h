@@ -39,6 +39,12 @@
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
+#if defined(__GNUC__)
+#define TTQ_API __attribute__((visibility("default")))
+#else
+#define TTQ_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -68,14 +74,14 @@ typedef struct {
 
 /* Number of uint32 words of packed codes for a [d_out, d] weight at q bits
  * (d_out * d * q / 32). Returns 0 when d is not a multiple of 32 or q is unsupported. */
-size_t ttq_codes_words(int64_t d_out, int64_t d, int32_t q);
+TTQ_API size_t ttq_codes_words(int64_t d_out, int64_t d, int32_t q);
 
 /* Bytes of scratch workspace that ttq_linear_prefill (and ttq_act_stats, and
  * ttq_linear_decode with T = b rows) needs for these sizes. The workspace holds the
  * partial column sums of the statistics, the folded activations X diag(1/s) in bf16,
  * the low-rank projection X A^T and split-K partial products. Contents need not be
  * initialised and are not preserved. */
-ttq_status ttq_workspace_size(int64_t T, int64_t d, int64_t d_out, const ttq_config* cfg,
+TTQ_API ttq_status ttq_workspace_size(int64_t T, int64_t d, int64_t d_out, const ttq_config* cfg,
                               size_t* bytes);
 
 /* Online activation statistics ([DR] section 2 online diagonal D of each prompt;
@@ -84,7 +90,7 @@ ttq_status ttq_workspace_size(int64_t T, int64_t d, int64_t d_out, const ttq_con
  *   s      device fp32 [d] output: s_j = (mean_t |x_tj|^p + lambda)^(alpha/p)
  *   ws     device scratch of at least ttq_workspace_size(T, d, 0, ...) bytes
  * The column sums accumulate in fp32 in a fixed order, so results are deterministic. */
-ttq_status ttq_act_stats(const void* X_bf16, int64_t T, int64_t d, int64_t ld_x, float alpha,
+TTQ_API ttq_status ttq_act_stats(const void* X_bf16, int64_t T, int64_t d, int64_t ld_x, float alpha,
                          float lambda, int32_t p, float* s, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
 
@@ -100,7 +106,7 @@ ttq_status ttq_act_stats(const void* X_bf16, int64_t T, int64_t d, int64_t ld_x,
  *   scale  device fp16 [d_out, d/g] output (sigma)
  *   zero   device fp16 [d_out, d/g] output (z, an integer held in fp16)
  * Needs no workspace. Bit-exact and deterministic for given (W, s). */
-ttq_status ttq_requant(const void* W_bf16, int64_t d_out, int64_t d, const float* s, int32_t q,
+TTQ_API ttq_status ttq_requant(const void* W_bf16, int64_t d_out, int64_t d, const float* s, int32_t q,
                        int32_t g, uint32_t* codes, void* scale_f16, void* zero_f16,
                        cudaStream_t stream);
 
@@ -117,7 +123,7 @@ ttq_status ttq_requant(const void* W_bf16, int64_t d_out, int64_t d, const float
  *          caller for the decode steps that follow
  *   Y      device bf16 [T, d_out] output
  *   ws     device scratch of at least ttq_workspace_size(T, d, d_out, cfg) bytes */
-ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const void* W_bf16,
+TTQ_API ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const void* W_bf16,
                               int64_t d_out, const void* A_bf16, const void* B_bf16,
                               const ttq_config* cfg, float* s, uint32_t* codes, void* scale_f16,
                               void* zero_f16, void* Y_bf16, void* ws, size_t ws_bytes,
@@ -129,7 +135,7 @@ ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const vo
  * ttq_act_stats + ttq_requant). Any b >= 1 is accepted.
  *   X      device bf16 [b, d], contiguous;  Y  device bf16 [b, d_out] output
  *   ws     device scratch of at least ttq_workspace_size(b, d, d_out, cfg) bytes */
-ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d_out,
+TTQ_API ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d_out,
                              const float* s, const uint32_t* codes, const void* scale_f16,
                              const void* zero_f16, const void* A_bf16, const void* B_bf16,
                              const ttq_config* cfg, void* Y_bf16, void* ws, size_t ws_bytes,
@@ -138,15 +144,24 @@ ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d
 /* Synchronises `stream`, then reads and clears the device error word: TTQ_OK, or
  * TTQ_ERR_TIMEOUT when a kernel gave up on a bounded wait since the last call, or
  * TTQ_ERR_CUDA when the synchronisation itself failed. */
-ttq_status ttq_device_status(cudaStream_t stream);
+TTQ_API ttq_status ttq_device_status(cudaStream_t stream);
 
 /* Sets the limit, in nanoseconds, after which a kernel waiting on an mbarrier gives up
  * and records TTQ_ERR_TIMEOUT (default 2e9, i.e. two seconds). Applies to launches made
  * after the call. A limit of 0 restores the default. */
-ttq_status ttq_set_wait_limit_ns(uint64_t ns);
+TTQ_API ttq_status ttq_set_wait_limit_ns(uint64_t ns);
+
+/* Stage tracing for measurement. With n >= 6 event handles (cudaEvent_t created by the
+ * caller with timing enabled), every later ttq_linear_prefill call records, on its
+ * stream: events[0] before the statistics, [1] after them, [2] after the fold (and the
+ * low-rank projection X A^T), [3] after the re-quantization, [4] after the tensor-core
+ * projection and [5] after the split-K reduction (when there is none, [5] directly
+ * follows [4]). n = 0 (or events = NULL) turns tracing off. The library keeps the
+ * handles, not copies: they must stay valid while tracing is on. Not thread-safe. */
+TTQ_API ttq_status ttq_set_trace_events(void* const* events, int32_t n);
 
 /* A static string naming a status code. */
-const char* ttq_status_string(ttq_status status);
+TTQ_API const char* ttq_status_string(ttq_status status);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,286 @@
+"""TTQ (activation-aware test-time quantization) on NVIDIA B200: Python binding.
+
+A thin ctypes layer over ``libttq.so`` (C ABI in ``include/ttq.h``). Every function
+here only checks and marshals its arguments (torch CUDA tensors -> device pointers,
+the current CUDA stream) and calls the library; all arithmetic of the hot path runs
+in the library's CUDA kernels. There is no CPU fallback: when the library is missing
+or a call fails, a ``TTQError`` is raised.
+
+Functions keep the C names without the ``ttq_`` prefix:
+``act_stats``, ``requant``, ``linear_prefill``, ``linear_decode``, ``workspace_size``,
+``codes_words``, ``device_status``, ``set_wait_limit_ns``. ``TTQLinear`` bundles one
+layer's weight and the per-prompt buffers (prefill, then decode reusing the codes).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libttq.so")
+
+STATUS = {0: "TTQ_OK", -1: "TTQ_ERR_INVALID_ARG", -2: "TTQ_ERR_UNSUPPORTED", -3: "TTQ_ERR_MISALIGNED",
+          -4: "TTQ_ERR_WORKSPACE", -5: "TTQ_ERR_CUDA", -6: "TTQ_ERR_TIMEOUT"}
+
+
+class TTQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+
+
+class Config(ctypes.Structure):
+    """Mirror of ``ttq_config``."""
+    _fields_ = [("q", ctypes.c_int32), ("g", ctypes.c_int32), ("alpha", ctypes.c_float),
+                ("lambda_", ctypes.c_float), ("p", ctypes.c_int32), ("r", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Loads libttq.so (once). Raises TTQError-compatible RuntimeError when it is absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m online_activation_aware_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    cfgp = ctypes.POINTER(Config)
+    lib.ttq_codes_words.argtypes = [i64, i64, i32]
+    lib.ttq_codes_words.restype = sz
+    lib.ttq_workspace_size.argtypes = [i64, i64, i64, cfgp, ctypes.POINTER(sz)]
+    lib.ttq_workspace_size.restype = i32
+    lib.ttq_act_stats.argtypes = [vp, i64, i64, i64, f32, f32, i32, vp, vp, sz, vp]
+    lib.ttq_act_stats.restype = i32
+    lib.ttq_requant.argtypes = [vp, i64, i64, vp, i32, i32, vp, vp, vp, vp]
+    lib.ttq_requant.restype = i32
+    lib.ttq_linear_prefill.argtypes = [vp, i64, i64, vp, i64, vp, vp, cfgp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.ttq_linear_prefill.restype = i32
+    lib.ttq_linear_decode.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, cfgp, vp, vp, sz, vp]
+    lib.ttq_linear_decode.restype = i32
+    lib.ttq_device_status.argtypes = [vp]
+    lib.ttq_device_status.restype = i32
+    lib.ttq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.ttq_set_wait_limit_ns.restype = i32
+    lib.ttq_set_trace_events.argtypes = [ctypes.POINTER(vp), i32]
+    lib.ttq_set_trace_events.restype = i32
+    lib.ttq_status_string.argtypes = [i32]
+    lib.ttq_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise TTQError(fn, status)
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_config(q: int, g: int, alpha: float, lam: float, p: int = 2, r: int = 0) -> Config:
+    return Config(int(q), int(g), float(alpha), float(lam), int(p), int(r))
+
+
+def codes_words(d_out: int, d: int, q: int) -> int:
+    return int(load_library().ttq_codes_words(d_out, d, q))
+
+
+def workspace_size(T: int, d: int, d_out: int, cfg: Config | None = None) -> int:
+    n = ctypes.c_size_t(0)
+    _check("ttq_workspace_size",
+           load_library().ttq_workspace_size(T, d, d_out, ctypes.byref(cfg) if cfg is not None else None,
+                                             ctypes.byref(n)))
+    return int(n.value)
+
+
+def alloc_workspace(T: int, d: int, d_out: int, cfg: Config | None = None, device="cuda"):
+    import torch
+
+    return torch.empty(max(workspace_size(T, d, d_out, cfg), 256), dtype=torch.uint8, device=device)
+
+
+def act_stats(X, alpha: float, lam: float, p: int = 2, s=None, ws=None, stream=None):
+    """s = (mean over tokens of |X|^p + lambda)^(alpha/p) per input channel; X [T, d] bf16."""
+    import torch
+
+    T, d = X.shape
+    if s is None:
+        s = torch.empty(d, dtype=torch.float32, device=X.device)
+    if ws is None:
+        ws = alloc_workspace(T, d, 0, None, X.device)
+    _check("ttq_act_stats", load_library().ttq_act_stats(
+        _ptr(X, torch.bfloat16, "X"), T, d, X.stride(0), alpha, lam, p, _ptr(s, torch.float32, "s"),
+        _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)))
+    return s
+
+
+def requant(W, s, q: int, g: int, codes=None, scale=None, zero=None, stream=None):
+    """Packed codes, fp16 scale and fp16 zero of Q[W diag(s)]; W [d_out, d] bf16."""
+    import torch
+
+    d_out, d = W.shape
+    dev = W.device
+    if codes is None:
+        codes = torch.empty(codes_words(d_out, d, q), dtype=torch.int32, device=dev)
+    if scale is None:
+        scale = torch.empty(d_out, d // g, dtype=torch.float16, device=dev)
+    if zero is None:
+        zero = torch.empty(d_out, d // g, dtype=torch.float16, device=dev)
+    _check("ttq_requant", load_library().ttq_requant(
+        _ptr(W, torch.bfloat16, "W"), d_out, d, _ptr(s, torch.float32, "s"), q, g,
+        _ptr(codes, torch.int32, "codes"), _ptr(scale, torch.float16, "scale"),
+        _ptr(zero, torch.float16, "zero"), _stream(stream)))
+    return codes, scale, zero
+
+
+def linear_prefill(X, W, cfg: Config, A=None, B=None, out=None, ws=None, stream=None):
+    """One prompt through a TTQ linear layer. Returns dict(s, codes, scale, zero, Y)."""
+    import torch
+
+    T, d = X.shape
+    d_out = W.shape[0]
+    dev = X.device
+    o = out or {}
+    s = o.get("s") if o.get("s") is not None else torch.empty(d, dtype=torch.float32, device=dev)
+    codes = o.get("codes") if o.get("codes") is not None else torch.empty(
+        codes_words(d_out, d, cfg.q), dtype=torch.int32, device=dev)
+    scale = o.get("scale") if o.get("scale") is not None else torch.empty(
+        d_out, d // cfg.g, dtype=torch.float16, device=dev)
+    zero = o.get("zero") if o.get("zero") is not None else torch.empty(
+        d_out, d // cfg.g, dtype=torch.float16, device=dev)
+    Y = o.get("Y") if o.get("Y") is not None else torch.empty(T, d_out, dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = alloc_workspace(T, d, d_out, cfg, dev)
+    _check("ttq_linear_prefill", load_library().ttq_linear_prefill(
+        _ptr(X, torch.bfloat16, "X"), T, d, _ptr(W, torch.bfloat16, "W"), d_out,
+        _ptr(A, torch.bfloat16, "A"), _ptr(B, torch.bfloat16, "B"), ctypes.byref(cfg),
+        _ptr(s, torch.float32, "s"), _ptr(codes, torch.int32, "codes"), _ptr(scale, torch.float16, "scale"),
+        _ptr(zero, torch.float16, "zero"), _ptr(Y, torch.bfloat16, "Y"), _ptr(ws, None, "ws"),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    return {"s": s, "codes": codes, "scale": scale, "zero": zero, "Y": Y}
+
+
+def linear_decode(X, s, codes, scale, zero, cfg: Config, d_out: int, A=None, B=None, Y=None, ws=None,
+                  stream=None):
+    """Y = (X diag(1/s)) deq(codes)^T (+ (X A^T) B^T) for b token rows, reusing a prefill's codes."""
+    import torch
+
+    b, d = X.shape
+    dev = X.device
+    if Y is None:
+        Y = torch.empty(b, d_out, dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = alloc_workspace(b, d, d_out, cfg, dev)
+    _check("ttq_linear_decode", load_library().ttq_linear_decode(
+        _ptr(X, torch.bfloat16, "X"), b, d, d_out, _ptr(s, torch.float32, "s"),
+        _ptr(codes, torch.int32, "codes"), _ptr(scale, torch.float16, "scale"),
+        _ptr(zero, torch.float16, "zero"), _ptr(A, torch.bfloat16, "A"), _ptr(B, torch.bfloat16, "B"),
+        ctypes.byref(cfg), _ptr(Y, torch.bfloat16, "Y"), _ptr(ws, None, "ws"),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    return Y
+
+
+def device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the library's device error status."""
+    return int(load_library().ttq_device_status(_stream(stream)))
+
+
+def set_wait_limit_ns(ns: int):
+    _check("ttq_set_wait_limit_ns", load_library().ttq_set_wait_limit_ns(int(ns)))
+
+
+def set_trace_events(events):
+    """Records stage boundaries of every later linear_prefill on these CUDA events
+    (a list of 6 ``torch.cuda.Event(enable_timing=True)``), or stops when None."""
+    lib = load_library()
+    if not events:
+        _check("ttq_set_trace_events", lib.ttq_set_trace_events(None, 0))
+        return
+    handles = []
+    for ev in events:
+        if ev.cuda_event == 0:  # torch creates the event lazily
+            ev.record()
+        handles.append(ev.cuda_event)
+    arr = (ctypes.c_void_p * len(handles))(*handles)
+    set_trace_events._keep = (arr, events)
+    _check("ttq_set_trace_events", lib.ttq_set_trace_events(arr, len(handles)))
+
+
+def lowrank_factors(W, r: int):
+    """Host set-up of the static low-rank side path (untimed, once per weight).
+
+    Returns bf16 CPU tensors (B [d_out, r], A [r, d], R [d_out, d]) with B = U_r S_r^(1/2),
+    A = S_r^(1/2) V_r^T from the fp64 SVD of W, and R = W - B A rounded to bf16, the
+    residual that is re-quantized per prompt (paper-daily.com deep reading of TTQ,
+    section 2: W_hat = W_q + BA with SVD-initialised factors, r = 16).
+    """
+    import torch
+
+    Wd = W.detach().to("cpu", torch.float64)
+    U, S, Vh = torch.linalg.svd(Wd, full_matrices=False)
+    root = S[:r].sqrt()
+    Bf = (U[:, :r] * root[None, :]).to(torch.bfloat16)
+    Af = (root[:, None] * Vh[:r, :]).to(torch.bfloat16)
+    R = (Wd - Bf.to(torch.float64) @ Af.to(torch.float64)).to(torch.bfloat16)
+    return Bf.contiguous(), Af.contiguous(), R.contiguous()
+
+
+class TTQLinear:
+    """One linear layer under TTQ: holds the bf16 weight (or residual R and the static
+    factors A, B when r > 0) and, after ``prefill``, the prompt's s and packed codes that
+    ``decode`` reuses."""
+
+    def __init__(self, W, q: int, g: int, alpha: float, lam: float, p: int = 2, r: int = 0,
+                 A=None, B=None):
+        import torch
+
+        self.cfg = make_config(q, g, alpha, lam, p, r)
+        self.W = W
+        self.A = A
+        self.B = B
+        self.d_out, self.d = W.shape
+        dev = W.device
+        self.s = torch.empty(self.d, dtype=torch.float32, device=dev)
+        self.codes = torch.empty(codes_words(self.d_out, self.d, q), dtype=torch.int32, device=dev)
+        self.scale = torch.empty(self.d_out, self.d // g, dtype=torch.float16, device=dev)
+        self.zero = torch.empty(self.d_out, self.d // g, dtype=torch.float16, device=dev)
+        self._ws = {}
+
+    def workspace(self, T: int):
+        if T not in self._ws:
+            self._ws[T] = alloc_workspace(T, self.d, self.d_out, self.cfg, self.W.device)
+        return self._ws[T]
+
+    def prefill(self, X, Y=None, stream=None):
+        out = {"s": self.s, "codes": self.codes, "scale": self.scale, "zero": self.zero, "Y": Y}
+        return linear_prefill(X, self.W, self.cfg, self.A, self.B, out=out, ws=self.workspace(X.shape[0]),
+                              stream=stream)["Y"]
+
+    def decode(self, X, Y=None, stream=None):
+        return linear_decode(X, self.s, self.codes, self.scale, self.zero, self.cfg, self.d_out, self.A,
+                             self.B, Y=Y, ws=self.workspace(X.shape[0]), stream=stream)

@@ -1,0 +1,271 @@
+// Kernels over the activations X [T, d] (bf16, row-major):
+//   act_stats   per-channel statistic s_j = (mean_t |x_tj|^p + lambda)^(alpha/p), the
+//               online diagonal D^(1/2) of the prompt (paper-daily.com deep reading of
+//               TTQ, section 2; gist.science German summary, section 2);
+//   fold        X diag(1/s) in bf16, the operand the projection multiplies (the
+//               D^(-1/2) of W_hat = Q[W D^(1/2)] D^(-1/2) moved onto the activations);
+//   lowrank_u   U = X A^T for the static low-rank side path (gist.science French
+//               summary, section 2B).
+// All three are HBM-bound streaming passes: a warp reads 512 contiguous bytes of a row
+// per step (32 lanes x 16 B), so every DRAM sector fetched is used in full.
+#include "ttq_internal.h"
+
+namespace ttq {
+
+namespace {
+
+constexpr int kColsPerBlock = 256;  // 32 lanes x 8 bf16
+constexpr int kRowWarps = 8;        // warps of a block walk rows 8 apart
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+template <int P>
+__device__ __forceinline__ void accum8(float (&acc)[8], const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float a = bf16lo_to_f32(w[j]);
+    const float b = bf16hi_to_f32(w[j]);
+    if (P == 2) {
+      acc[2 * j] = __fmaf_rn(a, a, acc[2 * j]);      // bf16^2 is exact in fp32
+      acc[2 * j + 1] = __fmaf_rn(b, b, acc[2 * j + 1]);
+    } else {
+      acc[2 * j] = __fadd_rn(acc[2 * j], fabsf(a));
+      acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], fabsf(b));
+    }
+  }
+}
+
+__device__ __forceinline__ float finalize_scale(float colsum, float T, float alpha_over_p,
+                                                float lambda) {
+  const float m = __fdiv_rn(colsum, T);  // mean over the prompt's tokens
+  return powf(__fadd_rn(m, lambda), alpha_over_p);
+}
+
+// grid: (col_blocks, nsplit); block: 256 threads. Each block reduces its rows for 256
+// columns into partial[split, col]; the last block of a column strip (in arrival order,
+// counted in `counters`) sums the strip's partials in split order and writes s. The
+// summation order is fixed, so the result does not depend on scheduling.
+template <int P>
+__global__ void __launch_bounds__(256) act_stats_kernel(const __nv_bfloat16* __restrict__ X,
+                                                        int64_t T, int d, int64_t ld_x,
+                                                        int64_t rows_per_split, int nsplit,
+                                                        float alpha_over_p, float lambda,
+                                                        float* __restrict__ partial,
+                                                        unsigned* __restrict__ counters,
+                                                        float* __restrict__ s) {
+  __shared__ float red[kRowWarps][kColsPerBlock];
+  __shared__ int is_last;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int col0 = blockIdx.x * kColsPerBlock + lane * 8;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
+  const int64_t r1 = min(T, r0 + rows_per_split);
+
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  if (col0 < d) {
+    const __nv_bfloat16* base = X + col0;
+    int64_t r = r0 + warp;
+    for (; r + 3 * kRowWarps < r1; r += 4 * kRowWarps) {
+      const uint4 v0 = ld_stream(base + r * ld_x);
+      const uint4 v1 = ld_stream(base + (r + kRowWarps) * ld_x);
+      const uint4 v2 = ld_stream(base + (r + 2 * kRowWarps) * ld_x);
+      const uint4 v3 = ld_stream(base + (r + 3 * kRowWarps) * ld_x);
+      accum8<P>(acc, v0);
+      accum8<P>(acc, v1);
+      accum8<P>(acc, v2);
+      accum8<P>(acc, v3);
+    }
+    for (; r < r1; r += kRowWarps) accum8<P>(acc, ld_stream(base + r * ld_x));
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) red[warp][lane * 8 + j] = acc[j];
+  __syncthreads();
+
+  const int col = blockIdx.x * kColsPerBlock + threadIdx.x;
+  float sum = 0.f;
+#pragma unroll
+  for (int w = 0; w < kRowWarps; ++w) sum = __fadd_rn(sum, red[w][threadIdx.x]);
+
+  if (nsplit == 1) {
+    if (col < d) s[col] = finalize_scale(sum, static_cast<float>(T), alpha_over_p, lambda);
+    return;
+  }
+  if (col < d) partial[static_cast<int64_t>(blockIdx.y) * d + col] = sum;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned prev = atomicAdd(&counters[blockIdx.x], 1u);
+    is_last = (prev == static_cast<unsigned>(nsplit - 1));
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  if (col < d) {
+    float tot = 0.f;
+    for (int sp = 0; sp < nsplit; ++sp) tot = __fadd_rn(tot, __ldcg(&partial[static_cast<int64_t>(sp) * d + col]));
+    s[col] = finalize_scale(tot, static_cast<float>(T), alpha_over_p, lambda);
+  }
+  if (threadIdx.x == 0) counters[blockIdx.x] = 0u;  // leave the strip counter ready
+}
+
+// grid: (col_blocks, row_splits); each thread owns 8 consecutive columns for all rows
+// of its split, so the 8 reciprocals 1/s are formed once per thread.
+__global__ void __launch_bounds__(256) fold_kernel(const __nv_bfloat16* __restrict__ X, int64_t T,
+                                                   int d, int64_t ld_x,
+                                                   const float* __restrict__ s,
+                                                   int64_t rows_per_split,
+                                                   __nv_bfloat16* __restrict__ Xf) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int col0 = blockIdx.x * kColsPerBlock + lane * 8;
+  if (col0 >= d) return;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
+  const int64_t r1 = min(T, r0 + rows_per_split);
+  const float4 sa = *reinterpret_cast<const float4*>(s + col0);
+  const float4 sb = *reinterpret_cast<const float4*>(s + col0 + 4);
+  const float rs[8] = {__frcp_rn(sa.x), __frcp_rn(sa.y), __frcp_rn(sa.z), __frcp_rn(sa.w),
+                       __frcp_rn(sb.x), __frcp_rn(sb.y), __frcp_rn(sb.z), __frcp_rn(sb.w)};
+  for (int64_t r = r0 + warp; r < r1; r += kRowWarps) {
+    const uint4 v = ld_stream(X + r * ld_x + col0);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      o[j] = pack_bf16x2(__fmul_rn(bf16lo_to_f32(w[j]), rs[2 * j]),
+                         __fmul_rn(bf16hi_to_f32(w[j]), rs[2 * j + 1]));
+    *reinterpret_cast<uint4*>(Xf + r * d + col0) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// U = X A^T. Block: 256 threads, 32 tokens; the token tile and a 64-column slice of A
+// are staged in shared memory (fp32); thread (token tid/8, ranks tid%8 + 8j) keeps 8
+// fp32 accumulators. Written for r <= 64 (the pages use r = 16).
+constexpr int kUTok = 32;
+constexpr int kUK = 64;
+__global__ void __launch_bounds__(256) lowrank_u_kernel(const __nv_bfloat16* __restrict__ X,
+                                                        int64_t T, int d,
+                                                        const __nv_bfloat16* __restrict__ A,
+                                                        int r, __nv_bfloat16* __restrict__ U) {
+  __shared__ float xs[kUTok][kUK + 1];
+  __shared__ float as[64][kUK + 1];
+  const int tid = threadIdx.x;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kUTok;
+  // thread -> (token tt = tid / 8, ranks rr = tid % 8 + 8*j for j < 8)
+  const int tt = tid >> 3;
+  const int rb = tid & 7;
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  for (int k0 = 0; k0 < d; k0 += kUK) {
+    // stage X tile [32 x 64] and A tile [r x 64]
+    for (int e = tid; e < kUTok * kUK; e += 256) {
+      const int a = e / kUK, b = e % kUK;
+      const int64_t t = t0 + a;
+      xs[a][b] = (t < T && k0 + b < d) ? __bfloat162float(X[t * d + k0 + b]) : 0.f;
+    }
+    for (int e = tid; e < 64 * kUK; e += 256) {
+      const int a = e / kUK, b = e % kUK;
+      as[a][b] = (a < r && k0 + b < d) ? __bfloat162float(A[static_cast<int64_t>(a) * d + k0 + b]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int k = 0; k < kUK; ++k) {
+      const float x = xs[tt][k];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] = __fmaf_rn(x, as[rb + 8 * j][k], acc[j]);
+    }
+    __syncthreads();
+  }
+  const int64_t t = t0 + tt;
+  if (t < T) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int rr = rb + 8 * j;
+      U[t * 64 + rr] = __float2bfloat16_rn(rr < r ? acc[j] : 0.f);
+    }
+  }
+}
+
+}  // namespace
+
+StatsPlan stats_plan(int64_t T, int64_t d) {
+  StatsPlan p;
+  p.col_blocks = static_cast<int>((d + kColsPerBlock - 1) / kColsPerBlock);
+  // aim for about 4 blocks of 256 threads per SM on a 148-SM part, with at least 64
+  // rows per split so each warp streams a few rows
+  const int64_t target_blocks = 148 * 4;
+  int64_t ns = (target_blocks + p.col_blocks - 1) / p.col_blocks;
+  const int64_t max_ns = (T + 63) / 64;
+  if (ns > max_ns) ns = max_ns;
+  if (ns < 1) ns = 1;
+  if (ns > 1024) ns = 1024;
+  p.rows_per_split = (T + ns - 1) / ns;
+  p.nsplit = static_cast<int>((T + p.rows_per_split - 1) / p.rows_per_split);
+  return p;
+}
+
+size_t stats_workspace_bytes(int64_t T, int64_t d) {
+  const StatsPlan p = stats_plan(T, d);
+  const size_t part = static_cast<size_t>(p.nsplit) * static_cast<size_t>(d) * sizeof(float);
+  const size_t cnt = static_cast<size_t>(p.col_blocks) * sizeof(unsigned);
+  return ((part + 255) / 256) * 256 + ((cnt + 255) / 256) * 256;
+}
+
+cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d, int64_t ld_x, float alpha,
+                             float lambda, int p, float* s, float* partial, unsigned* counters,
+                             cudaStream_t stream) {
+  const StatsPlan pl = stats_plan(T, d);
+  if (pl.nsplit > 1) {
+    cudaError_t e = cudaMemsetAsync(counters, 0, pl.col_blocks * sizeof(unsigned), stream);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(pl.col_blocks, pl.nsplit);
+  const float ap = alpha / static_cast<float>(p);
+  if (p == 2)
+    act_stats_kernel<2><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T,
+                                                  static_cast<int>(d), ld_x, pl.rows_per_split,
+                                                  pl.nsplit, ap, lambda, partial, counters, s);
+  else
+    act_stats_kernel<1><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T,
+                                                  static_cast<int>(d), ld_x, pl.rows_per_split,
+                                                  pl.nsplit, ap, lambda, partial, counters, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const float* s,
+                        void* Xf, cudaStream_t stream) {
+  const int col_blocks = static_cast<int>((d + kColsPerBlock - 1) / kColsPerBlock);
+  const int64_t target_blocks = 148 * 8;
+  int64_t ns = (target_blocks + col_blocks - 1) / col_blocks;
+  const int64_t max_ns = (T + 31) / 32;
+  if (ns > max_ns) ns = max_ns;
+  if (ns < 1) ns = 1;
+  if (ns > 65535) ns = 65535;
+  const int64_t rps = (T + ns - 1) / ns;
+  ns = (T + rps - 1) / rps;
+  dim3 grid(col_blocks, static_cast<unsigned>(ns));
+  fold_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T,
+                                        static_cast<int>(d), ld_x, s, rps,
+                                        static_cast<__nv_bfloat16*>(Xf));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A, int r, void* U,
+                             cudaStream_t stream) {
+  const int64_t blocks = (T + kUTok - 1) / kUTok;
+  lowrank_u_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(X), T, static_cast<int>(d),
+      static_cast<const __nv_bfloat16*>(A), r, static_cast<__nv_bfloat16*>(U));
+  return cudaGetLastError();
+}
+
+}  // namespace ttq

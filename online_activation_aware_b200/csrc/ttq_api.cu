@@ -1,0 +1,322 @@
+// C ABI of the TTQ hot path (declared in include/ttq.h): argument validation, workspace
+// layout and the launch sequence of each entry point. Every check happens before any
+// launch, so an argument error leaves the stream untouched.
+#include <atomic>
+#include <cmath>
+
+#include "ttq.h"
+#include "ttq_internal.h"
+
+namespace {
+
+__device__ unsigned g_ttq_error_word;
+
+constexpr int kMaxDevices = 64;
+std::atomic<uint64_t> g_wait_ns{2000000000ull};
+cudaEvent_t g_trace[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+bool g_trace_on = false;
+
+inline cudaError_t trace(int i, cudaStream_t stream) {
+  return g_trace_on ? cudaEventRecord(g_trace[i], stream) : cudaSuccess;
+}
+
+struct DeviceInfo {
+  bool init = false;
+  unsigned* err_word = nullptr;
+  int num_sms = 148;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+ttq_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TTQ_ERR_CUDA;
+  DeviceInfo& di = g_dev[dev];
+  if (!di.init) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_ttq_error_word) != cudaSuccess) return TTQ_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return TTQ_ERR_CUDA;
+    di.err_word = static_cast<unsigned*>(p);
+    di.num_sms = sms;
+    di.init = true;
+  }
+  *out = &di;
+  return TTQ_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+ttq_status check_qg(int32_t q, int32_t g, int64_t d) {
+  if (q < 2 || q > 4) return TTQ_ERR_UNSUPPORTED;
+  if (g != 32 && g != 64 && g != 128) return TTQ_ERR_UNSUPPORTED;
+  if (d % g != 0) return TTQ_ERR_INVALID_ARG;
+  return TTQ_OK;
+}
+
+ttq_status check_stats_args(float alpha, float lambda, int32_t p) {
+  if (p != 1 && p != 2) return TTQ_ERR_UNSUPPORTED;
+  if (!std::isfinite(alpha) || !std::isfinite(lambda) || alpha < 0.f || lambda < 0.f)
+    return TTQ_ERR_INVALID_ARG;
+  if (alpha > 0.f && !(lambda > 0.f)) return TTQ_ERR_INVALID_ARG;
+  return TTQ_OK;
+}
+
+ttq_status check_dims(int64_t T, int64_t d, int64_t d_out) {
+  const int64_t lim = (int64_t(1) << 31) - 1;
+  if (T < 1 || d < 1 || d_out < 1) return TTQ_ERR_INVALID_ARG;
+  if (T > lim || d > lim || d_out > lim || T * d > (int64_t(1) << 40) || d_out * d > (int64_t(1) << 40))
+    return TTQ_ERR_INVALID_ARG;
+  if (d % 8 != 0) return TTQ_ERR_INVALID_ARG;
+  return TTQ_OK;
+}
+
+ttq_status check_cfg(const ttq_config* cfg, int64_t d) {
+  if (!cfg) return TTQ_ERR_INVALID_ARG;
+  ttq_status st = check_qg(cfg->q, cfg->g, d);
+  if (st != TTQ_OK) return st;
+  st = check_stats_args(cfg->alpha, cfg->lambda, cfg->p);
+  if (st != TTQ_OK) return st;
+  if (cfg->r < 0 || cfg->r > 64) return TTQ_ERR_UNSUPPORTED;
+  if (cfg->r % 8 != 0) return TTQ_ERR_UNSUPPORTED;
+  return TTQ_OK;
+}
+
+struct WsLayout {
+  size_t stats_off, stats_bytes;
+  size_t xf_off, xf_bytes;
+  size_t u_off, u_bytes;
+  size_t part_off, part_bytes;
+  size_t total;
+  ttq::GemmPlan plan;
+};
+
+WsLayout ws_layout(int64_t T, int64_t d, int64_t d_out, int r, int num_sms) {
+  WsLayout L{};
+  L.stats_off = 0;
+  L.stats_bytes = round256(ttq::stats_workspace_bytes(T, d));
+  L.xf_off = L.stats_off + L.stats_bytes;
+  L.xf_bytes = d_out > 0 ? round256(static_cast<size_t>(T) * static_cast<size_t>(d) * 2) : 0;
+  L.u_off = L.xf_off + L.xf_bytes;
+  L.u_bytes = (d_out > 0 && r > 0) ? round256(static_cast<size_t>(T) * 64 * 2) : 0;
+  L.part_off = L.u_off + L.u_bytes;
+  if (d_out > 0) {
+    L.plan = ttq::gemm_plan(T, d, d_out, num_sms);
+    L.part_bytes = round256(ttq::gemm_partial_bytes(L.plan, T, d_out));
+  }
+  L.total = L.part_off + L.part_bytes;
+  return L;
+}
+
+ttq::DevErr dev_err(const DeviceInfo* di) { return ttq::DevErr{di->err_word, g_wait_ns.load()}; }
+
+inline ttq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TTQ_OK : TTQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t ttq_codes_words(int64_t d_out, int64_t d, int32_t q) {
+  if (d_out < 0 || d < 0 || d % 32 != 0 || q < 2 || q > 4) return 0;
+  return static_cast<size_t>(d_out) * static_cast<size_t>(d / 32) * static_cast<size_t>(q);
+}
+
+ttq_status ttq_workspace_size(int64_t T, int64_t d, int64_t d_out, const ttq_config* cfg,
+                              size_t* bytes) {
+  if (!bytes) return TTQ_ERR_INVALID_ARG;
+  if (d_out < 0) return TTQ_ERR_INVALID_ARG;
+  ttq_status st = check_dims(T, d, d_out > 0 ? d_out : 1);
+  if (st != TTQ_OK) return st;
+  const int r = cfg ? cfg->r : 0;
+  if (cfg) {
+    st = check_cfg(cfg, d);
+    if (st != TTQ_OK) return st;
+  }
+  int num_sms = 148;
+  DeviceInfo* di = nullptr;
+  if (d_out > 0) {
+    // the split-K plan depends on the SM count of the current device
+    if (device_info(&di) == TTQ_OK) num_sms = di->num_sms;
+  }
+  *bytes = ws_layout(T, d, d_out, r, num_sms).total;
+  return TTQ_OK;
+}
+
+ttq_status ttq_act_stats(const void* X_bf16, int64_t T, int64_t d, int64_t ld_x, float alpha,
+                         float lambda, int32_t p, float* s, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
+  ttq_status st = check_dims(T, d, 1);
+  if (st != TTQ_OK) return st;
+  if (ld_x < d || ld_x % 8 != 0) return TTQ_ERR_INVALID_ARG;
+  st = check_stats_args(alpha, lambda, p);
+  if (st != TTQ_OK) return st;
+  if (!X_bf16 || !s) return TTQ_ERR_INVALID_ARG;
+  if (!ws) return TTQ_ERR_WORKSPACE;
+  if (!aligned16(X_bf16) || !aligned16(s) || !aligned16(ws)) return TTQ_ERR_MISALIGNED;
+  if (ws_bytes < ws_layout(T, d, 0, 0, 148).total) return TTQ_ERR_WORKSPACE;
+  auto* base = static_cast<uint8_t*>(ws);
+  const size_t part_bytes = static_cast<size_t>(ttq::stats_plan(T, d).nsplit) * d * sizeof(float);
+  float* partial = reinterpret_cast<float*>(base);
+  unsigned* counters = reinterpret_cast<unsigned*>(base + round256(part_bytes));
+  return cuda_status(ttq::launch_act_stats(X_bf16, T, d, ld_x, alpha, lambda, p, s, partial,
+                                           counters, stream));
+}
+
+ttq_status ttq_requant(const void* W_bf16, int64_t d_out, int64_t d, const float* s, int32_t q,
+                       int32_t g, uint32_t* codes, void* scale_f16, void* zero_f16,
+                       cudaStream_t stream) {
+  ttq_status st = check_dims(1, d, d_out);
+  if (st != TTQ_OK) return st;
+  st = check_qg(q, g, d);
+  if (st != TTQ_OK) return st;
+  if (!W_bf16 || !s || !codes || !scale_f16 || !zero_f16) return TTQ_ERR_INVALID_ARG;
+  if (!aligned16(W_bf16) || !aligned16(s) || !aligned16(codes) || !aligned16(scale_f16) ||
+      !aligned16(zero_f16))
+    return TTQ_ERR_MISALIGNED;
+  return cuda_status(ttq::launch_requant(W_bf16, d_out, d, s, q, g, codes, scale_f16, zero_f16, stream));
+}
+
+static ttq_status check_lowrank(const ttq_config* cfg, const void* A, const void* B) {
+  if (cfg->r > 0) {
+    if (!A || !B) return TTQ_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B)) return TTQ_ERR_MISALIGNED;
+  } else if (A || B) {
+    return TTQ_ERR_INVALID_ARG;
+  }
+  return TTQ_OK;
+}
+
+ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const void* W_bf16,
+                              int64_t d_out, const void* A_bf16, const void* B_bf16,
+                              const ttq_config* cfg, float* s, uint32_t* codes, void* scale_f16,
+                              void* zero_f16, void* Y_bf16, void* ws, size_t ws_bytes,
+                              cudaStream_t stream) {
+  ttq_status st = check_dims(T, d, d_out);
+  if (st != TTQ_OK) return st;
+  st = check_cfg(cfg, d);
+  if (st != TTQ_OK) return st;
+  st = check_lowrank(cfg, A_bf16, B_bf16);
+  if (st != TTQ_OK) return st;
+  if (!X_bf16 || !W_bf16 || !s || !codes || !scale_f16 || !zero_f16 || !Y_bf16)
+    return TTQ_ERR_INVALID_ARG;
+  if (!ws) return TTQ_ERR_WORKSPACE;
+  if (!aligned16(X_bf16) || !aligned16(W_bf16) || !aligned16(s) || !aligned16(codes) ||
+      !aligned16(scale_f16) || !aligned16(zero_f16) || !aligned16(Y_bf16) || !aligned16(ws))
+    return TTQ_ERR_MISALIGNED;
+  DeviceInfo* di = nullptr;
+  st = device_info(&di);
+  if (st != TTQ_OK) return st;
+  const WsLayout L = ws_layout(T, d, d_out, cfg->r, di->num_sms);
+  if (ws_bytes < L.total) return TTQ_ERR_WORKSPACE;
+  auto* base = static_cast<uint8_t*>(ws);
+  const size_t part_bytes = static_cast<size_t>(ttq::stats_plan(T, d).nsplit) * d * sizeof(float);
+  float* spart = reinterpret_cast<float*>(base + L.stats_off);
+  unsigned* counters = reinterpret_cast<unsigned*>(base + L.stats_off + round256(part_bytes));
+  void* Xf = base + L.xf_off;
+  void* U = cfg->r > 0 ? base + L.u_off : nullptr;
+  float* gpart = L.part_bytes ? reinterpret_cast<float*>(base + L.part_off) : nullptr;
+
+  cudaError_t e = trace(0, stream);
+  if (e == cudaSuccess)
+    e = ttq::launch_act_stats(X_bf16, T, d, d, cfg->alpha, cfg->lambda, cfg->p, s, spart, counters, stream);
+  if (e == cudaSuccess) e = trace(1, stream);
+  if (e == cudaSuccess) e = ttq::launch_fold(X_bf16, T, d, d, s, Xf, stream);
+  if (e == cudaSuccess && cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, T, d, A_bf16, cfg->r, U, stream);
+  if (e == cudaSuccess) e = trace(2, stream);
+  if (e == cudaSuccess)
+    e = ttq::launch_requant(W_bf16, d_out, d, s, cfg->q, cfg->g, codes, scale_f16, zero_f16, stream);
+  if (e == cudaSuccess) e = trace(3, stream);
+  if (e == cudaSuccess) {
+    ttq::GemmArgs ga{Xf, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, T, d, d_out, cfg->q, cfg->g,
+                     Y_bf16, gpart};
+    e = ttq::launch_gemm_mainloop(ga, L.plan, dev_err(di), stream);
+    if (e == cudaSuccess) e = trace(4, stream);
+    if (e == cudaSuccess) e = ttq::launch_gemm_reduce(ga, L.plan, stream);
+  }
+  if (e == cudaSuccess) e = trace(5, stream);
+  return cuda_status(e);
+}
+
+ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d_out,
+                             const float* s, const uint32_t* codes, const void* scale_f16,
+                             const void* zero_f16, const void* A_bf16, const void* B_bf16,
+                             const ttq_config* cfg, void* Y_bf16, void* ws, size_t ws_bytes,
+                             cudaStream_t stream) {
+  ttq_status st = check_dims(b, d, d_out);
+  if (st != TTQ_OK) return st;
+  st = check_cfg(cfg, d);
+  if (st != TTQ_OK) return st;
+  st = check_lowrank(cfg, A_bf16, B_bf16);
+  if (st != TTQ_OK) return st;
+  if (!X_bf16 || !s || !codes || !scale_f16 || !zero_f16 || !Y_bf16) return TTQ_ERR_INVALID_ARG;
+  if (!ws) return TTQ_ERR_WORKSPACE;
+  if (!aligned16(X_bf16) || !aligned16(s) || !aligned16(codes) || !aligned16(scale_f16) ||
+      !aligned16(zero_f16) || !aligned16(Y_bf16) || !aligned16(ws))
+    return TTQ_ERR_MISALIGNED;
+  DeviceInfo* di = nullptr;
+  st = device_info(&di);
+  if (st != TTQ_OK) return st;
+  const WsLayout L = ws_layout(b, d, d_out, cfg->r, di->num_sms);
+  if (ws_bytes < L.total) return TTQ_ERR_WORKSPACE;
+  auto* base = static_cast<uint8_t*>(ws);
+  void* Xf = base + L.xf_off;
+  void* U = cfg->r > 0 ? base + L.u_off : nullptr;
+  float* gpart = L.part_bytes ? reinterpret_cast<float*>(base + L.part_off) : nullptr;
+  cudaError_t e = ttq::launch_fold(X_bf16, b, d, d, s, Xf, stream);
+  if (e == cudaSuccess && cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, stream);
+  if (e == cudaSuccess) {
+    ttq::GemmArgs ga{Xf, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g,
+                     Y_bf16, gpart};
+    e = ttq::launch_gemm(ga, L.plan, dev_err(di), stream);
+  }
+  return cuda_status(e);
+}
+
+ttq_status ttq_device_status(cudaStream_t stream) {
+  DeviceInfo* di = nullptr;
+  ttq_status st = device_info(&di);
+  if (st != TTQ_OK) return st;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return TTQ_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_ttq_error_word, sizeof(word)) != cudaSuccess) return TTQ_ERR_CUDA;
+  if (word != 0) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_ttq_error_word, &zero, sizeof(zero)) != cudaSuccess) return TTQ_ERR_CUDA;
+    return TTQ_ERR_TIMEOUT;
+  }
+  return TTQ_OK;
+}
+
+ttq_status ttq_set_wait_limit_ns(uint64_t ns) {
+  g_wait_ns.store(ns == 0 ? 2000000000ull : ns);
+  return TTQ_OK;
+}
+
+ttq_status ttq_set_trace_events(void* const* events, int32_t n) {
+  if (n == 0 || events == nullptr) {
+    g_trace_on = false;
+    return TTQ_OK;
+  }
+  if (n < 6) return TTQ_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i) {
+    if (!events[i]) return TTQ_ERR_INVALID_ARG;
+  }
+  for (int i = 0; i < 6; ++i) g_trace[i] = static_cast<cudaEvent_t>(events[i]);
+  g_trace_on = true;
+  return TTQ_OK;
+}
+
+const char* ttq_status_string(ttq_status status) {
+  switch (status) {
+    case TTQ_OK: return "TTQ_OK";
+    case TTQ_ERR_INVALID_ARG: return "TTQ_ERR_INVALID_ARG";
+    case TTQ_ERR_UNSUPPORTED: return "TTQ_ERR_UNSUPPORTED";
+    case TTQ_ERR_MISALIGNED: return "TTQ_ERR_MISALIGNED";
+    case TTQ_ERR_WORKSPACE: return "TTQ_ERR_WORKSPACE";
+    case TTQ_ERR_CUDA: return "TTQ_ERR_CUDA";
+    case TTQ_ERR_TIMEOUT: return "TTQ_ERR_TIMEOUT";
+  }
+  return "TTQ_ERR_UNKNOWN";
+}
+
+}  // extern "C"

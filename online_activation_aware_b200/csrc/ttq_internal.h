@@ -1,0 +1,85 @@
+// Internal launch interface between the C ABI (ttq_api.cu) and the kernel files.
+// Every launcher enqueues on `stream` and returns the launch status; none allocates.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ttq_common.cuh"
+
+namespace ttq {
+
+// ---------------------------------------------------------------- act_stats / fold
+
+// Column-split plan of the statistics kernel: blocks of 256 columns, T split in
+// `nsplit` row ranges of `rows_per_split` rows.
+struct StatsPlan {
+  int col_blocks;
+  int nsplit;
+  int64_t rows_per_split;
+};
+StatsPlan stats_plan(int64_t T, int64_t d);
+size_t stats_workspace_bytes(int64_t T, int64_t d);  // partial sums + counters
+
+// s = (mean_t |x|^p + lambda)^(alpha/p); partial/counters live in the workspace.
+cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d, int64_t ld_x, float alpha,
+                             float lambda, int p, float* s, float* partial, unsigned* counters,
+                             cudaStream_t stream);
+
+// Xf[t, j] = bf16(X[t, j] * (1 / s[j])), Xf contiguous [T, d].
+cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const float* s,
+                        void* Xf, cudaStream_t stream);
+
+// U[t, :] = X[t, :] A^T in fp32 accumulation, stored bf16 with row stride 64 (columns
+// r..63 zero). Requires r <= 64.
+cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A, int r, void* U,
+                             cudaStream_t stream);
+
+// ---------------------------------------------------------------- requant
+
+cudaError_t launch_requant(const void* W, int64_t d_out, int64_t d, const float* s, int q, int g,
+                           uint32_t* codes, void* scale, void* zero, cudaStream_t stream);
+
+// ---------------------------------------------------------------- GEMM
+
+struct GemmPlan {
+  int BN;           // tokens per CTA tile (MMA N): 16, 32, 64, 128 or 256
+  int m_tiles;      // ceil(d_out / 128)
+  int n_tiles;      // ceil(T / BN)
+  int nkb;          // K blocks of 64: ceil(d / 64)
+  int ksplit;       // split-K factor (1 = direct bf16 epilogue)
+  int kb_per_split;
+  size_t smem_bytes;
+};
+GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int num_sms);
+size_t gemm_partial_bytes(const GemmPlan& p, int64_t T, int64_t d_out);
+
+struct GemmArgs {
+  const void* Xf;        // bf16 [T, d] folded activations
+  const uint32_t* codes; // packed codes [d_out, d*q/32]
+  const void* scale;     // fp16 [d_out, d/g]
+  const void* zero;      // fp16 [d_out, d/g]
+  const void* U;         // bf16 [T, 64] low-rank projection (r > 0) or null
+  const void* Blr;       // bf16 [d_out, r] (r > 0) or null
+  int r;
+  int64_t T, d, d_out;
+  int q, g;
+  void* Y;               // bf16 [T, d_out]
+  float* partial;        // fp32 [ksplit, T, d_out] when ksplit > 1
+};
+
+// The tensor-core kernel (writes Y directly, or fp32 partials when plan.ksplit > 1) and
+// the split-K reduction (a no-op when plan.ksplit == 1); launch_gemm runs both.
+cudaError_t launch_gemm_mainloop(const GemmArgs& a, const GemmPlan& plan, const DevErr& err,
+                                 cudaStream_t stream);
+cudaError_t launch_gemm_reduce(const GemmArgs& a, const GemmPlan& plan, cudaStream_t stream);
+cudaError_t launch_gemm(const GemmArgs& a, const GemmPlan& plan, const DevErr& err,
+                        cudaStream_t stream);
+
+// Encodes a 2-D row-major bf16 tensor map with 128-byte swizzle and a box of
+// {64 columns, box_rows rows}. Returns false when the driver refuses it.
+bool encode_bf16_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                      uint64_t row_stride_elems, uint32_t box_rows);
+
+}  // namespace ttq

@@ -1,0 +1,137 @@
+"""The C-ABI library on the host, without a GPU: it loads, it exports every entry point
+include/ttq.h declares, and argument errors come back synchronously with the
+documented status before anything touches the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import online_activation_aware_b200 as ttq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, INVALID, UNSUPPORTED, MISALIGNED, WORKSPACE = 0, -1, -2, -3, -4
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from online_activation_aware_b200 import build
+
+    build.build()
+    return ttq.load_library()
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "ttq.h")) as f:
+        text = f.read()
+    return re.findall(r"TTQ_API\s+[\w\s\*]+?\b(ttq_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    for n in ("ttq_act_stats", "ttq_requant", "ttq_linear_prefill", "ttq_linear_decode",
+              "ttq_workspace_size", "ttq_codes_words", "ttq_device_status", "ttq_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_codes_words(lib):
+    assert ttq.codes_words(8192, 5120, 4) == 8192 * 5120 * 4 // 32
+    assert ttq.codes_words(3, 96, 3) == 3 * 3 * 3
+    assert lib.ttq_codes_words(4, 100, 4) == 0  # d not a multiple of 32
+    assert lib.ttq_codes_words(4, 64, 5) == 0
+
+
+def test_status_strings(lib):
+    for code, name in ttq.STATUS.items():
+        assert lib.ttq_status_string(code).decode() == name
+
+
+def test_workspace_size_components(lib):
+    cfg = ttq.make_config(4, 128, 0.5, 0.4)
+    ws_stats = ttq.workspace_size(4096, 5120, 0)
+    ws_full = ttq.workspace_size(4096, 5120, 8192, cfg)
+    assert ws_stats > 0
+    # the folded activations alone are T * d bf16
+    assert ws_full >= ws_stats + 4096 * 5120 * 2
+    cfg_r = ttq.make_config(4, 128, 0.5, 0.4, r=16)
+    assert ttq.workspace_size(4096, 5120, 8192, cfg_r) >= ws_full + 4096 * 64 * 2
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+def test_requant_argument_errors(lib):
+    a = 1 << 20  # a 16-byte-aligned fake address: never dereferenced on these paths
+    assert lib.ttq_requant(_p(a), 16, 64, _p(a), 5, 32, _p(a), _p(a), _p(a), None) == UNSUPPORTED
+    assert lib.ttq_requant(_p(a), 16, 64, _p(a), 4, 48, _p(a), _p(a), _p(a), None) == UNSUPPORTED
+    assert lib.ttq_requant(_p(a), 16, 96, _p(a), 4, 64, _p(a), _p(a), _p(a), None) == INVALID
+    assert lib.ttq_requant(None, 16, 64, _p(a), 4, 32, _p(a), _p(a), _p(a), None) == INVALID
+    assert lib.ttq_requant(_p(a + 8), 16, 64, _p(a), 4, 32, _p(a), _p(a), _p(a), None) == MISALIGNED
+    assert lib.ttq_requant(_p(a), 0, 64, _p(a), 4, 32, _p(a), _p(a), _p(a), None) == INVALID
+
+
+def test_act_stats_argument_errors(lib):
+    a = 1 << 20
+    f = ctypes.c_float
+    assert lib.ttq_act_stats(_p(a), 8, 64, 64, f(0.5), f(0.4), 3, _p(a), _p(a), 1 << 20, None) == UNSUPPORTED
+    assert lib.ttq_act_stats(_p(a), 8, 64, 64, f(-0.5), f(0.4), 2, _p(a), _p(a), 1 << 20, None) == INVALID
+    assert lib.ttq_act_stats(_p(a), 8, 64, 64, f(0.5), f(0.0), 2, _p(a), _p(a), 1 << 20, None) == INVALID
+    assert lib.ttq_act_stats(_p(a), 8, 64, 32, f(0.5), f(0.4), 2, _p(a), _p(a), 1 << 20, None) == INVALID
+    assert lib.ttq_act_stats(_p(a), 8, 60, 64, f(0.5), f(0.4), 2, _p(a), _p(a), 1 << 20, None) == INVALID
+    assert lib.ttq_act_stats(_p(a), 8, 64, 64, f(0.5), f(0.4), 2, _p(a), None, 1 << 20, None) == WORKSPACE
+    assert lib.ttq_act_stats(_p(a + 4), 8, 64, 64, f(0.5), f(0.4), 2, _p(a), _p(a), 1 << 20, None) == MISALIGNED
+    assert lib.ttq_act_stats(_p(a), 8, 64, 64, f(0.5), f(0.4), 2, _p(a), _p(a), 16, None) == WORKSPACE
+    assert lib.ttq_act_stats(_p(a), 0, 64, 64, f(0.5), f(0.4), 2, _p(a), _p(a), 1 << 20, None) == INVALID
+
+
+@pytest.mark.parametrize("cfg,status", [
+    (dict(q=4, g=32, alpha=0.5, lam=0.4, p=2, r=12), UNSUPPORTED),   # r not a multiple of 8
+    (dict(q=4, g=32, alpha=0.5, lam=0.4, p=2, r=72), UNSUPPORTED),   # r > 64
+    (dict(q=4, g=32, alpha=0.5, lam=0.4, p=4, r=0), UNSUPPORTED),
+    (dict(q=1, g=32, alpha=0.5, lam=0.4, p=2, r=0), UNSUPPORTED),
+    (dict(q=4, g=32, alpha=0.5, lam=0.0, p=2, r=0), INVALID),        # lambda must be > 0
+    (dict(q=4, g=32, alpha=float("nan"), lam=0.4, p=2, r=0), INVALID),
+])
+def test_prefill_config_errors(lib, cfg, status):
+    a = 1 << 20
+    c = ttq.make_config(cfg["q"], cfg["g"], cfg["alpha"], cfg["lam"], cfg["p"], cfg["r"])
+    A = _p(a) if cfg["r"] > 0 else None
+    rc = lib.ttq_linear_prefill(_p(a), 16, 128, _p(a), 64, A, A, ctypes.byref(c), _p(a), _p(a), _p(a),
+                                _p(a), _p(a), _p(a), 1 << 30, None)
+    assert rc == status
+
+
+def test_prefill_lowrank_pointer_rules(lib):
+    a = 1 << 20
+    c0 = ttq.make_config(4, 32, 0.5, 0.4, 2, 0)
+    c16 = ttq.make_config(4, 32, 0.5, 0.4, 2, 16)
+    args = (_p(a), _p(a), _p(a), _p(a), _p(a), _p(a), 1 << 30, None)
+    # factors given with r = 0, or missing with r > 0
+    assert lib.ttq_linear_prefill(_p(a), 16, 128, _p(a), 64, _p(a), _p(a), ctypes.byref(c0), *args) == INVALID
+    assert lib.ttq_linear_prefill(_p(a), 16, 128, _p(a), 64, None, None, ctypes.byref(c16), *args) == INVALID
+    assert lib.ttq_linear_prefill(_p(a), 16, 128, _p(a), 64, _p(a + 2), _p(a), ctypes.byref(c16), *args) == MISALIGNED
+
+
+def test_decode_argument_errors(lib):
+    a = 1 << 20
+    c = ttq.make_config(3, 128, 0.5, 0.4)
+    assert lib.ttq_linear_decode(_p(a), 1, 96, 64, _p(a), _p(a), _p(a), _p(a), None, None, ctypes.byref(c),
+                                 _p(a), _p(a), 1 << 30, None) == INVALID  # d % g != 0
+    c = ttq.make_config(3, 32, 0.5, 0.4)
+    assert lib.ttq_linear_decode(_p(a), 1, 96, 64, _p(a), _p(a), _p(a), _p(a), None, None, ctypes.byref(c),
+                                 _p(a), None, 1 << 30, None) == WORKSPACE
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    torch = pytest.importorskip("torch")
+    X = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ttq.act_stats(X, 0.5, 0.4, s=torch.zeros(64), ws=torch.zeros(1024, dtype=torch.uint8))
