@@ -76,6 +76,12 @@ def gemm_flops(T, d, d_out, r):
     return 2.0 * T * d * d_out + (2.0 * T * r * d_out if r else 0.0)
 
 
+def whole_job_ktoks(T, steps, world, t_max_ms):
+    """Whole-job throughput: every rank processed `steps` prompts of T tokens; the job
+    took as long as its slowest rank."""
+    return T * steps * world / (t_max_ms / 1e3) / 1e3
+
+
 def decode_bytes(b, d, d_out, q, g):
     return d_out * d * q // 8 + d_out * (d // g) * 4 + b * d * 2 + b * d_out * 2 + d * 4
 
@@ -367,8 +373,7 @@ def main():
     stage_names = ["stats", "fold", "requant", "gemm", "reduce"]
     stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
                 for j, n in enumerate(stage_names)}
-    tokens = T * K * world
-    value = tokens / (t_max_ms / 1e3) / 1e3
+    value = whole_job_ktoks(T, K, world, t_max_ms)
 
     plan_split = stage_ms["reduce"] > 0.002
     launches_per_step = 4 + (1 if r > 0 else 0) + (1 if plan_split else 0)
