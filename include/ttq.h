@@ -56,7 +56,8 @@ typedef enum {
   TTQ_ERR_MISALIGNED = -3,   /* a pointer (or leading dimension) is not 16-byte aligned */
   TTQ_ERR_WORKSPACE = -4,    /* ws is NULL or smaller than ttq_workspace_size()       */
   TTQ_ERR_CUDA = -5,         /* a CUDA runtime call or kernel launch failed            */
-  TTQ_ERR_TIMEOUT = -6       /* a kernel gave up on a bounded wait (device error word) */
+  TTQ_ERR_TIMEOUT = -6,      /* a kernel gave up on a bounded wait (device error word) */
+  TTQ_ERR_TOO_LARGE = -7     /* a size exceeds a fixed internal capacity               */
 } ttq_status;
 
 /* TTQ settings. q: bits per weight; g: group size along d; alpha, lambda, p: the
@@ -93,6 +94,27 @@ TTQ_API ttq_status ttq_workspace_size(int64_t T, int64_t d, int64_t d_out, const
 TTQ_API ttq_status ttq_act_stats(const void* X_bf16, int64_t T, int64_t d, int64_t ld_x, float alpha,
                          float lambda, int32_t p, float* s, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
+
+/* Allocation-free variant of ttq_act_stats, for callers that cannot allocate device
+ * memory: code running where cudaMalloc is unavailable or too costly (cudaMalloc can
+ * synchronise the whole device, which a latency-bound serving loop cannot afford), or
+ * code embedded in a program whose allocator has already reserved all device memory
+ * (for example a serving engine that claims the free HBM for its KV cache at start-up)
+ * and so cannot hand out a workspace. The paper has no counterpart: this is a
+ * deployment convenience of this library.
+ * Same inputs, output and numerics as ttq_act_stats, without the workspace argument:
+ * the partial sums live in a fixed scratch array in the library's device memory (1 MiB
+ * of fp32 partial sums plus 1 KiB of counters, held on every GPU that loads the library
+ * until the process exits). Limits: d <= 65536 channels, else TTQ_ERR_TOO_LARGE and
+ * nothing is launched; the row split of the reduction shrinks so that it fits.
+ * The first call on a device looks up the scratch array's device address (with that
+ * device current); make that first call before any stream capture. Every call on a
+ * device shares the one array and overwrites it (its counters are cleared by each
+ * call): calls whose kernels overlap on the GPU (other streams, other host threads)
+ * race and must be serialised by the caller. */
+TTQ_API ttq_status ttq_act_stats_noalloc(const void* X_bf16, int64_t T, int64_t d, int64_t ld_x,
+                                         float alpha, float lambda, int32_t p, float* s,
+                                         cudaStream_t stream);
 
 /* Re-quantization of W diag(s) ([DR] section 2 W_hat = Q[W D^(1/2)] D^(-1/2); [NR]
  * group-wise round-to-nearest quantize-dequantize). For each output row i and each

@@ -21,7 +21,7 @@ PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG_DIR, "libttq.so")
 
 STATUS = {0: "TTQ_OK", -1: "TTQ_ERR_INVALID_ARG", -2: "TTQ_ERR_UNSUPPORTED", -3: "TTQ_ERR_MISALIGNED",
-          -4: "TTQ_ERR_WORKSPACE", -5: "TTQ_ERR_CUDA", -6: "TTQ_ERR_TIMEOUT"}
+          -4: "TTQ_ERR_WORKSPACE", -5: "TTQ_ERR_CUDA", -6: "TTQ_ERR_TIMEOUT", -7: "TTQ_ERR_TOO_LARGE"}
 
 
 class TTQError(RuntimeError):
@@ -55,6 +55,8 @@ def load_library(path: str = LIB_PATH):
     lib.ttq_workspace_size.restype = i32
     lib.ttq_act_stats.argtypes = [vp, i64, i64, i64, f32, f32, i32, vp, vp, sz, vp]
     lib.ttq_act_stats.restype = i32
+    lib.ttq_act_stats_noalloc.argtypes = [vp, i64, i64, i64, f32, f32, i32, vp, vp]
+    lib.ttq_act_stats_noalloc.restype = i32
     lib.ttq_requant.argtypes = [vp, i64, i64, vp, i32, i32, vp, vp, vp, vp]
     lib.ttq_requant.restype = i32
     lib.ttq_linear_prefill.argtypes = [vp, i64, i64, vp, i64, vp, vp, cfgp, vp, vp, vp, vp, vp, vp, sz, vp]

@@ -241,6 +241,34 @@ cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d, int64_t ld_x, 
   return cudaGetLastError();
 }
 
+cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t ld_x, float alpha,
+                                    float lambda, int p, float* s, float* partial,
+                                    int64_t max_partial_floats, unsigned* counters,
+                                    cudaStream_t stream) {
+  StatsPlan pl = stats_plan(T, d);
+  if (static_cast<int64_t>(pl.nsplit) * d > max_partial_floats) {
+    int64_t ns = max_partial_floats / d;
+    if (ns < 1) ns = 1;
+    pl.rows_per_split = (T + ns - 1) / ns;
+    pl.nsplit = static_cast<int>((T + pl.rows_per_split - 1) / pl.rows_per_split);
+  }
+  if (pl.nsplit > 1) {
+    cudaError_t e = cudaMemsetAsync(counters, 0, pl.col_blocks * sizeof(unsigned), stream);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(pl.col_blocks, pl.nsplit);
+  const float ap = alpha / static_cast<float>(p);
+  if (p == 2)
+    act_stats_kernel<2><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T,
+                                                  static_cast<int>(d), ld_x, pl.rows_per_split,
+                                                  pl.nsplit, ap, lambda, partial, counters, s);
+  else
+    act_stats_kernel<1><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T,
+                                                  static_cast<int>(d), ld_x, pl.rows_per_split,
+                                                  pl.nsplit, ap, lambda, partial, counters, s);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const float* s,
                         void* Xf, cudaStream_t stream) {
   const int col_blocks = static_cast<int>((d + kColsPerBlock - 1) / kColsPerBlock);

@@ -315,6 +315,7 @@ const char* ttq_status_string(ttq_status status) {
     case TTQ_ERR_WORKSPACE: return "TTQ_ERR_WORKSPACE";
     case TTQ_ERR_CUDA: return "TTQ_ERR_CUDA";
     case TTQ_ERR_TIMEOUT: return "TTQ_ERR_TIMEOUT";
+    case TTQ_ERR_TOO_LARGE: return "TTQ_ERR_TOO_LARGE";
   }
   return "TTQ_ERR_UNKNOWN";
 }

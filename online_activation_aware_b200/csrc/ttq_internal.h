@@ -27,6 +27,13 @@ cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d, int64_t ld_x, 
                              float lambda, int p, float* s, float* partial, unsigned* counters,
                              cudaStream_t stream);
 
+// Same statistic, with at most `max_partial_floats` fp32 partial sums: the row split is
+// reduced until nsplit * d fits (used where the scratch has a fixed size).
+cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t ld_x, float alpha,
+                                    float lambda, int p, float* s, float* partial,
+                                    int64_t max_partial_floats, unsigned* counters,
+                                    cudaStream_t stream);
+
 // Xf[t, j] = bf16(X[t, j] * (1 / s[j])), Xf contiguous [T, d].
 cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const float* s,
                         void* Xf, cudaStream_t stream);
