@@ -173,6 +173,13 @@ TTQ_API ttq_status ttq_device_status(cudaStream_t stream);
  * after the call. A limit of 0 restores the default. */
 TTQ_API ttq_status ttq_set_wait_limit_ns(uint64_t ns);
 
+/* Test hook for failure detection: while enabled, every later launch of the tensor-core
+ * kernel first waits on a barrier that nothing ever arrives at, so that wait runs out
+ * after the limit set by ttq_set_wait_limit_ns; the kernel then records TTQ_ERR_TIMEOUT,
+ * drains its own copies, frees its tensor memory and returns without writing Y. Used to
+ * test the bounded waits; never enable it in production. */
+TTQ_API ttq_status ttq_debug_inject_stall(int32_t enable);
+
 /* Stage tracing for measurement. With n >= 6 event handles (cudaEvent_t created by the
  * caller with timing enabled), every later ttq_linear_prefill call records, on its
  * stream: events[0] before the statistics, [1] after them, [2] after the fold (and the
@@ -181,6 +188,11 @@ TTQ_API ttq_status ttq_set_wait_limit_ns(uint64_t ns);
  * follows [4]). n = 0 (or events = NULL) turns tracing off. The library keeps the
  * handles, not copies: they must stay valid while tracing is on. Not thread-safe. */
 TTQ_API ttq_status ttq_set_trace_events(void* const* events, int32_t n);
+
+/* The CUDA runtime error code behind the most recent TTQ_ERR_CUDA returned to this host
+ * thread (0 when there was none), and a static description of such a code. */
+TTQ_API int32_t ttq_last_cuda_error(void);
+TTQ_API const char* ttq_cuda_error_string(int32_t code);
 
 /* A static string naming a status code. */
 TTQ_API const char* ttq_status_string(ttq_status status);

@@ -25,9 +25,9 @@ STATUS = {0: "TTQ_OK", -1: "TTQ_ERR_INVALID_ARG", -2: "TTQ_ERR_UNSUPPORTED", -3:
 
 
 class TTQError(RuntimeError):
-    def __init__(self, fn: str, status: int):
+    def __init__(self, fn: str, status: int, detail: str = ""):
         self.status = status
-        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}{detail}")
 
 
 class Config(ctypes.Structure):
@@ -67,6 +67,12 @@ def load_library(path: str = LIB_PATH):
     lib.ttq_device_status.restype = i32
     lib.ttq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.ttq_set_wait_limit_ns.restype = i32
+    lib.ttq_last_cuda_error.argtypes = []
+    lib.ttq_last_cuda_error.restype = i32
+    lib.ttq_cuda_error_string.argtypes = [i32]
+    lib.ttq_cuda_error_string.restype = ctypes.c_char_p
+    lib.ttq_debug_inject_stall.argtypes = [i32]
+    lib.ttq_debug_inject_stall.restype = i32
     lib.ttq_set_trace_events.argtypes = [ctypes.POINTER(vp), i32]
     lib.ttq_set_trace_events.restype = i32
     lib.ttq_status_string.argtypes = [i32]
@@ -77,7 +83,11 @@ def load_library(path: str = LIB_PATH):
 
 def _check(fn: str, status: int):
     if status != 0:
-        raise TTQError(fn, status)
+        detail = ""
+        if status == -5 and _lib is not None:
+            code = int(_lib.ttq_last_cuda_error())
+            detail = f" (cuda error {code}: {_lib.ttq_cuda_error_string(code).decode()})"
+        raise TTQError(fn, status, detail)
 
 
 def _ptr(t, dtype=None, name="tensor"):
@@ -210,6 +220,11 @@ def linear_decode(X, s, codes, scale, zero, cfg: Config, d_out: int, A=None, B=N
 def device_status(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the library's device error status."""
     return int(load_library().ttq_device_status(_stream(stream)))
+
+
+def debug_inject_stall(enable: bool):
+    """Test hook: makes the tensor-core kernel wait on a barrier nothing arrives at."""
+    _check("ttq_debug_inject_stall", load_library().ttq_debug_inject_stall(1 if enable else 0))
 
 
 def set_wait_limit_ns(ns: int):

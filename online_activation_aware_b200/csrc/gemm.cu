@@ -5,17 +5,22 @@
 // (paper-daily.com deep reading of TTQ, section 2: W_hat = Q[W D^(1/2)] D^(-1/2) and
 // W_hat = W_q + BA; section 5 notes a kernel that fuses the pre-scaling).
 //
-// One CTA computes a 128 (weight rows) x BN (tokens) tile: D = A * B^T with
-// A = dequantised weight tile [128 x 64] and B = X' tile [BN x 64] per K block, the fp32
-// accumulator in tensor memory (128 lanes x BN columns). Warp roles:
+// Persistent kernel, one CTA per SM, walking 128 (weight rows) x BN (tokens) output
+// tiles: D = A * B^T per K block of 64, A = dequantised weight tile [128 x 64], B = X'
+// tile [BN x 64], fp32 accumulators in tensor memory, two of them so that the epilogue
+// of one tile overlaps the main loop of the next. Warp roles (14 warps):
 //   warp 0      TMA producer: X' tiles (and the low-rank U / B tiles) into a ring of
 //               shared-memory stages, completion counted in bytes on `full` barriers;
-//   warp 1      allocates tensor memory; one thread issues tcgen05.mma (M=128, N=BN,
-//               K=16, bf16 in, fp32 accumulate) and commits each stage back to `empty`;
-//   warps 2-5   dequantisers: each thread owns one weight row of the tile, streams its
-//               codes and group scale/zero through a private cp.async ring, writes 64
-//               bf16 per K block in the 128-byte-swizzled K-major layout the MMA reads,
-//               and arrives on `afull`; afterwards they are the epilogue (TMEM -> Y).
+//   warp 1      allocates tensor memory; one thread issues tcgen05.mma (M = 128,
+//               N = BN, K = 16, bf16 in, fp32 accumulate), commits each stage back to
+//               `empty` and each finished tile to `tfull`;
+//   warps 2-9   dequantisers: 256 threads, one per (tile row, half K block): each streams
+//               its 32 codes and the group's scale/zero per K block through a private
+//               cp.async ring, expands them to bf16 ((c - z) * sigma, exact in fp32, one
+//               rounding) in the 128-byte-swizzled K-major layout the MMA reads, and
+//               arrives on `afull`;
+//   warps 10-13 epilogue: tcgen05.ld of the finished accumulator, bf16 conversion,
+//               64-byte coalesced stores of Y (or fp32 split-K partials), then `tempty`.
 // No TMA multicast is used anywhere. Every mbarrier wait is bounded in time.
 #include "ttq_internal.h"
 
@@ -25,17 +30,25 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kMaxStages = 4;
-constexpr int kThreads = 192;
-constexpr int kDqThreads = 128;
-constexpr int kSlotBytes = 48;  // per thread per K block: 32 B codes + 8 B scale + 8 B zero
+constexpr int kNumDqWarps = 8;
+constexpr int kNumEpiWarps = 4;
+constexpr int kDqWarp0 = 2;
+constexpr int kEpiWarp0 = kDqWarp0 + kNumDqWarps;
+constexpr int kThreads = 32 * (kEpiWarp0 + kNumEpiWarps);  // 448
+constexpr int kDqThreads = 32 * kNumDqWarps;                // 256
+constexpr int kEpiThreads = 32 * kNumEpiWarps;              // 128
+constexpr int kSlotBytes = 32;  // per dequant thread per K block: 16 B codes, 4 B scale, 4 B zero
 constexpr uint32_t kATileBytes = kBM * kBK * 2;  // 16 KB
+constexpr int kMaxStages = 4;
 
 struct __align__(16) Tail {
   uint64_t full[kMaxStages];
   uint64_t afull[kMaxStages];
   uint64_t empty[kMaxStages];
-  uint64_t accum;
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint64_t stall;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -70,8 +83,34 @@ __device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint3
                : "memory");
 }
 
-// exact float value of a small non-negative integer code: 2^23 + c, as bits
-__device__ __forceinline__ float magic_code(uint32_t c) { return __uint_as_float(0x4B000000u | c); }
+// Two fp32 lanes at once (sm_100 packed fp32 arithmetic, each lane rounded to nearest).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// bf16x2 of the two fp32 lanes (round to nearest even), low lane in the low half.
+__device__ __forceinline__ uint32_t f2_to_bf16x2(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return pack_bf16x2(lo, hi);
+}
+
+// Bits of the float 2^23 + c for a code c held in byte `b` (0..3) of `x` (each byte
+// holding one code): byte permute with the exponent byte 0x4B of 2^23.
+__device__ __forceinline__ uint32_t magic_byte(uint32_t x, int b) {
+  return __byte_perm(x, 0x4B000000u, 0x7440u + static_cast<unsigned>(b));
+}
 
 struct KernelArgs {
   const uint32_t* codes;
@@ -79,19 +118,109 @@ struct KernelArgs {
   const __half* zero;
   __nv_bfloat16* Y;
   float* partial;
-  int T, d, d_out, g, BN, stages, nkb, kb_per_split, ksplit, has_lr;
+  int T, d, d_out, log2g, BN, nkb, kb_per_split, ksplit, has_lr;
+  int m_tiles, n_tiles, num_tiles;
+  int inject_stall;
   DevErr err;
 };
 
-template <int Q, int RING>
-__global__ void __launch_bounds__(kThreads, 2)
+// Output tile t: tokens fastest (neighbouring CTAs share weight rows), then weight
+// rows, then the K split.
+struct TileCoord {
+  int m0, n0, split, kb0, nk, items;
+  bool lr;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const KernelArgs& a, int t) {
+  TileCoord c;
+  const int n = t % a.n_tiles;
+  const int rest = t / a.n_tiles;
+  const int m = rest % a.m_tiles;
+  c.split = rest / a.m_tiles;
+  c.m0 = m * kBM;
+  c.n0 = n * a.BN;
+  c.kb0 = c.split * a.kb_per_split;
+  const int kb1 = min(a.nkb, c.kb0 + a.kb_per_split);
+  c.nk = kb1 - c.kb0;
+  c.lr = a.has_lr && c.split == a.ksplit - 1;
+  c.items = c.nk + (c.lr ? 1 : 0);
+  return c;
+}
+
+// Walks this CTA's sequence of K-block items (tile by tile), as every role does.
+struct ItemIter {
+  int t;
+  int j;
+  TileCoord c;
+  __device__ __forceinline__ void begin(const KernelArgs& a) {
+    t = blockIdx.x;
+    j = 0;
+    if (t < a.num_tiles) c = tile_coord(a, t);
+  }
+  __device__ __forceinline__ bool valid(const KernelArgs& a) const { return t < a.num_tiles; }
+  __device__ __forceinline__ void next(const KernelArgs& a) {
+    if (++j == c.items) {
+      j = 0;
+      t += gridDim.x;
+      if (t < a.num_tiles) c = tile_coord(a, t);
+    }
+  }
+  __device__ __forceinline__ bool is_lr() const { return c.lr && j == c.nk; }
+};
+
+// Expands the 32 codes of one half K block (4 chunks of 8 weights) to bf16 and stores
+// them in the swizzled A tile row `a_row`: chunk c of the row goes to 16-byte slot
+// c ^ (row & 7), the 128-byte swizzle TMA would apply.
+template <int Q>
+__device__ __forceinline__ void dequant_half(const uint32_t (&cw)[4], float sig, float zm,
+                                             uint32_t a_row, int half, int m) {
+  const uint64_t zm2 = f2_pack(zm, zm);
+  const uint64_t sg2 = f2_pack(sig, sig);
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t f[8];  // bits of the floats 2^23 + c
+    if (Q == 4) {
+      const uint32_t w = cw[cc];
+      const uint32_t lo = w & 0x0F0F0F0Fu;         // codes 0, 2, 4, 6 in bytes 0..3
+      const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // codes 1, 3, 5, 7
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        f[2 * b] = magic_byte(lo, b);
+        f[2 * b + 1] = magic_byte(hi, b);
+      }
+    } else if (Q == 2) {
+      const uint32_t x = cw[cc >> 1] >> ((cc & 1) * 16);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = 0x4B000000u | ((x >> (2 * e)) & 3u);
+    } else {  // Q == 3: bit planes, this chunk's 8 codes at bits [8cc, 8cc + 8)
+      const uint32_t p0 = cw[0] >> (8 * cc), p1 = cw[1] >> (8 * cc), p2 = cw[2] >> (8 * cc);
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        f[e] = 0x4B000000u | ((p0 >> e) & 1u) | (((p1 >> e) & 1u) << 1) | (((p2 >> e) & 1u) << 2);
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      // (2^23 + c) - (2^23 + z) = c - z exactly; times sigma exactly (<= 24 bits)
+      const uint64_t v = f2_pack(__uint_as_float(f[2 * p]), __uint_as_float(f[2 * p + 1]));
+      o[p] = f2_to_bf16x2(f2_mul(f2_sub(v, zm2), sg2));
+    }
+    const int c = half * 4 + cc;
+    sts128(a_row + ((c ^ (m & 7)) << 4), o[0], o[1], o[2], o[3]);
+  }
+}
+
+template <int Q, int S, int RING>
+__global__ void __launch_bounds__(kThreads, 1)
     ttq_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_u,
                     const __grid_constant__ CUtensorMap tm_b, const KernelArgs args) {
+  static_assert(S == 2 || S == 4, "stages");
+  static_assert(RING == 4 || RING == 8, "ring");
+  constexpr int LOG2S = S == 4 ? 2 : 1;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   const int BN = args.BN;
-  const int S = args.stages;
   const uint32_t b_bytes = static_cast<uint32_t>(BN) * kBK * 2;
   const uint32_t sA = base;
   const uint32_t sB = sA + S * kATileBytes;
@@ -99,24 +228,18 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t sTail = sRing + RING * kDqThreads * kSlotBytes;
   Tail* tail = reinterpret_cast<Tail*>(smem_raw + (sTail - raw));
   volatile int* abort_flag = &tail->abort_flag;
-
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * kBM;
-  const int n0 = blockIdx.x * BN;
-  const int split = blockIdx.z;
-  const int kb0 = split * args.kb_per_split;
-  const int kb1 = min(args.nkb, kb0 + args.kb_per_split);
-  const int nk = kb1 - kb0;  // weight K blocks of this CTA
-  const bool lr_here = args.has_lr && split == args.ksplit - 1;
-  const int nblocks = nk + (lr_here ? 1 : 0);
-  const uint32_t tmem_cols = BN < 32 ? 32u : static_cast<uint32_t>(BN);
+  const uint32_t tmem_cols = (2 * BN < 32) ? 32u : static_cast<uint32_t>(2 * BN);
   const DevErr err = args.err;
 
   const uint32_t bar_full = smem_addr(&tail->full[0]);
   const uint32_t bar_afull = smem_addr(&tail->afull[0]);
   const uint32_t bar_empty = smem_addr(&tail->empty[0]);
-  const uint32_t bar_accum = smem_addr(&tail->accum);
+  const uint32_t bar_tfull = smem_addr(&tail->tfull[0]);
+  const uint32_t bar_tempty = smem_addr(&tail->tempty[0]);
+  const uint32_t bar_drain = smem_addr(&tail->drain);
+  const uint32_t bar_stall = smem_addr(&tail->stall);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -124,7 +247,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(bar_afull + 8 * s, kDqThreads);
       mbar_init(bar_empty + 8 * s, 1);
     }
-    mbar_init(bar_accum, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_tfull + 8 * b, 1);
+      mbar_init(bar_tempty + 8 * b, kEpiThreads);
+    }
+    mbar_init(bar_drain, 1);
+    mbar_init(bar_stall, 1);  // nothing ever arrives here (test hook, see inject_stall)
     tail->abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tm_x);
@@ -145,208 +273,189 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int issued = 0;
-      for (int it = 0; it < nblocks; ++it) {
-        const int s = it % S;
-        if (it >= S && !mbar_wait(bar_empty + 8 * s, ((it / S) - 1) & 1, err, abort_flag)) break;
-        if (lr_here && it == nblocks - 1) {
+      uint32_t kc = 0;
+      ItemIter it;
+      for (it.begin(args); it.valid(args); it.next(args), ++kc) {
+        const uint32_t s = kc & (S - 1);
+        if (kc >= S && !mbar_wait(bar_empty + 8 * s, ((kc >> LOG2S) - 1) & 1, err, abort_flag)) break;
+        if (it.is_lr()) {
           mbar_arrive_expect_tx(bar_full + 8 * s, kATileBytes + b_bytes);
-          tma_load_2d(sA + s * kATileBytes, &tm_b, bar_full + 8 * s, 0, m0);
-          tma_load_2d(sB + s * b_bytes, &tm_u, bar_full + 8 * s, 0, n0);
+          tma_load_2d(sA + s * kATileBytes, &tm_b, bar_full + 8 * s, 0, it.c.m0);
+          tma_load_2d(sB + s * b_bytes, &tm_u, bar_full + 8 * s, 0, it.c.n0);
         } else {
           mbar_arrive_expect_tx(bar_full + 8 * s, b_bytes);
-          tma_load_2d(sB + s * b_bytes, &tm_x, bar_full + 8 * s, (kb0 + it) * kBK, n0);
+          tma_load_2d(sB + s * b_bytes, &tm_x, bar_full + 8 * s, (it.c.kb0 + it.j) * kBK, it.c.n0);
         }
-        issued = it + 1;
       }
       if (*abort_flag) {
         // let every copy this CTA started land before shared memory is released
-        for (int it = issued > S ? issued - S : 0; it < issued; ++it)
-          mbar_drain(bar_full + 8 * (it % S), (it / S) & 1, err);
+        for (uint32_t k = kc > S ? kc - S : 0; k < kc; ++k)
+          mbar_drain(bar_full + 8 * (k & (S - 1)), (k >> LOG2S) & 1, err);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      bool ok = true;
+      if (args.inject_stall) ok = mbar_wait(bar_stall, 0, err, abort_flag);
+      uint32_t kc = 0;
+      uint32_t tc = 0;
       const uint32_t idesc = idesc_bf16_f32(kBM, BN);
-      for (int it = 0; it < nblocks; ++it) {
-        const int s = it % S;
-        const uint32_t ph = (it / S) & 1;
-        const bool is_lr = lr_here && it == nblocks - 1;
-        if (!mbar_wait(bar_full + 8 * s, ph, err, abort_flag)) break;
-        if (!is_lr && !mbar_wait(bar_afull + 8 * s, ph, err, abort_flag)) break;
+      for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x, ++tc) {
+        const TileCoord c = tile_coord(args, t);
+        const uint32_t b = tc & 1;
+        if (tc >= 2 && !mbar_wait(bar_tempty + 8 * b, ((tc >> 1) - 1) & 1, err, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint64_t ad = sw128_kmajor_desc(sA + s * kATileBytes);
-        const uint64_t bd = sw128_kmajor_desc(sB + s * b_bytes);
+        const uint32_t dacc = tmem + b * static_cast<uint32_t>(BN);
+        for (int j = 0; j < c.items; ++j, ++kc) {
+          const uint32_t s = kc & (S - 1);
+          const uint32_t ph = (kc >> LOG2S) & 1;
+          if (!mbar_wait(bar_full + 8 * s, ph, err, abort_flag) ||
+              !mbar_wait(bar_afull + 8 * s, ph, err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = sw128_kmajor_desc(sA + s * kATileBytes);
+          const uint64_t bd = sw128_kmajor_desc(sB + s * b_bytes);
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k)
-          umma_bf16(tmem, ad + 2 * k, bd + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
-        umma_commit(bar_empty + 8 * s);
+          for (int k = 0; k < kBK / 16; ++k)
+            umma_bf16(dacc, ad + 2 * k, bd + 2 * k, idesc, (j > 0 || k > 0) ? 1u : 0u);
+          umma_commit(bar_empty + 8 * s);
+        }
+        if (ok) umma_commit(bar_tfull + 8 * b);
       }
-      umma_commit(bar_accum);  // arrives once every MMA issued above has completed
-      mbar_drain(bar_accum, 0, err);
+      umma_commit(bar_drain);  // arrives once every MMA issued above has completed
+      mbar_drain(bar_drain, 0, err);
     }
     __syncwarp();
-  } else {
+  } else if (warp < kEpiWarp0) {
     // ------------------------------------------------------------ dequantisers
-    const int dt = threadIdx.x - 64;  // 0..127: tile row
-    const int i = m0 + dt;
-    const bool row_ok = i < args.d_out;
+    const int dt = threadIdx.x - 32 * kDqWarp0;  // 0..255
+    const int m = dt & (kBM - 1);                // tile row
+    const int half = dt >> 7;                    // which 32 of the K block's 64 weights
     const int d = args.d;
-    const int g = args.g;
-    const int gpr = d / g;  // groups per row
+    const int log2g = args.log2g;
+    const int gpr = d >> log2g;  // groups per row
     const int64_t meta_total = static_cast<int64_t>(args.d_out) * gpr;
     const int64_t wpr = static_cast<int64_t>(d) * Q / 32;
-    const uint32_t* crow = args.codes + static_cast<int64_t>(row_ok ? i : 0) * wpr;
-    const int64_t meta_row = static_cast<int64_t>(row_ok ? i : 0) * gpr;
     const uint32_t my_slot0 = sRing + dt * kSlotBytes;
+    constexpr uint32_t kRingStride = kDqThreads * kSlotBytes;
 
-    auto issue = [&](int j) {
-      if (j < nk && row_ok) {
-        const int kb = kb0 + j;
-        const uint32_t dst = my_slot0 + (j % RING) * (kDqThreads * kSlotBytes);
-        const int kvalid = min(kBK, d - kb * kBK);  // 64, or 32 on a ragged last block
-        const int nwords = kvalid * Q / 32;
-        const uint32_t* src = crow + static_cast<int64_t>(kb) * 2 * Q;
-        if (Q == 4) {
-          cp_async_16(dst, src);
-          if (nwords == 8) cp_async_16(dst + 16, src + 4);
-        } else {
-          for (int w = 0; w < nwords; ++w) cp_async_4(dst + 4 * w, src + w);
-        }
-        // group scale/zero: the 4-byte-aligned fp16 pairs covering this block's groups
-        const int64_t e = meta_row + (static_cast<int64_t>(kb) * kBK) / g;
-        const int64_t e0 = e & ~int64_t(1);
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          if (e0 + 2 * w + 1 < meta_total) {
-            cp_async_4(dst + 32 + 4 * w, args.scale + e0 + 2 * w);
-            cp_async_4(dst + 40 + 4 * w, args.zero + e0 + 2 * w);
+    // prefetch side: issues the cp.async copies of one item into ring slot (item % RING)
+    ItemIter pf;
+    pf.begin(args);
+    uint32_t pf_k = 0;
+    auto issue = [&]() {
+      if (pf.valid(args) && !pf.is_lr()) {
+        const int i = pf.c.m0 + m;
+        const int kb = pf.c.kb0 + pf.j;
+        const int k0 = kb * kBK + half * 32;
+        if (i < args.d_out && k0 < d) {
+          const uint32_t dst = my_slot0 + (pf_k & (RING - 1)) * kRingStride;
+          const uint32_t* src = args.codes + static_cast<int64_t>(i) * wpr + (k0 >> 5) * Q;
+          if (Q == 4) {
+            cp_async_16(dst, src);
+          } else if (Q == 2) {
+            cp_async_8(dst, src);
+          } else {
+            cp_async_4(dst, src);
+            cp_async_4(dst + 4, src + 1);
+            cp_async_4(dst + 8, src + 2);
+          }
+          const int64_t ge = static_cast<int64_t>(i) * gpr + (k0 >> log2g);
+          const int64_t e0 = ge & ~int64_t(1);
+          if (e0 + 1 < meta_total) {
+            cp_async_4(dst + 16, args.scale + e0);
+            cp_async_4(dst + 20, args.zero + e0);
           }
         }
       }
       cp_async_commit();
+      if (pf.valid(args)) pf.next(args);
+      ++pf_k;
     };
-
 #pragma unroll
-    for (int j = 0; j < RING - 1; ++j) issue(j);
+    for (int p = 0; p < RING - 1; ++p) issue();
 
-    for (int j = 0; j < nk; ++j) {
-      issue(j + RING - 1);
+    uint32_t kc = 0;
+    ItemIter it;
+    for (it.begin(args); it.valid(args); it.next(args), ++kc) {
+      issue();
       cp_async_wait<RING - 1>();
-      const int s = j % S;
-      if (j >= S && !mbar_wait(bar_empty + 8 * s, ((j / S) - 1) & 1, err, abort_flag)) break;
-      const uint32_t slot = my_slot0 + (j % RING) * (kDqThreads * kSlotBytes);
-      const uint32_t a_row = sA + s * kATileBytes + dt * 128;
-      const int kb = kb0 + j;
-      if (row_ok) {
-        const uint4 c0 = lds128(slot);
-        const uint4 c1 = lds128(slot + 16);
-        const uint4 mt = lds128(slot + 32);
-        const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const uint32_t sw[2] = {mt.x, mt.y};
-        const uint32_t zw[2] = {mt.z, mt.w};
-        const int64_t e = meta_row + (static_cast<int64_t>(kb) * kBK) / g;
-        const int64_t e0 = e & ~int64_t(1);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int kk = kb * kBK + c * 8;
-          uint32_t o0 = 0, o1 = 0, o2 = 0, o3 = 0;
-          if (kk < d) {
-            const int64_t ge = meta_row + kk / g;
-            const int off = static_cast<int>(ge - e0);  // 0..2
-            const uint32_t sbits = (sw[off >> 1] >> ((off & 1) * 16)) & 0xFFFFu;
-            const uint32_t zbits = (zw[off >> 1] >> ((off & 1) * 16)) & 0xFFFFu;
-            float sig = __half2float(__ushort_as_half(static_cast<unsigned short>(sbits)));
-            float zf = __half2float(__ushort_as_half(static_cast<unsigned short>(zbits)));
-            if (ge == meta_total - 1 && (meta_total & 1)) {  // last element of an odd-length array
-              sig = __half2float(args.scale[ge]);
-              zf = __half2float(args.zero[ge]);
-            }
-            const float zm = 8388608.0f + zf;  // exact: |z| <= 2048
-            uint32_t cc[8];
-            if (Q == 4) {
-              const uint32_t w = cw[c];
-#pragma unroll
-              for (int e2 = 0; e2 < 8; ++e2) cc[e2] = (w >> (4 * e2)) & 0xFu;
-            } else if (Q == 2) {
-              const uint32_t w = cw[c >> 1] >> ((c & 1) * 16);
-#pragma unroll
-              for (int e2 = 0; e2 < 8; ++e2) cc[e2] = (w >> (2 * e2)) & 0x3u;
-            } else {
-              const int u = c >> 2;
-              const int sh = (c & 3) * 8;
-              const uint32_t p0 = cw[3 * u] >> sh, p1 = cw[3 * u + 1] >> sh, p2 = cw[3 * u + 2] >> sh;
-#pragma unroll
-              for (int e2 = 0; e2 < 8; ++e2)
-                cc[e2] = ((p0 >> e2) & 1u) | (((p1 >> e2) & 1u) << 1) | (((p2 >> e2) & 1u) << 2);
-            }
-            float f[8];
-#pragma unroll
-            for (int e2 = 0; e2 < 8; ++e2) f[e2] = __fmul_rn(__fsub_rn(magic_code(cc[e2]), zm), sig);
-            o0 = pack_bf16x2(f[0], f[1]);
-            o1 = pack_bf16x2(f[2], f[3]);
-            o2 = pack_bf16x2(f[4], f[5]);
-            o3 = pack_bf16x2(f[6], f[7]);
+      const uint32_t s = kc & (S - 1);
+      if (kc >= S && !mbar_wait(bar_empty + 8 * s, ((kc >> LOG2S) - 1) & 1, err, abort_flag)) break;
+      if (!it.is_lr()) {
+        const int i = it.c.m0 + m;
+        const int k0 = (it.c.kb0 + it.j) * kBK + half * 32;
+        const uint32_t a_row = sA + s * kATileBytes + m * 128;
+        if (i < args.d_out && k0 < d) {
+          const uint32_t slot = my_slot0 + (kc & (RING - 1)) * kRingStride;
+          const uint4 cv = lds128(slot);
+          const uint4 mv = lds128(slot + 16);
+          const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+          const int64_t ge = static_cast<int64_t>(i) * gpr + (k0 >> log2g);
+          uint32_t sbits, zbits;
+          if (((ge & ~int64_t(1)) + 1) < meta_total) {
+            const int sh = static_cast<int>(ge & 1) * 16;
+            sbits = (mv.x >> sh) & 0xFFFFu;
+            zbits = (mv.y >> sh) & 0xFFFFu;
+          } else {  // last element of an odd-length scale/zero array
+            sbits = __half_as_ushort(args.scale[ge]);
+            zbits = __half_as_ushort(args.zero[ge]);
           }
-          sts128(a_row + ((c ^ (dt & 7)) << 4), o0, o1, o2, o3);
-        }
-      } else {
+          const float sig = __half2float(__ushort_as_half(static_cast<unsigned short>(sbits)));
+          const float zm = 8388608.0f + __half2float(__ushort_as_half(static_cast<unsigned short>(zbits)));
+          dequant_half<Q>(cw, sig, zm, a_row, half, m);
+        } else {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) sts128(a_row + ((c ^ (dt & 7)) << 4), 0u, 0u, 0u, 0u);
+          for (int cc = 0; cc < 4; ++cc) {
+            const int c = half * 4 + cc;
+            sts128(a_row + ((c ^ (m & 7)) << 4), 0u, 0u, 0u, 0u);
+          }
+        }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
       mbar_arrive(bar_afull + 8 * s);
     }
     cp_async_wait<0>();
-
+  } else {
     // ------------------------------------------------------------ epilogue
-    // tcgen05.ld is warp-collective: take the TMEM path only when every lane saw the
-    // accumulator complete
-    const bool acc_ok = __all_sync(0xffffffffu, mbar_wait(bar_accum, 0, err, abort_flag) ? 1 : 0);
-    if (acc_ok) {
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    uint32_t tc = 0;
+    for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x, ++tc) {
+      const TileCoord c = tile_coord(args, t);
+      const uint32_t b = tc & 1;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(bar_tfull + 8 * b, (tc >> 1) & 1, err, abort_flag) ? 1 : 0);
+      if (!ok) break;
       tc_fence_after();
-      const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
-      const int row = m0 + quarter * 32 + lane;
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+      const int row = c.m0 + quarter * 32 + lane;
       const bool rok = row < args.d_out;
-      if (BN >= 32) {
-        for (int cc0 = 0; cc0 < BN; cc0 += 32) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + cc0, r);
-          tmem_ld_wait();
-          if (rok) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int t = n0 + cc0 + j;
-              if (t < args.T) {
-                const float v = __uint_as_float(r[j]);
-                if (args.ksplit == 1)
-                  args.Y[static_cast<int64_t>(t) * args.d_out + row] = __float2bfloat16_rn(v);
-                else
-                  args.partial[(static_cast<int64_t>(split) * args.T + t) * args.d_out + row] = v;
-              }
-            }
-          }
-        }
-      } else {
+      const uint32_t taddr = lane_base + b * static_cast<uint32_t>(BN);
+      for (int cc0 = 0; cc0 < BN; cc0 += 16) {
         uint32_t r[16];
-        tmem_ld_32x32b_x16(taddr, r);
+        tmem_ld_32x32b_x16(taddr + cc0, r);
         tmem_ld_wait();
         if (rok) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int t = n0 + j;
-            if (t < args.T) {
+            const int tok = c.n0 + cc0 + j;
+            if (tok < args.T) {
               const float v = __uint_as_float(r[j]);
               if (args.ksplit == 1)
-                args.Y[static_cast<int64_t>(t) * args.d_out + row] = __float2bfloat16_rn(v);
+                args.Y[static_cast<int64_t>(tok) * args.d_out + row] = __float2bfloat16_rn(v);
               else
-                args.partial[(static_cast<int64_t>(split) * args.T + t) * args.d_out + row] = v;
+                args.partial[(static_cast<int64_t>(c.split) * args.T + tok) * args.d_out + row] = v;
             }
           }
         }
       }
+      tc_fence_before();
+      mbar_arrive(bar_tempty + 8 * b);
     }
   }
 
@@ -384,12 +493,36 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
+}  // namespace
+
+namespace {
+bool g_inject_stall = false;
+
+int plan_stages(int /*BN*/) { return 4; }
+int plan_ring(int BN) { return BN >= 256 ? 4 : 8; }
+int ilog2(int v) {
+  int r = 0;
+  while ((1 << r) < v) ++r;
+  return r;
+}
+
 size_t smem_bytes_for(int BN, int stages, int ring) {
   return 1024 + static_cast<size_t>(stages) * kATileBytes + static_cast<size_t>(stages) * BN * kBK * 2 +
          static_cast<size_t>(ring) * kDqThreads * kSlotBytes + sizeof(Tail);
 }
 
+template <int Q, int S, int RING>
+cudaError_t launch_q(const CUtensorMap& tx, const CUtensorMap& tu, const CUtensorMap& tb,
+                     const KernelArgs& ka, int grid, size_t smem, cudaStream_t stream) {
+  auto kern = ttq_gemm_kernel<Q, S, RING>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, stream>>>(tx, tu, tb, ka);
+  return cudaGetLastError();
+}
 }  // namespace
+
+void set_inject_stall(bool on) { g_inject_stall = on; }
 
 bool encode_bf16_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                       uint64_t row_stride_elems, uint32_t box_rows) {
@@ -405,9 +538,6 @@ bool encode_bf16_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_
   return r == CUDA_SUCCESS;
 }
 
-static int plan_ring(int BN) { return BN >= 256 ? 4 : 8; }
-static int plan_stages(int BN) { return BN >= 128 ? 4 : 2; }
-
 GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int num_sms) {
   GemmPlan p{};
   int BN = 16;
@@ -417,14 +547,11 @@ GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int num_sms) {
   p.n_tiles = static_cast<int>((T + BN - 1) / BN);
   p.nkb = static_cast<int>((d + kBK - 1) / kBK);
   p.smem_bytes = smem_bytes_for(BN, plan_stages(BN), plan_ring(BN));
-  const size_t per_sm = 233472;  // 228 KB of shared memory per SM
-  int per = static_cast<int>(per_sm / (p.smem_bytes + 1024));
-  if (per < 1) per = 1;
-  if (per > 2) per = 2;
-  const int64_t slots = static_cast<int64_t>(num_sms) * per;
+  // One persistent CTA per SM. Split K only when the tiles cannot fill one wave of
+  // the machine, and then just enough to fill it: every split adds an fp32 partial
+  // write and read of Y.
+  const int64_t slots = num_sms;
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
-  // Split K only when the tiles cannot fill one wave of the machine, and then just
-  // enough to fill that one wave: every split adds an fp32 partial write and read of Y.
   int best = 1;
   if (tiles < slots) {
     int64_t ns = slots / tiles;
@@ -433,7 +560,6 @@ GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int num_sms) {
     if (ns < 1) ns = 1;
     best = static_cast<int>(ns);
   }
-  p.ksplit = best;
   p.kb_per_split = (p.nkb + best - 1) / best;
   p.ksplit = (p.nkb + p.kb_per_split - 1) / p.kb_per_split;  // no empty split
   return p;
@@ -442,16 +568,6 @@ GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int num_sms) {
 size_t gemm_partial_bytes(const GemmPlan& p, int64_t T, int64_t d_out) {
   if (p.ksplit <= 1) return 0;
   return static_cast<size_t>(p.ksplit) * static_cast<size_t>(T) * static_cast<size_t>(d_out) * sizeof(float);
-}
-
-template <int Q, int RING>
-static cudaError_t launch_q(const CUtensorMap& tx, const CUtensorMap& tu, const CUtensorMap& tb,
-                            const KernelArgs& ka, dim3 grid, size_t smem, cudaStream_t stream) {
-  auto kern = ttq_gemm_kernel<Q, RING>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, stream>>>(tx, tu, tb, ka);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_mainloop(const GemmArgs& a, const GemmPlan& plan, const DevErr& err,
@@ -470,6 +586,8 @@ cudaError_t launch_gemm_mainloop(const GemmArgs& a, const GemmPlan& plan, const 
     tu = tx;
     tb = tx;
   }
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   KernelArgs ka;
   ka.codes = a.codes;
   ka.scale = static_cast<const __half*>(a.scale);
@@ -479,31 +597,30 @@ cudaError_t launch_gemm_mainloop(const GemmArgs& a, const GemmPlan& plan, const 
   ka.T = static_cast<int>(a.T);
   ka.d = static_cast<int>(a.d);
   ka.d_out = static_cast<int>(a.d_out);
-  ka.g = a.g;
+  ka.log2g = ilog2(a.g);
   ka.BN = plan.BN;
-  ka.stages = plan_stages(plan.BN);
   ka.nkb = plan.nkb;
   ka.kb_per_split = plan.kb_per_split;
   ka.ksplit = plan.ksplit;
   ka.has_lr = a.r > 0 ? 1 : 0;
+  ka.m_tiles = plan.m_tiles;
+  ka.n_tiles = plan.n_tiles;
+  ka.num_tiles = plan.m_tiles * plan.n_tiles * plan.ksplit;
+  ka.inject_stall = g_inject_stall ? 1 : 0;
   ka.err = err;
-  dim3 grid(plan.n_tiles, plan.m_tiles, plan.ksplit);
-  const int ring = plan_ring(plan.BN);
-  cudaError_t e;
-  if (ring == 4) {
+  const int grid = ka.num_tiles < sms ? ka.num_tiles : sms;
+  if (plan_ring(plan.BN) == 4) {
     switch (a.q) {
-      case 2: e = launch_q<2, 4>(tx, tu, tb, ka, grid, plan.smem_bytes, stream); break;
-      case 3: e = launch_q<3, 4>(tx, tu, tb, ka, grid, plan.smem_bytes, stream); break;
-      default: e = launch_q<4, 4>(tx, tu, tb, ka, grid, plan.smem_bytes, stream); break;
-    }
-  } else {
-    switch (a.q) {
-      case 2: e = launch_q<2, 8>(tx, tu, tb, ka, grid, plan.smem_bytes, stream); break;
-      case 3: e = launch_q<3, 8>(tx, tu, tb, ka, grid, plan.smem_bytes, stream); break;
-      default: e = launch_q<4, 8>(tx, tu, tb, ka, grid, plan.smem_bytes, stream); break;
+      case 2: return launch_q<2, 4, 4>(tx, tu, tb, ka, grid, plan.smem_bytes, stream);
+      case 3: return launch_q<3, 4, 4>(tx, tu, tb, ka, grid, plan.smem_bytes, stream);
+      default: return launch_q<4, 4, 4>(tx, tu, tb, ka, grid, plan.smem_bytes, stream);
     }
   }
-  return e;
+  switch (a.q) {
+    case 2: return launch_q<2, 4, 8>(tx, tu, tb, ka, grid, plan.smem_bytes, stream);
+    case 3: return launch_q<3, 4, 8>(tx, tu, tb, ka, grid, plan.smem_bytes, stream);
+    default: return launch_q<4, 4, 8>(tx, tu, tb, ka, grid, plan.smem_bytes, stream);
+  }
 }
 
 cudaError_t launch_gemm_reduce(const GemmArgs& a, const GemmPlan& plan, cudaStream_t stream) {

@@ -110,7 +110,13 @@ WsLayout ws_layout(int64_t T, int64_t d, int64_t d_out, int r, int num_sms) {
 
 ttq::DevErr dev_err(const DeviceInfo* di) { return ttq::DevErr{di->err_word, g_wait_ns.load()}; }
 
-inline ttq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TTQ_OK : TTQ_ERR_CUDA; }
+thread_local int g_last_cuda_error = 0;
+
+inline ttq_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return TTQ_OK;
+  g_last_cuda_error = static_cast<int>(e);
+  return TTQ_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -289,6 +295,17 @@ ttq_status ttq_device_status(cudaStream_t stream) {
 
 ttq_status ttq_set_wait_limit_ns(uint64_t ns) {
   g_wait_ns.store(ns == 0 ? 2000000000ull : ns);
+  return TTQ_OK;
+}
+
+int32_t ttq_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* ttq_cuda_error_string(int32_t code) {
+  return cudaGetErrorString(static_cast<cudaError_t>(code));
+}
+
+ttq_status ttq_debug_inject_stall(int32_t enable) {
+  ttq::set_inject_stall(enable != 0);
   return TTQ_OK;
 }
 

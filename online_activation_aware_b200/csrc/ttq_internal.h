@@ -84,6 +84,10 @@ cudaError_t launch_gemm_reduce(const GemmArgs& a, const GemmPlan& plan, cudaStre
 cudaError_t launch_gemm(const GemmArgs& a, const GemmPlan& plan, const DevErr& err,
                         cudaStream_t stream);
 
+// Test hook: when on, the tensor-core kernel's MMA thread first waits on a barrier that
+// nothing arrives at, so its bounded wait runs out (see ttq_debug_inject_stall).
+void set_inject_stall(bool on);
+
 // Encodes a 2-D row-major bf16 tensor map with 128-byte swizzle and a box of
 // {64 columns, box_rows rows}. Returns false when the driver refuses it.
 bool encode_bf16_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
