@@ -39,7 +39,12 @@ constexpr int kDqThreads = 32 * kNumDqWarps;                // 256
 constexpr int kEpiThreads = 32 * kNumEpiWarps;              // 128
 constexpr int kSlotBytes = 32;  // per dequant thread per K block: 16 B codes, 4 B scale, 4 B zero
 constexpr uint32_t kATileBytes = kBM * kBK * 2;  // 16 KB
-constexpr int kMaxStages = 4;
+// TMA-fed codes: per stage a [128 rows x 32 B] codes tile (32-byte swizzle) and two
+// [128 rows x 8 groups] fp16 tiles of scale and zero.
+constexpr uint32_t kCodeTileBytes = kBM * 32;
+constexpr uint32_t kMetaTileBytes = kBM * 16;
+constexpr uint32_t kCStageBytes = kCodeTileBytes + 2 * kMetaTileBytes;  // 8 KB
+constexpr int kMaxStages = 8;
 
 struct __align__(16) Tail {
   uint64_t full[kMaxStages];
@@ -78,38 +83,14 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
                : "r"(a));
   return v;
 }
+__device__ __forceinline__ uint32_t lds16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
 __device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w)
                : "memory");
-}
-
-// Two fp32 lanes at once (sm_100 packed fp32 arithmetic, each lane rounded to nearest).
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-// bf16x2 of the two fp32 lanes (round to nearest even), low lane in the low half.
-__device__ __forceinline__ uint32_t f2_to_bf16x2(uint64_t v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return pack_bf16x2(lo, hi);
-}
-
-// Bits of the float 2^23 + c for a code c held in byte `b` (0..3) of `x` (each byte
-// holding one code): byte permute with the exponent byte 0x4B of 2^23.
-__device__ __forceinline__ uint32_t magic_byte(uint32_t x, int b) {
-  return __byte_perm(x, 0x4B000000u, 0x7440u + static_cast<unsigned>(b));
 }
 
 struct KernelArgs {
@@ -168,55 +149,64 @@ struct ItemIter {
   __device__ __forceinline__ bool is_lr() const { return c.lr && j == c.nk; }
 };
 
+// Float 128 + c for a code c (< 128) held in byte `b` of `x`: byte permute of the code
+// into mantissa bits 16-22 under the exponent of 128 (0x43000000).
+__device__ __forceinline__ float code_plus_128(uint32_t x, int b) {
+  return __uint_as_float(__byte_perm(x, 0x43000000u, 0x7044u + (static_cast<unsigned>(b) << 8)));
+}
+
 // Expands the 32 codes of one half K block (4 chunks of 8 weights) to bf16 and stores
 // them in the swizzled A tile row `a_row`: chunk c of the row goes to 16-byte slot
 // c ^ (row & 7), the 128-byte swizzle TMA would apply.
+// Each weight is fma(128 + c, sigma, -(128 + z) * sigma): both products are exact in
+// fp32 (at most 12 + 11 significant bits), so the result is (c - z) * sigma exactly,
+// then rounded once to bf16.
 template <int Q>
-__device__ __forceinline__ void dequant_half(const uint32_t (&cw)[4], float sig, float zm,
+__device__ __forceinline__ void dequant_half(const uint32_t (&cw)[4], float sig, float negk,
                                              uint32_t a_row, int half, int m) {
-  const uint64_t zm2 = f2_pack(zm, zm);
-  const uint64_t sg2 = f2_pack(sig, sig);
 #pragma unroll
   for (int cc = 0; cc < 4; ++cc) {
-    uint32_t f[8];  // bits of the floats 2^23 + c
+    float f[8];
     if (Q == 4) {
       const uint32_t w = cw[cc];
       const uint32_t lo = w & 0x0F0F0F0Fu;         // codes 0, 2, 4, 6 in bytes 0..3
       const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // codes 1, 3, 5, 7
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        f[2 * b] = magic_byte(lo, b);
-        f[2 * b + 1] = magic_byte(hi, b);
+        f[2 * b] = code_plus_128(lo, b);
+        f[2 * b + 1] = code_plus_128(hi, b);
       }
     } else if (Q == 2) {
       const uint32_t x = cw[cc >> 1] >> ((cc & 1) * 16);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = 0x4B000000u | ((x >> (2 * e)) & 3u);
+      for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(0x43000000u | (((x >> (2 * e)) & 3u) << 16));
     } else {  // Q == 3: bit planes, this chunk's 8 codes at bits [8cc, 8cc + 8)
       const uint32_t p0 = cw[0] >> (8 * cc), p1 = cw[1] >> (8 * cc), p2 = cw[2] >> (8 * cc);
 #pragma unroll
       for (int e = 0; e < 8; ++e)
-        f[e] = 0x4B000000u | ((p0 >> e) & 1u) | (((p1 >> e) & 1u) << 1) | (((p2 >> e) & 1u) << 2);
+        f[e] = __uint_as_float(0x43000000u | ((((p0 >> e) & 1u) | (((p1 >> e) & 1u) << 1) |
+                                              (((p2 >> e) & 1u) << 2)) << 16));
     }
     uint32_t o[4];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      // (2^23 + c) - (2^23 + z) = c - z exactly; times sigma exactly (<= 24 bits)
-      const uint64_t v = f2_pack(__uint_as_float(f[2 * p]), __uint_as_float(f[2 * p + 1]));
-      o[p] = f2_to_bf16x2(f2_mul(f2_sub(v, zm2), sg2));
-    }
+    for (int p = 0; p < 4; ++p)
+      o[p] = pack_bf16x2(__fmaf_rn(f[2 * p], sig, negk), __fmaf_rn(f[2 * p + 1], sig, negk));
     const int c = half * 4 + cc;
     sts128(a_row + ((c ^ (m & 7)) << 4), o[0], o[1], o[2], o[3]);
   }
 }
 
-template <int Q, int S, int RING>
+// TQ: codes, scale and zero arrive by TMA in each stage (rows of 16-byte multiples);
+// otherwise each dequantiser streams its own row through a private cp.async ring.
+template <int Q, int S, int RING, bool TQ>
 __global__ void __launch_bounds__(kThreads, 1)
     ttq_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_u,
-                    const __grid_constant__ CUtensorMap tm_b, const KernelArgs args) {
-  static_assert(S == 2 || S == 4, "stages");
+                    const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
+                    const __grid_constant__ CUtensorMap tm_sc, const __grid_constant__ CUtensorMap tm_z,
+                    const KernelArgs args) {
+  static_assert(S == 2 || S == 4 || S == 8, "stages");
   static_assert(RING == 4 || RING == 8, "ring");
-  constexpr int LOG2S = S == 4 ? 2 : 1;
+  constexpr int LOG2S = S == 8 ? 3 : (S == 4 ? 2 : 1);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -224,8 +214,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t b_bytes = static_cast<uint32_t>(BN) * kBK * 2;
   const uint32_t sA = base;
   const uint32_t sB = sA + S * kATileBytes;
-  const uint32_t sRing = sB + S * b_bytes;
-  const uint32_t sTail = sRing + RING * kDqThreads * kSlotBytes;
+  const uint32_t sRing = sB + S * b_bytes;  // cp.async ring, or (TQ) the codes stages
+  const uint32_t sTail = sRing + (TQ ? S * kCStageBytes : RING * kDqThreads * kSlotBytes);
   Tail* tail = reinterpret_cast<Tail*>(smem_raw + (sTail - raw));
   volatile int* abort_flag = &tail->abort_flag;
   const int warp = threadIdx.x >> 5;
@@ -256,6 +246,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tail->abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tm_x);
+    if (TQ) {
+      prefetch_tensormap(&tm_c);
+      prefetch_tensormap(&tm_sc);
+      prefetch_tensormap(&tm_z);
+    }
     if (args.has_lr) {
       prefetch_tensormap(&tm_u);
       prefetch_tensormap(&tm_b);
@@ -283,8 +278,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sA + s * kATileBytes, &tm_b, bar_full + 8 * s, 0, it.c.m0);
           tma_load_2d(sB + s * b_bytes, &tm_u, bar_full + 8 * s, 0, it.c.n0);
         } else {
-          mbar_arrive_expect_tx(bar_full + 8 * s, b_bytes);
-          tma_load_2d(sB + s * b_bytes, &tm_x, bar_full + 8 * s, (it.c.kb0 + it.j) * kBK, it.c.n0);
+          const int kb = it.c.kb0 + it.j;
+          mbar_arrive_expect_tx(bar_full + 8 * s, b_bytes + (TQ ? kCStageBytes : 0u));
+          tma_load_2d(sB + s * b_bytes, &tm_x, bar_full + 8 * s, kb * kBK, it.c.n0);
+          if (TQ) {
+            const uint32_t cst = sRing + s * kCStageBytes;
+            tma_load_2d(cst, &tm_c, bar_full + 8 * s, (2 * Q * kb) & ~3, it.c.m0);
+            const int gx = ((kb * kBK) >> args.log2g) & ~7;
+            tma_load_2d(cst + kCodeTileBytes, &tm_sc, bar_full + 8 * s, gx, it.c.m0);
+            tma_load_2d(cst + kCodeTileBytes + kMetaTileBytes, &tm_z, bar_full + 8 * s, gx, it.c.m0);
+          }
         }
       }
       if (*abort_flag) {
@@ -345,83 +348,140 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t my_slot0 = sRing + dt * kSlotBytes;
     constexpr uint32_t kRingStride = kDqThreads * kSlotBytes;
 
-    // prefetch side: issues the cp.async copies of one item into ring slot (item % RING)
-    ItemIter pf;
-    pf.begin(args);
-    uint32_t pf_k = 0;
-    auto issue = [&]() {
-      if (pf.valid(args) && !pf.is_lr()) {
-        const int i = pf.c.m0 + m;
-        const int kb = pf.c.kb0 + pf.j;
-        const int k0 = kb * kBK + half * 32;
-        if (i < args.d_out && k0 < d) {
-          const uint32_t dst = my_slot0 + (pf_k & (RING - 1)) * kRingStride;
-          const uint32_t* src = args.codes + static_cast<int64_t>(i) * wpr + (k0 >> 5) * Q;
-          if (Q == 4) {
-            cp_async_16(dst, src);
-          } else if (Q == 2) {
-            cp_async_8(dst, src);
+    if constexpr (TQ) {
+      // codes, scale and zero of each item arrive with the stage's TMA copies
+      uint32_t kc = 0;
+      ItemIter it;
+      const uint32_t swz = static_cast<uint32_t>((m >> 2) & 1);  // 32-byte swizzle of row m
+      for (it.begin(args); it.valid(args); it.next(args), ++kc) {
+        const uint32_t s = kc & (S - 1);
+        if (!mbar_wait(bar_full + 8 * s, (kc >> LOG2S) & 1, err, abort_flag)) break;
+        if (!it.is_lr()) {
+          const int i = it.c.m0 + m;
+          const int kb = it.c.kb0 + it.j;
+          const int k0 = kb * kBK + half * 32;
+          const uint32_t a_row = sA + s * kATileBytes + m * 128;
+          if (i < args.d_out && k0 < d) {
+            const uint32_t cst = sRing + s * kCStageBytes;
+            const uint32_t crow = cst + m * 32;
+            uint32_t cw[4];
+            if (Q == 4) {
+              const uint4 v = lds128(crow + ((static_cast<uint32_t>(half) ^ swz) << 4));
+              cw[0] = v.x; cw[1] = v.y; cw[2] = v.z; cw[3] = v.w;
+            } else {
+              const uint4 v0 = lds128(crow + ((0u ^ swz) << 4));
+              const uint4 v1 = lds128(crow + ((1u ^ swz) << 4));
+              const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+              const int woff = (2 * Q * kb) - ((2 * Q * kb) & ~3) + half * Q;  // first word of this half
+              if (Q == 2) {
+                cw[0] = woff == 0 ? w[0] : (woff == 2 ? w[2] : (woff == 4 ? w[4] : w[6]));
+                cw[1] = woff == 0 ? w[1] : (woff == 2 ? w[3] : (woff == 4 ? w[5] : w[7]));
+                cw[2] = cw[3] = 0u;
+              } else {  // Q == 3: woff in {0, 2, 3, 5}
+                cw[0] = woff == 0 ? w[0] : (woff == 2 ? w[2] : (woff == 3 ? w[3] : w[5]));
+                cw[1] = woff == 0 ? w[1] : (woff == 2 ? w[3] : (woff == 3 ? w[4] : w[6]));
+                cw[2] = woff == 0 ? w[2] : (woff == 2 ? w[4] : (woff == 3 ? w[5] : w[7]));
+                cw[3] = 0u;
+              }
+            }
+            const int goff = (k0 >> log2g) - (((kb * kBK) >> log2g) & ~7);  // 0..7
+            const uint32_t sbits = lds16(cst + kCodeTileBytes + m * 16 + 2 * goff);
+            const uint32_t zbits = lds16(cst + kCodeTileBytes + kMetaTileBytes + m * 16 + 2 * goff);
+            const float sig = __half2float(__ushort_as_half(static_cast<unsigned short>(sbits)));
+            const float z = __half2float(__ushort_as_half(static_cast<unsigned short>(zbits)));
+            const float negk = -__fmul_rn(128.0f + z, sig);  // exact: |128 + z| < 2^12
+            dequant_half<Q>(cw, sig, negk, a_row, half, m);
           } else {
-            cp_async_4(dst, src);
-            cp_async_4(dst + 4, src + 1);
-            cp_async_4(dst + 8, src + 2);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const int c = half * 4 + cc;
+              sts128(a_row + ((c ^ (m & 7)) << 4), 0u, 0u, 0u, 0u);
+            }
           }
-          const int64_t ge = static_cast<int64_t>(i) * gpr + (k0 >> log2g);
-          const int64_t e0 = ge & ~int64_t(1);
-          if (e0 + 1 < meta_total) {
-            cp_async_4(dst + 16, args.scale + e0);
-            cp_async_4(dst + 20, args.zero + e0);
+          fence_proxy_async_smem();
+        }
+        mbar_arrive(bar_afull + 8 * s);
+      }
+    } else {
+      // prefetch side: issues the cp.async copies of one item into ring slot (item % RING)
+      ItemIter pf;
+      pf.begin(args);
+      uint32_t pf_k = 0;
+      auto issue = [&]() {
+        if (pf.valid(args) && !pf.is_lr()) {
+          const int i = pf.c.m0 + m;
+          const int kb = pf.c.kb0 + pf.j;
+          const int k0 = kb * kBK + half * 32;
+          if (i < args.d_out && k0 < d) {
+            const uint32_t dst = my_slot0 + (pf_k & (RING - 1)) * kRingStride;
+            const uint32_t* src = args.codes + static_cast<int64_t>(i) * wpr + (k0 >> 5) * Q;
+            if (Q == 4) {
+              cp_async_16(dst, src);
+            } else if (Q == 2) {
+              cp_async_8(dst, src);
+            } else {
+              cp_async_4(dst, src);
+              cp_async_4(dst + 4, src + 1);
+              cp_async_4(dst + 8, src + 2);
+            }
+            const int64_t ge = static_cast<int64_t>(i) * gpr + (k0 >> log2g);
+            const int64_t e0 = ge & ~int64_t(1);
+            if (e0 + 1 < meta_total) {
+              cp_async_4(dst + 16, args.scale + e0);
+              cp_async_4(dst + 20, args.zero + e0);
+            }
           }
         }
-      }
-      cp_async_commit();
-      if (pf.valid(args)) pf.next(args);
-      ++pf_k;
-    };
-#pragma unroll
-    for (int p = 0; p < RING - 1; ++p) issue();
+        cp_async_commit();
+        if (pf.valid(args)) pf.next(args);
+        ++pf_k;
+      };
+  #pragma unroll
+      for (int p = 0; p < RING - 1; ++p) issue();
 
-    uint32_t kc = 0;
-    ItemIter it;
-    for (it.begin(args); it.valid(args); it.next(args), ++kc) {
-      issue();
-      cp_async_wait<RING - 1>();
-      const uint32_t s = kc & (S - 1);
-      if (kc >= S && !mbar_wait(bar_empty + 8 * s, ((kc >> LOG2S) - 1) & 1, err, abort_flag)) break;
-      if (!it.is_lr()) {
-        const int i = it.c.m0 + m;
-        const int k0 = (it.c.kb0 + it.j) * kBK + half * 32;
-        const uint32_t a_row = sA + s * kATileBytes + m * 128;
-        if (i < args.d_out && k0 < d) {
-          const uint32_t slot = my_slot0 + (kc & (RING - 1)) * kRingStride;
-          const uint4 cv = lds128(slot);
-          const uint4 mv = lds128(slot + 16);
-          const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
-          const int64_t ge = static_cast<int64_t>(i) * gpr + (k0 >> log2g);
-          uint32_t sbits, zbits;
-          if (((ge & ~int64_t(1)) + 1) < meta_total) {
-            const int sh = static_cast<int>(ge & 1) * 16;
-            sbits = (mv.x >> sh) & 0xFFFFu;
-            zbits = (mv.y >> sh) & 0xFFFFu;
-          } else {  // last element of an odd-length scale/zero array
-            sbits = __half_as_ushort(args.scale[ge]);
-            zbits = __half_as_ushort(args.zero[ge]);
+      uint32_t kc = 0;
+      ItemIter it;
+      for (it.begin(args); it.valid(args); it.next(args), ++kc) {
+        issue();
+        cp_async_wait<RING - 1>();
+        const uint32_t s = kc & (S - 1);
+        if (kc >= S && !mbar_wait(bar_empty + 8 * s, ((kc >> LOG2S) - 1) & 1, err, abort_flag)) break;
+        if (!it.is_lr()) {
+          const int i = it.c.m0 + m;
+          const int k0 = (it.c.kb0 + it.j) * kBK + half * 32;
+          const uint32_t a_row = sA + s * kATileBytes + m * 128;
+          if (i < args.d_out && k0 < d) {
+            const uint32_t slot = my_slot0 + (kc & (RING - 1)) * kRingStride;
+            const uint4 cv = lds128(slot);
+            const uint4 mv = lds128(slot + 16);
+            const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+            const int64_t ge = static_cast<int64_t>(i) * gpr + (k0 >> log2g);
+            uint32_t sbits, zbits;
+            if (((ge & ~int64_t(1)) + 1) < meta_total) {
+              const int sh = static_cast<int>(ge & 1) * 16;
+              sbits = (mv.x >> sh) & 0xFFFFu;
+              zbits = (mv.y >> sh) & 0xFFFFu;
+            } else {  // last element of an odd-length scale/zero array
+              sbits = __half_as_ushort(args.scale[ge]);
+              zbits = __half_as_ushort(args.zero[ge]);
+            }
+            const float sig = __half2float(__ushort_as_half(static_cast<unsigned short>(sbits)));
+            const float z = __half2float(__ushort_as_half(static_cast<unsigned short>(zbits)));
+            const float negk = -__fmul_rn(128.0f + z, sig);  // exact: |128 + z| < 2^12
+            dequant_half<Q>(cw, sig, negk, a_row, half, m);
+          } else {
+  #pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const int c = half * 4 + cc;
+              sts128(a_row + ((c ^ (m & 7)) << 4), 0u, 0u, 0u, 0u);
+            }
           }
-          const float sig = __half2float(__ushort_as_half(static_cast<unsigned short>(sbits)));
-          const float zm = 8388608.0f + __half2float(__ushort_as_half(static_cast<unsigned short>(zbits)));
-          dequant_half<Q>(cw, sig, zm, a_row, half, m);
-        } else {
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            const int c = half * 4 + cc;
-            sts128(a_row + ((c ^ (m & 7)) << 4), 0u, 0u, 0u, 0u);
-          }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
+        mbar_arrive(bar_afull + 8 * s);
       }
-      mbar_arrive(bar_afull + 8 * s);
+  cp_async_wait<0>();
     }
-    cp_async_wait<0>();
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
@@ -498,26 +558,41 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 namespace {
 bool g_inject_stall = false;
 
-int plan_stages(int /*BN*/) { return 4; }
-int plan_ring(int BN) { return BN >= 256 ? 4 : 8; }
+// Small N tiles (decode, short prompts) are bound by the latency of their loads, so they
+// get deeper pipelines; the stage counts keep shared memory within 227 KB.
+int plan_stages(int BN, bool tq) {
+  if (tq) return BN <= 32 ? 8 : 4;
+  return BN <= 64 ? 8 : 4;
+}
+int plan_ring(int BN) { return (BN >= 256 || BN == 64) ? 4 : 8; }
 int ilog2(int v) {
   int r = 0;
   while ((1 << r) < v) ++r;
   return r;
 }
 
-size_t smem_bytes_for(int BN, int stages, int ring) {
-  return 1024 + static_cast<size_t>(stages) * kATileBytes + static_cast<size_t>(stages) * BN * kBK * 2 +
-         static_cast<size_t>(ring) * kDqThreads * kSlotBytes + sizeof(Tail);
+size_t smem_bytes_for(int BN, int stages, int ring, bool tq) {
+  const size_t per_stage = kATileBytes + static_cast<size_t>(BN) * kBK * 2 + (tq ? kCStageBytes : 0);
+  return 1024 + static_cast<size_t>(stages) * per_stage +
+         (tq ? 0 : static_cast<size_t>(ring) * kDqThreads * kSlotBytes) + sizeof(Tail);
 }
 
-template <int Q, int S, int RING>
-cudaError_t launch_q(const CUtensorMap& tx, const CUtensorMap& tu, const CUtensorMap& tb,
-                     const KernelArgs& ka, int grid, size_t smem, cudaStream_t stream) {
-  auto kern = ttq_gemm_kernel<Q, S, RING>;
+// Codes and group scale/zero rows can be TMA-loaded when their row pitches are 16-byte
+// multiples (every hidden size divisible by 128, with d / g divisible by 8).
+bool tma_codes_ok(int64_t d, int q, int g) {
+  return ((d * q / 8) % 16 == 0) && (((d / g) * 2) % 16 == 0);
+}
+
+struct Maps {
+  CUtensorMap x, u, b, c, sc, z;
+};
+
+template <int Q, int S, int RING, bool TQ>
+cudaError_t launch_q(const Maps& mp, const KernelArgs& ka, int grid, size_t smem, cudaStream_t stream) {
+  auto kern = ttq_gemm_kernel<Q, S, RING, TQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, stream>>>(tx, tu, tb, ka);
+  kern<<<grid, kThreads, smem, stream>>>(mp.x, mp.u, mp.b, mp.c, mp.sc, mp.z, ka);
   return cudaGetLastError();
 }
 }  // namespace
@@ -538,6 +613,24 @@ bool encode_bf16_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_
   return r == CUDA_SUCCESS;
 }
 
+namespace {
+// 2-D row-major tensor map of `elem_bytes`-sized elements with a {box_cols, box_rows} box.
+bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, uint32_t elem_bytes, const void* base,
+                 uint64_t rows, uint64_t cols, uint64_t row_stride_elems, uint32_t box_cols,
+                 uint32_t box_rows, CUtensorMapSwizzle swz) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {cols, rows};
+  cuuint64_t gstride[1] = {row_stride_elems * elem_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), gdim, gstride, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+}  // namespace
+
 GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int num_sms) {
   GemmPlan p{};
   int BN = 16;
@@ -546,7 +639,7 @@ GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int num_sms) {
   p.m_tiles = static_cast<int>((d_out + kBM - 1) / kBM);
   p.n_tiles = static_cast<int>((T + BN - 1) / BN);
   p.nkb = static_cast<int>((d + kBK - 1) / kBK);
-  p.smem_bytes = smem_bytes_for(BN, plan_stages(BN), plan_ring(BN));
+  p.smem_bytes = smem_bytes_for(BN, plan_stages(BN, false), plan_ring(BN), false);
   // One persistent CTA per SM. Split K only when the tiles cannot fill one wave of
   // the machine, and then just enough to fill it: every split adds an fp32 partial
   // write and read of Y.
@@ -572,19 +665,33 @@ size_t gemm_partial_bytes(const GemmPlan& p, int64_t T, int64_t d_out) {
 
 cudaError_t launch_gemm_mainloop(const GemmArgs& a, const GemmPlan& plan, const DevErr& err,
                                  cudaStream_t stream) {
-  CUtensorMap tx, tu, tb;
-  if (!encode_bf16_tmap(&tx, a.Xf, static_cast<uint64_t>(a.T), static_cast<uint64_t>(a.d),
+  Maps mp;
+  if (!encode_bf16_tmap(&mp.x, a.Xf, static_cast<uint64_t>(a.T), static_cast<uint64_t>(a.d),
                         static_cast<uint64_t>(a.d), static_cast<uint32_t>(plan.BN)))
     return cudaErrorInvalidValue;
   if (a.r > 0) {
-    if (!encode_bf16_tmap(&tu, a.U, static_cast<uint64_t>(a.T), 64, 64, static_cast<uint32_t>(plan.BN)))
+    if (!encode_bf16_tmap(&mp.u, a.U, static_cast<uint64_t>(a.T), 64, 64, static_cast<uint32_t>(plan.BN)))
       return cudaErrorInvalidValue;
-    if (!encode_bf16_tmap(&tb, a.Blr, static_cast<uint64_t>(a.d_out), static_cast<uint64_t>(a.r),
+    if (!encode_bf16_tmap(&mp.b, a.Blr, static_cast<uint64_t>(a.d_out), static_cast<uint64_t>(a.r),
                           static_cast<uint64_t>(a.r), kBM))
       return cudaErrorInvalidValue;
   } else {
-    tu = tx;
-    tb = tx;
+    mp.u = mp.x;
+    mp.b = mp.x;
+  }
+  const bool tq = tma_codes_ok(a.d, a.q, a.g);
+  if (tq) {
+    const uint64_t wpr = static_cast<uint64_t>(a.d) * a.q / 32;
+    const uint64_t gpr = static_cast<uint64_t>(a.d / a.g);
+    if (!encode_tmap(&mp.c, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.codes, a.d_out, wpr, wpr, 8, kBM,
+                     CU_TENSOR_MAP_SWIZZLE_32B) ||
+        !encode_tmap(&mp.sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.scale, a.d_out, gpr, gpr, 8, kBM,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_tmap(&mp.z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.zero, a.d_out, gpr, gpr, 8, kBM,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  } else {
+    mp.c = mp.sc = mp.z = mp.x;
   }
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -609,18 +716,24 @@ cudaError_t launch_gemm_mainloop(const GemmArgs& a, const GemmPlan& plan, const 
   ka.inject_stall = g_inject_stall ? 1 : 0;
   ka.err = err;
   const int grid = ka.num_tiles < sms ? ka.num_tiles : sms;
-  if (plan_ring(plan.BN) == 4) {
-    switch (a.q) {
-      case 2: return launch_q<2, 4, 4>(tx, tu, tb, ka, grid, plan.smem_bytes, stream);
-      case 3: return launch_q<3, 4, 4>(tx, tu, tb, ka, grid, plan.smem_bytes, stream);
-      default: return launch_q<4, 4, 4>(tx, tu, tb, ka, grid, plan.smem_bytes, stream);
-    }
+  const int S = plan_stages(plan.BN, tq);
+  const int R = plan_ring(plan.BN);
+  const size_t smem = smem_bytes_for(plan.BN, S, R, tq);
+#define TTQ_LAUNCH(SS, RR, TT)                                              \
+  switch (a.q) {                                                            \
+    case 2: return launch_q<2, SS, RR, TT>(mp, ka, grid, smem, stream);     \
+    case 3: return launch_q<3, SS, RR, TT>(mp, ka, grid, smem, stream);     \
+    default: return launch_q<4, SS, RR, TT>(mp, ka, grid, smem, stream);    \
   }
-  switch (a.q) {
-    case 2: return launch_q<2, 4, 8>(tx, tu, tb, ka, grid, plan.smem_bytes, stream);
-    case 3: return launch_q<3, 4, 8>(tx, tu, tb, ka, grid, plan.smem_bytes, stream);
-    default: return launch_q<4, 4, 8>(tx, tu, tb, ka, grid, plan.smem_bytes, stream);
+  if (tq) {
+    if (S == 4) { TTQ_LAUNCH(4, 4, true) }
+    TTQ_LAUNCH(8, 4, true)
   }
+  if (S == 4 && R == 4) { TTQ_LAUNCH(4, 4, false) }
+  if (S == 4 && R == 8) { TTQ_LAUNCH(4, 8, false) }
+  if (S == 8 && R == 4) { TTQ_LAUNCH(8, 4, false) }
+  TTQ_LAUNCH(8, 8, false)
+#undef TTQ_LAUNCH
 }
 
 cudaError_t launch_gemm_reduce(const GemmArgs& a, const GemmPlan& plan, cudaStream_t stream) {
