@@ -234,12 +234,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_afull + 8 * s, kDqThreads);
+      mbar_init(bar_afull + 8 * s, kNumDqWarps);  // one arrival per dequant warp
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_tfull + 8 * b, 1);
-      mbar_init(bar_tempty + 8 * b, kEpiThreads);
+      mbar_init(bar_tempty + 8 * b, kNumEpiWarps);
     }
     mbar_init(bar_drain, 1);
     mbar_init(bar_stall, 1);  // nothing ever arrives here (test hook, see inject_stall)
@@ -355,7 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t swz = static_cast<uint32_t>((m >> 2) & 1);  // 32-byte swizzle of row m
       for (it.begin(args); it.valid(args); it.next(args), ++kc) {
         const uint32_t s = kc & (S - 1);
-        if (!mbar_wait(bar_full + 8 * s, (kc >> LOG2S) & 1, err, abort_flag)) break;
+        if (!__all_sync(0xffffffffu, (mbar_wait(bar_full + 8 * s, (kc >> LOG2S) & 1, err, abort_flag)) ? 1 : 0))
+          break;  // warp-uniform: the warp arrives below as one
         if (!it.is_lr()) {
           const int i = it.c.m0 + m;
           const int kb = it.c.kb0 + it.j;
@@ -400,7 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
         }
-        mbar_arrive(bar_afull + 8 * s);
+        __syncwarp();  // the warp's shared-memory writes are ordered before its one arrival
+        if (lane == 0) mbar_arrive(bar_afull + 8 * s);
       }
     } else {
       // prefetch side: issues the cp.async copies of one item into ring slot (item % RING)
@@ -445,7 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue();
         cp_async_wait<RING - 1>();
         const uint32_t s = kc & (S - 1);
-        if (kc >= S && !mbar_wait(bar_empty + 8 * s, ((kc >> LOG2S) - 1) & 1, err, abort_flag)) break;
+        if (!__all_sync(0xffffffffu, (kc < S || mbar_wait(bar_empty + 8 * s, ((kc >> LOG2S) - 1) & 1, err, abort_flag)) ? 1 : 0))
+          break;  // warp-uniform: the warp arrives below as one
         if (!it.is_lr()) {
           const int i = it.c.m0 + m;
           const int k0 = (it.c.kb0 + it.j) * kBK + half * 32;
@@ -478,7 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
         }
-        mbar_arrive(bar_afull + 8 * s);
+        __syncwarp();  // the warp's shared-memory writes are ordered before its one arrival
+        if (lane == 0) mbar_arrive(bar_afull + 8 * s);
       }
   cp_async_wait<0>();
     }
@@ -515,7 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar_tempty + 8 * b);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_tempty + 8 * b);
     }
   }
 
@@ -577,11 +582,6 @@ size_t smem_bytes_for(int BN, int stages, int ring, bool tq) {
          (tq ? 0 : static_cast<size_t>(ring) * kDqThreads * kSlotBytes) + sizeof(Tail);
 }
 
-// Codes and group scale/zero rows can be TMA-loaded when their row pitches are 16-byte
-// multiples (every hidden size divisible by 128, with d / g divisible by 8).
-bool tma_codes_ok(int64_t d, int q, int g) {
-  return ((d * q / 8) % 16 == 0) && (((d / g) * 2) % 16 == 0);
-}
 
 struct Maps {
   CUtensorMap x, u, b, c, sc, z;
@@ -599,6 +599,13 @@ cudaError_t launch_q(const Maps& mp, const KernelArgs& ka, int grid, size_t smem
 
 void set_inject_stall(bool on) { g_inject_stall = on; }
 
+// Codes and group scale/zero rows can be TMA-loaded when their row pitches are 16-byte
+// multiples (every hidden size divisible by 128, with d / g divisible by 8).
+bool tma_codes_ok(int64_t d, int q, int g) {
+  return ((d * q / 8) % 16 == 0) && (((d / g) * 2) % 16 == 0);
+}
+
+
 bool encode_bf16_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                       uint64_t row_stride_elems, uint32_t box_rows) {
   auto fn = get_encode_fn();
@@ -613,9 +620,8 @@ bool encode_bf16_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_
   return r == CUDA_SUCCESS;
 }
 
-namespace {
 // 2-D row-major tensor map of `elem_bytes`-sized elements with a {box_cols, box_rows} box.
-bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, uint32_t elem_bytes, const void* base,
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, uint32_t elem_bytes, const void* base,
                  uint64_t rows, uint64_t cols, uint64_t row_stride_elems, uint32_t box_cols,
                  uint32_t box_rows, CUtensorMapSwizzle swz) {
   auto fn = get_encode_fn();
@@ -629,21 +635,25 @@ bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, uint32_t elem_bytes, 
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
-}  // namespace
 
-GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int num_sms) {
+GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int q, int g, int num_sms) {
   GemmPlan p{};
   int BN = 16;
   while (BN < 256 && BN < T) BN *= 2;
   p.BN = BN;
-  p.m_tiles = static_cast<int>((d_out + kBM - 1) / kBM);
+  // CTA pairs (2-SM MMA, half of X' per SM) for full 256-token tiles whenever the codes
+  // can be TMA-loaded and there are at least two 128-row blocks of weights; short prompts
+  // and decode steps (N <= 128) run faster on single CTAs
+  p.pair = BN == 256 && tma_codes_ok(d, q, g) && d_out > kBM;
+  const int rows_per_tile = p.pair ? 2 * kBM : kBM;
+  p.m_tiles = static_cast<int>((d_out + rows_per_tile - 1) / rows_per_tile);
   p.n_tiles = static_cast<int>((T + BN - 1) / BN);
   p.nkb = static_cast<int>((d + kBK - 1) / kBK);
-  p.smem_bytes = smem_bytes_for(BN, plan_stages(BN, false), plan_ring(BN), false);
-  // One persistent CTA per SM. Split K only when the tiles cannot fill one wave of
-  // the machine, and then just enough to fill it: every split adds an fp32 partial
-  // write and read of Y.
-  const int64_t slots = num_sms;
+  p.smem_bytes = 0;
+  // One persistent CTA (or CTA pair) per SM (pair of SMs). Split K only when the tiles
+  // cannot fill one wave, and then just enough to fill it: every split adds an fp32
+  // partial write and read of Y.
+  const int64_t slots = p.pair ? num_sms / 2 : num_sms;
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
   int best = 1;
   if (tiles < slots) {
@@ -665,6 +675,7 @@ size_t gemm_partial_bytes(const GemmPlan& p, int64_t T, int64_t d_out) {
 
 cudaError_t launch_gemm_mainloop(const GemmArgs& a, const GemmPlan& plan, const DevErr& err,
                                  cudaStream_t stream) {
+  if (plan.pair) return launch_gemm2sm(a, plan, err, g_inject_stall ? 1 : 0, stream);
   Maps mp;
   if (!encode_bf16_tmap(&mp.x, a.Xf, static_cast<uint64_t>(a.T), static_cast<uint64_t>(a.d),
                         static_cast<uint64_t>(a.d), static_cast<uint32_t>(plan.BN)))
@@ -683,11 +694,11 @@ cudaError_t launch_gemm_mainloop(const GemmArgs& a, const GemmPlan& plan, const 
   if (tq) {
     const uint64_t wpr = static_cast<uint64_t>(a.d) * a.q / 32;
     const uint64_t gpr = static_cast<uint64_t>(a.d / a.g);
-    if (!encode_tmap(&mp.c, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.codes, a.d_out, wpr, wpr, 8, kBM,
+    if (!encode_tmap_2d(&mp.c, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.codes, a.d_out, wpr, wpr, 8, kBM,
                      CU_TENSOR_MAP_SWIZZLE_32B) ||
-        !encode_tmap(&mp.sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.scale, a.d_out, gpr, gpr, 8, kBM,
+        !encode_tmap_2d(&mp.sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.scale, a.d_out, gpr, gpr, 8, kBM,
                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_tmap(&mp.z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.zero, a.d_out, gpr, gpr, 8, kBM,
+        !encode_tmap_2d(&mp.z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.zero, a.d_out, gpr, gpr, 8, kBM,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   } else {

@@ -91,7 +91,7 @@ struct WsLayout {
   ttq::GemmPlan plan;
 };
 
-WsLayout ws_layout(int64_t T, int64_t d, int64_t d_out, int r, int num_sms) {
+WsLayout ws_layout(int64_t T, int64_t d, int64_t d_out, int r, int q, int g, int num_sms) {
   WsLayout L{};
   L.stats_off = 0;
   L.stats_bytes = round256(ttq::stats_workspace_bytes(T, d));
@@ -101,7 +101,7 @@ WsLayout ws_layout(int64_t T, int64_t d, int64_t d_out, int r, int num_sms) {
   L.u_bytes = (d_out > 0 && r > 0) ? round256(static_cast<size_t>(T) * 64 * 2) : 0;
   L.part_off = L.u_off + L.u_bytes;
   if (d_out > 0) {
-    L.plan = ttq::gemm_plan(T, d, d_out, num_sms);
+    L.plan = ttq::gemm_plan(T, d, d_out, q, g, num_sms);
     L.part_bytes = round256(ttq::gemm_partial_bytes(L.plan, T, d_out));
   }
   L.total = L.part_off + L.part_bytes;
@@ -144,7 +144,9 @@ ttq_status ttq_workspace_size(int64_t T, int64_t d, int64_t d_out, const ttq_con
     // the split-K plan depends on the SM count of the current device
     if (device_info(&di) == TTQ_OK) num_sms = di->num_sms;
   }
-  *bytes = ws_layout(T, d, d_out, r, num_sms).total;
+  const int q = cfg ? cfg->q : 4;
+  const int g = cfg ? cfg->g : 128;
+  *bytes = ws_layout(T, d, d_out, r, q, g, num_sms).total;
   return TTQ_OK;
 }
 
@@ -159,7 +161,7 @@ ttq_status ttq_act_stats(const void* X_bf16, int64_t T, int64_t d, int64_t ld_x,
   if (!X_bf16 || !s) return TTQ_ERR_INVALID_ARG;
   if (!ws) return TTQ_ERR_WORKSPACE;
   if (!aligned16(X_bf16) || !aligned16(s) || !aligned16(ws)) return TTQ_ERR_MISALIGNED;
-  if (ws_bytes < ws_layout(T, d, 0, 0, 148).total) return TTQ_ERR_WORKSPACE;
+  if (ws_bytes < ws_layout(T, d, 0, 0, 4, 128, 148).total) return TTQ_ERR_WORKSPACE;
   auto* base = static_cast<uint8_t*>(ws);
   const size_t part_bytes = static_cast<size_t>(ttq::stats_plan(T, d).nsplit) * d * sizeof(float);
   float* partial = reinterpret_cast<float*>(base);
@@ -212,7 +214,7 @@ ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const vo
   DeviceInfo* di = nullptr;
   st = device_info(&di);
   if (st != TTQ_OK) return st;
-  const WsLayout L = ws_layout(T, d, d_out, cfg->r, di->num_sms);
+  const WsLayout L = ws_layout(T, d, d_out, cfg->r, cfg->q, cfg->g, di->num_sms);
   if (ws_bytes < L.total) return TTQ_ERR_WORKSPACE;
   auto* base = static_cast<uint8_t*>(ws);
   const size_t part_bytes = static_cast<size_t>(ttq::stats_plan(T, d).nsplit) * d * sizeof(float);
@@ -262,7 +264,7 @@ ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d
   DeviceInfo* di = nullptr;
   st = device_info(&di);
   if (st != TTQ_OK) return st;
-  const WsLayout L = ws_layout(b, d, d_out, cfg->r, di->num_sms);
+  const WsLayout L = ws_layout(b, d, d_out, cfg->r, cfg->q, cfg->g, di->num_sms);
   if (ws_bytes < L.total) return TTQ_ERR_WORKSPACE;
   auto* base = static_cast<uint8_t*>(ws);
   void* Xf = base + L.xf_off;

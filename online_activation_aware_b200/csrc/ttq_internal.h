@@ -51,15 +51,18 @@ cudaError_t launch_requant(const void* W, int64_t d_out, int64_t d, const float*
 // ---------------------------------------------------------------- GEMM
 
 struct GemmPlan {
-  int BN;           // tokens per CTA tile (MMA N): 16, 32, 64, 128 or 256
-  int m_tiles;      // ceil(d_out / 128)
+  bool pair;        // 2-SM kernel (tcgen05 cta_group::2, 256-row tiles per CTA pair)
+  int BN;           // tokens per tile (MMA N): 16, 32, 64, 128 or 256
+  int m_tiles;      // ceil(d_out / 128), or ceil(d_out / 256) for the 2-SM kernel
   int n_tiles;      // ceil(T / BN)
   int nkb;          // K blocks of 64: ceil(d / 64)
   int ksplit;       // split-K factor (1 = direct bf16 epilogue)
   int kb_per_split;
   size_t smem_bytes;
 };
-GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int num_sms);
+GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int q, int g, int num_sms);
+// Codes and group scale/zero rows have 16-byte pitches, so TMA can load them.
+bool tma_codes_ok(int64_t d, int q, int g);
 size_t gemm_partial_bytes(const GemmPlan& p, int64_t T, int64_t d_out);
 
 struct GemmArgs {
@@ -87,6 +90,15 @@ cudaError_t launch_gemm(const GemmArgs& a, const GemmPlan& plan, const DevErr& e
 // Test hook: when on, the tensor-core kernel's MMA thread first waits on a barrier that
 // nothing arrives at, so its bounded wait runs out (see ttq_debug_inject_stall).
 void set_inject_stall(bool on);
+
+// 2-D row-major tensor map of `elem_bytes`-sized elements with a {box_cols, box_rows}
+// box and the given swizzle.
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, uint32_t elem_bytes, const void* base,
+                    uint64_t rows, uint64_t cols, uint64_t row_stride_elems, uint32_t box_cols,
+                    uint32_t box_rows, CUtensorMapSwizzle swz);
+// The 2-SM tensor-core kernel (launched by launch_gemm_mainloop when plan.pair).
+cudaError_t launch_gemm2sm(const GemmArgs& a, const GemmPlan& plan, const DevErr& err, int inject_stall,
+                           cudaStream_t stream);
 
 // Encodes a 2-D row-major bf16 tensor map with 128-byte swizzle and a box of
 // {64 columns, box_rows rows}. Returns false when the driver refuses it.
