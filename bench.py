@@ -370,18 +370,21 @@ def main():
     assert ttq.device_status() == 0
     t_ms = start.elapsed_time(end)
     t_max_ms = D.max_over_ranks(t_ms, dev)
-    stage_names = ["stats", "fold", "requant", "gemm", "reduce"]
+    stage_names = ["stats_fold", "lowrank_u", "requant", "gemm", "reduce"]
     stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
                 for j, n in enumerate(stage_names)}
     value = whole_job_ktoks(T, K, world, t_max_ms)
 
     plan_split = stage_ms["reduce"] > 0.002
-    launches_per_step = 4 + (1 if r > 0 else 0) + (1 if plan_split else 0)
+    # kernels of ours per step: stats+fold, (low-rank X A^T), requant, tensor-core GEMM,
+    # (split-K reduce); the zeroing of the grid-barrier word is a memset, not counted
+    launches_per_step = 3 + (1 if r > 0 else 0) + (1 if plan_split else 0)
 
     kern = {
-        "stats": {"ms": stage_ms["stats"], "bound": "hbm", "bytes": stats_bytes(T, d)},
-        "fold": {"ms": stage_ms["fold"], "bound": "hbm", "bytes": fold_bytes(T, d) + (T * d * 2 if r else 0)},
+        "stats_fold": {"ms": stage_ms["stats_fold"], "bound": "hbm", "bytes": stats_bytes(T, d) + T * d * 2 + 4 * d},
         "requant": {"ms": stage_ms["requant"], "bound": "hbm", "bytes": requant_bytes(d, d_out, q, g)},
+        **({"lowrank_u": {"ms": stage_ms["lowrank_u"], "bound": "hbm", "bytes": T * d * 2 + r * d * 2 + T * 128}}
+           if r > 0 else {}),
         "gemm": {"ms": stage_ms["gemm"] + stage_ms["reduce"], "bound": "tensor", "flops": gemm_flops(T, d, d_out, r)},
     }
     for k_, v in kern.items():
@@ -397,13 +400,14 @@ def main():
     dk = kern[dom]
     wkey = f"{wl.name}_T{T}_r{r}"
     if dk["bound"] == "tensor":
-        roof = {"kernel": "ttq_gemm_kernel", "bound": "tensor", "achieved": dk["TFLOPs"], "peak": tc_peak,
+        roof = {"kernel": "ttq_gemm2sm_kernel" if T > 128 else "ttq_gemm_kernel", "bound": "tensor", "achieved": dk["TFLOPs"], "peak": tc_peak,
                 "unit": "TFLOP/s", "frac": dk["frac"],
-                "traffic": profiled_traffic("ttq_gemm_kernel", wkey),
+                "traffic": profiled_traffic("ttq_gemm2sm_kernel" if T > 128 else "ttq_gemm_kernel", wkey),
                 "algorithmic": f"2*T*d*d_out flops per launch = {dk['flops']:.4g}",
                 "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"}
     else:
-        roof = {"kernel": {"requant": "requant_kernel", "stats": "act_stats_kernel", "fold": "fold_kernel"}[dom],
+        roof = {"kernel": {"requant": "requant_kernel", "stats_fold": "stats_fold_kernel",
+                           "lowrank_u": "lowrank_u_kernel"}[dom],
                 "bound": "hbm", "achieved": dk["GBps"], "peak": hbm_peak, "unit": "GB/s", "frac": dk["frac"],
                 "traffic": profiled_traffic(dom, wkey), "algorithmic": f"{dk['bytes']} bytes per launch",
                 "peak_source": f"{peak_src} HBM copy (MEASURED_PEAKS.json)"}
@@ -418,7 +422,7 @@ def main():
         "requant_gbs": kern["requant"]["GBps"],
         "roofline": roof,
         "kernels": kern,
-        "rho_measured": round((stage_ms["stats"] + stage_ms["requant"]) / (stage_ms["gemm"] + stage_ms["reduce"]), 4),
+        "rho_measured": round((stage_ms["stats_fold"] + stage_ms["requant"]) / (stage_ms["gemm"] + stage_ms["reduce"]), 4),
         "gpu_launches": K * launches_per_step,
         "clocks": clocks,
         "wall_s_timed": round(wall, 3),
@@ -469,12 +473,16 @@ def main():
 
 def decode_leg(torch, ttq, wl, cfg, X, W, A, B, dev, hbm_peak):
     """Decode steps reusing one prefill's codes, b tokens per step, each step a CUDA
-    graph replay timed with events; L2 is flushed between steps (outside the events)."""
+    graph replay timed with events; L2 is flushed between steps by a read of 256 MB
+    (outside the events)."""
     lin = wl.layers[0]
     d, d_out = lin.d, lin.d_out
     layer_ = ttq.TTQLinear(W, cfg.q, cfg.g, cfg.alpha, cfg.lambda_, cfg.p, cfg.r, A, B)
     layer_.prefill(X)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    # L2 flush by reading a 256 MB buffer: it evicts the codes without leaving dirty lines
+    # whose write-back would be charged to the timed step
+    flush = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
     out = {}
     for b in wl.decode_batches or (1,):
         xt = synthetic.as_bf16(synthetic.draw_tokens(b, d, seed=1234 + b)).to(dev)
@@ -494,7 +502,7 @@ def decode_leg(torch, ttq, wl, cfg, X, W, A, B, dev, hbm_peak):
         times = []
         n = 64
         for i in range(n + 4):
-            flush.fill_(i & 0xFF)
+            torch.sum(flush, dim=0, out=sink)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record()

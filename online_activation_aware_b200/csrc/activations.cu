@@ -117,6 +117,98 @@ __global__ void __launch_bounds__(256) act_stats_kernel(const __nv_bfloat16* __r
   if (threadIdx.x == 0) counters[blockIdx.x] = 0u;  // leave the strip counter ready
 }
 
+// Statistics and fold in one cooperative launch (all blocks resident). Phase 1: each
+// block reduces its rows of a 256-column strip into partial[split, col] (as
+// act_stats_kernel). A grid barrier (bounded spin on a counter the host zeroes before
+// the launch) then lets every block form s for its strip from all partials, in split
+// order, so every block gets the same s; the blocks of split 0 write s. Phase 2 folds the
+// same rows, X' = bf16(X * (1/s)), while they are still in L2.
+template <int P>
+__global__ void __launch_bounds__(256) stats_fold_kernel(const __nv_bfloat16* __restrict__ X, int64_t T,
+                                                         int d, int64_t ld_x, int64_t rows_per_split,
+                                                         int nsplit, float alpha_over_p, float lambda,
+                                                         float* __restrict__ partial,
+                                                         unsigned* __restrict__ grid_counter,
+                                                         float* __restrict__ s,
+                                                         __nv_bfloat16* __restrict__ Xf, DevErr err) {
+  __shared__ float red[kRowWarps][kColsPerBlock];
+  __shared__ float rs_sm[kColsPerBlock];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int col0 = blockIdx.x * kColsPerBlock + lane * 8;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
+  const int64_t r1 = min(T, r0 + rows_per_split);
+
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  if (col0 < d) {
+    const __nv_bfloat16* base = X + col0;
+    int64_t r = r0 + warp;
+    for (; r + 3 * kRowWarps < r1; r += 4 * kRowWarps) {
+      const uint4 v0 = ld_stream(base + r * ld_x);
+      const uint4 v1 = ld_stream(base + (r + kRowWarps) * ld_x);
+      const uint4 v2 = ld_stream(base + (r + 2 * kRowWarps) * ld_x);
+      const uint4 v3 = ld_stream(base + (r + 3 * kRowWarps) * ld_x);
+      accum8<P>(acc, v0);
+      accum8<P>(acc, v1);
+      accum8<P>(acc, v2);
+      accum8<P>(acc, v3);
+    }
+    for (; r < r1; r += kRowWarps) accum8<P>(acc, ld_stream(base + r * ld_x));
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) red[warp][lane * 8 + j] = acc[j];
+  __syncthreads();
+  const int col = blockIdx.x * kColsPerBlock + threadIdx.x;
+  {
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kRowWarps; ++w) sum = __fadd_rn(sum, red[w][threadIdx.x]);
+    if (col < d) partial[static_cast<int64_t>(blockIdx.y) * d + col] = sum;
+  }
+
+  // grid barrier: every block's partial sums are written before anyone reads them
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned nblocks = gridDim.x * gridDim.y;
+    atomicAdd(grid_counter, 1u);
+    volatile unsigned* vc = grid_counter;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0; *vc < nblocks; ++it) {
+      if ((it & 255u) == 255u && globaltimer_ns() - t0 > err.wait_ns) {
+        atomicOr(err.word, kErrTimeout);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+  __threadfence();
+
+  if (col < d) {
+    float tot = 0.f;
+    for (int sp = 0; sp < nsplit; ++sp) tot = __fadd_rn(tot, __ldcg(&partial[static_cast<int64_t>(sp) * d + col]));
+    const float sv = finalize_scale(tot, static_cast<float>(T), alpha_over_p, lambda);
+    if (blockIdx.y == 0) s[col] = sv;
+    rs_sm[threadIdx.x] = __frcp_rn(sv);
+  }
+  __syncthreads();
+  if (col0 >= d) return;
+  float rs[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) rs[j] = rs_sm[lane * 8 + j];
+  for (int64_t r = r0 + warp; r < r1; r += kRowWarps) {
+    const uint4 v = ld_stream(X + r * ld_x + col0);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      o[j] = pack_bf16x2(__fmul_rn(bf16lo_to_f32(w[j]), rs[2 * j]), __fmul_rn(bf16hi_to_f32(w[j]), rs[2 * j + 1]));
+    *reinterpret_cast<uint4*>(Xf + r * d + col0) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 // grid: (col_blocks, row_splits); each thread owns 8 consecutive columns for all rows
 // of its split, so the 8 reciprocals 1/s are formed once per thread.
 __global__ void __launch_bounds__(256) fold_kernel(const __nv_bfloat16* __restrict__ X, int64_t T,
@@ -267,6 +359,49 @@ cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t
                                                   static_cast<int>(d), ld_x, pl.rows_per_split,
                                                   pl.nsplit, ap, lambda, partial, counters, s);
   return cudaGetLastError();
+}
+
+cudaError_t launch_stats_fold(const void* X, int64_t T, int64_t d, float alpha, float lambda, int p, float* s,
+                              float* partial, unsigned* counter, void* Xf, const DevErr& err,
+                              cudaStream_t stream) {
+  static int resident[2] = {0, 0};  // blocks per SM of the p = 1 / p = 2 kernels
+  const int pi = p == 2 ? 1 : 0;
+  if (resident[pi] == 0) {
+    int n = 0;
+    cudaError_t e = p == 2 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, stats_fold_kernel<2>, 256, 0)
+                           : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, stats_fold_kernel<1>, 256, 0);
+    if (e != cudaSuccess) return e;
+    resident[pi] = n > 0 ? n : 1;
+  }
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const StatsPlan base = stats_plan(T, d);
+  // as many row splits as the plan wants, within what can be resident at once
+  int64_t ns = base.nsplit;
+  const int64_t cap = static_cast<int64_t>(resident[pi]) * sms / base.col_blocks;
+  if (ns > cap) ns = cap;
+  if (ns < 1) ns = 1;
+  const int64_t rps = (T + ns - 1) / ns;
+  ns = (T + rps - 1) / rps;
+  cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(unsigned), stream);
+  if (e != cudaSuccess) return e;
+  dim3 grid(base.col_blocks, static_cast<unsigned>(ns));
+  const float ap = alpha / static_cast<float>(p);
+  const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
+  __nv_bfloat16* Xo = static_cast<__nv_bfloat16*>(Xf);
+  int di = static_cast<int>(d);
+  int nsi = static_cast<int>(ns);
+  int64_t ld = d;
+  DevErr er = err;
+  void* args[] = {&Xb, &T, &di, &ld, const_cast<int64_t*>(&rps), &nsi, const_cast<float*>(&ap), &lambda,
+                  &partial, &counter, &s, &Xo, &er};
+  if (p == 2)
+    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(stats_fold_kernel<2>), grid, dim3(256), args, 0,
+                                    stream);
+  else
+    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(stats_fold_kernel<1>), grid, dim3(256), args, 0,
+                                    stream);
+  return e;
 }
 
 cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const float* s,

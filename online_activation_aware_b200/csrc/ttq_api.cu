@@ -226,9 +226,9 @@ ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const vo
 
   cudaError_t e = trace(0, stream);
   if (e == cudaSuccess)
-    e = ttq::launch_act_stats(X_bf16, T, d, d, cfg->alpha, cfg->lambda, cfg->p, s, spart, counters, stream);
+    e = ttq::launch_stats_fold(X_bf16, T, d, cfg->alpha, cfg->lambda, cfg->p, s, spart, counters, Xf, dev_err(di),
+                               stream);
   if (e == cudaSuccess) e = trace(1, stream);
-  if (e == cudaSuccess) e = ttq::launch_fold(X_bf16, T, d, d, s, Xf, stream);
   if (e == cudaSuccess && cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, T, d, A_bf16, cfg->r, U, stream);
   if (e == cudaSuccess) e = trace(2, stream);
   if (e == cudaSuccess)
@@ -270,6 +270,16 @@ ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d
   void* Xf = base + L.xf_off;
   void* U = cfg->r > 0 ? base + L.u_off : nullptr;
   float* gpart = L.part_bytes ? reinterpret_cast<float*>(base + L.part_off) : nullptr;
+  if (ttq::decode_gemv_ok(b, d)) {
+    // few tokens: the CUDA-core GEMV folds them itself and streams the codes once
+    cudaError_t e = cudaSuccess;
+    if (cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, stream);
+    if (e == cudaSuccess) {
+      ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16};
+      e = ttq::launch_decode_gemv(da, stream);
+    }
+    return cuda_status(e);
+  }
   cudaError_t e = ttq::launch_fold(X_bf16, b, d, d, s, Xf, stream);
   if (e == cudaSuccess && cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, stream);
   if (e == cudaSuccess) {

@@ -34,6 +34,12 @@ cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t
                                     int64_t max_partial_floats, unsigned* counters,
                                     cudaStream_t stream);
 
+// Statistic and fold in one cooperative launch (X contiguous): writes s and
+// Xf = bf16(X * (1/s)); `counter` (one word of workspace) is zeroed on the stream first.
+cudaError_t launch_stats_fold(const void* X, int64_t T, int64_t d, float alpha, float lambda, int p, float* s,
+                              float* partial, unsigned* counter, void* Xf, const DevErr& err,
+                              cudaStream_t stream);
+
 // Xf[t, j] = bf16(X[t, j] * (1 / s[j])), Xf contiguous [T, d].
 cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const float* s,
                         void* Xf, cudaStream_t stream);
@@ -42,6 +48,26 @@ cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const
 // r..63 zero). Requires r <= 64.
 cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A, int r, void* U,
                              cudaStream_t stream);
+
+// ---------------------------------------------------------------- decode (b <= 8)
+
+constexpr int kGemvMaxTokens = 8;
+struct DecodeArgs {
+  const void* X;          // bf16 [b, d] new tokens (not folded)
+  const float* s;         // fp32 [d] the prefill's statistic
+  const uint32_t* codes;  // packed codes [d_out, d*q/32]
+  const void* scale;      // fp16 [d_out, d/g]
+  const void* zero;       // fp16 [d_out, d/g]
+  const void* U;          // bf16 [b, 64] = X A^T (r > 0) or null
+  const void* Blr;        // bf16 [d_out, r] or null
+  int r;
+  int64_t b, d, d_out;
+  int q, g;
+  void* Y;                // bf16 [b, d_out]
+};
+// True when the CUDA-core GEMV handles these decode sizes (b <= 8, x' fits in shared memory).
+bool decode_gemv_ok(int64_t b, int64_t d);
+cudaError_t launch_decode_gemv(const DecodeArgs& a, cudaStream_t stream);
 
 // ---------------------------------------------------------------- requant
 

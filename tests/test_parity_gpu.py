@@ -293,3 +293,17 @@ def test_zero_weight_and_zero_activation():
     out = ttq.linear_prefill(X, W, ttq.make_config(4, 32, 0.5, 0.4))
     assert torch.count_nonzero(out["Y"]) == 0
     np.testing.assert_array_equal(out["s"].cpu().numpy(), np.full(d, np.float32(0.4) ** np.float32(0.25), np.float32))
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("q,g,r,d_out", [(4, 128, 0, 384), (3, 32, 0, 300), (2, 32, 16, 256), (4, 64, 8, 130)])
+def test_decode_few_tokens_parity(b, q, g, r, d_out):
+    # few decode tokens run on the CUDA-core GEMV (codes streamed once); same bar as the GEMM
+    d = 1024
+    Xb, X, s32, oc, osc, oz, A, B = oracle_inputs(256, d, d_out, q, g, r, seed=900 + b * 10 + q)
+    xt = synthetic.as_bf16(synthetic.draw_tokens(b, d, seed=31 + b))
+    Yg = gpu_linear_with_oracle_codes(xt, s32, oc, osc, oz, A, B, q, g, r, d_out)
+    Yo = O.linear(synthetic.bf16_values(xt), s32, oc, osc, oz, g, A, B)
+    assert np.isfinite(Yg).all()
+    err = rel_fro(Yg, Yo)
+    assert err <= Y_RTOL, err
