@@ -1,221 +1,333 @@
-// Decode steps with few tokens (b <= 8): the projection as a CUDA-core GEMV that streams
+// Decode steps with few tokens (b <= 2): the projection as a CUDA-core GEMV that streams
 // the prefill's packed codes once (paper-daily.com deep reading of TTQ, section 6:
 // quantisation parameters are computed at prefill and reused at decode).
 //
-// For a weight row i and a unit of 32 consecutive inputs (all in one group g >= 32):
-//   sum_k x'_tk (c_ik - z) sigma = sigma * ( sum_k (128 + c_ik) x'_tk - (128 + z) sum_k x'_tk )
-// so each weight costs one byte permute (128 + c as a float) and one FMA per token; the
-// per-unit sums of x' are formed once per CTA. x' = bf16(x * (1/s)) is formed in the
-// prologue (the same rounding as the tensor-core path's fold), kept as fp32 in shared
-// memory with each unit's 8 chunks of 4 floats rotated by (unit & 7), so the lanes of a
-// warp, which read 8 different units at the same chunk, hit different banks.
-// One warp per output row: lanes stride over the row's units with 16-byte code loads
-// (512 contiguous bytes per warp step, q = 4), then reduce by shuffles.
+// For a weight row i and a group G of g inputs, cut into 32-input units V:
+//   sum_{k in G} x'_tk (c_ik - z) sigma
+//     = sigma * sum_{V in G} ( sum_{k in V} (128 + c_ik) x'_tk - (128 + z) sum_{k in V} x'_tk )
+// so each weight costs one byte permute (128 + c as an fp32, exact) and one FMA per token;
+// each unit is finished on its own (scale and zero of its group), so a lane may take any
+// set of units; the unit sums of x' come with x' from a small prep kernel.
+//
+// Layout of the work: one warp per 4 weight rows, the 32 lanes spanning the inputs (lane j
+// takes the rows' 32-input units j, j + 32, ...), so that each row's lanes read 512
+// contiguous bytes of codes per step (16-byte loads that bypass L1) and every x' value a
+// lane loads (16-byte loads through L1, contiguous across the warp) serves 4 weights: a
+// load's cost is its per-lane register writeback, so the reuse in registers is what keeps
+// x' traffic below the code traffic. The next unit's codes are in flight while one is
+// consumed; the 32 lanes are summed by shuffles in a fixed order. CTAs of 8 rows put about
+// 7 CTAs on each SM, all in one wave, with the rows' scale and zero staged in shared
+// memory. x' (fp32, chunk-major, see xoff) and the unit sums come from a prep kernel
+// chained to the GEMV by programmatic dependent launch: the GEMV issues its first code
+// loads before waiting for x'.
 #include "ttq_internal.h"
 
 namespace ttq {
 
 namespace {
 
+constexpr int kRowsPerWarp = 4;
+constexpr int kGemvThreads = 64;                                  // 2 warps
+constexpr int kRowsPerCta = kRowsPerWarp * kGemvThreads / 32;     // 8: about 7 CTAs per SM, one wave
+
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 __device__ __forceinline__ float code_plus_128f(uint32_t x, int b) {
   return __uint_as_float(__byte_perm(x, 0x43000000u, 0x7044u + (static_cast<unsigned>(b) << 8)));
 }
 
-// The packed codes of one 32-input unit (Q words) and their expansion to 32 floats
-// 128 + c.
+// The Q words holding one row's codes for one 32-input unit.
 template <int Q>
-__device__ __forceinline__ uint4 load_unit(const uint32_t* __restrict__ src) {
-  if (Q == 4) return __ldg(reinterpret_cast<const uint4*>(src));
-  if (Q == 2) return make_uint4(__ldg(src), __ldg(src + 1), 0u, 0u);
-  return make_uint4(__ldg(src), __ldg(src + 1), __ldg(src + 2), 0u);
-}
+struct UnitWords {
+  uint32_t w[Q];
+};
 
+// Codes are read once: they bypass L1 (no_allocate) so that x', which every warp reads
+// again and again, stays there.
 template <int Q>
-__device__ __forceinline__ void unit_codes(const uint4& v, float (&f)[32]) {
+__device__ __forceinline__ UnitWords<Q> load_unit(const uint32_t* __restrict__ src) {
+  UnitWords<Q> u;
   if (Q == 4) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t lo = w[j] & 0x0F0F0F0Fu, hi = (w[j] >> 4) & 0x0F0F0F0Fu;
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        f[8 * j + 2 * b] = code_plus_128f(lo, b);
-        f[8 * j + 2 * b + 1] = code_plus_128f(hi, b);
-      }
-    }
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(u.w[0]), "=r"(u.w[1]), "=r"(u.w[2]), "=r"(u.w[3])
+                 : "l"(src));
   } else if (Q == 2) {
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      f[e] = __uint_as_float(0x43000000u | (((v.x >> (2 * e)) & 3u) << 16));
-      f[16 + e] = __uint_as_float(0x43000000u | (((v.y >> (2 * e)) & 3u) << 16));
-    }
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(u.w[0]), "=r"(u.w[1]) : "l"(src));
   } else {
 #pragma unroll
-    for (int e = 0; e < 32; ++e)
-      f[e] = __uint_as_float(0x43000000u |
-                             ((((v.x >> e) & 1u) | (((v.y >> e) & 1u) << 1) | (((v.z >> e) & 1u) << 2)) << 16));
+    for (int i = 0; i < Q; ++i)
+      asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(u.w[i]) : "l"(src + i));
+  }
+  return u;
+}
+
+// 128 + c (as fp32) of the unit's inputs 4*c4 .. 4*c4 + 3.
+template <int Q>
+__device__ __forceinline__ void codes4(const UnitWords<Q>& u, int c4, float (&f)[4]) {
+  if (Q == 4) {
+    // word c4 / 2 holds inputs 8j .. 8j + 7 as nibbles (input 8j + e at bits 4e)
+    const uint32_t w = u.w[c4 >> 1];
+    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;  // even, odd inputs
+    const int b0 = (c4 & 1) * 2;
+    f[0] = code_plus_128f(lo, b0);
+    f[1] = code_plus_128f(hi, b0);
+    f[2] = code_plus_128f(lo, b0 + 1);
+    f[3] = code_plus_128f(hi, b0 + 1);
+  } else if (Q == 2) {
+    const uint32_t w = u.w[c4 >> 2] >> (8 * (c4 & 3));  // input 16v + e at bits 2e
+#pragma unroll
+    for (int e = 0; e < 4; ++e) f[e] = __uint_as_float(0x43000000u | (((w >> (2 * e)) & 3u) << 16));
+  } else {
+    // three bit planes: bit b of input k at bit k of word b
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int k = 4 * c4 + e;
+      const uint32_t c = ((u.w[0] >> k) & 1u) | (((u.w[1] >> k) & 1u) << 1) | (((u.w[2] >> k) & 1u) << 2);
+      f[e] = __uint_as_float(0x43000000u | (c << 16));
+    }
   }
 }
 
-template <int Q, int B>
-__global__ void __launch_bounds__(256) decode_gemv_kernel(
-    const __nv_bfloat16* __restrict__ X, const float* __restrict__ s, const uint32_t* __restrict__ codes,
-    const __half* __restrict__ scale, const __half* __restrict__ zero, int d, int d_out, int log2g,
-    const __nv_bfloat16* __restrict__ U, const __nv_bfloat16* __restrict__ Blr, int r,
-    __nv_bfloat16* __restrict__ Y, int nb) {
-  // nb <= B real token rows; rows nb..B-1 are zero and never written
-  extern __shared__ float sm[];
-  const int upr = d >> 5;          // units per row
-  float* xs = sm;                  // [B][d], unit chunks rotated
-  float* xsum = sm + B * d;        // [B][upr]
-  // prologue: x' = bf16(x / s) as fp32, rotated layout; 8 inputs per step (16-byte loads)
-  for (int c = threadIdx.x; c < (B * d) >> 3; c += blockDim.x) {
-    const int t = c / (d >> 3);
-    const int k0 = (c - t * (d >> 3)) << 3;
-    const uint4 xv = t < nb ? __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(t) * d + k0))
-                            : make_uint4(0u, 0u, 0u, 0u);
-    const float4 sa = __ldg(reinterpret_cast<const float4*>(s + k0));
-    const float4 sb = __ldg(reinterpret_cast<const float4*>(s + k0 + 4));
-    const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
-    const float sv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
-    float xp[8];
+// B floats of x' (or of the unit sums) for one input, token-minor.
+template <int B>
+struct TokVec {
+  float v[B];
+};
+template <int B>
+__device__ __forceinline__ TokVec<B> load_tok(const float* p) {
+  TokVec<B> r;
+  if (B == 1) {
+    r.v[0] = p[0];
+  } else if (B == 2) {
+    const float2 a = *reinterpret_cast<const float2*>(p);
+    r.v[0] = a.x; r.v[1] = a.y;
+  } else {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float lo = __uint_as_float(w[j] << 16), hi = __uint_as_float(w[j] & 0xFFFF0000u);
-      xp[2 * j] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lo, __frcp_rn(sv[2 * j]))));
-      xp[2 * j + 1] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(hi, __frcp_rn(sv[2 * j + 1]))));
-    }
-    const int u = k0 >> 5, q0 = (k0 & 31) >> 2;  // unit and first 4-float chunk
-    float4* dst = reinterpret_cast<float4*>(xs + t * d + u * 32);
-    dst[q0 ^ (u & 7)] = make_float4(xp[0], xp[1], xp[2], xp[3]);
-    dst[(q0 + 1) ^ (u & 7)] = make_float4(xp[4], xp[5], xp[6], xp[7]);
-  }
-  __syncthreads();
-  {
-    // per-unit sums: one warp per unit, one element per lane, shuffle reduction
-    const int ln = threadIdx.x & 31;
-    for (int e = threadIdx.x >> 5; e < B * upr; e += blockDim.x >> 5) {
-      float a = xs[(e / upr) * d + (e % upr) * 32 + ln];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-      if (ln == 0) xsum[e] = a;
+    for (int i = 0; i < B; i += 4) {
+      const float4 a = *reinterpret_cast<const float4*>(p + i);
+      r.v[i] = a.x; r.v[i + 1] = a.y; r.v[i + 2] = a.z; r.v[i + 3] = a.w;
     }
   }
-  __syncthreads();
+  return r;
+}
 
+// x' layout, chunk-major: input k = 32 u + 4 c + e of token t sits at
+// ((c * units + u) * 4 + e) * B + t, so that 32 lanes reading chunk c of 32 consecutive
+// units read one contiguous block.
+__host__ __device__ __forceinline__ int64_t xoff(int c, int u, int units, int B) {
+  return (static_cast<int64_t>(c) * units + u) * 4 * B;
+}
+
+// One warp per kRowsPerWarp weight rows; lane j takes the rows' 32-input units j, j + 32,
+// j + 64, ... so that each row's 32 lanes read 512 contiguous bytes of codes per step, and
+// every x' value a lane loads serves all kRowsPerWarp rows (a load's cost is its per-lane
+// register writeback, so reuse in registers is what cuts it). The next unit's codes are in
+// flight while one is consumed.
+template <int Q, int B>
+__global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
+    const uint32_t* __restrict__ codes, const __half* __restrict__ scale, const __half* __restrict__ zero,
+    const float* xp, const float* usum, int d, int d_out, int log2g, const __nv_bfloat16* __restrict__ U,
+    const __nv_bfloat16* __restrict__ Blr, int r, __nv_bfloat16* __restrict__ Y, int nb) {
+  extern __shared__ __align__(16) float2 meta_sm[];  // [kRowsPerCta][gpr]: (sigma, 128 + z)
+  constexpr int R = kRowsPerWarp;
   const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int upr = d >> 5;                            // 32-input units per row
+  const int lgu = log2g - 5;                         // log2 of units per group
   const int gpr = d >> log2g;
-  const int64_t wpr = static_cast<int64_t>(upr) * Q;
-  const int warps_total = gridDim.x * (blockDim.x >> 5);
-  for (int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); i < d_out; i += warps_total) {
-    float part[B];
+  const int row0 = blockIdx.x * kRowsPerCta + R * warp;  // the warp's first row
+  const uint32_t* crow[R];
 #pragma unroll
-    for (int t = 0; t < B; ++t) part[t] = 0.f;
-    const uint32_t* crow = codes + static_cast<int64_t>(i) * wpr;
-    constexpr int kBatch = 8;  // units of a row whose loads are in flight together
-    for (int u0 = lane; u0 < upr; u0 += 32 * kBatch) {
-      uint4 cv[kBatch];
-      float sg[kBatch], zp[kBatch];
+  for (int i = 0; i < R; ++i) crow[i] = codes + static_cast<int64_t>(row0 + i < d_out ? row0 + i : 0) * upr * Q;
+  const int nsteps = (upr - lane + 31) >> 5;         // units of this lane: lane, lane + 32, ...
+
+  // the first unit's codes, and the CTA's scale/zero into shared memory, before x' is ready
+  UnitWords<Q> cb[2][R];
+  if (nsteps > 0) {
 #pragma unroll
-      for (int kq = 0; kq < kBatch; ++kq) {
-        const int u = u0 + 32 * kq;
-        if (u < upr) {
-          cv[kq] = load_unit<Q>(crow + static_cast<int64_t>(u) * Q);
-          const int64_t gi = static_cast<int64_t>(i) * gpr + ((u << 5) >> log2g);
-          sg[kq] = __half2float(scale[gi]);
-          zp[kq] = 128.0f + __half2float(zero[gi]);
+    for (int i = 0; i < R; ++i) cb[0][i] = load_unit<Q>(crow[i] + static_cast<int64_t>(lane) * Q);
+  }
+  for (int e = threadIdx.x; e < kRowsPerCta * gpr; e += blockDim.x) {
+    const int rr = e / gpr, gi = e - rr * gpr;
+    const int mrow = blockIdx.x * kRowsPerCta + rr;
+    float2 v = make_float2(0.f, 128.f);
+    if (mrow < d_out) {
+      const int64_t o = static_cast<int64_t>(mrow) * gpr + gi;
+      v = make_float2(__half2float(scale[o]), 128.0f + __half2float(zero[o]));
+    }
+    meta_sm[e] = v;
+  }
+  grid_dep_wait();  // x' and its unit sums are written by the prep kernel
+  __syncthreads();  // meta is in place
+
+  float pacc[R][B];
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int t = 0; t < B; ++t) pacc[i][t] = 0.f;
+  for (int s0 = 0; s0 < nsteps; s0 += 2) {
+#pragma unroll
+    for (int hb = 0; hb < 2; ++hb) {
+      const int st = s0 + hb;
+      if (st < nsteps) {
+        const int u = lane + 32 * st;
+        if (st + 1 < nsteps) {  // the next unit's codes into the other buffer
+#pragma unroll
+          for (int i = 0; i < R; ++i) cb[hb ^ 1][i] = load_unit<Q>(crow[i] + static_cast<int64_t>(u + 32) * Q);
         }
-      }
+        float acc[R][B];
 #pragma unroll
-      for (int kq = 0; kq < kBatch; ++kq) {
-        const int u = u0 + 32 * kq;
-        if (u < upr) {
-          float f[32];
-          unit_codes<Q>(cv[kq], f);
+        for (int i = 0; i < R; ++i)
 #pragma unroll
-          for (int t = 0; t < B; ++t) {
-            const float4* xu = reinterpret_cast<const float4*>(xs + t * d + u * 32);
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+          for (int t = 0; t < B; ++t) acc[i][t] = 0.f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float4 x4 = xu[j ^ (u & 7)];
-              a0 = __fmaf_rn(f[4 * j], x4.x, a0);
-              a1 = __fmaf_rn(f[4 * j + 1], x4.y, a1);
-              a2 = __fmaf_rn(f[4 * j + 2], x4.z, a2);
-              a3 = __fmaf_rn(f[4 * j + 3], x4.w, a3);
-            }
-            const float acc = (a0 + a1) + (a2 + a3);
-            part[t] = __fmaf_rn(sg[kq], __fmaf_rn(-zp[kq], xsum[t * upr + u], acc), part[t]);
+        for (int c4 = 0; c4 < 8; ++c4) {
+          // x' of inputs 4 c4 .. 4 c4 + 3 of unit u for all B tokens
+          float x[4 * B];
+          const float* xb = xp + xoff(c4, u, upr, B);
+#pragma unroll
+          for (int i2 = 0; i2 < B; ++i2) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(xb + 4 * i2));
+            x[4 * i2] = v.x; x[4 * i2 + 1] = v.y; x[4 * i2 + 2] = v.z; x[4 * i2 + 3] = v.w;
+          }
+#pragma unroll
+          for (int i = 0; i < R; ++i) {
+            float f[4];
+            codes4<Q>(cb[hb][i], c4, f);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+              for (int t = 0; t < B; ++t) acc[i][t] = __fmaf_rn(f[e], x[e * B + t], acc[i][t]);
           }
         }
+        // sigma * (sum (128 + c) x' - (128 + z) sum x') for this unit's group, per row
+        const TokVec<B> xs = load_tok<B>(usum + static_cast<int64_t>(u) * B);
+        const int grp = u >> lgu;
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+          const float2 sz = meta_sm[(R * warp + i) * gpr + grp];
+#pragma unroll
+          for (int t = 0; t < B; ++t) pacc[i][t] = __fmaf_rn(sz.x, __fmaf_rn(-sz.y, xs.v[t], acc[i][t]), pacc[i][t]);
+        }
       }
     }
+  }
+  // the warp's 32 lanes in a fixed order (butterfly: every lane ends with the same sums)
 #pragma unroll
-    for (int t = 0; t < B; ++t) {
+  for (int i = 0; i < R; ++i)
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) part[t] += __shfl_xor_sync(0xffffffffu, part[t], off);
-    }
-    if (lane < nb) {
-      float y = 0.f;
+    for (int t = 0; t < B; ++t)
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) pacc[i][t] += __shfl_xor_sync(0xffffffffu, pacc[i][t], off);
+  // lane i * B + t stores token t of row i
+  const int oi = lane / B, ot = lane - oi * B;
+  const int orow = row0 + oi;
+  if (oi < R && ot < nb && orow < d_out) {
+    float y = 0.f;
+#pragma unroll
+    for (int i = 0; i < R; ++i)
 #pragma unroll
       for (int t = 0; t < B; ++t)
-        if (t == lane) y = part[t];
-      if (r > 0) {
-        for (int q = 0; q < r; ++q)
-          y = __fmaf_rn(__bfloat162float(U[static_cast<int64_t>(lane) * 64 + q]),
-                        __bfloat162float(Blr[static_cast<int64_t>(i) * r + q]), y);
-      }
-      Y[static_cast<int64_t>(lane) * d_out + i] = __float2bfloat16_rn(y);
-    }
+        if (i == oi && t == ot) y = pacc[i][t];
+    for (int q = 0; q < r; ++q)
+      y = __fmaf_rn(__bfloat162float(U[static_cast<int64_t>(ot) * 64 + q]),
+                    __bfloat162float(Blr[static_cast<int64_t>(orow) * r + q]), y);
+    Y[static_cast<int64_t>(ot) * d_out + orow] = __float2bfloat16_rn(y);
   }
 }
 
+// x'[k][t] = bf16(x[t][k] * (1 / s_k)) as fp32 (rows t >= nb zero), the same rounding as
+// the prefill's fold, in the chunk-major layout of xoff, and usum[v][t] = sum of x' over
+// the 32-input unit v. One warp per (unit, token).
+template <int B>
+__global__ void __launch_bounds__(256) decode_prep_kernel(const __nv_bfloat16* __restrict__ X, int nb, int d,
+                                                          const float* __restrict__ s, float* __restrict__ xp,
+                                                          float* __restrict__ usum) {
+  grid_dep_launch();  // the GEMV may start loading codes
+  const int lane = threadIdx.x & 31;
+  const int pair = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int units = d >> 5;
+  if (pair >= units * B) return;
+  const int v = pair / B;
+  const int t = pair - v * B;
+  const int k = 32 * v + lane;
+  float x = 0.f;
+  if (t < nb)
+    x = __bfloat162float(__float2bfloat16_rn(
+        __fmul_rn(__bfloat162float(X[static_cast<int64_t>(t) * d + k]), __frcp_rn(s[k]))));
+  xp[xoff(lane >> 2, v, units, B) + (lane & 3) * B + t] = x;
+  float sum = x;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane == 0) usum[static_cast<int64_t>(v) * B + t] = sum;
+}
+
+int gemv_tokens(int64_t b) { return b <= 1 ? 1 : 2; }
+
+size_t round16(size_t v) { return (v + 15) & ~static_cast<size_t>(15); }
+
+// Workspace of the decode: x' [d][B] (chunks rotated per unit) and the unit sums [d / 32][B].
+size_t gemv_ws_bytes(int64_t b, int64_t d) {
+  const int B = gemv_tokens(b);
+  return round16(static_cast<size_t>(d) * B * 4) + round16(static_cast<size_t>(d / 32) * B * 4);
+}
+
 template <int Q, int B>
-cudaError_t launch_b(const DecodeArgs& a, cudaStream_t stream) {
-  const size_t smem = (static_cast<size_t>(B) * a.d + static_cast<size_t>(B) * (a.d / 32)) * sizeof(float);
-  auto kern = decode_gemv_kernel<Q, B>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int per_sm = 1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem) != cudaSuccess || per_sm < 1)
-    per_sm = 1;
-  int64_t blocks = (a.d_out + 7) / 8;
-  if (blocks > static_cast<int64_t>(sms) * per_sm) blocks = static_cast<int64_t>(sms) * per_sm;
+cudaError_t launch_qb(const DecodeArgs& a, uint8_t* ws, cudaStream_t stream) {
   int lg = 0;
   while ((1 << lg) < a.g) ++lg;
-  kern<<<static_cast<unsigned>(blocks), 256, smem, stream>>>(
-      static_cast<const __nv_bfloat16*>(a.X), a.s, a.codes, static_cast<const __half*>(a.scale),
-      static_cast<const __half*>(a.zero), static_cast<int>(a.d), static_cast<int>(a.d_out), lg,
-      static_cast<const __nv_bfloat16*>(a.U), static_cast<const __nv_bfloat16*>(a.Blr), a.r,
-      static_cast<__nv_bfloat16*>(a.Y), static_cast<int>(a.b));
+  float* xp = reinterpret_cast<float*>(ws);
+  float* usum = reinterpret_cast<float*>(ws + round16(static_cast<size_t>(a.d) * B * 4));
+  const int units = static_cast<int>(a.d / 32);
+  decode_prep_kernel<B><<<(units * B + 7) / 8, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(a.X), static_cast<int>(a.b), static_cast<int>(a.d), a.s, xp, usum);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  const size_t smem = static_cast<size_t>(kRowsPerCta) * (a.d / a.g) * sizeof(float2);
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(decode_gemv_kernel<Q, B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  cfg.gridDim = dim3(static_cast<unsigned>((a.d_out + kRowsPerCta - 1) / kRowsPerCta));
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_gemv_kernel<Q, B>, static_cast<const uint32_t*>(a.codes),
+                         static_cast<const __half*>(a.scale), static_cast<const __half*>(a.zero),
+                         static_cast<const float*>(xp), static_cast<const float*>(usum), static_cast<int>(a.d),
+                         static_cast<int>(a.d_out), lg, static_cast<const __nv_bfloat16*>(a.U),
+                         static_cast<const __nv_bfloat16*>(a.Blr), a.r, static_cast<__nv_bfloat16*>(a.Y),
+                         static_cast<int>(a.b));
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <int Q>
-cudaError_t launch_q(const DecodeArgs& a, cudaStream_t stream) {
-  switch (a.b) {
-    case 1: return launch_b<Q, 1>(a, stream);
-    case 2: return launch_b<Q, 2>(a, stream);
-    case 3: case 4: return launch_b<Q, 4>(a, stream);
-    default: return launch_b<Q, 8>(a, stream);
-  }
+cudaError_t launch_q(const DecodeArgs& a, uint8_t* ws, cudaStream_t stream) {
+  if (gemv_tokens(a.b) == 1) return launch_qb<Q, 1>(a, ws, stream);
+  return launch_qb<Q, 2>(a, ws, stream);
 }
 
 }  // namespace
 
-bool decode_gemv_ok(int64_t b, int64_t d) {
-  if (b < 1 || b > kGemvMaxTokens) return false;
-  const int64_t B = b <= 2 ? b : (b <= 4 ? 4 : 8);  // the kernel instance that serves b
-  return (static_cast<size_t>(B) * d + static_cast<size_t>(B) * (d / 32)) * sizeof(float) <= 200 * 1024;
-}
+bool decode_gemv_ok(int64_t b, int64_t d) { return b >= 1 && b <= kGemvMaxTokens && d % 32 == 0; }
 
-cudaError_t launch_decode_gemv(const DecodeArgs& a, cudaStream_t stream) {
+size_t decode_gemv_ws_bytes(int64_t b, int64_t d) { return gemv_ws_bytes(b, d); }
+
+cudaError_t launch_decode_gemv(const DecodeArgs& a, void* ws, cudaStream_t stream) {
+  auto* w = static_cast<uint8_t*>(ws);
   switch (a.q) {
-    case 2: return launch_q<2>(a, stream);
-    case 3: return launch_q<3>(a, stream);
-    default: return launch_q<4>(a, stream);
+    case 2: return launch_q<2>(a, w, stream);
+    case 3: return launch_q<3>(a, w, stream);
+    default: return launch_q<4>(a, w, stream);
   }
 }
 

@@ -87,6 +87,7 @@ struct WsLayout {
   size_t xf_off, xf_bytes;
   size_t u_off, u_bytes;
   size_t part_off, part_bytes;
+  size_t dec_off, dec_bytes;  // CUDA-core decode (b <= 2): x' and its unit sums
   size_t total;
   ttq::GemmPlan plan;
 };
@@ -104,7 +105,9 @@ WsLayout ws_layout(int64_t T, int64_t d, int64_t d_out, int r, int q, int g, int
     L.plan = ttq::gemm_plan(T, d, d_out, q, g, num_sms);
     L.part_bytes = round256(ttq::gemm_partial_bytes(L.plan, T, d_out));
   }
-  L.total = L.part_off + L.part_bytes;
+  L.dec_off = L.part_off + L.part_bytes;
+  if (d_out > 0 && ttq::decode_gemv_ok(T, d)) L.dec_bytes = round256(ttq::decode_gemv_ws_bytes(T, d));
+  L.total = L.dec_off + L.dec_bytes;
   return L;
 }
 
@@ -270,13 +273,13 @@ ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d
   void* Xf = base + L.xf_off;
   void* U = cfg->r > 0 ? base + L.u_off : nullptr;
   float* gpart = L.part_bytes ? reinterpret_cast<float*>(base + L.part_off) : nullptr;
-  if (ttq::decode_gemv_ok(b, d)) {
-    // few tokens: the CUDA-core GEMV folds them itself and streams the codes once
+  if (L.dec_bytes > 0) {
+    // few tokens: the CUDA-core GEMV streams the codes once
     cudaError_t e = cudaSuccess;
     if (cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, stream);
     if (e == cudaSuccess) {
       ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16};
-      e = ttq::launch_decode_gemv(da, stream);
+      e = ttq::launch_decode_gemv(da, base + L.dec_off, stream);
     }
     return cuda_status(e);
   }

@@ -49,9 +49,9 @@ cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const
 cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A, int r, void* U,
                              cudaStream_t stream);
 
-// ---------------------------------------------------------------- decode (b <= 8)
+// ---------------------------------------------------------------- decode
 
-constexpr int kGemvMaxTokens = 8;
+constexpr int kGemvMaxTokens = 2;  // larger decode batches run on the tensor cores
 struct DecodeArgs {
   const void* X;          // bf16 [b, d] new tokens (not folded)
   const float* s;         // fp32 [d] the prefill's statistic
@@ -65,9 +65,12 @@ struct DecodeArgs {
   int q, g;
   void* Y;                // bf16 [b, d_out]
 };
-// True when the CUDA-core GEMV handles these decode sizes (b <= 8, x' fits in shared memory).
+// True when the CUDA-core GEMV handles these decode sizes (b <= 2).
 bool decode_gemv_ok(int64_t b, int64_t d);
-cudaError_t launch_decode_gemv(const DecodeArgs& a, cudaStream_t stream);
+// Workspace bytes of launch_decode_gemv: x' (fp32, [d][B]) and its 32-input unit sums.
+size_t decode_gemv_ws_bytes(int64_t b, int64_t d);
+// The prep kernel and the GEMV (launched as its programmatic dependent).
+cudaError_t launch_decode_gemv(const DecodeArgs& a, void* ws, cudaStream_t stream);
 
 // ---------------------------------------------------------------- requant
 

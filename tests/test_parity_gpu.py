@@ -307,3 +307,73 @@ def test_decode_few_tokens_parity(b, q, g, r, d_out):
     assert np.isfinite(Yg).all()
     err = rel_fro(Yg, Yo)
     assert err <= Y_RTOL, err
+
+
+@pytest.mark.parametrize("b,d,d_out,q,g,r", [
+    (1, 1024, 384, 4, 128, 0),
+    (16, 1024, 300, 3, 32, 0),    # ragged last row block, g = 32
+    (17, 512, 640, 2, 64, 16),    # low rank
+    (33, 2048, 256, 4, 32, 8),
+    (64, 768, 520, 4, 128, 0),
+    (5, 256, 128 * 300, 4, 128, 0),  # many row blocks
+    (2, 5120, 1024, 4, 128, 16),  # the Qwen3-32B hidden size with low rank
+    (3, 5120, 520, 3, 64, 0),     # 3-bit bit planes, 10 slices of 10 units per row
+])
+def test_decode_parity_shapes(b, d, d_out, q, g, r):
+    # b <= 8 runs on the CUDA-core GEMV (one lane per weight row), larger b on the tensor cores
+    Xb, X, s32, oc, osc, oz, A, B = oracle_inputs(128, d, d_out, q, g, r, seed=700 + b + d_out)
+    xt = synthetic.as_bf16(synthetic.draw_tokens(b, d, seed=5 + b))
+    Yg = gpu_linear_with_oracle_codes(xt, s32, oc, osc, oz, A, B, q, g, r, d_out)
+    Yo = O.linear(synthetic.bf16_values(xt), s32, oc, osc, oz, g, A, B)
+    assert np.isfinite(Yg).all()
+    err = rel_fro(Yg, Yo)
+    assert err <= Y_RTOL, err
+
+
+@pytest.mark.parametrize("b,d", [(1, 992), (2, 160), (2, 96), (3, 992), (8, 160), (7, 96)])
+def test_decode_small_hidden_parity(b, d):
+    # hidden sizes with fewer 32-input units than lanes in a warp, and ragged unit counts
+    d_out, q, g = 200, 4, 32
+    Xb, X, s32, oc, osc, oz, A, B = oracle_inputs(64, d, d_out, q, g, 0, seed=b * 11 + d)
+    xt = synthetic.as_bf16(synthetic.draw_tokens(b, d, seed=9 + b))
+    Yg = gpu_linear_with_oracle_codes(xt, s32, oc, osc, oz, None, None, q, g, 0, d_out)
+    Yo = O.linear(synthetic.bf16_values(xt), s32, oc, osc, oz, g)
+    err = rel_fro(Yg, Yo)
+    assert err <= Y_RTOL, err
+
+
+@pytest.mark.parametrize("b", [1, 8])
+def test_decode_is_deterministic(b):
+    # every reduction (GEMV lanes, split-K partials) runs in a fixed order: repeated steps
+    # agree bit for bit
+    d, d_out, q, g = 1024, 384, 4, 128
+    Xb, X, s32, oc, osc, oz, A, B = oracle_inputs(64, d, d_out, q, g, 0, seed=42)
+    xt = synthetic.as_bf16(synthetic.draw_tokens(b, d, seed=43))
+    Y1 = gpu_linear_with_oracle_codes(xt, s32, oc, osc, oz, None, None, q, g, 0, d_out)
+    Y2 = gpu_linear_with_oracle_codes(xt, s32, oc, osc, oz, None, None, q, g, 0, d_out)
+    np.testing.assert_array_equal(Y1, Y2)
+
+
+@pytest.mark.parametrize("b", [2, 6])
+@pytest.mark.parametrize("g", [32, 128])
+def test_decode_far_zero_points(g, b):
+    # groups whose scaled weights all share one sign get zero points far outside [0, 2^q - 1]
+    # (up to the +-2048 clamp): (128 + z) sum x' must stay exact
+    d, d_out, q = 1024, 256, 4
+    Xb, Wb, X, W = layer(128, d, d_out, seed=77)
+    _, s32 = O.act_stats(X, 0.5, 0.4)
+    W = W.copy()
+    rng = np.random.default_rng(5)
+    for i in range(0, 40):
+        k = slice((i % (d // g)) * g, (i % (d // g) + 1) * g)
+        # scaled weights w * s of one sign in a narrow band
+        W[i, k] = (0.05 + 1e-4 * rng.standard_normal(g)) / s32[k]
+        W[i + 40, k] = (-0.03 + 2e-5 * rng.standard_normal(g)) / s32[k]
+    W = synthetic.bf16_values(synthetic.as_bf16(W))
+    oc, osc, oz = O.requant(W, s32, q, g)
+    assert np.abs(oz).max() > 128
+    xt = synthetic.as_bf16(synthetic.draw_tokens(b, d, seed=12))
+    Yg = gpu_linear_with_oracle_codes(xt, s32, oc, osc, oz, None, None, q, g, 0, d_out)
+    Yo = O.linear(synthetic.bf16_values(xt), s32, oc, osc, oz, g)
+    err = rel_fro(Yg, Yo)
+    assert err <= Y_RTOL, err
