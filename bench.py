@@ -155,7 +155,7 @@ def gpu_uuid(torch, dev):
 
 def kernel_hash():
     h = hashlib.sha256()
-    for name in ("gemm.cu", "ttq_common.cuh"):
+    for name in ("gemm.cu", "gemm2sm.cu", "ttq_common.cuh"):
         with open(os.path.join(ROOT, "online_activation_aware_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
