@@ -117,27 +117,34 @@ __global__ void __launch_bounds__(256) act_stats_kernel(const __nv_bfloat16* __r
   if (threadIdx.x == 0) counters[blockIdx.x] = 0u;  // leave the strip counter ready
 }
 
-// Statistics and fold in one cooperative launch (all blocks resident). Phase 1: each
-// block reduces its rows of a 256-column strip into partial[split, col] (as
-// act_stats_kernel). A grid barrier (bounded spin on a counter the host zeroes before
-// the launch) then lets every block form s for its strip from all partials, in split
-// order, so every block gets the same s; the blocks of split 0 write s. Phase 2 folds the
-// same rows, X' = bf16(X * (1/s)), while they are still in L2.
+// Statistics and fold in one launch whose blocks are all resident at once (cooperative).
+// Phase 1: each block reduces its rows of a 256-column strip into partial[split, col] (as
+// act_stats_kernel). The blocks of a strip then meet at a per-strip barrier: the last to
+// arrive sums the strip's partials in split order (a fixed order, so s does not depend on
+// scheduling), writes s for the strip and publishes it by bumping the strip's epoch; the
+// others wait (bounded in time) for the epoch to change. A block reads the epoch before it
+// arrives, so the change it waits for is this launch's. Phase 2 folds the same rows,
+// X' = bf16(X * (1/s)), while they are still in L2. `strip_sync` holds a counter (zeroed
+// by the host before the launch, and left zero by the kernel) and an epoch per strip.
 template <int P>
 __global__ void __launch_bounds__(256) stats_fold_kernel(const __nv_bfloat16* __restrict__ X, int64_t T,
                                                          int d, int64_t ld_x, int64_t rows_per_split,
                                                          int nsplit, float alpha_over_p, float lambda,
                                                          float* __restrict__ partial,
-                                                         unsigned* __restrict__ grid_counter,
+                                                         unsigned* __restrict__ strip_sync,
                                                          float* __restrict__ s,
                                                          __nv_bfloat16* __restrict__ Xf, DevErr err) {
   __shared__ float red[kRowWarps][kColsPerBlock];
   __shared__ float rs_sm[kColsPerBlock];
+  __shared__ unsigned epoch0;
+  __shared__ int is_last;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int col0 = blockIdx.x * kColsPerBlock + lane * 8;
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
   const int64_t r1 = min(T, r0 + rows_per_split);
+  unsigned* counter = strip_sync + 2 * blockIdx.x;
+  unsigned* epoch = counter + 1;
 
   float acc[8];
 #pragma unroll
@@ -145,15 +152,12 @@ __global__ void __launch_bounds__(256) stats_fold_kernel(const __nv_bfloat16* __
   if (col0 < d) {
     const __nv_bfloat16* base = X + col0;
     int64_t r = r0 + warp;
-    for (; r + 3 * kRowWarps < r1; r += 4 * kRowWarps) {
-      const uint4 v0 = ld_stream(base + r * ld_x);
-      const uint4 v1 = ld_stream(base + (r + kRowWarps) * ld_x);
-      const uint4 v2 = ld_stream(base + (r + 2 * kRowWarps) * ld_x);
-      const uint4 v3 = ld_stream(base + (r + 3 * kRowWarps) * ld_x);
-      accum8<P>(acc, v0);
-      accum8<P>(acc, v1);
-      accum8<P>(acc, v2);
-      accum8<P>(acc, v3);
+    for (; r + 7 * kRowWarps < r1; r += 8 * kRowWarps) {  // 8 loads in flight per lane
+      uint4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = ld_stream(base + (r + i * kRowWarps) * ld_x);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) accum8<P>(acc, v[i]);
     }
     for (; r < r1; r += kRowWarps) accum8<P>(acc, ld_stream(base + r * ld_x));
   }
@@ -168,45 +172,65 @@ __global__ void __launch_bounds__(256) stats_fold_kernel(const __nv_bfloat16* __
     if (col < d) partial[static_cast<int64_t>(blockIdx.y) * d + col] = sum;
   }
 
-  // grid barrier: every block's partial sums are written before anyone reads them
-  __threadfence();
+  // per-strip barrier: the strip's partial sums are written before the last block reads them
+  if (threadIdx.x == 0) epoch0 = atomicOr(epoch, 0u);
+  __threadfence();  // partials (every thread) and the epoch read (thread 0) before the arrival
   __syncthreads();
-  if (threadIdx.x == 0) {
-    const unsigned nblocks = gridDim.x * gridDim.y;
-    atomicAdd(grid_counter, 1u);
-    volatile unsigned* vc = grid_counter;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 0; *vc < nblocks; ++it) {
-      if ((it & 255u) == 255u && globaltimer_ns() - t0 > err.wait_ns) {
-        atomicOr(err.word, kErrTimeout);
-        break;
+  if (threadIdx.x == 0) is_last = atomicAdd(counter, 1u) == static_cast<unsigned>(nsplit - 1) ? 1 : 0;
+  __syncthreads();
+  if (is_last) {
+    __threadfence();
+    if (col < d) {
+      float tot = 0.f;
+      for (int sp = 0; sp < nsplit; ++sp) tot = __fadd_rn(tot, __ldcg(&partial[static_cast<int64_t>(sp) * d + col]));
+      const float sv = finalize_scale(tot, static_cast<float>(T), alpha_over_p, lambda);
+      s[col] = sv;
+      rs_sm[threadIdx.x] = __frcp_rn(sv);
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      *counter = 0u;  // ready for the next launch
+      __threadfence();
+      atomicAdd(epoch, 1u);  // publish s
+    }
+  } else {
+    if (threadIdx.x == 0) {
+      volatile unsigned* ve = epoch;
+      const uint64_t t0 = globaltimer_ns();
+      for (uint32_t it = 0; *ve == epoch0; ++it) {
+        if ((it & 255u) == 255u && globaltimer_ns() - t0 > err.wait_ns) {
+          atomicOr(err.word, kErrTimeout);
+          break;
+        }
       }
     }
-  }
-  __syncthreads();
-  __threadfence();
-
-  if (col < d) {
-    float tot = 0.f;
-    for (int sp = 0; sp < nsplit; ++sp) tot = __fadd_rn(tot, __ldcg(&partial[static_cast<int64_t>(sp) * d + col]));
-    const float sv = finalize_scale(tot, static_cast<float>(T), alpha_over_p, lambda);
-    if (blockIdx.y == 0) s[col] = sv;
-    rs_sm[threadIdx.x] = __frcp_rn(sv);
+    __syncthreads();
+    __threadfence();
+    if (col < d) rs_sm[threadIdx.x] = __frcp_rn(__ldcg(&s[col]));
   }
   __syncthreads();
   if (col0 >= d) return;
   float rs[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) rs[j] = rs_sm[lane * 8 + j];
-  for (int64_t r = r0 + warp; r < r1; r += kRowWarps) {
-    const uint4 v = ld_stream(X + r * ld_x + col0);
+  auto fold1 = [&](const uint4& v, int64_t r) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t o[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
       o[j] = pack_bf16x2(__fmul_rn(bf16lo_to_f32(w[j]), rs[2 * j]), __fmul_rn(bf16hi_to_f32(w[j]), rs[2 * j + 1]));
     *reinterpret_cast<uint4*>(Xf + r * d + col0) = make_uint4(o[0], o[1], o[2], o[3]);
+  };
+  int64_t r = r0 + warp;
+  for (; r + 3 * kRowWarps < r1; r += 4 * kRowWarps) {  // 4 loads in flight per lane
+    uint4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = ld_stream(X + (r + i * kRowWarps) * ld_x + col0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) fold1(v[i], r + i * kRowWarps);
   }
+  for (; r < r1; r += kRowWarps) fold1(ld_stream(X + r * ld_x + col0), r);
 }
 
 // grid: (col_blocks, row_splits); each thread owns 8 consecutive columns for all rows
@@ -308,7 +332,7 @@ StatsPlan stats_plan(int64_t T, int64_t d) {
 size_t stats_workspace_bytes(int64_t T, int64_t d) {
   const StatsPlan p = stats_plan(T, d);
   const size_t part = static_cast<size_t>(p.nsplit) * static_cast<size_t>(d) * sizeof(float);
-  const size_t cnt = static_cast<size_t>(p.col_blocks) * sizeof(unsigned);
+  const size_t cnt = 2 * static_cast<size_t>(p.col_blocks) * sizeof(unsigned);  // counter, epoch per strip
   return ((part + 255) / 256) * 256 + ((cnt + 255) / 256) * 256;
 }
 
@@ -362,7 +386,7 @@ cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t
 }
 
 cudaError_t launch_stats_fold(const void* X, int64_t T, int64_t d, float alpha, float lambda, int p, float* s,
-                              float* partial, unsigned* counter, void* Xf, const DevErr& err,
+                              float* partial, unsigned* strip_sync, void* Xf, const DevErr& err,
                               cudaStream_t stream) {
   static int resident[2] = {0, 0};  // blocks per SM of the p = 1 / p = 2 kernels
   const int pi = p == 2 ? 1 : 0;
@@ -383,7 +407,7 @@ cudaError_t launch_stats_fold(const void* X, int64_t T, int64_t d, float alpha, 
   if (ns < 1) ns = 1;
   const int64_t rps = (T + ns - 1) / ns;
   ns = (T + rps - 1) / rps;
-  cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(unsigned), stream);
+  cudaError_t e = cudaMemsetAsync(strip_sync, 0, 2 * sizeof(unsigned) * base.col_blocks, stream);
   if (e != cudaSuccess) return e;
   dim3 grid(base.col_blocks, static_cast<unsigned>(ns));
   const float ap = alpha / static_cast<float>(p);
@@ -394,7 +418,8 @@ cudaError_t launch_stats_fold(const void* X, int64_t T, int64_t d, float alpha, 
   int64_t ld = d;
   DevErr er = err;
   void* args[] = {&Xb, &T, &di, &ld, const_cast<int64_t*>(&rps), &nsi, const_cast<float*>(&ap), &lambda,
-                  &partial, &counter, &s, &Xo, &er};
+                  &partial, &strip_sync, &s, &Xo, &er};
+  // cooperative: the blocks of a strip wait for one another, so all must be resident
   if (p == 2)
     e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(stats_fold_kernel<2>), grid, dim3(256), args, 0,
                                     stream);

@@ -35,9 +35,10 @@ cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t
                                     cudaStream_t stream);
 
 // Statistic and fold in one cooperative launch (X contiguous): writes s and
-// Xf = bf16(X * (1/s)); `counter` (one word of workspace) is zeroed on the stream first.
+// Xf = bf16(X * (1/s)); `strip_sync` (two words of workspace per 256-column strip: a
+// counter, zeroed on the stream first, and an epoch) carries the per-strip barrier.
 cudaError_t launch_stats_fold(const void* X, int64_t T, int64_t d, float alpha, float lambda, int p, float* s,
-                              float* partial, unsigned* counter, void* Xf, const DevErr& err,
+                              float* partial, unsigned* strip_sync, void* Xf, const DevErr& err,
                               cudaStream_t stream);
 
 // Xf[t, j] = bf16(X[t, j] * (1 / s[j])), Xf contiguous [T, d].
