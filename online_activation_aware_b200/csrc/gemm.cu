@@ -298,16 +298,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // the whole warp walks the tiles (waits and loop values warp-uniform); one elected
+    // lane issues the MMAs and commits
+    {
       bool ok = true;
-      if (args.inject_stall) ok = mbar_wait(bar_stall, 0, err, abort_flag);
+      if (args.inject_stall) ok = __all_sync(0xffffffffu, mbar_wait(bar_stall, 0, err, abort_flag) ? 1 : 0);
       uint32_t kc = 0;
       uint32_t tc = 0;
       const uint32_t idesc = idesc_bf16_f32(kBM, BN);
       for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x, ++tc) {
         const TileCoord c = tile_coord(args, t);
         const uint32_t b = tc & 1;
-        if (tc >= 2 && !mbar_wait(bar_tempty + 8 * b, ((tc >> 1) - 1) & 1, err, abort_flag)) {
+        if (tc >= 2 &&
+            !__all_sync(0xffffffffu, mbar_wait(bar_tempty + 8 * b, ((tc >> 1) - 1) & 1, err, abort_flag) ? 1 : 0)) {
           ok = false;
           break;
         }
@@ -316,23 +319,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < c.items; ++j, ++kc) {
           const uint32_t s = kc & (S - 1);
           const uint32_t ph = (kc >> LOG2S) & 1;
-          if (!mbar_wait(bar_full + 8 * s, ph, err, abort_flag) ||
-              !mbar_wait(bar_afull + 8 * s, ph, err, abort_flag)) {
+          const bool ready = mbar_wait(bar_full + 8 * s, ph, err, abort_flag) &&
+                             mbar_wait(bar_afull + 8 * s, ph, err, abort_flag);
+          if (!__all_sync(0xffffffffu, ready ? 1 : 0)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint64_t ad = sw128_kmajor_desc(sA + s * kATileBytes);
           const uint64_t bd = sw128_kmajor_desc(sB + s * b_bytes);
+          if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            umma_bf16(dacc, ad + 2 * k, bd + 2 * k, idesc, (j > 0 || k > 0) ? 1u : 0u);
-          umma_commit(bar_empty + 8 * s);
+            for (int k = 0; k < kBK / 16; ++k)
+              umma_bf16(dacc, ad + 2 * k, bd + 2 * k, idesc, (j > 0 || k > 0) ? 1u : 0u);
+            umma_commit(bar_empty + 8 * s);
+          }
+          __syncwarp();
         }
-        if (ok) umma_commit(bar_tfull + 8 * b);
+        if (ok && elect_one()) umma_commit(bar_tfull + 8 * b);
+        __syncwarp();
       }
-      umma_commit(bar_drain);  // arrives once every MMA issued above has completed
-      mbar_drain(bar_drain, 0, err);
+      if (elect_one()) {
+        umma_commit(bar_drain);  // arrives once every MMA issued above has completed
+        mbar_drain(bar_drain, 0, err);
+      }
     }
     __syncwarp();
   } else if (warp < kEpiWarp0) {

@@ -366,16 +366,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
-    if (rank == 0 && lane == 0) {
+    // the whole warp walks the tiles (waits and loop values warp-uniform); one elected
+    // lane issues the MMAs and commits
+    if (rank == 0) {
       bool ok = true;
-      if (args.inject_stall) ok = mbar_wait(bar_stall, 0, err, abort_flag);
+      if (args.inject_stall) ok = __all_sync(0xffffffffu, mbar_wait(bar_stall, 0, err, abort_flag) ? 1 : 0);
       Pipe p;
       uint32_t tc = 0;
       const uint32_t idesc = idesc_bf16_f32(2 * kBM, BN);
       for (int t = blockIdx.x >> 1; ok && t < args.num_tiles; t += gridDim.x >> 1, ++tc) {
         const TileCoord2 c = tile_coord2(args, t);
         const uint32_t b = tc & 1;
-        if (tc >= 2 && !mbar_wait(bar_tempty + 8 * b, ((tc >> 1) - 1) & 1, err, abort_flag)) {
+        if (tc >= 2 &&
+            !__all_sync(0xffffffffu, mbar_wait(bar_tempty + 8 * b, ((tc >> 1) - 1) & 1, err, abort_flag) ? 1 : 0)) {
           ok = false;
           break;
         }
@@ -383,23 +386,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t dacc = tmem + b * static_cast<uint32_t>(BN);
         for (int j = 0; j < c.items; ++j, p.advance(S)) {
           const uint32_t s = p.stage;
-          if (!mbar_wait(bar_full + 8 * s, p.phase, err, abort_flag) ||
-              !mbar_wait(bar_afull + 8 * s, p.phase, err, abort_flag)) {
+          const bool ready = mbar_wait(bar_full + 8 * s, p.phase, err, abort_flag) &&
+                             mbar_wait(bar_afull + 8 * s, p.phase, err, abort_flag);
+          if (!__all_sync(0xffffffffu, ready ? 1 : 0)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint64_t ad = sw128_kmajor_desc(sA + s * kATileBytes);
           const uint64_t bd = sw128_kmajor_desc(sB + s * b_bytes);
+          if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            umma2_bf16(dacc, ad + 2 * k, bd + 2 * k, idesc, (j > 0 || k > 0) ? 1u : 0u);
-          umma2_commit_both(bar_empty + 8 * s);
+            for (int k = 0; k < kBK / 16; ++k)
+              umma2_bf16(dacc, ad + 2 * k, bd + 2 * k, idesc, (j > 0 || k > 0) ? 1u : 0u);
+            umma2_commit_both(bar_empty + 8 * s);
+          }
+          __syncwarp();
         }
-        if (ok) umma2_commit_both(bar_tfull + 8 * b);
+        if (ok && elect_one()) umma2_commit_both(bar_tfull + 8 * b);
+        __syncwarp();
       }
-      umma2_commit_both(bar_drain);  // arrives once every MMA issued above has completed
-      mbar_drain(bar_drain, 0, err);
+      if (elect_one()) {
+        umma2_commit_both(bar_drain);  // arrives once every MMA issued above has completed
+        mbar_drain(bar_drain, 0, err);
+      }
     }
     __syncwarp();
   } else if (warp < kEpiWarp0) {
