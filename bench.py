@@ -376,9 +376,9 @@ def main():
     value = whole_job_ktoks(T, K, world, t_max_ms)
 
     plan_split = stage_ms["reduce"] > 0.002
-    # kernels of ours per step: stats+fold, (low-rank X A^T), requant, tensor-core GEMM,
-    # (split-K reduce); the zeroing of the grid-barrier word is a memset, not counted
-    launches_per_step = 3 + (1 if r > 0 else 0) + (1 if plan_split else 0)
+    # kernels of ours per step: statistic partial sums, statistic + fold, (low-rank X A^T),
+    # requant, tensor-core GEMM, (split-K reduce)
+    launches_per_step = 4 + (1 if r > 0 else 0) + (1 if plan_split else 0)
 
     kern = {
         "stats_fold": {"ms": stage_ms["stats_fold"], "bound": "hbm", "bytes": stats_bytes(T, d) + T * d * 2 + 4 * d},

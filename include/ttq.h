@@ -77,11 +77,12 @@ typedef struct {
  * (d_out * d * q / 32). Returns 0 when d is not a multiple of 32 or q is unsupported. */
 TTQ_API size_t ttq_codes_words(int64_t d_out, int64_t d, int32_t q);
 
-/* Bytes of scratch workspace that ttq_linear_prefill (and ttq_act_stats, and
- * ttq_linear_decode with T = b rows) needs for these sizes. The workspace holds the
- * partial column sums of the statistics, the folded activations X diag(1/s) in bf16,
- * the low-rank projection X A^T and split-K partial products. Contents need not be
- * initialised and are not preserved. */
+/* Bytes of scratch workspace that ttq_linear_prefill (and ttq_linear_decode with
+ * T = b rows; and ttq_act_stats with d_out = 0) needs for these sizes. For the prefill
+ * and decode it holds the folded activations X diag(1/s) in bf16, the low-rank
+ * projection X A^T, split-K partial products and the decode GEMV's operands; for
+ * ttq_act_stats (d_out = 0) the partial column sums of the statistic. Contents need
+ * not be initialised and are not preserved. */
 TTQ_API ttq_status ttq_workspace_size(int64_t T, int64_t d, int64_t d_out, const ttq_config* cfg,
                               size_t* bytes);
 

@@ -8,6 +8,9 @@
 //               summary, section 2B).
 // All three are HBM-bound streaming passes: a warp reads 512 contiguous bytes of a row
 // per step (32 lanes x 16 B), so every DRAM sector fetched is used in full.
+#include <algorithm>
+#include <climits>
+
 #include "ttq_internal.h"
 
 namespace ttq {
@@ -117,104 +120,148 @@ __global__ void __launch_bounds__(256) act_stats_kernel(const __nv_bfloat16* __r
   if (threadIdx.x == 0) counters[blockIdx.x] = 0u;  // leave the strip counter ready
 }
 
-// Statistics and fold in one launch whose blocks are all resident at once (cooperative).
-// Phase 1: each block reduces its rows of a 256-column strip into partial[split, col] (as
-// act_stats_kernel). The blocks of a strip then meet at a per-strip barrier: the last to
-// arrive sums the strip's partials in split order (a fixed order, so s does not depend on
-// scheduling), writes s for the strip and publishes it by bumping the strip's epoch; the
-// others wait (bounded in time) for the epoch to change. A block reads the epoch before it
-// arrives, so the change it waits for is this launch's. Phase 2 folds the same rows,
-// X' = bf16(X * (1/s)), while they are still in L2. `strip_sync` holds a counter (zeroed
-// by the host before the launch, and left zero by the kernel) and an epoch per strip.
+// Statistic, then fold, as two launches that need no grid-wide synchronisation:
+//   stats_partial_kernel  block (strip c, split k) sums |x|^p over its rows of a 256-column
+//                         strip into partial[k, strip columns] (fp32, fixed order);
+//   stats_fold_kernel     launched as the programmatic dependent of the first, so its
+//                         blocks are resident and waiting when the partial sums land;
+//                         block (c, k) reduces the strip's partials in a fixed order
+//                         (warp w takes splits w, w + 8, ...; the eight warp sums are then
+//                         added in warp order), forms s for the strip (the blocks of split 0
+//                         write it out) and folds its rows, X' = bf16(X * (1/s)), re-reading
+//                         them from L2 (those loads mark the lines evict-first: X is dead
+//                         after them).
+// Every block of a strip reduces the same values in the same order, so all hold the same
+// s. Both grids are sized to a whole number of waves over the SMs.
 template <int P>
-__global__ void __launch_bounds__(256) stats_fold_kernel(const __nv_bfloat16* __restrict__ X, int64_t T,
-                                                         int d, int64_t ld_x, int64_t rows_per_split,
-                                                         int nsplit, float alpha_over_p, float lambda,
-                                                         float* __restrict__ partial,
-                                                         unsigned* __restrict__ strip_sync,
-                                                         float* __restrict__ s,
-                                                         __nv_bfloat16* __restrict__ Xf, DevErr err) {
+__global__ void __launch_bounds__(256, 5) stats_partial_kernel(const __nv_bfloat16* __restrict__ X, int64_t T,
+                                                            int d, int64_t ld_x, int64_t rows_per_split,
+                                                            float* __restrict__ partial) {
   __shared__ float red[kRowWarps][kColsPerBlock];
-  __shared__ float rs_sm[kColsPerBlock];
-  __shared__ unsigned epoch0;
-  __shared__ int is_last;
+  grid_dep_launch();  // the fold kernel's blocks may take their places now
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int col0 = blockIdx.x * kColsPerBlock + lane * 8;
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
   const int64_t r1 = min(T, r0 + rows_per_split);
-  unsigned* counter = strip_sync + 2 * blockIdx.x;
-  unsigned* epoch = counter + 1;
-
   float acc[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) acc[j] = 0.f;
   if (col0 < d) {
     const __nv_bfloat16* base = X + col0;
+    // batches of 8 rows with all 8 loads in flight per lane, then the rest in predicated
+    // batches of 4 (a row past the end reads as zero, which adds nothing)
     int64_t r = r0 + warp;
-    for (; r + 7 * kRowWarps < r1; r += 8 * kRowWarps) {  // 8 loads in flight per lane
+    for (; r + 7 * kRowWarps < r1; r += 8 * kRowWarps) {
       uint4 v[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] = ld_stream(base + (r + i * kRowWarps) * ld_x);
 #pragma unroll
       for (int i = 0; i < 8; ++i) accum8<P>(acc, v[i]);
     }
-    for (; r < r1; r += kRowWarps) accum8<P>(acc, ld_stream(base + r * ld_x));
+    for (; r < r1; r += 4 * kRowWarps) {
+      uint4 v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int64_t rr = r + i * kRowWarps;
+        v[i] = rr < r1 ? ld_stream(base + rr * ld_x) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) accum8<P>(acc, v[i]);
+    }
   }
 #pragma unroll
   for (int j = 0; j < 8; ++j) red[warp][lane * 8 + j] = acc[j];
   __syncthreads();
   const int col = blockIdx.x * kColsPerBlock + threadIdx.x;
-  {
-    float sum = 0.f;
+  float sum = 0.f;
 #pragma unroll
-    for (int w = 0; w < kRowWarps; ++w) sum = __fadd_rn(sum, red[w][threadIdx.x]);
-    if (col < d) partial[static_cast<int64_t>(blockIdx.y) * d + col] = sum;
-  }
+  for (int w = 0; w < kRowWarps; ++w) sum = __fadd_rn(sum, red[w][threadIdx.x]);
+  if (col < d) partial[static_cast<int64_t>(blockIdx.y) * d + col] = sum;
+}
 
-  // per-strip barrier: the strip's partial sums are written before the last block reads them
-  if (threadIdx.x == 0) epoch0 = atomicOr(epoch, 0u);
-  __threadfence();  // partials (every thread) and the epoch read (thread 0) before the arrival
-  __syncthreads();
-  if (threadIdx.x == 0) is_last = atomicAdd(counter, 1u) == static_cast<unsigned>(nsplit - 1) ? 1 : 0;
-  __syncthreads();
-  if (is_last) {
-    __threadfence();
-    if (col < d) {
-      float tot = 0.f;
-      for (int sp = 0; sp < nsplit; ++sp) tot = __fadd_rn(tot, __ldcg(&partial[static_cast<int64_t>(sp) * d + col]));
-      const float sv = finalize_scale(tot, static_cast<float>(T), alpha_over_p, lambda);
-      s[col] = sv;
-      rs_sm[threadIdx.x] = __frcp_rn(sv);
-    }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      *counter = 0u;  // ready for the next launch
-      __threadfence();
-      atomicAdd(epoch, 1u);  // publish s
-    }
-  } else {
-    if (threadIdx.x == 0) {
-      volatile unsigned* ve = epoch;
-      const uint64_t t0 = globaltimer_ns();
-      for (uint32_t it = 0; *ve == epoch0; ++it) {
-        if ((it & 255u) == 255u && globaltimer_ns() - t0 > err.wait_ns) {
-          atomicOr(err.word, kErrTimeout);
-          break;
+// s for the 256 columns of strip blockIdx.x from partial[nsplit, d], into s_out (shared
+// memory, 256 floats; columns past d get 1). Needs all 256 threads; `red` is 8 x 256
+// floats of shared scratch.
+__device__ __forceinline__ void strip_scale(const float* __restrict__ partial, int d, int nsplit, float T,
+                                            float alpha_over_p, float lambda, float (*red)[kColsPerBlock],
+                                            float* s_out) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int col0 = blockIdx.x * kColsPerBlock + lane * 8;
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  if (col0 < d) {
+    constexpr int U = 2;  // splits in flight per warp
+    for (int k0 = warp; k0 < nsplit; k0 += U * kRowWarps) {
+      float4 va[U], vb[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int k = k0 + u * kRowWarps;
+        if (k < nsplit) {
+          const float* p = partial + static_cast<int64_t>(k) * d + col0;
+          va[u] = __ldcg(reinterpret_cast<const float4*>(p));
+          vb[u] = __ldcg(reinterpret_cast<const float4*>(p + 4));
+        } else {
+          va[u] = vb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
-    }
-    __syncthreads();
-    __threadfence();
-    if (col < d) rs_sm[threadIdx.x] = __frcp_rn(__ldcg(&s[col]));
-  }
-  __syncthreads();
-  if (col0 >= d) return;
-  float rs[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) rs[j] = rs_sm[lane * 8 + j];
+      for (int u = 0; u < U; ++u) {
+        acc[0] = __fadd_rn(acc[0], va[u].x);
+        acc[1] = __fadd_rn(acc[1], va[u].y);
+        acc[2] = __fadd_rn(acc[2], va[u].z);
+        acc[3] = __fadd_rn(acc[3], va[u].w);
+        acc[4] = __fadd_rn(acc[4], vb[u].x);
+        acc[5] = __fadd_rn(acc[5], vb[u].y);
+        acc[6] = __fadd_rn(acc[6], vb[u].z);
+        acc[7] = __fadd_rn(acc[7], vb[u].w);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) red[warp][lane * 8 + j] = acc[j];
+  __syncthreads();
+  const int col = blockIdx.x * kColsPerBlock + threadIdx.x;
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < kRowWarps; ++w) tot = __fadd_rn(tot, red[w][threadIdx.x]);
+  s_out[threadIdx.x] = col < d ? finalize_scale(tot, T, alpha_over_p, lambda) : 1.f;
+  __syncthreads();
+}
+
+template <int P>
+__global__ void __launch_bounds__(256, 5) stats_fold_kernel(const __nv_bfloat16* __restrict__ X, int64_t T, int d,
+                                                         int64_t rows_per_split, int nsplit,
+                                                         const float* __restrict__ partial,
+                                                         float alpha_over_p, float lambda,
+                                                         float* __restrict__ s, __nv_bfloat16* __restrict__ Xf) {
+  __shared__ float red[kRowWarps][kColsPerBlock];
+  __shared__ float s_sm[kColsPerBlock];
+  grid_dep_wait();  // the partial sums are complete and visible
+  grid_dep_launch();
+  strip_scale(partial, d, nsplit, static_cast<float>(T), alpha_over_p, lambda, red, s_sm);
+  const int col = blockIdx.x * kColsPerBlock + threadIdx.x;
+  if (blockIdx.y == 0 && col < d) s[col] = s_sm[threadIdx.x];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int col0 = blockIdx.x * kColsPerBlock + lane * 8;
+  if (col0 >= d) return;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
+  const int64_t r1 = min(T, r0 + rows_per_split);
+  __syncwarp();
+  {
+    float* rsw = &red[0][0];  // reciprocals, this lane's 8 columns (the reduction scratch is free now)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) rsw[threadIdx.x * 8 + ((j + lane) & 7)] = __frcp_rn(s_sm[lane * 8 + ((j + lane) & 7)]);
+  }
+  __syncwarp();
+  const float4* rs4 = reinterpret_cast<const float4*>(&red[0][0]) + threadIdx.x * 2;
+  const uint64_t pol = l2_evict_first_policy();
   auto fold1 = [&](const uint4& v, int64_t r) {
+    const float4 ra = rs4[0], rb = rs4[1];
+    const float rs[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t o[4];
 #pragma unroll
@@ -222,15 +269,28 @@ __global__ void __launch_bounds__(256) stats_fold_kernel(const __nv_bfloat16* __
       o[j] = pack_bf16x2(__fmul_rn(bf16lo_to_f32(w[j]), rs[2 * j]), __fmul_rn(bf16hi_to_f32(w[j]), rs[2 * j + 1]));
     *reinterpret_cast<uint4*>(Xf + r * d + col0) = make_uint4(o[0], o[1], o[2], o[3]);
   };
-  int64_t r = r0 + warp;
-  for (; r + 3 * kRowWarps < r1; r += 4 * kRowWarps) {  // 4 loads in flight per lane
+  for (int64_t r = r0 + warp; r < r1; r += 4 * kRowWarps) {  // predicated batches of 4 rows (from L2)
     uint4 v[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = ld_stream(X + (r + i * kRowWarps) * ld_x + col0);
+    for (int i = 0; i < 4; ++i)
+      if (r + i * kRowWarps < r1) v[i] = ld_stream_hint(X + (r + i * kRowWarps) * d + col0, pol);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) fold1(v[i], r + i * kRowWarps);
+    for (int i = 0; i < 4; ++i)
+      if (r + i * kRowWarps < r1) fold1(v[i], r + i * kRowWarps);
   }
-  for (; r < r1; r += kRowWarps) fold1(ld_stream(X + r * ld_x + col0), r);
+}
+
+// s alone from the partial sums: one block per strip (the finishing step of ttq_act_stats).
+__global__ void __launch_bounds__(256) stats_finish_kernel(const float* __restrict__ partial, int d, int nsplit,
+                                                           float T, float alpha_over_p, float lambda,
+                                                           float* __restrict__ s) {
+  __shared__ float red[kRowWarps][kColsPerBlock];
+  __shared__ float s_sm[kColsPerBlock];
+  grid_dep_wait();
+  grid_dep_launch();
+  strip_scale(partial, d, nsplit, T, alpha_over_p, lambda, red, s_sm);
+  const int col = blockIdx.x * kColsPerBlock + threadIdx.x;
+  if (col < d) s[col] = s_sm[threadIdx.x];
 }
 
 // grid: (col_blocks, row_splits); each thread owns 8 consecutive columns for all rows
@@ -329,32 +389,69 @@ StatsPlan stats_plan(int64_t T, int64_t d) {
   return p;
 }
 
-size_t stats_workspace_bytes(int64_t T, int64_t d) {
-  const StatsPlan p = stats_plan(T, d);
-  const size_t part = static_cast<size_t>(p.nsplit) * static_cast<size_t>(d) * sizeof(float);
-  const size_t cnt = 2 * static_cast<size_t>(p.col_blocks) * sizeof(unsigned);  // counter, epoch per strip
-  return ((part + 255) / 256) * 256 + ((cnt + 255) / 256) * 256;
+StatsPlan split_plan(int64_t T, int64_t d, int num_sms) {
+  StatsPlan p;
+  p.col_blocks = static_cast<int>((d + kColsPerBlock - 1) / kColsPerBlock);
+  if (num_sms < 1) num_sms = 1;
+  // the row split that best balances the rows each SM reduces (blocks per SM rounded up,
+  // times rows per block), with at least 32 rows per split; fewer splits win ties
+  const int64_t max_ns = std::max<int64_t>(1, std::min<int64_t>(1024, (T + 31) / 32));
+  int64_t best_ns = 1, best_cost = INT64_MAX;
+  for (int64_t ns = 1; ns <= max_ns; ++ns) {
+    const int64_t per_sm = (static_cast<int64_t>(p.col_blocks) * ns + num_sms - 1) / num_sms;
+    const int64_t cost = per_sm * ((T + ns - 1) / ns);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best_ns = ns;
+    }
+  }
+  p.rows_per_split = (T + best_ns - 1) / best_ns;
+  p.nsplit = static_cast<int>((T + p.rows_per_split - 1) / p.rows_per_split);
+  return p;
 }
 
-cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d, int64_t ld_x, float alpha,
-                             float lambda, int p, float* s, float* partial, unsigned* counters,
-                             cudaStream_t stream) {
-  const StatsPlan pl = stats_plan(T, d);
-  if (pl.nsplit > 1) {
-    cudaError_t e = cudaMemsetAsync(counters, 0, pl.col_blocks * sizeof(unsigned), stream);
-    if (e != cudaSuccess) return e;
-  }
-  dim3 grid(pl.col_blocks, pl.nsplit);
-  const float ap = alpha / static_cast<float>(p);
-  if (p == 2)
-    act_stats_kernel<2><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T,
-                                                  static_cast<int>(d), ld_x, pl.rows_per_split,
-                                                  pl.nsplit, ap, lambda, partial, counters, s);
-  else
-    act_stats_kernel<1><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T,
-                                                  static_cast<int>(d), ld_x, pl.rows_per_split,
-                                                  pl.nsplit, ap, lambda, partial, counters, s);
+size_t split_partial_bytes(int64_t T, int64_t d, int num_sms) {
+  return static_cast<size_t>(split_plan(T, d, num_sms).nsplit) * static_cast<size_t>(d) * sizeof(float);
+}
+
+namespace {
+
+template <typename K, typename... Args>
+cudaError_t launch_dependent(K kernel, dim3 grid, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+template <int P>
+cudaError_t launch_partials(const __nv_bfloat16* X, int64_t T, int d, int64_t ld_x, const StatsPlan& pl,
+                            float* partial, cudaStream_t stream) {
+  stats_partial_kernel<P><<<dim3(pl.col_blocks, pl.nsplit), 256, 0, stream>>>(X, T, d, ld_x, pl.rows_per_split,
+                                                                               partial);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d, int64_t ld_x, float alpha, float lambda, int p,
+                             float* s, float* partial, int num_sms, cudaStream_t stream) {
+  const StatsPlan pl = split_plan(T, d, num_sms);
+  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
+  const int di = static_cast<int>(d);
+  cudaError_t e = p == 2 ? launch_partials<2>(Xb, T, di, ld_x, pl, partial, stream)
+                         : launch_partials<1>(Xb, T, di, ld_x, pl, partial, stream);
+  if (e != cudaSuccess) return e;
+  const float ap = alpha / static_cast<float>(p);
+  return launch_dependent(stats_finish_kernel, dim3(pl.col_blocks), stream, static_cast<const float*>(partial), di,
+                          pl.nsplit, static_cast<float>(T), ap, lambda, s);
 }
 
 cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t ld_x, float alpha,
@@ -386,47 +483,22 @@ cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t
 }
 
 cudaError_t launch_stats_fold(const void* X, int64_t T, int64_t d, float alpha, float lambda, int p, float* s,
-                              float* partial, unsigned* strip_sync, void* Xf, const DevErr& err,
-                              cudaStream_t stream) {
-  static int resident[2] = {0, 0};  // blocks per SM of the p = 1 / p = 2 kernels
-  const int pi = p == 2 ? 1 : 0;
-  if (resident[pi] == 0) {
-    int n = 0;
-    cudaError_t e = p == 2 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, stats_fold_kernel<2>, 256, 0)
-                           : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, stats_fold_kernel<1>, 256, 0);
-    if (e != cudaSuccess) return e;
-    resident[pi] = n > 0 ? n : 1;
-  }
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const StatsPlan base = stats_plan(T, d);
-  // as many row splits as the plan wants, within what can be resident at once
-  int64_t ns = base.nsplit;
-  const int64_t cap = static_cast<int64_t>(resident[pi]) * sms / base.col_blocks;
-  if (ns > cap) ns = cap;
-  if (ns < 1) ns = 1;
-  const int64_t rps = (T + ns - 1) / ns;
-  ns = (T + rps - 1) / rps;
-  cudaError_t e = cudaMemsetAsync(strip_sync, 0, 2 * sizeof(unsigned) * base.col_blocks, stream);
+                              float* partial, void* Xf, int num_sms, cudaStream_t stream) {
+  const StatsPlan pl = split_plan(T, d, num_sms);
+  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
+  const int di = static_cast<int>(d);
+  cudaError_t e = p == 2 ? launch_partials<2>(Xb, T, di, d, pl, partial, stream)
+                         : launch_partials<1>(Xb, T, di, d, pl, partial, stream);
   if (e != cudaSuccess) return e;
-  dim3 grid(base.col_blocks, static_cast<unsigned>(ns));
   const float ap = alpha / static_cast<float>(p);
-  const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
-  __nv_bfloat16* Xo = static_cast<__nv_bfloat16*>(Xf);
-  int di = static_cast<int>(d);
-  int nsi = static_cast<int>(ns);
-  int64_t ld = d;
-  DevErr er = err;
-  void* args[] = {&Xb, &T, &di, &ld, const_cast<int64_t*>(&rps), &nsi, const_cast<float*>(&ap), &lambda,
-                  &partial, &strip_sync, &s, &Xo, &er};
-  // cooperative: the blocks of a strip wait for one another, so all must be resident
+  const dim3 grid(pl.col_blocks, pl.nsplit);
+  auto* Xo = static_cast<__nv_bfloat16*>(Xf);
+  const float* part = partial;
   if (p == 2)
-    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(stats_fold_kernel<2>), grid, dim3(256), args, 0,
-                                    stream);
-  else
-    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(stats_fold_kernel<1>), grid, dim3(256), args, 0,
-                                    stream);
-  return e;
+    return launch_dependent(stats_fold_kernel<2>, grid, stream, Xb, T, di, pl.rows_per_split, pl.nsplit, part, ap,
+                            lambda, s, Xo);
+  return launch_dependent(stats_fold_kernel<1>, grid, stream, Xb, T, di, pl.rows_per_split, pl.nsplit, part, ap,
+                          lambda, s, Xo);
 }
 
 cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const float* s,

@@ -30,9 +30,6 @@ constexpr int kRowsPerWarp = 4;
 constexpr int kGemvThreads = 64;                                  // 2 warps
 constexpr int kRowsPerCta = kRowsPerWarp * kGemvThreads / 32;     // 8: about 7 CTAs per SM, one wave
 
-__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
-
 __device__ __forceinline__ float code_plus_128f(uint32_t x, int b) {
   return __uint_as_float(__byte_perm(x, 0x43000000u, 0x7044u + (static_cast<unsigned>(b) << 8)));
 }

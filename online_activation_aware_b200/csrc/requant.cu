@@ -16,25 +16,18 @@
 // step and writes the row's packed codes as 512 contiguous bytes (q = 4). A group spans
 // g/32 adjacent lanes, which exchange min/max by warp shuffles.
 //
-// The per-element division v / sigma is the hot spot. It is computed as v * (1/sigma)
-// and rounded with the 1.5 * 2^23 add (round half to even on the integer), which equals
-// rint(fl32(v / sigma)) except when the quotient lies within a few ulps of a half
-// integer; a unit whose closest quotient falls inside that window (|q| * 2^-21, far
-// wider than the 2^-22.9 relative error of v * RN(1/sigma)) is recomputed with the
-// IEEE-rounded division, so every code equals the one the rules above define.
+// The per-element division v / sigma is the hot spot. It is computed as v * RN(1/sigma)
+// fused with the 1.5 * 2^23 + z add that rounds it to an integer (half to even), which
+// equals rint(fl32(v / sigma)) + z except when the quotient lies within a few ulps of a
+// half integer; a unit whose closest quotient falls inside a window of (|z| + N) * 2^-21
+// around one (far wider than the 2^-24 relative error of v * RN(1/sigma)) is recomputed
+// with the IEEE-rounded division, so every code equals the one the rules above define.
+// W is read once with an evict-first L2 policy.
 #include "ttq_internal.h"
 
 namespace ttq {
 
 namespace {
-
-__device__ __forceinline__ uint4 ld_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
 
 // Smallest fp16 >= x (x > 0), kept within the finite positive range [2^-24, 65504].
 __device__ __forceinline__ __half fp16_up_sat(float x) {
@@ -42,25 +35,6 @@ __device__ __forceinline__ __half fp16_up_sat(float x) {
   __half h = __float2half_ru(x);
   if (__half_as_ushort(h) == 0u) h = __ushort_as_half(static_cast<unsigned short>(0x0001u));
   return h;
-}
-
-// v = fl32(w * s) for one unit: its 32 bf16 weights in `wv` (4 x 8), the strip's s in
-// shared memory, chunk jj of lane l stored at l * 8 + (jj ^ (l & 7)) (conflict-free).
-__device__ __forceinline__ void scale_unit(const uint4 (&wv)[4], const uint4* s_sm, int lane,
-                                           float (&v)[32]) {
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint4 sa = s_sm[lane * 8 + ((2 * j) ^ (lane & 7))];
-    const uint4 sb = s_sm[lane * 8 + ((2 * j + 1) ^ (lane & 7))];
-    v[8 * j + 0] = __fmul_rn(bf16lo_to_f32(wv[j].x), __uint_as_float(sa.x));
-    v[8 * j + 1] = __fmul_rn(bf16hi_to_f32(wv[j].x), __uint_as_float(sa.y));
-    v[8 * j + 2] = __fmul_rn(bf16lo_to_f32(wv[j].y), __uint_as_float(sa.z));
-    v[8 * j + 3] = __fmul_rn(bf16hi_to_f32(wv[j].y), __uint_as_float(sa.w));
-    v[8 * j + 4] = __fmul_rn(bf16lo_to_f32(wv[j].z), __uint_as_float(sb.x));
-    v[8 * j + 5] = __fmul_rn(bf16hi_to_f32(wv[j].z), __uint_as_float(sb.y));
-    v[8 * j + 6] = __fmul_rn(bf16lo_to_f32(wv[j].w), __uint_as_float(sb.z));
-    v[8 * j + 7] = __fmul_rn(bf16hi_to_f32(wv[j].w), __uint_as_float(sb.w));
-  }
 }
 
 __device__ __forceinline__ float min3f(float a, float b, float c) {
@@ -86,82 +60,119 @@ __device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
-__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
 __device__ __forceinline__ uint64_t f2sub(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
 
-// Packs 32 codes held in the low bytes of `cb` (float bits 1.5 * 2^23 + code: the low
-// byte of such a float is the code) into Q words at `dst`.
+// A lane's 64 B of weights (one unit) sit in its warp's ring slot as four 16-byte chunks,
+// chunk j of lane l at l * 4 + ((j + (l >> 1)) & 3): a quarter warp reading chunk j then
+// touches eight different 16-byte bank groups (conflict-free).
+__device__ __forceinline__ int wchunk(int lane, int j) { return lane * 4 + ((j + (lane >> 1)) & 3); }
+
+// v[0..8) = fl32(w * s) for chunk j (8 weights) of the lane's unit; the strip's s in
+// shared memory, chunk jj of lane l stored at l * 8 + (jj ^ (l & 7)) (conflict-free).
+// Two products per packed f32x2 multiply (each lane of it rounds like __fmul_rn).
+__device__ __forceinline__ void scale_chunk(const uint4* slot, const uint4* s_sm, int lane, int j,
+                                            float* v) {
+  const uint4 wq = slot[wchunk(lane, j)];
+  const uint4 sa = s_sm[lane * 8 + ((2 * j) ^ (lane & 7))];
+  const uint4 sb = s_sm[lane * 8 + ((2 * j + 1) ^ (lane & 7))];
+  const uint32_t w[4] = {wq.x, wq.y, wq.z, wq.w};
+  const float sv[8] = {__uint_as_float(sa.x), __uint_as_float(sa.y), __uint_as_float(sa.z),
+                       __uint_as_float(sa.w), __uint_as_float(sb.x), __uint_as_float(sb.y),
+                       __uint_as_float(sb.z), __uint_as_float(sb.w)};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint64_t p = f2mul(f2(bf16lo_to_f32(w[k]), bf16hi_to_f32(w[k])), f2(sv[2 * k], sv[2 * k + 1]));
+    unf2(p, v[2 * k], v[2 * k + 1]);
+  }
+}
+
+// Packing of a unit's 32 codes, 8 at a time (chunk j = codes 8j .. 8j + 7). A code is the
+// low byte of c[k]: either the bits of the float 1.5 * 2^23 + code (whose low byte is the
+// code) or the plain integer.
+//   q = 4: acc[j] is the finished word (LSB-first nibbles);
+//   q = 2: acc[j] holds 16 bits (LSB-first 2-bit fields) in its low half;
+//   q = 3: acc[b] collects bit plane b of all 32 codes.
 template <int Q>
-__device__ __forceinline__ void store_code_bytes(uint32_t* dst, const uint32_t (&cb)[32]) {
+__device__ __forceinline__ void put_chunk(uint32_t (&acc)[4], int j, const uint32_t (&c)[8]) {
   if (Q == 4) {
-    uint32_t w[4];
+    uint32_t p[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t p[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) p[k] = cb[8 * j + 2 * k] + 16u * cb[8 * j + 2 * k + 1];  // low byte
-      const uint32_t u = __byte_perm(p[0], p[1], 0x5140u);
-      const uint32_t v = __byte_perm(p[2], p[3], 0x5140u);
-      w[j] = __byte_perm(u, v, 0x5410u);
-    }
-    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    for (int k = 0; k < 4; ++k) p[k] = c[2 * k] + 16u * c[2 * k + 1];  // low byte: two nibbles
+    acc[j] = __byte_perm(__byte_perm(p[0], p[1], 0x5140u), __byte_perm(p[2], p[3], 0x5140u), 0x5410u);
   } else if (Q == 2) {
-    uint32_t w[2];
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      uint32_t p[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int e = 16 * j + 4 * k;
-        p[k] = (cb[e] + 4u * cb[e + 1]) + 16u * (cb[e + 2] + 4u * cb[e + 3]);  // low byte
-      }
-      const uint32_t u = __byte_perm(p[0], p[1], 0x5140u);
-      const uint32_t v = __byte_perm(p[2], p[3], 0x5140u);
-      w[j] = __byte_perm(u, v, 0x5410u);
-    }
-    *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
-  } else {  // Q == 3: three bit planes
+    const uint32_t lo = (c[0] + 4u * c[1]) + 16u * (c[2] + 4u * c[3]);  // low byte: four fields
+    const uint32_t hi = (c[4] + 4u * c[5]) + 16u * (c[6] + 4u * c[7]);
+    acc[j] = __byte_perm(lo, hi, 0x0040u);
+  } else {
 #pragma unroll
     for (int b = 0; b < 3; ++b) {
       uint32_t a = 0;
 #pragma unroll
-      for (int k = 0; k < 32; ++k) a |= ((cb[k] >> b) & 1u) << k;
-      dst[b] = a;
+      for (int k = 0; k < 8; ++k) a |= ((c[k] >> b) & 1u) << k;
+      acc[b] |= a << (8 * j);
     }
+  }
+}
+
+template <int Q>
+__device__ __forceinline__ void store_codes(uint32_t* dst, const uint32_t (&acc)[4]) {
+  if (Q == 4) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(acc[0], acc[1], acc[2], acc[3]);
+  } else if (Q == 2) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(__byte_perm(acc[0], acc[1], 0x5410u), __byte_perm(acc[2], acc[3], 0x5410u));
+  } else {
+    dst[0] = acc[0];
+    dst[1] = acc[1];
+    dst[2] = acc[2];
   }
 }
 
 // Group parameters, codes and stores for one unit of 32 scaled weights. Every lane of
 // the warp calls this together (the group's lanes exchange min/max by shuffles).
 //
-// Fast path (no clamp): when z is not clamped, every exact quotient v / sigma lies in
-// [min v / sigma, max v / sigma] and rint of that interval is within [-z, N - z] except
-// at exact half-integer ties, so the code needs no clamping unless some quotient is
-// near a tie; units with a quotient within |q| * 2^-21 of a half integer, or whose
-// group's z was clamped, take the exact path with IEEE division and the clamp.
+// Fast path: t = fl32(v * rcp + (1.5 * 2^23 + z)) with one rounding (packed FMA) holds
+// 1.5 * 2^23 + rint(v * rcp + z) whenever that integer is in range, and its low byte is
+// the code; fr = fl32((t - 1.5 * 2^23 - z) - v * rcp) is the distance of v * rcp from
+// that integer. rcp = RN(1 / sigma) is within 2^-24 relative of 1 / sigma, so v * rcp is
+// within |v / sigma| * 2^-24 of the exact quotient: rounding it gives rint(v / sigma)
+// except within that distance of a half integer. When z is not clamped and sigma is not
+// saturated, every exact quotient lies in [-z - 1/2, N - z + 1/2] up to the rounding of
+// the range (sigma is rounded up to fp16), so the code needs no clamp either except at
+// a half integer. A unit with some |fr| >= 1/2 - (|z| + N) * 2^-21 (a window far wider
+// than those errors), or whose group has a clamped z or a saturated sigma, is recomputed
+// with the IEEE-rounded division and the clamp, so every code equals the rule's.
 template <int Q, int G>
-__device__ __forceinline__ void quantize_unit(const float (&v)[32], int lane, bool store_ok,
-                                              uint32_t* codes_dst, __half* scale_dst,
-                                              __half* zero_dst) {
+__device__ __forceinline__ void quantize_unit(const float (&v)[32], const uint4* slot, const uint4* s_sm,
+                                              int lane, bool store_ok, uint32_t* codes_dst,
+                                              __half* scale_dst, __half* zero_dst) {
   constexpr int LPG = G / 32;  // lanes per group
   constexpr float NQ = static_cast<float>((1 << Q) - 1);
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  float mn = v[0], mx = v[0];
+  // min / max as four short chains (depth 6 instead of 16)
+  float m4[4], x4[4];
 #pragma unroll
-  for (int k = 1; k < 31; k += 2) {
-    mn = min3f(mn, v[k], v[k + 1]);
-    mx = max3f(mx, v[k], v[k + 1]);
+  for (int c = 0; c < 4; ++c) {
+    const float* u = &v[8 * c];
+    float mn_ = min3f(u[0], u[1], u[2]);
+    float mx_ = max3f(u[0], u[1], u[2]);
+    mn_ = min3f(mn_, u[3], u[4]);
+    mx_ = max3f(mx_, u[3], u[4]);
+    mn_ = min3f(mn_, u[5], u[6]);
+    mx_ = max3f(mx_, u[5], u[6]);
+    m4[c] = fminf(mn_, u[7]);
+    x4[c] = fmaxf(mx_, u[7]);
   }
-  mn = fminf(mn, v[31]);
-  mx = fmaxf(mx, v[31]);
+  float mn = fminf(min3f(m4[0], m4[1], m4[2]), m4[3]);
+  float mx = fmaxf(max3f(x4[0], x4[1], x4[2]), x4[3]);
 #pragma unroll
   for (int off = 1; off < LPG; off <<= 1) {
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
@@ -169,41 +180,57 @@ __device__ __forceinline__ void quantize_unit(const float (&v)[32], int lane, bo
   }
   float rng = __fsub_rn(mx, mn);
   if (rng == 0.f) rng = (mn != 0.f) ? fabsf(mn) : 1.0f;
-  const __half sig16 = fp16_up_sat(__fdiv_rn(rng, NQ));
+  const float sig32 = __fdiv_rn(rng, NQ);
+  const __half sig16 = fp16_up_sat(sig32);
   const float sig = __half2float(sig16);
   const float zr = rintf(__fdiv_rn(-mn, sig));
   const float zf = fminf(fmaxf(zr, -2048.f), 2048.f);
 
   const float rcp = __frcp_rn(sig);
-  const float margin = (fabsf(zf) + NQ) * 4.76837158203125e-7f;  // >= max(|lo|, |hi|) * 2^-21
+  const float margin = (fabsf(zf) + NQ) * 4.76837158203125e-7f;  // >= max |v / sigma| * 2^-21
+  const float mz = __fadd_rn(kMagic, zf);                         // exact
   const uint64_t rcp2 = f2(rcp, rcp);
-  const uint64_t magic2 = f2(kMagic, kMagic);
-  const uint64_t z2 = f2(zf, zf);
-  uint32_t cb[32];
+  const uint64_t nrcp2 = f2(-rcp, -rcp);
+  const uint64_t mz2 = f2(mz, mz);
+  uint32_t acc[4] = {0u, 0u, 0u, 0u};
   float fmax_ = 0.f;
 #pragma unroll
-  for (int k = 0; k < 32; k += 2) {
-    const uint64_t q = f2mul(f2(v[k], v[k + 1]), rcp2);
-    const uint64_t t = f2add(q, magic2);      // rounds q to an integer, half to even
-    const uint64_t fr = f2sub(q, f2sub(t, magic2));  // q - rint(q), exact
-    const uint64_t tz = f2add(t, z2);         // 1.5 * 2^23 + rint(q) + z, exact
-    float f0, f1, c0, c1;
-    unf2(fr, f0, f1);
-    unf2(tz, c0, c1);
-    fmax_ = max3f(fmax_, fabsf(f0), fabsf(f1));
-    cb[k] = __float_as_uint(c0);
-    cb[k + 1] = __float_as_uint(c1);
-  }
-  if (fmax_ >= 0.5f - margin || fabsf(zf) >= 2048.f) {
-    // a quotient is near a rounding tie, or z was clamped: the exact definition
+  for (int j = 0; j < 4; ++j) {
+    uint32_t c8[8];
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const float qe = __fadd_rn(rintf(__fdiv_rn(v[k], sig)), zf);
-      cb[k] = static_cast<uint32_t>(fminf(fmaxf(qe, 0.f), NQ));
+    for (int k = 0; k < 8; k += 2) {
+      const uint64_t vv = f2(v[8 * j + k], v[8 * j + k + 1]);
+      const uint64_t t = f2fma(vv, rcp2, mz2);        // 1.5 * 2^23 + rint(v * rcp + z)
+      const uint64_t kk = f2sub(t, mz2);              // rint(v * rcp + z) - z, exact
+      const uint64_t fr = f2fma(vv, nrcp2, kk);       // that - v * rcp, one rounding
+      float f0, f1, c0, c1;
+      unf2(fr, f0, f1);
+      unf2(t, c0, c1);
+      fmax_ = max3f(fmax_, fabsf(f0), fabsf(f1));
+      c8[k] = __float_as_uint(c0);
+      c8[k + 1] = __float_as_uint(c1);
+    }
+    put_chunk<Q>(acc, j, c8);
+  }
+  if (fmax_ >= 0.5f - margin || fabsf(zf) >= 2048.f || sig32 > 65504.f) {
+    // a quotient is near a rounding tie, z was clamped or sigma saturated: the exact rule
+    // (v is formed again from the weights still in the ring slot, 8 at a time)
+    acc[0] = acc[1] = acc[2] = acc[3] = 0u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float v8[8];
+      scale_chunk(slot, s_sm, lane, j, v8);
+      uint32_t c8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float qe = __fadd_rn(rintf(__fdiv_rn(v8[k], sig)), zf);
+        c8[k] = static_cast<uint32_t>(fminf(fmaxf(qe, 0.f), NQ));
+      }
+      put_chunk<Q>(acc, j, c8);
     }
   }
   if (store_ok) {
-    store_code_bytes<Q>(codes_dst, cb);
+    store_codes<Q>(codes_dst, acc);
     if ((lane % LPG) == 0) {
       *scale_dst = sig16;
       *zero_dst = __float2half_rn(zf);
@@ -211,17 +238,33 @@ __device__ __forceinline__ void quantize_unit(const float (&v)[32], int lane, bo
   }
 }
 
-// grid: (column strips of 32 units, row blocks); block: 8 warps. Warp w handles rows
-// r0 + w, r0 + w + 8, ... of the block's range, two rows in flight ahead of the one it
-// quantizes. Lanes past the end of a row compute on clamped data and store nothing.
+constexpr int kRqWarps = 8;   // warps per CTA
+constexpr int kRqStages = 3;  // ring slots per warp (rows in flight: kRqStages - 1 ahead)
+constexpr size_t kRqSmem = (32 * 8 + kRqWarps * kRqStages * 32 * 4) * sizeof(uint4);  // 52 KB
+
+__device__ __forceinline__ void cp_async_16_hint(uint32_t dst, const void* src, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(pol)
+               : "memory");
+}
+
+// grid: (column strips of 32 units, row blocks); block: 8 warps, 4 blocks per SM (3 for
+// q = 3, whose bit-plane packing needs more registers). Warp w
+// handles rows r0 + w, r0 + w + 8, ... of the block's range. Each lane copies its own 64 B
+// of a row (cp.async, L2 evict-first: W is read once, so the folded activations written
+// just before, which the projection reads next, stay in L2) into its warp's ring of
+// kRqStages slots, two rows ahead of the one it quantizes; the lane reads back only what
+// it copied, so no barrier is needed. Lanes past the end of a row work on clamped
+// addresses and store nothing.
 template <int Q, int G>
-__global__ void __launch_bounds__(256, 2) requant_kernel(const __nv_bfloat16* __restrict__ W,
+__global__ void __launch_bounds__(kRqWarps * 32, Q == 3 ? 3 : 4) requant_kernel(const __nv_bfloat16* __restrict__ W,
                                                          const float* __restrict__ s, int d_out,
                                                          int units_per_row, int rows_per_cta,
                                                          uint32_t* __restrict__ codes,
                                                          __half* __restrict__ scale,
                                                          __half* __restrict__ zero) {
-  __shared__ uint4 s_sm[32 * 8];
+  extern __shared__ uint4 rq_smem[];
+  uint4* s_sm = rq_smem;                 // [32 lanes x 8 chunks]
+  uint4* ring = rq_smem + 32 * 8;        // [warp][stage][32 lanes x 4 chunks]
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int unit = blockIdx.x * 32 + lane;
@@ -229,6 +272,34 @@ __global__ void __launch_bounds__(256, 2) requant_kernel(const __nv_bfloat16* __
   const int ucl = col_ok ? unit : units_per_row - 1;
   const int d = units_per_row * 32;
   const int gpr = d / G;
+  const int r0 = blockIdx.y * rows_per_cta;
+  const int r1 = min(d_out, r0 + rows_per_cta);
+  int r = r0 + warp;
+  // per-lane cursors, advanced by 8 rows per step
+  const __nv_bfloat16* wnext = W + static_cast<int64_t>(r) * d + static_cast<int64_t>(ucl) * 32;
+  uint32_t* cdst = codes + (static_cast<int64_t>(r) * units_per_row + ucl) * Q;
+  const int64_t g0 = static_cast<int64_t>(r) * gpr + (ucl * 32) / G;
+  __half* sdst = scale + g0;
+  __half* zdst = zero + g0;
+  const uint32_t ring0 = smem_addr(ring + warp * (kRqStages * 32 * 4));
+  int ahead = r;  // next row to copy
+  auto issue = [&](int stage) {
+    if (ahead < r1) {
+      const uint64_t pol = l2_evict_first_policy();
+      const uint32_t base = ring0 + static_cast<uint32_t>(stage) * (32 * 4 * 16);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) cp_async_16_hint(base + 16u * wchunk(lane, j), wnext + 8 * j, pol);
+    }
+    cp_async_commit();  // one group per row, empty past the end, so the counting stays uniform
+    ahead += 8;
+    wnext += static_cast<int64_t>(8) * d;
+  };
+#pragma unroll
+  for (int i = 0; i < kRqStages - 1; ++i) issue(i);
+  // W does not depend on the kernel ahead in the stream; s does. When launched as a
+  // programmatic dependent, the first rows of W are in flight before this wait.
+  grid_dep_wait();
+  grid_dep_launch();
   {
     const int l = threadIdx.x >> 3;
     const int jj = threadIdx.x & 7;
@@ -238,48 +309,58 @@ __global__ void __launch_bounds__(256, 2) requant_kernel(const __nv_bfloat16* __
     s_sm[l * 8 + (jj ^ (l & 7))] = val;
   }
   __syncthreads();
-
-  const int r0 = blockIdx.y * rows_per_cta;
-  const int r1 = min(d_out, r0 + rows_per_cta);
-  const __nv_bfloat16* wcol = W + static_cast<int64_t>(ucl) * 32;
-  uint4 A[4], B[4];
-  auto load = [&](uint4(&buf)[4], int row) {
-    if (row < r1) {
-      const __nv_bfloat16* p = wcol + static_cast<int64_t>(row) * d;
+  for (int stage = 0; r < r1; r += 8) {
+    issue(stage == 0 ? kRqStages - 1 : stage - 1);
+    cp_async_wait<kRqStages - 1>();  // this lane's copy of row r has landed
+    const uint4* slot = ring + warp * (kRqStages * 32 * 4) + stage * (32 * 4);
+    float v[32];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) buf[j] = ld_stream(p + 8 * j);
-    }
-  };
-  auto finish = [&](const float(&v)[32], int row) {
-    const int64_t u = static_cast<int64_t>(row) * units_per_row + ucl;
-    const int64_t gi = static_cast<int64_t>(row) * gpr + (ucl * 32) / G;
-    quantize_unit<Q, G>(v, lane, col_ok, codes + u * Q, scale + gi, zero + gi);
-  };
-  int r = r0 + warp;
-  load(A, r);
-  load(B, r + 8);
-  for (; r < r1; r += 16) {
-    {
-      float v[32];
-      scale_unit(A, s_sm, lane, v);
-      load(A, r + 16);
-      finish(v, r);
-    }
-    if (r + 8 < r1) {
-      float v[32];
-      scale_unit(B, s_sm, lane, v);
-      load(B, r + 24);
-      finish(v, r + 8);
-    }
+    for (int j = 0; j < 4; ++j) scale_chunk(slot, s_sm, lane, j, &v[8 * j]);
+    quantize_unit<Q, G>(v, slot, s_sm, lane, col_ok, cdst, sdst, zdst);
+    cdst += static_cast<int64_t>(8) * units_per_row * Q;
+    sdst += static_cast<int64_t>(8) * gpr;
+    zdst += static_cast<int64_t>(8) * gpr;
+    stage = stage + 1 == kRqStages ? 0 : stage + 1;
   }
+  cp_async_wait<0>();
+}
+
+template <int Q, int G>
+cudaError_t launch_qg(dim3 grid, const __nv_bfloat16* W, const float* s, int d_out, int units_per_row,
+                      int rows_per_cta, uint32_t* codes, __half* scale, __half* zero, bool pdl,
+                      cudaStream_t stream) {
+  static bool attr_set[64] = {};  // per instantiation and device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(requant_kernel<Q, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kRqSmem));
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kRqWarps * 32);
+  cfg.dynamicSmemBytes = kRqSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, requant_kernel<Q, G>, W, s, d_out, units_per_row, rows_per_cta, codes, scale,
+                            zero);
 }
 
 template <int Q>
 cudaError_t launch_q(int g, const __nv_bfloat16* W, const float* s, int64_t d_out, int units_per_row,
-                     uint32_t* codes, __half* scale, __half* zero, cudaStream_t stream) {
+                     uint32_t* codes, __half* scale, __half* zero, bool pdl, cudaStream_t stream) {
   const int strips = (units_per_row + 31) / 32;
-  // about one wave of 2 CTAs per SM on a 148-SM part, at least 8 rows per CTA
-  int64_t row_blocks = 296 / strips;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // about one wave of resident CTAs, at least 8 rows per CTA
+  int64_t row_blocks = ((Q == 3 ? 3 : 4) * static_cast<int64_t>(sms)) / strips;
   const int64_t max_blocks = (d_out + 7) / 8;
   if (row_blocks > max_blocks) row_blocks = max_blocks;
   if (row_blocks < 1) row_blocks = 1;
@@ -288,31 +369,24 @@ cudaError_t launch_q(int g, const __nv_bfloat16* W, const float* s, int64_t d_ou
   dim3 grid(strips, static_cast<unsigned>(row_blocks));
   const int dout = static_cast<int>(d_out);
   switch (g) {
-    case 32:
-      requant_kernel<Q, 32><<<grid, 256, 0, stream>>>(W, s, dout, units_per_row, rows_per_cta, codes, scale, zero);
-      break;
-    case 64:
-      requant_kernel<Q, 64><<<grid, 256, 0, stream>>>(W, s, dout, units_per_row, rows_per_cta, codes, scale, zero);
-      break;
-    default:
-      requant_kernel<Q, 128><<<grid, 256, 0, stream>>>(W, s, dout, units_per_row, rows_per_cta, codes, scale, zero);
-      break;
+    case 32: return launch_qg<Q, 32>(grid, W, s, dout, units_per_row, rows_per_cta, codes, scale, zero, pdl, stream);
+    case 64: return launch_qg<Q, 64>(grid, W, s, dout, units_per_row, rows_per_cta, codes, scale, zero, pdl, stream);
+    default: return launch_qg<Q, 128>(grid, W, s, dout, units_per_row, rows_per_cta, codes, scale, zero, pdl, stream);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_requant(const void* W, int64_t d_out, int64_t d, const float* s, int q, int g,
-                           uint32_t* codes, void* scale, void* zero, cudaStream_t stream) {
+                           uint32_t* codes, void* scale, void* zero, bool pdl, cudaStream_t stream) {
   const int units_per_row = static_cast<int>(d / 32);
   const auto* Wb = static_cast<const __nv_bfloat16*>(W);
   auto* sc = static_cast<__half*>(scale);
   auto* zr = static_cast<__half*>(zero);
   switch (q) {
-    case 2: return launch_q<2>(g, Wb, s, d_out, units_per_row, codes, sc, zr, stream);
-    case 3: return launch_q<3>(g, Wb, s, d_out, units_per_row, codes, sc, zr, stream);
-    default: return launch_q<4>(g, Wb, s, d_out, units_per_row, codes, sc, zr, stream);
+    case 2: return launch_q<2>(g, Wb, s, d_out, units_per_row, codes, sc, zr, pdl, stream);
+    case 3: return launch_q<3>(g, Wb, s, d_out, units_per_row, codes, sc, zr, pdl, stream);
+    default: return launch_q<4>(g, Wb, s, d_out, units_per_row, codes, sc, zr, pdl, stream);
   }
 }
 

@@ -95,7 +95,7 @@ struct WsLayout {
 WsLayout ws_layout(int64_t T, int64_t d, int64_t d_out, int r, int q, int g, int num_sms) {
   WsLayout L{};
   L.stats_off = 0;
-  L.stats_bytes = round256(ttq::stats_workspace_bytes(T, d));
+  L.stats_bytes = round256(ttq::split_partial_bytes(T, d, num_sms));  // per-split partial sums
   L.xf_off = L.stats_off + L.stats_bytes;
   L.xf_bytes = d_out > 0 ? round256(static_cast<size_t>(T) * static_cast<size_t>(d) * 2) : 0;
   L.u_off = L.xf_off + L.xf_bytes;
@@ -141,12 +141,11 @@ ttq_status ttq_workspace_size(int64_t T, int64_t d, int64_t d_out, const ttq_con
     st = check_cfg(cfg, d);
     if (st != TTQ_OK) return st;
   }
+  // the statistic's row split and the split-K plan depend on the SM count of the current
+  // device (148 when no device can be queried)
   int num_sms = 148;
   DeviceInfo* di = nullptr;
-  if (d_out > 0) {
-    // the split-K plan depends on the SM count of the current device
-    if (device_info(&di) == TTQ_OK) num_sms = di->num_sms;
-  }
+  if (device_info(&di) == TTQ_OK) num_sms = di->num_sms;
   const int q = cfg ? cfg->q : 4;
   const int g = cfg ? cfg->g : 128;
   *bytes = ws_layout(T, d, d_out, r, q, g, num_sms).total;
@@ -164,13 +163,12 @@ ttq_status ttq_act_stats(const void* X_bf16, int64_t T, int64_t d, int64_t ld_x,
   if (!X_bf16 || !s) return TTQ_ERR_INVALID_ARG;
   if (!ws) return TTQ_ERR_WORKSPACE;
   if (!aligned16(X_bf16) || !aligned16(s) || !aligned16(ws)) return TTQ_ERR_MISALIGNED;
-  if (ws_bytes < ws_layout(T, d, 0, 0, 4, 128, 148).total) return TTQ_ERR_WORKSPACE;
-  auto* base = static_cast<uint8_t*>(ws);
-  const size_t part_bytes = static_cast<size_t>(ttq::stats_plan(T, d).nsplit) * d * sizeof(float);
-  float* partial = reinterpret_cast<float*>(base);
-  unsigned* counters = reinterpret_cast<unsigned*>(base + round256(part_bytes));
-  return cuda_status(ttq::launch_act_stats(X_bf16, T, d, ld_x, alpha, lambda, p, s, partial,
-                                           counters, stream));
+  DeviceInfo* di = nullptr;
+  const int num_sms = device_info(&di) == TTQ_OK ? di->num_sms : 148;
+  if (ws_bytes < ws_layout(T, d, 0, 0, 4, 128, num_sms).total) return TTQ_ERR_WORKSPACE;
+  if (!di) return TTQ_ERR_CUDA;
+  float* partial = static_cast<float*>(ws);
+  return cuda_status(ttq::launch_act_stats(X_bf16, T, d, ld_x, alpha, lambda, p, s, partial, num_sms, stream));
 }
 
 ttq_status ttq_requant(const void* W_bf16, int64_t d_out, int64_t d, const float* s, int32_t q,
@@ -184,7 +182,7 @@ ttq_status ttq_requant(const void* W_bf16, int64_t d_out, int64_t d, const float
   if (!aligned16(W_bf16) || !aligned16(s) || !aligned16(codes) || !aligned16(scale_f16) ||
       !aligned16(zero_f16))
     return TTQ_ERR_MISALIGNED;
-  return cuda_status(ttq::launch_requant(W_bf16, d_out, d, s, q, g, codes, scale_f16, zero_f16, stream));
+  return cuda_status(ttq::launch_requant(W_bf16, d_out, d, s, q, g, codes, scale_f16, zero_f16, false, stream));
 }
 
 static ttq_status check_lowrank(const ttq_config* cfg, const void* A, const void* B) {
@@ -220,22 +218,19 @@ ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const vo
   const WsLayout L = ws_layout(T, d, d_out, cfg->r, cfg->q, cfg->g, di->num_sms);
   if (ws_bytes < L.total) return TTQ_ERR_WORKSPACE;
   auto* base = static_cast<uint8_t*>(ws);
-  const size_t part_bytes = static_cast<size_t>(ttq::stats_plan(T, d).nsplit) * d * sizeof(float);
   float* spart = reinterpret_cast<float*>(base + L.stats_off);
-  unsigned* counters = reinterpret_cast<unsigned*>(base + L.stats_off + round256(part_bytes));
   void* Xf = base + L.xf_off;
   void* U = cfg->r > 0 ? base + L.u_off : nullptr;
   float* gpart = L.part_bytes ? reinterpret_cast<float*>(base + L.part_off) : nullptr;
 
   cudaError_t e = trace(0, stream);
   if (e == cudaSuccess)
-    e = ttq::launch_stats_fold(X_bf16, T, d, cfg->alpha, cfg->lambda, cfg->p, s, spart, counters, Xf, dev_err(di),
-                               stream);
+    e = ttq::launch_stats_fold(X_bf16, T, d, cfg->alpha, cfg->lambda, cfg->p, s, spart, Xf, di->num_sms, stream);
   if (e == cudaSuccess) e = trace(1, stream);
   if (e == cudaSuccess && cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, T, d, A_bf16, cfg->r, U, stream);
   if (e == cudaSuccess) e = trace(2, stream);
   if (e == cudaSuccess)
-    e = ttq::launch_requant(W_bf16, d_out, d, s, cfg->q, cfg->g, codes, scale_f16, zero_f16, stream);
+    e = ttq::launch_requant(W_bf16, d_out, d, s, cfg->q, cfg->g, codes, scale_f16, zero_f16, true, stream);
   if (e == cudaSuccess) e = trace(3, stream);
   if (e == cudaSuccess) {
     ttq::GemmArgs ga{Xf, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, T, d, d_out, cfg->q, cfg->g,

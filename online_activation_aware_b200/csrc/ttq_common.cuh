@@ -225,6 +225,35 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// A kernel launched with programmatic stream serialization may start before the kernel
+// ahead of it in the stream has finished; grid_dep_wait() blocks until that kernel has
+// completed and its memory writes are visible (a no-op for a normally launched kernel).
+// grid_dep_launch() lets the next kernel of the stream start launching.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+// ------------------------------------------------------------------ L2 eviction hints
+
+// Cache policy that marks the lines an access touches as the first to evict from L2:
+// for data read (or written) for the last time, so that it does not push out data a
+// later kernel of the same step reads again.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 16-byte read-only load that bypasses L1 and applies an L2 cache policy.
+__device__ __forceinline__ uint4 ld_stream_hint(const void* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
 // ------------------------------------------------------------------ numeric helpers
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -12,20 +12,26 @@ namespace ttq {
 
 // ---------------------------------------------------------------- act_stats / fold
 
-// Column-split plan of the statistics kernel: blocks of 256 columns, T split in
+// Column-split plan of the statistics kernels: blocks of 256 columns, T split in
 // `nsplit` row ranges of `rows_per_split` rows.
 struct StatsPlan {
   int col_blocks;
   int nsplit;
   int64_t rows_per_split;
 };
+// Plan of the single-kernel statistic with arrival counters (launch_act_stats_capped).
 StatsPlan stats_plan(int64_t T, int64_t d);
-size_t stats_workspace_bytes(int64_t T, int64_t d);  // partial sums + counters
 
-// s = (mean_t |x|^p + lambda)^(alpha/p); partial/counters live in the workspace.
-cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d, int64_t ld_x, float alpha,
-                             float lambda, int p, float* s, float* partial, unsigned* counters,
-                             cudaStream_t stream);
+// Row split of the statistic over `num_sms` SMs: blocks of 256 columns x rows_per_split
+// rows, chosen to balance the rows each SM reduces. The partial sums take
+// split_partial_bytes() of workspace.
+StatsPlan split_plan(int64_t T, int64_t d, int num_sms);
+size_t split_partial_bytes(int64_t T, int64_t d, int num_sms);
+
+// s = (mean_t |x|^p + lambda)^(alpha/p): per-split partial sums into `partial` (workspace),
+// then a finishing kernel (programmatic dependent launch) that adds them in a fixed order.
+cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d, int64_t ld_x, float alpha, float lambda, int p,
+                             float* s, float* partial, int num_sms, cudaStream_t stream);
 
 // Same statistic, with at most `max_partial_floats` fp32 partial sums: the row split is
 // reduced until nsplit * d fits (used where the scratch has a fixed size).
@@ -34,12 +40,11 @@ cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t
                                     int64_t max_partial_floats, unsigned* counters,
                                     cudaStream_t stream);
 
-// Statistic and fold in one cooperative launch (X contiguous): writes s and
-// Xf = bf16(X * (1/s)); `strip_sync` (two words of workspace per 256-column strip: a
-// counter, zeroed on the stream first, and an epoch) carries the per-strip barrier.
+// Statistic and fold (X contiguous): the partial sums of launch_act_stats, then a kernel
+// (programmatic dependent launch) whose every block forms s for its strip from the partials
+// and folds its rows, Xf = bf16(X * (1/s)); the blocks of split 0 write s.
 cudaError_t launch_stats_fold(const void* X, int64_t T, int64_t d, float alpha, float lambda, int p, float* s,
-                              float* partial, unsigned* strip_sync, void* Xf, const DevErr& err,
-                              cudaStream_t stream);
+                              float* partial, void* Xf, int num_sms, cudaStream_t stream);
 
 // Xf[t, j] = bf16(X[t, j] * (1 / s[j])), Xf contiguous [T, d].
 cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const float* s,
@@ -75,8 +80,10 @@ cudaError_t launch_decode_gemv(const DecodeArgs& a, void* ws, cudaStream_t strea
 
 // ---------------------------------------------------------------- requant
 
+// pdl: launch as the programmatic dependent of the kernel ahead in the stream (only where
+// that kernel does not write W; the kernel waits for it before it reads s).
 cudaError_t launch_requant(const void* W, int64_t d_out, int64_t d, const float* s, int q, int g,
-                           uint32_t* codes, void* scale, void* zero, cudaStream_t stream);
+                           uint32_t* codes, void* scale, void* zero, bool pdl, cudaStream_t stream);
 
 // ---------------------------------------------------------------- GEMM
 

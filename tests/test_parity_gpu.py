@@ -152,6 +152,23 @@ def test_requant_degenerate_groups():
     requant_check(Wb, synthetic.bf16_values(Wb), np.full(d, 0.3, np.float32), 4, 64)
 
 
+@pytest.mark.parametrize("q", [2, 3, 4])
+def test_requant_saturated_scale_and_clamped_zero(q):
+    # groups whose range is so large that sigma saturates at the largest fp16 (every
+    # quotient then needs the clamp), and groups whose spread is tiny next to their
+    # offset (s varies by a few ulps across the group), so z is clamped to +-2048
+    d_out, d, g = 6, 128, 32
+    W = np.ones((d_out, d))
+    W[0] = np.tile([3.0e6, -3.0e6, 1.0e5, -2.5e4], d // 4)
+    W[1, ::3] = 2.0e7
+    W[2] = -1.0
+    W[3] = np.linspace(-4.0e6, 1.0e4, d)
+    W[4, 64:] = 7.0e6
+    Wb = synthetic.as_bf16(W)
+    s = (1.0 + np.arange(d) * 2.0 ** -20).astype(np.float32)
+    requant_check(Wb, synthetic.bf16_values(Wb), s, q, g)
+
+
 def test_requant_fullsize_qwen3_32b_qproj_sampled_rows():
     # the 5120 -> 8192 projection at its full size; the oracle checks 64 sampled rows
     T, d, d_out, q, g = 4096, 5120, 8192, 4, 128
