@@ -120,19 +120,15 @@ __global__ void __launch_bounds__(256) act_stats_kernel(const __nv_bfloat16* __r
   if (threadIdx.x == 0) counters[blockIdx.x] = 0u;  // leave the strip counter ready
 }
 
-// Statistic, then fold, as two launches that need no grid-wide synchronisation:
+// The statistic as two launches that need no grid-wide synchronisation:
 //   stats_partial_kernel  block (strip c, split k) sums |x|^p over its rows of a 256-column
 //                         strip into partial[k, strip columns] (fp32, fixed order);
-//   stats_fold_kernel     launched as the programmatic dependent of the first, so its
-//                         blocks are resident and waiting when the partial sums land;
-//                         block (c, k) reduces the strip's partials in a fixed order
-//                         (warp w takes splits w, w + 8, ...; the eight warp sums are then
-//                         added in warp order), forms s for the strip (the blocks of split 0
-//                         write it out) and folds its rows, X' = bf16(X * (1/s)), re-reading
-//                         them from L2 (those loads mark the lines evict-first: X is dead
-//                         after them).
-// Every block of a strip reduces the same values in the same order, so all hold the same
-// s. Both grids are sized to a whole number of waves over the SMs.
+//   stats_finish_kernel   launched as the programmatic dependent of the first (its blocks
+//                         are resident and waiting when the partial sums land); block c
+//                         reduces strip c's partials in a fixed order (warp w takes splits
+//                         w, w + 8, ...; the eight warp sums are then added in warp order)
+//                         and writes s for the strip.
+// The partial grid is sized to balance the rows each SM reads.
 template <int P>
 __global__ void __launch_bounds__(256, 5) stats_partial_kernel(const __nv_bfloat16* __restrict__ X, int64_t T,
                                                             int d, int64_t ld_x, int64_t rows_per_split,
@@ -229,55 +225,6 @@ __device__ __forceinline__ void strip_scale(const float* __restrict__ partial, i
   for (int w = 0; w < kRowWarps; ++w) tot = __fadd_rn(tot, red[w][threadIdx.x]);
   s_out[threadIdx.x] = col < d ? finalize_scale(tot, T, alpha_over_p, lambda) : 1.f;
   __syncthreads();
-}
-
-template <int P>
-__global__ void __launch_bounds__(256, 5) stats_fold_kernel(const __nv_bfloat16* __restrict__ X, int64_t T, int d,
-                                                         int64_t rows_per_split, int nsplit,
-                                                         const float* __restrict__ partial,
-                                                         float alpha_over_p, float lambda,
-                                                         float* __restrict__ s, __nv_bfloat16* __restrict__ Xf) {
-  __shared__ float red[kRowWarps][kColsPerBlock];
-  __shared__ float s_sm[kColsPerBlock];
-  grid_dep_wait();  // the partial sums are complete and visible
-  grid_dep_launch();
-  strip_scale(partial, d, nsplit, static_cast<float>(T), alpha_over_p, lambda, red, s_sm);
-  const int col = blockIdx.x * kColsPerBlock + threadIdx.x;
-  if (blockIdx.y == 0 && col < d) s[col] = s_sm[threadIdx.x];
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int col0 = blockIdx.x * kColsPerBlock + lane * 8;
-  if (col0 >= d) return;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
-  const int64_t r1 = min(T, r0 + rows_per_split);
-  __syncwarp();
-  {
-    float* rsw = &red[0][0];  // reciprocals, this lane's 8 columns (the reduction scratch is free now)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) rsw[threadIdx.x * 8 + ((j + lane) & 7)] = __frcp_rn(s_sm[lane * 8 + ((j + lane) & 7)]);
-  }
-  __syncwarp();
-  const float4* rs4 = reinterpret_cast<const float4*>(&red[0][0]) + threadIdx.x * 2;
-  const uint64_t pol = l2_evict_first_policy();
-  auto fold1 = [&](const uint4& v, int64_t r) {
-    const float4 ra = rs4[0], rb = rs4[1];
-    const float rs[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      o[j] = pack_bf16x2(__fmul_rn(bf16lo_to_f32(w[j]), rs[2 * j]), __fmul_rn(bf16hi_to_f32(w[j]), rs[2 * j + 1]));
-    *reinterpret_cast<uint4*>(Xf + r * d + col0) = make_uint4(o[0], o[1], o[2], o[3]);
-  };
-  for (int64_t r = r0 + warp; r < r1; r += 4 * kRowWarps) {  // predicated batches of 4 rows (from L2)
-    uint4 v[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (r + i * kRowWarps < r1) v[i] = ld_stream_hint(X + (r + i * kRowWarps) * d + col0, pol);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (r + i * kRowWarps < r1) fold1(v[i], r + i * kRowWarps);
-  }
 }
 
 // s alone from the partial sums: one block per strip (the finishing step of ttq_act_stats).
@@ -480,25 +427,6 @@ cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t
                                                   static_cast<int>(d), ld_x, pl.rows_per_split,
                                                   pl.nsplit, ap, lambda, partial, counters, s);
   return cudaGetLastError();
-}
-
-cudaError_t launch_stats_fold(const void* X, int64_t T, int64_t d, float alpha, float lambda, int p, float* s,
-                              float* partial, void* Xf, int num_sms, cudaStream_t stream) {
-  const StatsPlan pl = split_plan(T, d, num_sms);
-  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
-  const int di = static_cast<int>(d);
-  cudaError_t e = p == 2 ? launch_partials<2>(Xb, T, di, d, pl, partial, stream)
-                         : launch_partials<1>(Xb, T, di, d, pl, partial, stream);
-  if (e != cudaSuccess) return e;
-  const float ap = alpha / static_cast<float>(p);
-  const dim3 grid(pl.col_blocks, pl.nsplit);
-  auto* Xo = static_cast<__nv_bfloat16*>(Xf);
-  const float* part = partial;
-  if (p == 2)
-    return launch_dependent(stats_fold_kernel<2>, grid, stream, Xb, T, di, pl.rows_per_split, pl.nsplit, part, ap,
-                            lambda, s, Xo);
-  return launch_dependent(stats_fold_kernel<1>, grid, stream, Xb, T, di, pl.rows_per_split, pl.nsplit, part, ap,
-                          lambda, s, Xo);
 }
 
 cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const float* s,

@@ -263,6 +263,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // launched as a programmatic dependent: the set-up above overlaps the end of the kernel
+  // that writes X' (and the codes); no global memory is touched before this wait
+  grid_dep_wait();
   const uint32_t tmem = tail->tmem_base;
 
   if (warp == 0) {
@@ -602,8 +605,17 @@ cudaError_t launch_q(const Maps& mp, const KernelArgs& ka, int grid, size_t smem
   auto kern = ttq_gemm_kernel<Q, S, RING, TQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, stream>>>(mp.x, mp.u, mp.b, mp.c, mp.sc, mp.z, ka);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mp.x, mp.u, mp.b, mp.c, mp.sc, mp.z, ka);
 }
 }  // namespace
 

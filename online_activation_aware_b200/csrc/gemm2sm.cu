@@ -316,6 +316,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __syncthreads();
   cluster_sync();  // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
+  // launched as a programmatic dependent: the set-up above overlaps the end of the kernel
+  // that writes X' and the codes; no global memory is touched before this wait
+  grid_dep_wait();
   const uint32_t tmem = tail->tmem_base;
 
   if (warp == 0) {
@@ -551,8 +554,17 @@ cudaError_t launch_2sm_q(const CUtensorMap* m, const KernelArgs2& ka, int grid, 
   auto kern = ttq_gemm2sm_kernel<Q, S>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, stream>>>(m[0], m[1], m[2], m[3], m[4], m[5], ka);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], m[5], ka);
 }
 
 template <int S>

@@ -238,49 +238,82 @@ __device__ __forceinline__ void quantize_unit(const float (&v)[32], const uint4*
   }
 }
 
-constexpr int kRqWarps = 8;   // warps per CTA
-constexpr int kRqStages = 3;  // ring slots per warp (rows in flight: kRqStages - 1 ahead)
-constexpr size_t kRqSmem = (32 * 8 + kRqWarps * kRqStages * 32 * 4) * sizeof(uint4);  // 52 KB
+constexpr int kRqWarps = 8;    // re-quantization warps per CTA
+constexpr int kFoldWarps = 2;  // activation-folding warps per CTA (fused form)
+constexpr int kRqStages = 3;   // ring slots per warp (rows in flight: kRqStages - 1 ahead)
+
+__host__ __device__ constexpr size_t rq_smem_bytes(bool fold) {
+  // s (and, fused, 1/s) for the strip, then one ring per warp
+  return ((fold ? 2 : 1) * 32 * 8 + (kRqWarps + (fold ? kFoldWarps : 0)) * kRqStages * 32 * 4) * sizeof(uint4);
+}
 
 __device__ __forceinline__ void cp_async_16_hint(uint32_t dst, const void* src, uint64_t pol) {
   asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(pol)
                : "memory");
 }
 
-// grid: (column strips of 32 units, row blocks); block: 8 warps, 4 blocks per SM (3 for
-// q = 3, whose bit-plane packing needs more registers). Warp w
-// handles rows r0 + w, r0 + w + 8, ... of the block's range. Each lane copies its own 64 B
-// of a row (cp.async, L2 evict-first: W is read once, so the folded activations written
-// just before, which the projection reads next, stay in L2) into its warp's ring of
-// kRqStages slots, two rows ahead of the one it quantizes; the lane reads back only what
-// it copied, so no barrier is needed. Lanes past the end of a row work on clamped
-// addresses and store nothing.
-template <int Q, int G>
-__global__ void __launch_bounds__(kRqWarps * 32, Q == 3 ? 3 : 4) requant_kernel(const __nv_bfloat16* __restrict__ W,
-                                                         const float* __restrict__ s, int d_out,
-                                                         int units_per_row, int rows_per_cta,
-                                                         uint32_t* __restrict__ codes,
-                                                         __half* __restrict__ scale,
-                                                         __half* __restrict__ zero) {
+// X' = bf16(x * (1/s)) for one lane's 32 activations of a row (4 chunks of 8, read from the
+// lane's ring slot), with the strip's reciprocals rs_sm laid out like s_sm.
+__device__ __forceinline__ void fold_unit(const uint4* slot, const uint4* rs_sm, int lane, __nv_bfloat16* dst) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 xq = slot[wchunk(lane, j)];
+    const uint4 ra = rs_sm[lane * 8 + ((2 * j) ^ (lane & 7))];
+    const uint4 rb = rs_sm[lane * 8 + ((2 * j + 1) ^ (lane & 7))];
+    const float r[8] = {__uint_as_float(ra.x), __uint_as_float(ra.y), __uint_as_float(ra.z), __uint_as_float(ra.w),
+                        __uint_as_float(rb.x), __uint_as_float(rb.y), __uint_as_float(rb.z), __uint_as_float(rb.w)};
+    const uint32_t w[4] = {xq.x, xq.y, xq.z, xq.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      o[k] = pack_bf16x2(__fmul_rn(bf16lo_to_f32(w[k]), r[2 * k]), __fmul_rn(bf16hi_to_f32(w[k]), r[2 * k + 1]));
+    *reinterpret_cast<uint4*>(dst + 8 * j) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// grid: (column strips of 32 units, row blocks). Every warp streams rows through its own
+// ring of kRqStages shared-memory slots: each lane copies its own 64 B of a row (cp.async,
+// L2 evict-first: the data is read once) two rows ahead of the one it works on, and reads
+// back only what it copied, so no barrier is needed. Warps 0..7 re-quantize rows r0 + w,
+// r0 + w + 8, ... of the block's range of W. In the fused form (FOLD), warps 8..9 at the
+// same time fold the block's share of the activation rows over the same 1024 columns,
+// X' = bf16(x * RN(1/s)), so the W stream and the X stream share the DRAM pipe instead of
+// following one another. Lanes past the end of a row work on clamped addresses and store
+// nothing.
+template <int Q, int G, bool FOLD>
+__global__ void __launch_bounds__((kRqWarps + (FOLD ? kFoldWarps : 0)) * 32, FOLD ? (Q == 3 ? 2 : 3) : (Q == 3 ? 3 : 4))
+    requant_kernel(const __nv_bfloat16* __restrict__ W, const float* __restrict__ s, int d_out, int units_per_row,
+                   int rows_per_cta, uint32_t* __restrict__ codes, __half* __restrict__ scale,
+                   __half* __restrict__ zero, const __nv_bfloat16* __restrict__ X, __nv_bfloat16* __restrict__ Xf,
+                   int T, int x_rows_per_cta) {
   extern __shared__ uint4 rq_smem[];
-  uint4* s_sm = rq_smem;                 // [32 lanes x 8 chunks]
-  uint4* ring = rq_smem + 32 * 8;        // [warp][stage][32 lanes x 4 chunks]
+  uint4* s_sm = rq_smem;                            // [32 lanes x 8 chunks]
+  uint4* rs_sm = rq_smem + 32 * 8;                  // fused: 1/s, same layout
+  uint4* ring = rq_smem + (FOLD ? 2 : 1) * 32 * 8;  // [warp][stage][32 lanes x 4 chunks]
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  const bool folder = FOLD && warp >= kRqWarps;
   const int unit = blockIdx.x * 32 + lane;
   const bool col_ok = unit < units_per_row;
   const int ucl = col_ok ? unit : units_per_row - 1;
   const int d = units_per_row * 32;
-  const int gpr = d / G;
-  const int r0 = blockIdx.y * rows_per_cta;
-  const int r1 = min(d_out, r0 + rows_per_cta);
-  int r = r0 + warp;
-  // per-lane cursors, advanced by 8 rows per step
-  const __nv_bfloat16* wnext = W + static_cast<int64_t>(r) * d + static_cast<int64_t>(ucl) * 32;
-  uint32_t* cdst = codes + (static_cast<int64_t>(r) * units_per_row + ucl) * Q;
-  const int64_t g0 = static_cast<int64_t>(r) * gpr + (ucl * 32) / G;
-  __half* sdst = scale + g0;
-  __half* zdst = zero + g0;
+  // rows this warp streams: W rows r0 + w (step 8), or X rows t0 + (w - 8) (step kFoldWarps)
+  int r, r1, step;
+  const __nv_bfloat16* src;
+  if (folder) {
+    const int t0 = blockIdx.y * x_rows_per_cta;
+    r = t0 + warp - kRqWarps;
+    r1 = min(T, t0 + x_rows_per_cta);
+    step = kFoldWarps;
+    src = X;
+  } else {
+    const int w0 = blockIdx.y * rows_per_cta;
+    r = w0 + warp;
+    r1 = min(d_out, w0 + rows_per_cta);
+    step = kRqWarps;
+    src = W;
+  }
+  const __nv_bfloat16* next = src + static_cast<int64_t>(r) * d + static_cast<int64_t>(ucl) * 32;
   const uint32_t ring0 = smem_addr(ring + warp * (kRqStages * 32 * 4));
   int ahead = r;  // next row to copy
   auto issue = [&](int stage) {
@@ -288,90 +321,136 @@ __global__ void __launch_bounds__(kRqWarps * 32, Q == 3 ? 3 : 4) requant_kernel(
       const uint64_t pol = l2_evict_first_policy();
       const uint32_t base = ring0 + static_cast<uint32_t>(stage) * (32 * 4 * 16);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) cp_async_16_hint(base + 16u * wchunk(lane, j), wnext + 8 * j, pol);
+      for (int j = 0; j < 4; ++j) cp_async_16_hint(base + 16u * wchunk(lane, j), next + 8 * j, pol);
     }
     cp_async_commit();  // one group per row, empty past the end, so the counting stays uniform
-    ahead += 8;
-    wnext += static_cast<int64_t>(8) * d;
+    ahead += step;
+    next += static_cast<int64_t>(step) * d;
   };
 #pragma unroll
   for (int i = 0; i < kRqStages - 1; ++i) issue(i);
-  // W does not depend on the kernel ahead in the stream; s does. When launched as a
-  // programmatic dependent, the first rows of W are in flight before this wait.
+  // W and X do not depend on the kernel ahead in the stream; s does. When launched as a
+  // programmatic dependent, the first rows are in flight before this wait.
   grid_dep_wait();
   grid_dep_launch();
-  {
+  if (threadIdx.x < 256) {
     const int l = threadIdx.x >> 3;
     const int jj = threadIdx.x & 7;
     const int u = blockIdx.x * 32 + l;
     uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (u < units_per_row) val = __ldg(reinterpret_cast<const uint4*>(s + static_cast<int64_t>(u) * 32 + jj * 4));
+    if (u < units_per_row) val = __ldcg(reinterpret_cast<const uint4*>(s + static_cast<int64_t>(u) * 32 + jj * 4));
     s_sm[l * 8 + (jj ^ (l & 7))] = val;
+    if (FOLD) {
+      const uint4 rv = make_uint4(__float_as_uint(__frcp_rn(__uint_as_float(val.x))),
+                                  __float_as_uint(__frcp_rn(__uint_as_float(val.y))),
+                                  __float_as_uint(__frcp_rn(__uint_as_float(val.z))),
+                                  __float_as_uint(__frcp_rn(__uint_as_float(val.w))));
+      rs_sm[l * 8 + (jj ^ (l & 7))] = rv;
+    }
   }
   __syncthreads();
-  for (int stage = 0; r < r1; r += 8) {
+  const uint4* wring = ring + warp * (kRqStages * 32 * 4);
+  if (folder) {
+    __nv_bfloat16* dst = Xf + static_cast<int64_t>(r) * d + static_cast<int64_t>(ucl) * 32;
+    for (int stage = 0; r < r1; r += step) {
+      issue(stage == 0 ? kRqStages - 1 : stage - 1);
+      cp_async_wait<kRqStages - 1>();  // this lane's copy of row r has landed
+      if (col_ok) fold_unit(wring + stage * (32 * 4), rs_sm, lane, dst);
+      dst += static_cast<int64_t>(step) * d;
+      stage = stage + 1 == kRqStages ? 0 : stage + 1;
+    }
+    cp_async_wait<0>();
+    return;
+  }
+  const int gpr = d / G;
+  uint32_t* cdst = codes + (static_cast<int64_t>(r) * units_per_row + ucl) * Q;
+  const int64_t g0 = static_cast<int64_t>(r) * gpr + (ucl * 32) / G;
+  __half* sdst = scale + g0;
+  __half* zdst = zero + g0;
+  for (int stage = 0; r < r1; r += step) {
     issue(stage == 0 ? kRqStages - 1 : stage - 1);
     cp_async_wait<kRqStages - 1>();  // this lane's copy of row r has landed
-    const uint4* slot = ring + warp * (kRqStages * 32 * 4) + stage * (32 * 4);
+    const uint4* slot = wring + stage * (32 * 4);
     float v[32];
 #pragma unroll
     for (int j = 0; j < 4; ++j) scale_chunk(slot, s_sm, lane, j, &v[8 * j]);
     quantize_unit<Q, G>(v, slot, s_sm, lane, col_ok, cdst, sdst, zdst);
-    cdst += static_cast<int64_t>(8) * units_per_row * Q;
-    sdst += static_cast<int64_t>(8) * gpr;
-    zdst += static_cast<int64_t>(8) * gpr;
+    cdst += static_cast<int64_t>(kRqWarps) * units_per_row * Q;
+    sdst += static_cast<int64_t>(kRqWarps) * gpr;
+    zdst += static_cast<int64_t>(kRqWarps) * gpr;
     stage = stage + 1 == kRqStages ? 0 : stage + 1;
   }
   cp_async_wait<0>();
 }
 
-template <int Q, int G>
-cudaError_t launch_qg(dim3 grid, const __nv_bfloat16* W, const float* s, int d_out, int units_per_row,
-                      int rows_per_cta, uint32_t* codes, __half* scale, __half* zero, bool pdl,
-                      cudaStream_t stream) {
+struct RqArgs {
+  const __nv_bfloat16* W;
+  const float* s;
+  int d_out, units_per_row, rows_per_cta;
+  uint32_t* codes;
+  __half* scale;
+  __half* zero;
+  const __nv_bfloat16* X;
+  __nv_bfloat16* Xf;
+  int T, x_rows_per_cta;
+};
+
+template <int Q, int G, bool FOLD>
+cudaError_t launch_qg(dim3 grid, const RqArgs& args, bool pdl, cudaStream_t stream) {
   static bool attr_set[64] = {};  // per instantiation and device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(requant_kernel<Q, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kRqSmem));
+    e = cudaFuncSetAttribute(requant_kernel<Q, G, FOLD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(rq_smem_bytes(FOLD)));
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kRqWarps * 32);
-  cfg.dynamicSmemBytes = kRqSmem;
+  cfg.blockDim = dim3((kRqWarps + (FOLD ? kFoldWarps : 0)) * 32);
+  cfg.dynamicSmemBytes = rq_smem_bytes(FOLD);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, requant_kernel<Q, G>, W, s, d_out, units_per_row, rows_per_cta, codes, scale,
-                            zero);
+  return cudaLaunchKernelEx(&cfg, requant_kernel<Q, G, FOLD>, args.W, args.s, args.d_out, args.units_per_row,
+                            args.rows_per_cta, args.codes, args.scale, args.zero, args.X, args.Xf, args.T,
+                            args.x_rows_per_cta);
 }
 
-template <int Q>
-cudaError_t launch_q(int g, const __nv_bfloat16* W, const float* s, int64_t d_out, int units_per_row,
-                     uint32_t* codes, __half* scale, __half* zero, bool pdl, cudaStream_t stream) {
-  const int strips = (units_per_row + 31) / 32;
+template <int Q, bool FOLD>
+cudaError_t launch_q(int g, RqArgs args, bool pdl, cudaStream_t stream) {
+  const int strips = (args.units_per_row + 31) / 32;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // about one wave of resident CTAs, at least 8 rows per CTA
-  int64_t row_blocks = ((Q == 3 ? 3 : 4) * static_cast<int64_t>(sms)) / strips;
+  // about one wave of resident CTAs, at least 8 rows of W per CTA
+  const int per_sm = FOLD ? (Q == 3 ? 2 : 3) : (Q == 3 ? 3 : 4);  // resident CTAs (launch bounds)
+  const int64_t d_out = args.d_out;
+  int64_t row_blocks = (per_sm * static_cast<int64_t>(sms)) / strips;
   const int64_t max_blocks = (d_out + 7) / 8;
   if (row_blocks > max_blocks) row_blocks = max_blocks;
   if (row_blocks < 1) row_blocks = 1;
-  const int rows_per_cta = static_cast<int>((d_out + row_blocks - 1) / row_blocks);
-  row_blocks = (d_out + rows_per_cta - 1) / rows_per_cta;
-  dim3 grid(strips, static_cast<unsigned>(row_blocks));
-  const int dout = static_cast<int>(d_out);
+  args.rows_per_cta = static_cast<int>((d_out + row_blocks - 1) / row_blocks);
+  row_blocks = (d_out + args.rows_per_cta - 1) / args.rows_per_cta;
+  args.x_rows_per_cta = FOLD ? static_cast<int>((args.T + row_blocks - 1) / row_blocks) : 0;
+  const dim3 grid(strips, static_cast<unsigned>(row_blocks));
   switch (g) {
-    case 32: return launch_qg<Q, 32>(grid, W, s, dout, units_per_row, rows_per_cta, codes, scale, zero, pdl, stream);
-    case 64: return launch_qg<Q, 64>(grid, W, s, dout, units_per_row, rows_per_cta, codes, scale, zero, pdl, stream);
-    default: return launch_qg<Q, 128>(grid, W, s, dout, units_per_row, rows_per_cta, codes, scale, zero, pdl, stream);
+    case 32: return launch_qg<Q, 32, FOLD>(grid, args, pdl, stream);
+    case 64: return launch_qg<Q, 64, FOLD>(grid, args, pdl, stream);
+    default: return launch_qg<Q, 128, FOLD>(grid, args, pdl, stream);
+  }
+}
+
+template <bool FOLD>
+cudaError_t launch_any(int q, int g, const RqArgs& args, bool pdl, cudaStream_t stream) {
+  switch (q) {
+    case 2: return launch_q<2, FOLD>(g, args, pdl, stream);
+    case 3: return launch_q<3, FOLD>(g, args, pdl, stream);
+    default: return launch_q<4, FOLD>(g, args, pdl, stream);
   }
 }
 
@@ -379,15 +458,18 @@ cudaError_t launch_q(int g, const __nv_bfloat16* W, const float* s, int64_t d_ou
 
 cudaError_t launch_requant(const void* W, int64_t d_out, int64_t d, const float* s, int q, int g,
                            uint32_t* codes, void* scale, void* zero, bool pdl, cudaStream_t stream) {
-  const int units_per_row = static_cast<int>(d / 32);
-  const auto* Wb = static_cast<const __nv_bfloat16*>(W);
-  auto* sc = static_cast<__half*>(scale);
-  auto* zr = static_cast<__half*>(zero);
-  switch (q) {
-    case 2: return launch_q<2>(g, Wb, s, d_out, units_per_row, codes, sc, zr, pdl, stream);
-    case 3: return launch_q<3>(g, Wb, s, d_out, units_per_row, codes, sc, zr, pdl, stream);
-    default: return launch_q<4>(g, Wb, s, d_out, units_per_row, codes, sc, zr, pdl, stream);
-  }
+  RqArgs args{static_cast<const __nv_bfloat16*>(W), s, static_cast<int>(d_out), static_cast<int>(d / 32), 0, codes,
+              static_cast<__half*>(scale), static_cast<__half*>(zero), nullptr, nullptr, 0, 0};
+  return launch_any<false>(q, g, args, pdl, stream);
+}
+
+cudaError_t launch_fold_requant(const void* X, int64_t T, void* Xf, const void* W, int64_t d_out, int64_t d,
+                                const float* s, int q, int g, uint32_t* codes, void* scale, void* zero,
+                                cudaStream_t stream) {
+  RqArgs args{static_cast<const __nv_bfloat16*>(W), s, static_cast<int>(d_out), static_cast<int>(d / 32), 0, codes,
+              static_cast<__half*>(scale), static_cast<__half*>(zero), static_cast<const __nv_bfloat16*>(X),
+              static_cast<__nv_bfloat16*>(Xf), static_cast<int>(T), 0};
+  return launch_any<true>(q, g, args, true, stream);
 }
 
 }  // namespace ttq

@@ -223,14 +223,17 @@ ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const vo
   void* U = cfg->r > 0 ? base + L.u_off : nullptr;
   float* gpart = L.part_bytes ? reinterpret_cast<float*>(base + L.part_off) : nullptr;
 
+  // statistic (partial sums, then s) -> (X A^T) -> fold of X fused with the requant of
+  // W -> projection
   cudaError_t e = trace(0, stream);
   if (e == cudaSuccess)
-    e = ttq::launch_stats_fold(X_bf16, T, d, cfg->alpha, cfg->lambda, cfg->p, s, spart, Xf, di->num_sms, stream);
+    e = ttq::launch_act_stats(X_bf16, T, d, d, cfg->alpha, cfg->lambda, cfg->p, s, spart, di->num_sms, stream);
   if (e == cudaSuccess) e = trace(1, stream);
   if (e == cudaSuccess && cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, T, d, A_bf16, cfg->r, U, stream);
   if (e == cudaSuccess) e = trace(2, stream);
   if (e == cudaSuccess)
-    e = ttq::launch_requant(W_bf16, d_out, d, s, cfg->q, cfg->g, codes, scale_f16, zero_f16, true, stream);
+    e = ttq::launch_fold_requant(X_bf16, T, Xf, W_bf16, d_out, d, s, cfg->q, cfg->g, codes, scale_f16, zero_f16,
+                                 stream);
   if (e == cudaSuccess) e = trace(3, stream);
   if (e == cudaSuccess) {
     ttq::GemmArgs ga{Xf, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, T, d, d_out, cfg->q, cfg->g,

@@ -40,12 +40,6 @@ cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t
                                     int64_t max_partial_floats, unsigned* counters,
                                     cudaStream_t stream);
 
-// Statistic and fold (X contiguous): the partial sums of launch_act_stats, then a kernel
-// (programmatic dependent launch) whose every block forms s for its strip from the partials
-// and folds its rows, Xf = bf16(X * (1/s)); the blocks of split 0 write s.
-cudaError_t launch_stats_fold(const void* X, int64_t T, int64_t d, float alpha, float lambda, int p, float* s,
-                              float* partial, void* Xf, int num_sms, cudaStream_t stream);
-
 // Xf[t, j] = bf16(X[t, j] * (1 / s[j])), Xf contiguous [T, d].
 cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const float* s,
                         void* Xf, cudaStream_t stream);
@@ -84,6 +78,14 @@ cudaError_t launch_decode_gemv(const DecodeArgs& a, void* ws, cudaStream_t strea
 // that kernel does not write W; the kernel waits for it before it reads s).
 cudaError_t launch_requant(const void* W, int64_t d_out, int64_t d, const float* s, int q, int g,
                            uint32_t* codes, void* scale, void* zero, bool pdl, cudaStream_t stream);
+
+// The prefill's fused form: the re-quantization of W and, in the same launch (extra warps
+// per CTA), the fold Xf = bf16(X * (1/s)) of the contiguous [T, d] activations. Launched
+// as the programmatic dependent of the kernel ahead in the stream, which must write
+// neither W nor X (it waits for that kernel before it reads s).
+cudaError_t launch_fold_requant(const void* X, int64_t T, void* Xf, const void* W, int64_t d_out, int64_t d,
+                                const float* s, int q, int g, uint32_t* codes, void* scale, void* zero,
+                                cudaStream_t stream);
 
 // ---------------------------------------------------------------- GEMM
 
