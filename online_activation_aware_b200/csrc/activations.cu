@@ -4,9 +4,7 @@
 //               TTQ, section 2; gist.science German summary, section 2);
 //   fold        X diag(1/s) in bf16, the operand the projection multiplies (the
 //               D^(-1/2) of W_hat = Q[W D^(1/2)] D^(-1/2) moved onto the activations);
-//   lowrank_u   U = X A^T for the static low-rank side path (gist.science French
-//               summary, section 2B).
-// All three are HBM-bound streaming passes: a warp reads 512 contiguous bytes of a row
+// Both are HBM-bound streaming passes: a warp reads 512 contiguous bytes of a row
 // per step (32 lanes x 16 B), so every DRAM sector fetched is used in full.
 #include <algorithm>
 #include <climits>
@@ -269,55 +267,6 @@ __global__ void __launch_bounds__(256) fold_kernel(const __nv_bfloat16* __restri
   }
 }
 
-// U = X A^T. Block: 256 threads, 32 tokens; the token tile and a 64-column slice of A
-// are staged in shared memory (fp32); thread (token tid/8, ranks tid%8 + 8j) keeps 8
-// fp32 accumulators. Written for r <= 64 (the pages use r = 16).
-constexpr int kUTok = 32;
-constexpr int kUK = 64;
-__global__ void __launch_bounds__(256) lowrank_u_kernel(const __nv_bfloat16* __restrict__ X,
-                                                        int64_t T, int d,
-                                                        const __nv_bfloat16* __restrict__ A,
-                                                        int r, __nv_bfloat16* __restrict__ U) {
-  __shared__ float xs[kUTok][kUK + 1];
-  __shared__ float as[64][kUK + 1];
-  const int tid = threadIdx.x;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kUTok;
-  // thread -> (token tt = tid / 8, ranks rr = tid % 8 + 8*j for j < 8)
-  const int tt = tid >> 3;
-  const int rb = tid & 7;
-  float acc[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-  for (int k0 = 0; k0 < d; k0 += kUK) {
-    // stage X tile [32 x 64] and A tile [r x 64]
-    for (int e = tid; e < kUTok * kUK; e += 256) {
-      const int a = e / kUK, b = e % kUK;
-      const int64_t t = t0 + a;
-      xs[a][b] = (t < T && k0 + b < d) ? __bfloat162float(X[t * d + k0 + b]) : 0.f;
-    }
-    for (int e = tid; e < 64 * kUK; e += 256) {
-      const int a = e / kUK, b = e % kUK;
-      as[a][b] = (a < r && k0 + b < d) ? __bfloat162float(A[static_cast<int64_t>(a) * d + k0 + b]) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int k = 0; k < kUK; ++k) {
-      const float x = xs[tt][k];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[j] = __fmaf_rn(x, as[rb + 8 * j][k], acc[j]);
-    }
-    __syncthreads();
-  }
-  const int64_t t = t0 + tt;
-  if (t < T) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int rr = rb + 8 * j;
-      U[t * 64 + rr] = __float2bfloat16_rn(rr < r ? acc[j] : 0.f);
-    }
-  }
-}
-
 }  // namespace
 
 StatsPlan stats_plan(int64_t T, int64_t d) {
@@ -444,15 +393,6 @@ cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const
   fold_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T,
                                         static_cast<int>(d), ld_x, s, rps,
                                         static_cast<__nv_bfloat16*>(Xf));
-  return cudaGetLastError();
-}
-
-cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A, int r, void* U,
-                             cudaStream_t stream) {
-  const int64_t blocks = (T + kUTok - 1) / kUTok;
-  lowrank_u_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(X), T, static_cast<int>(d),
-      static_cast<const __nv_bfloat16*>(A), r, static_cast<__nv_bfloat16*>(U));
   return cudaGetLastError();
 }
 

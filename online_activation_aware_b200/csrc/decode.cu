@@ -14,8 +14,8 @@
 // contiguous bytes of codes per step (16-byte loads that bypass L1) and every x' value a
 // lane loads (16-byte loads through L1, contiguous across the warp) serves 4 weights: a
 // load's cost is its per-lane register writeback, so the reuse in registers is what keeps
-// x' traffic below the code traffic. The next unit's codes are in flight while one is
-// consumed; the 32 lanes are summed by shuffles in a fixed order. CTAs of 8 rows put about
+// x' traffic below the code traffic. The codes of the next kDepth units are in flight
+// while one is consumed; the 32 lanes are summed by shuffles in a fixed order. CTAs of 8 rows put about
 // 7 CTAs on each SM, all in one wave, with the rows' scale and zero staged in shared
 // memory. x' (fp32, chunk-major, see xoff) and the unit sums come from a prep kernel
 // chained to the GEMV by programmatic dependent launch: the GEMV issues its first code
@@ -27,6 +27,7 @@ namespace ttq {
 namespace {
 
 constexpr int kRowsPerWarp = 4;
+constexpr int kDepth = 4;  // 32-input units of codes in flight per lane (for each of its rows)
 constexpr int kGemvThreads = 64;                                  // 2 warps
 constexpr int kRowsPerCta = kRowsPerWarp * kGemvThreads / 32;     // 8: about 7 CTAs per SM, one wave
 
@@ -119,8 +120,9 @@ __host__ __device__ __forceinline__ int64_t xoff(int c, int u, int units, int B)
 // One warp per kRowsPerWarp weight rows; lane j takes the rows' 32-input units j, j + 32,
 // j + 64, ... so that each row's 32 lanes read 512 contiguous bytes of codes per step, and
 // every x' value a lane loads serves all kRowsPerWarp rows (a load's cost is its per-lane
-// register writeback, so reuse in registers is what cuts it). The next unit's codes are in
-// flight while one is consumed.
+// register writeback, so reuse in registers is what cuts it). The codes of the next
+// kDepth units are in flight while one is consumed (at d = 5120 a lane's five units are
+// nearly all requested at once).
 template <int Q, int B>
 __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
     const uint32_t* __restrict__ codes, const __half* __restrict__ scale, const __half* __restrict__ zero,
@@ -139,11 +141,15 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
   for (int i = 0; i < R; ++i) crow[i] = codes + static_cast<int64_t>(row0 + i < d_out ? row0 + i : 0) * upr * Q;
   const int nsteps = (upr - lane + 31) >> 5;         // units of this lane: lane, lane + 32, ...
 
-  // the first unit's codes, and the CTA's scale/zero into shared memory, before x' is ready
-  UnitWords<Q> cb[2][R];
-  if (nsteps > 0) {
+  // the first kDepth units' codes, and the CTA's scale/zero into shared memory, before x'
+  // is ready
+  UnitWords<Q> cb[kDepth][R];
 #pragma unroll
-    for (int i = 0; i < R; ++i) cb[0][i] = load_unit<Q>(crow[i] + static_cast<int64_t>(lane) * Q);
+  for (int k = 0; k < kDepth; ++k) {
+    if (k < nsteps) {
+#pragma unroll
+      for (int i = 0; i < R; ++i) cb[k][i] = load_unit<Q>(crow[i] + static_cast<int64_t>(lane + 32 * k) * Q);
+    }
   }
   for (int e = threadIdx.x; e < kRowsPerCta * gpr; e += blockDim.x) {
     const int rr = e / gpr, gi = e - rr * gpr;
@@ -163,16 +169,12 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
   for (int i = 0; i < R; ++i)
 #pragma unroll
     for (int t = 0; t < B; ++t) pacc[i][t] = 0.f;
-  for (int s0 = 0; s0 < nsteps; s0 += 2) {
+  for (int s0 = 0; s0 < nsteps; s0 += kDepth) {
 #pragma unroll
-    for (int hb = 0; hb < 2; ++hb) {
+    for (int hb = 0; hb < kDepth; ++hb) {
       const int st = s0 + hb;
       if (st < nsteps) {
         const int u = lane + 32 * st;
-        if (st + 1 < nsteps) {  // the next unit's codes into the other buffer
-#pragma unroll
-          for (int i = 0; i < R; ++i) cb[hb ^ 1][i] = load_unit<Q>(crow[i] + static_cast<int64_t>(u + 32) * Q);
-        }
         float acc[R][B];
 #pragma unroll
         for (int i = 0; i < R; ++i)
@@ -197,6 +199,11 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
 #pragma unroll
               for (int t = 0; t < B; ++t) acc[i][t] = __fmaf_rn(f[e], x[e * B + t], acc[i][t]);
           }
+        }
+        if (st + kDepth < nsteps) {  // refill the slot just consumed, kDepth units ahead
+#pragma unroll
+          for (int i = 0; i < R; ++i)
+            cb[hb][i] = load_unit<Q>(crow[i] + static_cast<int64_t>(u + 32 * kDepth) * Q);
         }
         // sigma * (sum (128 + c) x' - (128 + z) sum x') for this unit's group, per row
         const TokVec<B> xs = load_tok<B>(usum + static_cast<int64_t>(u) * B);

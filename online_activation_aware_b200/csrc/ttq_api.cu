@@ -99,7 +99,10 @@ WsLayout ws_layout(int64_t T, int64_t d, int64_t d_out, int r, int q, int g, int
   L.xf_off = L.stats_off + L.stats_bytes;
   L.xf_bytes = d_out > 0 ? round256(static_cast<size_t>(T) * static_cast<size_t>(d) * 2) : 0;
   L.u_off = L.xf_off + L.xf_bytes;
-  L.u_bytes = (d_out > 0 && r > 0) ? round256(static_cast<size_t>(T) * 64 * 2) : 0;
+  // U (bf16 [T, 64]) and the fp32 partial sums of its K splits
+  L.u_bytes = (d_out > 0 && r > 0)
+                  ? round256(static_cast<size_t>(T) * 64 * 2) + round256(ttq::lowrank_partial_bytes(T, d, r, num_sms))
+                  : 0;
   L.part_off = L.u_off + L.u_bytes;
   if (d_out > 0) {
     L.plan = ttq::gemm_plan(T, d, d_out, q, g, num_sms);
@@ -221,6 +224,8 @@ ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const vo
   float* spart = reinterpret_cast<float*>(base + L.stats_off);
   void* Xf = base + L.xf_off;
   void* U = cfg->r > 0 ? base + L.u_off : nullptr;
+  float* upart = cfg->r > 0 ? reinterpret_cast<float*>(base + L.u_off + round256(static_cast<size_t>(T) * 64 * 2))
+                            : nullptr;
   float* gpart = L.part_bytes ? reinterpret_cast<float*>(base + L.part_off) : nullptr;
 
   // statistic (partial sums, then s) -> (X A^T) -> fold of X fused with the requant of
@@ -229,7 +234,8 @@ ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const vo
   if (e == cudaSuccess)
     e = ttq::launch_act_stats(X_bf16, T, d, d, cfg->alpha, cfg->lambda, cfg->p, s, spart, di->num_sms, stream);
   if (e == cudaSuccess) e = trace(1, stream);
-  if (e == cudaSuccess && cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, T, d, A_bf16, cfg->r, U, stream);
+  if (e == cudaSuccess && cfg->r > 0)
+    e = ttq::launch_lowrank_u(X_bf16, T, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
   if (e == cudaSuccess) e = trace(2, stream);
   if (e == cudaSuccess)
     e = ttq::launch_fold_requant(X_bf16, T, Xf, W_bf16, d_out, d, s, cfg->q, cfg->g, codes, scale_f16, zero_f16,
@@ -270,11 +276,13 @@ ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d
   auto* base = static_cast<uint8_t*>(ws);
   void* Xf = base + L.xf_off;
   void* U = cfg->r > 0 ? base + L.u_off : nullptr;
+  float* upart = cfg->r > 0 ? reinterpret_cast<float*>(base + L.u_off + round256(static_cast<size_t>(b) * 64 * 2))
+                            : nullptr;
   float* gpart = L.part_bytes ? reinterpret_cast<float*>(base + L.part_off) : nullptr;
   if (L.dec_bytes > 0) {
     // few tokens: the CUDA-core GEMV streams the codes once
     cudaError_t e = cudaSuccess;
-    if (cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, stream);
+    if (cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
     if (e == cudaSuccess) {
       ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16};
       e = ttq::launch_decode_gemv(da, base + L.dec_off, stream);
@@ -282,7 +290,8 @@ ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d
     return cuda_status(e);
   }
   cudaError_t e = ttq::launch_fold(X_bf16, b, d, d, s, Xf, stream);
-  if (e == cudaSuccess && cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, stream);
+  if (e == cudaSuccess && cfg->r > 0)
+    e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
   if (e == cudaSuccess) {
     ttq::GemmArgs ga{Xf, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g,
                      Y_bf16, gpart};

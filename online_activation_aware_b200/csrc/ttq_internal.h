@@ -44,10 +44,14 @@ cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t
 cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const float* s,
                         void* Xf, cudaStream_t stream);
 
-// U[t, :] = X[t, :] A^T in fp32 accumulation, stored bf16 with row stride 64 (columns
-// r..63 zero). Requires r <= 64.
-cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A, int r, void* U,
-                             cudaStream_t stream);
+// U[t, :] = X[t, :] A^T in fp32 accumulation (tensor cores, K split over blocks, the
+// splits added in a fixed order by a dependent kernel), stored bf16 with row stride 64
+// (columns r..63 zero). Requires r % 8 == 0, r <= 64; `partial` holds
+// lowrank_partial_bytes() of workspace.
+int lowrank_splits(int64_t T, int64_t d, int num_sms);
+size_t lowrank_partial_bytes(int64_t T, int64_t d, int r, int num_sms);
+cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A, int r, void* U, float* partial,
+                             int num_sms, cudaStream_t stream);
 
 // ---------------------------------------------------------------- decode
 
