@@ -381,9 +381,10 @@ def main():
     value = whole_job_ktoks(T, K, world, t_max_ms)
 
     plan_split = stage_ms["reduce"] > 0.002
-    # kernels of ours per step: statistic partial sums, statistic finish, (low-rank X A^T),
-    # fold + requant, tensor-core GEMM, (split-K reduce)
-    launches_per_step = 4 + (1 if r > 0 else 0) + (1 if plan_split else 0)
+    # kernels of ours per step: statistic partial sums, statistic finish, (low-rank X A^T
+    # partial products and their reduction), fold + requant, tensor-core GEMM, (split-K
+    # reduce)
+    launches_per_step = 4 + (2 if r > 0 else 0) + (1 if plan_split else 0)
 
     kern = {
         "stats": {"ms": stage_ms["stats"], "bound": "hbm", "bytes": stats_bytes(T, d)},
@@ -470,6 +471,8 @@ def main():
         result["cpu_baseline"] = cpu_baseline(Xv, Wv, wl, args.cpu_seconds)
         result["decode"] = decode_leg(torch, ttq, wl, cfg, Xs[0], Ws[0], A, B, dev, hbm_peak)
         result["sweep"] = sweep_leg(torch, ttq, wl, cfg, Wb, A, B, dev, r)
+        if r == 0:
+            result["lowrank_r16"] = lowrank_leg(torch, ttq, wl, Xs, Ws, dev)
     if rank == 0:
         print(json.dumps(result), flush=True)
     D.barrier()
@@ -548,6 +551,33 @@ def decode_leg(torch, ttq, wl, cfg, X, W, A, B, dev, hbm_peak):
                         "GBps": round(by / t / 1e9, 1), "frac_hbm": round(by / t / 1e9 / hbm_peak, 4)}
     assert ttq.device_status() == 0
     return out
+
+
+def lowrank_leg(torch, ttq, wl, Xs, Ws, dev, r=16, K=30):
+    """The same prefill with the low-rank side path (rank r): seeded random bf16 factors
+    B [d_out, r], A [r, d] of the right shapes stand in for the SVD factors (the kernels'
+    time does not depend on their values); rotating buffer sets as in the main run."""
+    lin = wl.layers[0]
+    d, d_out, T = lin.d, lin.d_out, Xs[0].shape[0]
+    g_ = torch.Generator(device="cpu").manual_seed(16)
+    A = (torch.randn(r, d, generator=g_) * 0.02).to(torch.bfloat16).to(dev)
+    B = (torch.randn(d_out, r, generator=g_) * 0.02).to(torch.bfloat16).to(dev)
+    cfg = ttq.make_config(wl.q, wl.g, wl.alpha, wl.lam, wl.p, r)
+    ws = ttq.alloc_workspace(T, d, d_out, cfg, dev)
+    n = len(Xs)
+    outs = [ttq.linear_prefill(Xs[i], Ws[i], cfg, A, B, ws=ws) for i in range(n)]
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(K):
+        ttq.linear_prefill(Xs[i % n], Ws[i % n], cfg, A, B, out=outs[i % n], ws=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / K
+    assert ttq.device_status() == 0
+    return {"r": r, "T": T, "k_tokens_per_s": round(T / t / 1e3, 2), "us_per_prompt": round(t * 1e6, 1),
+            "factors": "seeded random bf16 of the SVD factors' shapes"}
 
 
 def sweep_leg(torch, ttq, wl, cfg, Wb, A, B, dev, r):

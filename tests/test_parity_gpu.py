@@ -211,6 +211,9 @@ def gpu_linear_with_oracle_codes(Xb, s32, oc, osc, oz, A, B, q, g, r, d_out):
     (128, 512, 256, 4, 128, 0), (300, 320, 200, 4, 64, 0), (1024, 768, 768, 4, 32, 0),
     (64, 256, 128, 4, 32, 16), (300, 512, 384, 3, 32, 16), (2048, 768, 3072, 4, 32, 0),
     (513, 1024, 640, 2, 32, 8), (4096, 512, 256, 4, 128, 0),
+    # low rank: odd number of 8-rank tiles, the largest rank, K not a multiple of the
+    # low-rank kernel's 64-wide stages, ragged token blocks
+    (70, 96, 64, 3, 32, 24), (200, 1088, 256, 4, 64, 64), (1, 160, 96, 4, 32, 40),
 ])
 def test_gemm_parity_with_oracle_codes(T, d, d_out, q, g, r):
     Xb, X, s32, oc, osc, oz, A, B = oracle_inputs(T, d, d_out, q, g, r, seed=T * 3 + d)
@@ -313,7 +316,8 @@ def test_zero_weight_and_zero_activation():
 
 
 @pytest.mark.parametrize("b", [1, 2, 3, 4, 5, 8])
-@pytest.mark.parametrize("q,g,r,d_out", [(4, 128, 0, 384), (3, 32, 0, 300), (2, 32, 16, 256), (4, 64, 8, 130)])
+@pytest.mark.parametrize("q,g,r,d_out", [(4, 128, 0, 384), (3, 32, 0, 300), (2, 32, 16, 256), (4, 64, 8, 130),
+                                         (4, 32, 64, 192)])
 def test_decode_few_tokens_parity(b, q, g, r, d_out):
     # few decode tokens run on the CUDA-core GEMV (codes streamed once); same bar as the GEMM
     d = 1024
