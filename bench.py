@@ -427,6 +427,7 @@ def main():
                    "q": q, "g": g, "alpha": wl.alpha, "lambda": wl.lam, "r": r, "parallelism": f"replicas{world}",
                    "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.0f} MB (> 126 MB L2)"},
         "requant_gbs": requant_leg(torch, ttq, Ws, outs, d, d_out, q, g),
+        "requant_batched": requant_batched_leg(torch, ttq, Ws, outs, d, d_out, q, g),
         "roofline": roof,
         "kernels": kern,
         "rho_measured": round((stage_ms["stats"] + stage_ms["fold_requant"]) / (stage_ms["gemm"] + stage_ms["reduce"]), 4),
@@ -502,6 +503,46 @@ def requant_leg(torch, ttq, Ws, outs, d, d_out, q, g, reps=100):
     torch.cuda.synchronize()
     sec = e0.elapsed_time(e1) / 1e3 / reps
     return round(requant_bytes(d, d_out, q, g) / sec / 1e9, 1)
+
+
+def requant_batched_leg(torch, ttq, Ws, outs, d, d_out, q, g, P=4, reps=50):
+    """One weight re-quantized for P prompts per launch (ttq_requant_batched: W read once,
+    P sets of codes / scale / zero written), rotating weight sets; compared with P
+    single-prompt launches (ttq_requant) over the same sets."""
+    n = len(Ws)
+    S = torch.stack([outs[i % n]["s"] for i in range(P)]).contiguous()
+    dev = Ws[0].device
+    res_ = [ttq.requant_batched(Ws[0], S, q, g) for _ in range(2)]
+
+    def timed(fn):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(reps):
+            fn(i)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3 / reps
+
+    def batched(i):
+        c, s_, z = res_[i % 2]
+        ttq.requant_batched(Ws[i % n], S, q, g, codes=c, scale=s_, zero=z)
+
+    def singles(i):
+        c, s_, z = res_[i % 2]
+        for p in range(P):
+            ttq.requant(Ws[i % n], S[p], q, g, codes=c[p], scale=s_[p], zero=z[p])
+
+    tb = timed(batched)
+    ts = timed(singles)
+    by = d_out * d * 2 + P * (d * 4 + d_out * d * q // 8 + d_out * (d // g) * 4)
+    del res_, S
+    return {"prompts": P, "us_per_launch": round(tb * 1e6, 2), "us_per_prompt": round(tb * 1e6 / P, 2),
+            "GBps": round(by / tb / 1e9, 1), "single_prompt_launches_us": round(ts * 1e6, 2),
+            "speedup_vs_single": round(ts / tb, 3)}
 
 
 def decode_leg(torch, ttq, wl, cfg, X, W, A, B, dev, hbm_peak):

@@ -133,6 +133,19 @@ TTQ_API ttq_status ttq_requant(const void* W_bf16, int64_t d_out, int64_t d, con
                        int32_t g, uint32_t* codes, void* scale_f16, void* zero_f16,
                        cudaStream_t stream);
 
+/* Re-quantization of one weight for P prompts at once (P = 1 .. 8), each against its own
+ * statistic, from a single read of W: the multi-prompt case that [DR] section 5 leaves
+ * open (every request of a serving batch carries its own D). Prompt p's results equal
+ * ttq_requant(W, s + p * d, ...) bit for bit.
+ *   W      device bf16 [d_out, d]
+ *   s      device fp32 [P, d], prompt-major
+ *   codes  device uint32 [P, ttq_codes_words(d_out, d, q)] output
+ *   scale  device fp16 [P, d_out, d/g] output;  zero  device fp16 [P, d_out, d/g] output
+ * P outside 1 .. 8 returns TTQ_ERR_UNSUPPORTED. Needs no workspace. */
+TTQ_API ttq_status ttq_requant_batched(const void* W_bf16, int64_t d_out, int64_t d, const float* s,
+                                       int32_t prompts, int32_t q, int32_t g, uint32_t* codes, void* scale_f16,
+                                       void* zero_f16, cudaStream_t stream);
+
 /* One prompt through a TTQ linear layer ([DR] section 2 and section 6: statistics and
  * scale-quantize-rescale at prefill): s = stats(X); (codes, scale, zero) = requant(W, s);
  * Y = (X diag(1/s)) deq(codes)^T + (X A^T) B^T, where deq(c) = (c - z) * sigma is the

@@ -7,7 +7,7 @@ in the library's CUDA kernels. There is no CPU fallback: when the library is mis
 or a call fails, a ``TTQError`` is raised.
 
 Functions keep the C names without the ``ttq_`` prefix:
-``act_stats``, ``requant``, ``linear_prefill``, ``linear_decode``, ``workspace_size``,
+``act_stats``, ``requant``, ``requant_batched``, ``linear_prefill``, ``linear_decode``, ``workspace_size``,
 ``codes_words``, ``device_status``, ``set_wait_limit_ns``. ``TTQLinear`` bundles one
 layer's weight and the per-prompt buffers (prefill, then decode reusing the codes).
 """
@@ -59,6 +59,8 @@ def load_library(path: str = LIB_PATH):
     lib.ttq_act_stats_noalloc.restype = i32
     lib.ttq_requant.argtypes = [vp, i64, i64, vp, i32, i32, vp, vp, vp, vp]
     lib.ttq_requant.restype = i32
+    lib.ttq_requant_batched.argtypes = [vp, i64, i64, vp, i32, i32, i32, vp, vp, vp, vp]
+    lib.ttq_requant_batched.restype = i32
     lib.ttq_linear_prefill.argtypes = [vp, i64, i64, vp, i64, vp, vp, cfgp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.ttq_linear_prefill.restype = i32
     lib.ttq_linear_decode.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, cfgp, vp, vp, sz, vp]
@@ -165,6 +167,29 @@ def requant(W, s, q: int, g: int, codes=None, scale=None, zero=None, stream=None
         zero = torch.empty(d_out, d // g, dtype=torch.float16, device=dev)
     _check("ttq_requant", load_library().ttq_requant(
         _ptr(W, torch.bfloat16, "W"), d_out, d, _ptr(s, torch.float32, "s"), q, g,
+        _ptr(codes, torch.int32, "codes"), _ptr(scale, torch.float16, "scale"),
+        _ptr(zero, torch.float16, "zero"), _stream(stream)))
+    return codes, scale, zero
+
+
+def requant_batched(W, S, q: int, g: int, codes=None, scale=None, zero=None, stream=None):
+    """Codes, scale and zero of Q[W diag(s_p)] for P prompts from one read of W.
+
+    W [d_out, d] bf16; S [P, d] fp32 (P = 1 .. 8). Returns (codes [P, words] int32,
+    scale [P, d_out, d/g] fp16, zero [P, d_out, d/g] fp16)."""
+    import torch
+
+    d_out, d = W.shape
+    P = S.shape[0]
+    dev = W.device
+    if codes is None:
+        codes = torch.empty(P, codes_words(d_out, d, q), dtype=torch.int32, device=dev)
+    if scale is None:
+        scale = torch.empty(P, d_out, d // g, dtype=torch.float16, device=dev)
+    if zero is None:
+        zero = torch.empty(P, d_out, d // g, dtype=torch.float16, device=dev)
+    _check("ttq_requant_batched", load_library().ttq_requant_batched(
+        _ptr(W, torch.bfloat16, "W"), d_out, d, _ptr(S, torch.float32, "S"), P, q, g,
         _ptr(codes, torch.int32, "codes"), _ptr(scale, torch.float16, "scale"),
         _ptr(zero, torch.float16, "zero"), _stream(stream)))
     return codes, scale, zero

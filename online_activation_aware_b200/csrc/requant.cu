@@ -242,9 +242,18 @@ constexpr int kRqWarps = 8;    // re-quantization warps per CTA
 constexpr int kFoldWarps = 2;  // activation-folding warps per CTA (fused form)
 constexpr int kRqStages = 3;   // ring slots per warp (rows in flight: kRqStages - 1 ahead)
 
-__host__ __device__ constexpr size_t rq_smem_bytes(bool fold) {
-  // s (and, fused, 1/s) for the strip, then one ring per warp
-  return ((fold ? 2 : 1) * 32 * 8 + (kRqWarps + (fold ? kFoldWarps : 0)) * kRqStages * 32 * 4) * sizeof(uint4);
+// Forms of the kernel: one prompt; one prompt with the fold of its activations; P prompts
+// sharing one read of W.
+enum RqMode { kRqSingle = 0, kRqFold = 1, kRqBatch = 2 };
+
+__host__ __device__ constexpr size_t rq_smem_bytes(int mode, int prompts) {
+  // s of every prompt (and, fused, 1/s) for the strip, then one ring per warp
+  return ((mode == kRqFold ? 2 : prompts) * 32 * 8 + (kRqWarps + (mode == kRqFold ? kFoldWarps : 0)) * kRqStages * 32 * 4) *
+         sizeof(uint4);
+}
+
+__host__ __device__ constexpr int rq_ctas_per_sm(int mode, int q) {
+  return mode == kRqFold ? (q == 3 ? 2 : 3) : mode == kRqBatch ? 2 : (q == 3 ? 3 : 4);
 }
 
 __device__ __forceinline__ void cp_async_16_hint(uint32_t dst, const void* src, uint64_t pol) {
@@ -275,21 +284,25 @@ __device__ __forceinline__ void fold_unit(const uint4* slot, const uint4* rs_sm,
 // ring of kRqStages shared-memory slots: each lane copies its own 64 B of a row (cp.async,
 // L2 evict-first: the data is read once) two rows ahead of the one it works on, and reads
 // back only what it copied, so no barrier is needed. Warps 0..7 re-quantize rows r0 + w,
-// r0 + w + 8, ... of the block's range of W. In the fused form (FOLD), warps 8..9 at the
+// r0 + w + 8, ... of the block's range of W. In the fused form (kRqFold), warps 8..9 at the
 // same time fold the block's share of the activation rows over the same 1024 columns,
 // X' = bf16(x * RN(1/s)), so the W stream and the X stream share the DRAM pipe instead of
-// following one another. Lanes past the end of a row work on clamped addresses and store
-// nothing.
-template <int Q, int G, bool FOLD>
-__global__ void __launch_bounds__((kRqWarps + (FOLD ? kFoldWarps : 0)) * 32, FOLD ? (Q == 3 ? 2 : 3) : (Q == 3 ? 3 : 4))
+// following one another. In the batched form (kRqBatch) each row of W, once in shared
+// memory, is re-quantized against the statistic of each of P prompts in turn (prompt p
+// writes codes + p * cstride, scale / zero + p * mstride). Lanes past the end of a row
+// work on clamped addresses and store nothing.
+template <int Q, int G, int MODE>
+__global__ void __launch_bounds__((kRqWarps + (MODE == kRqFold ? kFoldWarps : 0)) * 32, rq_ctas_per_sm(MODE, Q))
     requant_kernel(const __nv_bfloat16* __restrict__ W, const float* __restrict__ s, int d_out, int units_per_row,
                    int rows_per_cta, uint32_t* __restrict__ codes, __half* __restrict__ scale,
                    __half* __restrict__ zero, const __nv_bfloat16* __restrict__ X, __nv_bfloat16* __restrict__ Xf,
-                   int T, int x_rows_per_cta) {
+                   int T, int x_rows_per_cta, int prompts, int64_t cstride, int64_t mstride) {
+  constexpr bool FOLD = MODE == kRqFold;
+  const int P = MODE == kRqBatch ? prompts : 1;
   extern __shared__ uint4 rq_smem[];
-  uint4* s_sm = rq_smem;                            // [32 lanes x 8 chunks]
+  uint4* s_sm = rq_smem;                            // [prompt][32 lanes x 8 chunks]
   uint4* rs_sm = rq_smem + 32 * 8;                  // fused: 1/s, same layout
-  uint4* ring = rq_smem + (FOLD ? 2 : 1) * 32 * 8;  // [warp][stage][32 lanes x 4 chunks]
+  uint4* ring = rq_smem + (FOLD ? 2 : P) * 32 * 8;  // [warp][stage][32 lanes x 4 chunks]
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const bool folder = FOLD && warp >= kRqWarps;
@@ -340,6 +353,13 @@ __global__ void __launch_bounds__((kRqWarps + (FOLD ? kFoldWarps : 0)) * 32, FOL
     uint4 val = make_uint4(0u, 0u, 0u, 0u);
     if (u < units_per_row) val = __ldcg(reinterpret_cast<const uint4*>(s + static_cast<int64_t>(u) * 32 + jj * 4));
     s_sm[l * 8 + (jj ^ (l & 7))] = val;
+    for (int p = 1; p < P; ++p) {  // batched: the other prompts' statistics
+      uint4 vp = make_uint4(0u, 0u, 0u, 0u);
+      if (u < units_per_row)
+        vp = __ldcg(reinterpret_cast<const uint4*>(s + static_cast<int64_t>(p) * d + static_cast<int64_t>(u) * 32 +
+                                                   jj * 4));
+      s_sm[p * 256 + l * 8 + (jj ^ (l & 7))] = vp;
+    }
     if (FOLD) {
       const uint4 rv = make_uint4(__float_as_uint(__frcp_rn(__uint_as_float(val.x))),
                                   __float_as_uint(__frcp_rn(__uint_as_float(val.y))),
@@ -371,10 +391,21 @@ __global__ void __launch_bounds__((kRqWarps + (FOLD ? kFoldWarps : 0)) * 32, FOL
     issue(stage == 0 ? kRqStages - 1 : stage - 1);
     cp_async_wait<kRqStages - 1>();  // this lane's copy of row r has landed
     const uint4* slot = wring + stage * (32 * 4);
-    float v[32];
+    if (MODE == kRqBatch) {
+#pragma unroll 1
+      for (int p = 0; p < P; ++p) {
+        const uint4* sp = s_sm + p * 256;
+        float v[32];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) scale_chunk(slot, s_sm, lane, j, &v[8 * j]);
-    quantize_unit<Q, G>(v, slot, s_sm, lane, col_ok, cdst, sdst, zdst);
+        for (int j = 0; j < 4; ++j) scale_chunk(slot, sp, lane, j, &v[8 * j]);
+        quantize_unit<Q, G>(v, slot, sp, lane, col_ok, cdst + p * cstride, sdst + p * mstride, zdst + p * mstride);
+      }
+    } else {
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) scale_chunk(slot, s_sm, lane, j, &v[8 * j]);
+      quantize_unit<Q, G>(v, slot, s_sm, lane, col_ok, cdst, sdst, zdst);
+    }
     cdst += static_cast<int64_t>(kRqWarps) * units_per_row * Q;
     sdst += static_cast<int64_t>(kRqWarps) * gpr;
     zdst += static_cast<int64_t>(kRqWarps) * gpr;
@@ -393,42 +424,44 @@ struct RqArgs {
   const __nv_bfloat16* X;
   __nv_bfloat16* Xf;
   int T, x_rows_per_cta;
+  int prompts;
+  int64_t cstride, mstride;
 };
 
-template <int Q, int G, bool FOLD>
+template <int Q, int G, int MODE>
 cudaError_t launch_qg(dim3 grid, const RqArgs& args, bool pdl, cudaStream_t stream) {
-  static bool attr_set[64] = {};  // per instantiation and device
+  static bool attr_set[64] = {};  // per instantiation and device (set for the largest batch)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(requant_kernel<Q, G, FOLD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(rq_smem_bytes(FOLD)));
+    e = cudaFuncSetAttribute(requant_kernel<Q, G, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(rq_smem_bytes(MODE, MODE == kRqBatch ? kRequantMaxPrompts : 1)));
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3((kRqWarps + (FOLD ? kFoldWarps : 0)) * 32);
-  cfg.dynamicSmemBytes = rq_smem_bytes(FOLD);
+  cfg.blockDim = dim3((kRqWarps + (MODE == kRqFold ? kFoldWarps : 0)) * 32);
+  cfg.dynamicSmemBytes = rq_smem_bytes(MODE, args.prompts);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, requant_kernel<Q, G, FOLD>, args.W, args.s, args.d_out, args.units_per_row,
+  return cudaLaunchKernelEx(&cfg, requant_kernel<Q, G, MODE>, args.W, args.s, args.d_out, args.units_per_row,
                             args.rows_per_cta, args.codes, args.scale, args.zero, args.X, args.Xf, args.T,
-                            args.x_rows_per_cta);
+                            args.x_rows_per_cta, args.prompts, args.cstride, args.mstride);
 }
 
-template <int Q, bool FOLD>
+template <int Q, int MODE>
 cudaError_t launch_q(int g, RqArgs args, bool pdl, cudaStream_t stream) {
   const int strips = (args.units_per_row + 31) / 32;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // about one wave of resident CTAs, at least 8 rows of W per CTA
-  const int per_sm = FOLD ? (Q == 3 ? 2 : 3) : (Q == 3 ? 3 : 4);  // resident CTAs (launch bounds)
+  // about one wave of resident CTAs (launch bounds), at least 8 rows of W per CTA
+  const int per_sm = rq_ctas_per_sm(MODE, Q);
   const int64_t d_out = args.d_out;
   int64_t row_blocks = (per_sm * static_cast<int64_t>(sms)) / strips;
   const int64_t max_blocks = (d_out + 7) / 8;
@@ -436,21 +469,21 @@ cudaError_t launch_q(int g, RqArgs args, bool pdl, cudaStream_t stream) {
   if (row_blocks < 1) row_blocks = 1;
   args.rows_per_cta = static_cast<int>((d_out + row_blocks - 1) / row_blocks);
   row_blocks = (d_out + args.rows_per_cta - 1) / args.rows_per_cta;
-  args.x_rows_per_cta = FOLD ? static_cast<int>((args.T + row_blocks - 1) / row_blocks) : 0;
+  args.x_rows_per_cta = MODE == kRqFold ? static_cast<int>((args.T + row_blocks - 1) / row_blocks) : 0;
   const dim3 grid(strips, static_cast<unsigned>(row_blocks));
   switch (g) {
-    case 32: return launch_qg<Q, 32, FOLD>(grid, args, pdl, stream);
-    case 64: return launch_qg<Q, 64, FOLD>(grid, args, pdl, stream);
-    default: return launch_qg<Q, 128, FOLD>(grid, args, pdl, stream);
+    case 32: return launch_qg<Q, 32, MODE>(grid, args, pdl, stream);
+    case 64: return launch_qg<Q, 64, MODE>(grid, args, pdl, stream);
+    default: return launch_qg<Q, 128, MODE>(grid, args, pdl, stream);
   }
 }
 
-template <bool FOLD>
+template <int MODE>
 cudaError_t launch_any(int q, int g, const RqArgs& args, bool pdl, cudaStream_t stream) {
   switch (q) {
-    case 2: return launch_q<2, FOLD>(g, args, pdl, stream);
-    case 3: return launch_q<3, FOLD>(g, args, pdl, stream);
-    default: return launch_q<4, FOLD>(g, args, pdl, stream);
+    case 2: return launch_q<2, MODE>(g, args, pdl, stream);
+    case 3: return launch_q<3, MODE>(g, args, pdl, stream);
+    default: return launch_q<4, MODE>(g, args, pdl, stream);
   }
 }
 
@@ -459,8 +492,16 @@ cudaError_t launch_any(int q, int g, const RqArgs& args, bool pdl, cudaStream_t 
 cudaError_t launch_requant(const void* W, int64_t d_out, int64_t d, const float* s, int q, int g,
                            uint32_t* codes, void* scale, void* zero, bool pdl, cudaStream_t stream) {
   RqArgs args{static_cast<const __nv_bfloat16*>(W), s, static_cast<int>(d_out), static_cast<int>(d / 32), 0, codes,
-              static_cast<__half*>(scale), static_cast<__half*>(zero), nullptr, nullptr, 0, 0};
-  return launch_any<false>(q, g, args, pdl, stream);
+              static_cast<__half*>(scale), static_cast<__half*>(zero), nullptr, nullptr, 0, 0, 1, 0, 0};
+  return launch_any<kRqSingle>(q, g, args, pdl, stream);
+}
+
+cudaError_t launch_requant_batched(const void* W, int64_t d_out, int64_t d, const float* s, int prompts, int q,
+                                   int g, uint32_t* codes, void* scale, void* zero, cudaStream_t stream) {
+  RqArgs args{static_cast<const __nv_bfloat16*>(W), s, static_cast<int>(d_out), static_cast<int>(d / 32), 0, codes,
+              static_cast<__half*>(scale), static_cast<__half*>(zero), nullptr, nullptr, 0, 0, prompts,
+              d_out * (d / 32) * q, d_out * (d / g)};
+  return launch_any<kRqBatch>(q, g, args, false, stream);
 }
 
 cudaError_t launch_fold_requant(const void* X, int64_t T, void* Xf, const void* W, int64_t d_out, int64_t d,
@@ -468,8 +509,8 @@ cudaError_t launch_fold_requant(const void* X, int64_t T, void* Xf, const void* 
                                 cudaStream_t stream) {
   RqArgs args{static_cast<const __nv_bfloat16*>(W), s, static_cast<int>(d_out), static_cast<int>(d / 32), 0, codes,
               static_cast<__half*>(scale), static_cast<__half*>(zero), static_cast<const __nv_bfloat16*>(X),
-              static_cast<__nv_bfloat16*>(Xf), static_cast<int>(T), 0};
-  return launch_any<true>(q, g, args, true, stream);
+              static_cast<__nv_bfloat16*>(Xf), static_cast<int>(T), 0, 1, 0, 0};
+  return launch_any<kRqFold>(q, g, args, true, stream);
 }
 
 }  // namespace ttq

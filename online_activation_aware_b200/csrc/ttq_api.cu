@@ -188,6 +188,22 @@ ttq_status ttq_requant(const void* W_bf16, int64_t d_out, int64_t d, const float
   return cuda_status(ttq::launch_requant(W_bf16, d_out, d, s, q, g, codes, scale_f16, zero_f16, false, stream));
 }
 
+ttq_status ttq_requant_batched(const void* W_bf16, int64_t d_out, int64_t d, const float* s, int32_t prompts,
+                               int32_t q, int32_t g, uint32_t* codes, void* scale_f16, void* zero_f16,
+                               cudaStream_t stream) {
+  ttq_status st = check_dims(1, d, d_out);
+  if (st != TTQ_OK) return st;
+  st = check_qg(q, g, d);
+  if (st != TTQ_OK) return st;
+  if (prompts < 1 || prompts > ttq::kRequantMaxPrompts) return TTQ_ERR_UNSUPPORTED;
+  if (!W_bf16 || !s || !codes || !scale_f16 || !zero_f16) return TTQ_ERR_INVALID_ARG;
+  if (!aligned16(W_bf16) || !aligned16(s) || !aligned16(codes) || !aligned16(scale_f16) ||
+      !aligned16(zero_f16))
+    return TTQ_ERR_MISALIGNED;
+  return cuda_status(
+      ttq::launch_requant_batched(W_bf16, d_out, d, s, prompts, q, g, codes, scale_f16, zero_f16, stream));
+}
+
 static ttq_status check_lowrank(const ttq_config* cfg, const void* A, const void* B) {
   if (cfg->r > 0) {
     if (!A || !B) return TTQ_ERR_INVALID_ARG;

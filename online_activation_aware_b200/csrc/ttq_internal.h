@@ -83,6 +83,13 @@ cudaError_t launch_decode_gemv(const DecodeArgs& a, void* ws, cudaStream_t strea
 cudaError_t launch_requant(const void* W, int64_t d_out, int64_t d, const float* s, int q, int g,
                            uint32_t* codes, void* scale, void* zero, bool pdl, cudaStream_t stream);
 
+// P prompts (1 <= P <= kRequantMaxPrompts) re-quantized from one read of W: s is [P, d],
+// prompt p's codes / scale / zero start P strides into the outputs (strides of one
+// prompt's output sizes).
+constexpr int kRequantMaxPrompts = 8;
+cudaError_t launch_requant_batched(const void* W, int64_t d_out, int64_t d, const float* s, int prompts, int q,
+                                   int g, uint32_t* codes, void* scale, void* zero, cudaStream_t stream);
+
 // The prefill's fused form: the re-quantization of W and, in the same launch (extra warps
 // per CTA), the fold Xf = bf16(X * (1/s)) of the contiguous [T, d] activations. Launched
 // as the programmatic dependent of the kernel ahead in the stream, which must write

@@ -80,6 +80,15 @@ def test_requant_argument_errors(lib):
     assert lib.ttq_requant(_p(a), 0, 64, _p(a), 4, 32, _p(a), _p(a), _p(a), None) == INVALID
 
 
+def test_requant_batched_argument_errors(lib):
+    a = 1 << 20
+    assert lib.ttq_requant_batched(_p(a), 16, 64, _p(a), 0, 4, 32, _p(a), _p(a), _p(a), None) == UNSUPPORTED
+    assert lib.ttq_requant_batched(_p(a), 16, 64, _p(a), 9, 4, 32, _p(a), _p(a), _p(a), None) == UNSUPPORTED
+    assert lib.ttq_requant_batched(_p(a), 16, 64, _p(a), 2, 5, 32, _p(a), _p(a), _p(a), None) == UNSUPPORTED
+    assert lib.ttq_requant_batched(_p(a), 16, 64, _p(a + 4), 2, 4, 32, _p(a), _p(a), _p(a), None) == MISALIGNED
+    assert lib.ttq_requant_batched(_p(a), 16, 64, None, 2, 4, 32, _p(a), _p(a), _p(a), None) == INVALID
+
+
 def test_act_stats_argument_errors(lib):
     a = 1 << 20
     f = ctypes.c_float

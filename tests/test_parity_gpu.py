@@ -169,6 +169,25 @@ def test_requant_saturated_scale_and_clamped_zero(q):
     requant_check(Wb, synthetic.bf16_values(Wb), s, q, g)
 
 
+@pytest.mark.parametrize("P,d_out,d,q,g", [(1, 130, 512, 4, 128), (3, 64, 96, 3, 32), (8, 257, 1024, 2, 64),
+                                           (5, 200, 768, 4, 32)])
+def test_requant_batched_matches_oracle_per_prompt(P, d_out, d, q, g):
+    # one read of W, P statistics (each prompt's own activations): every prompt's codes,
+    # scales and zeros equal the single-prompt oracle's bit for bit
+    _, Wb, _, W = layer(8, d, d_out, seed=700 + P)
+    S = []
+    for p in range(P):
+        Xp = synthetic.bf16_values(synthetic.as_bf16(synthetic.draw_layer(32, d, 1, seed=7000 + 13 * p)[0]))
+        S.append(O.act_stats(Xp, 0.5 + 0.05 * p, 0.4)[1])
+    S = np.stack(S).astype(np.float32)
+    codes, scale, zero = ttq.requant_batched(gpu(Wb), gpu(torch.from_numpy(S)), q, g)
+    for p in range(P):
+        oc, osc, oz = O.requant(W, S[p], q, g)
+        np.testing.assert_array_equal(packed_np(codes[p], q, d_out, d), O.pack_codes(oc, q))
+        np.testing.assert_array_equal(scale[p].cpu().numpy().view(np.uint16), osc.view(np.uint16))
+        np.testing.assert_array_equal(zero[p].cpu().numpy().view(np.uint16), oz.view(np.uint16))
+
+
 def test_requant_fullsize_qwen3_32b_qproj_sampled_rows():
     # the 5120 -> 8192 projection at its full size; the oracle checks 64 sampled rows
     T, d, d_out, q, g = 4096, 5120, 8192, 4, 128
