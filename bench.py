@@ -15,6 +15,7 @@ Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -471,6 +472,7 @@ def main():
         Xv, Wv = synthetic.bf16_values(Xb), synthetic.bf16_values(Wb)
         result["cpu_baseline"] = cpu_baseline(Xv, Wv, wl, args.cpu_seconds)
         result["decode"] = decode_leg(torch, ttq, wl, cfg, Xs[0], Ws[0], A, B, dev, hbm_peak)
+        result["decode_batched"] = decode_batched_leg(torch, ttq, wl, cfg, Ws[0], outs, dev, hbm_peak)
         result["sweep"] = sweep_leg(torch, ttq, wl, cfg, Wb, A, B, dev, r)
         if r == 0:
             result["lowrank_r16"] = lowrank_leg(torch, ttq, wl, Xs, Ws, dev)
@@ -543,6 +545,55 @@ def requant_batched_leg(torch, ttq, Ws, outs, d, d_out, q, g, P=4, reps=50):
     return {"prompts": P, "us_per_launch": round(tb * 1e6, 2), "us_per_prompt": round(tb * 1e6 / P, 2),
             "GBps": round(by / tb / 1e9, 1), "single_prompt_launches_us": round(ts * 1e6, 2),
             "speedup_vs_single": round(ts / tb, 3)}
+
+
+def decode_batched_leg(torch, ttq, wl, cfg, W, outs, dev, hbm_peak, P=8, b=1):
+    """Decode steps of P requests with their own prefill parameters (statistic and codes
+    from one weight re-quantized per request), b tokens each, in one call
+    (ttq_linear_decode_batched), each step a CUDA graph replay with L2 flushed by a read of
+    256 MB outside the events; compared with one request's step."""
+    lin = wl.layers[0]
+    d, d_out = lin.d, lin.d_out
+    n = len(outs)
+    S = torch.stack([outs[i % n]["s"] * (1.0 + 0.01 * i) for i in range(P)]).contiguous()
+    codes, scale, zero = ttq.requant_batched(W, S, cfg.q, cfg.g)
+    xt = synthetic.as_bf16(synthetic.draw_tokens(P * b, d, seed=77)).reshape(P, b, d).to(dev)
+    Y = torch.empty(P, b, d_out, dtype=torch.bfloat16, device=dev)
+    flush = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    nws = ctypes.c_size_t(0)
+    assert ttq.load_library().ttq_decode_batched_workspace_size(P, b, d, d_out, ctypes.byref(cfg),
+                                                                ctypes.byref(nws)) == 0
+    ws = torch.empty(max(int(nws.value), 256), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        ttq.linear_decode_batched(xt, S, codes, scale, zero, cfg, d_out, Y=Y, ws=ws)
+    torch.cuda.synchronize()
+    g_ = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g_, stream=s):
+            ttq.linear_decode_batched(xt, S, codes, scale, zero, cfg, d_out, Y=Y, ws=ws, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    times = []
+    for i in range(36):
+        torch.sum(flush, dim=0, out=sink)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g_.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 4:
+            times.append(e0.elapsed_time(e1))
+    del g_
+    t = statistics.median(times) / 1e3
+    by = P * decode_bytes(b, d, d_out, cfg.q, cfg.g)
+    assert ttq.device_status() == 0
+    return {"requests": P, "tokens_per_request": b, "us_per_step": round(t * 1e6, 2),
+            "k_tokens_per_s": round(P * b / t / 1e3, 2), "GBps": round(by / t / 1e9, 1),
+            "frac_hbm": round(by / t / 1e9 / hbm_peak, 4)}
 
 
 def decode_leg(torch, ttq, wl, cfg, X, W, A, B, dev, hbm_peak):

@@ -177,6 +177,26 @@ TTQ_API ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, i
                              const ttq_config* cfg, void* Y_bf16, void* ws, size_t ws_bytes,
                              cudaStream_t stream);
 
+/* Decode steps of several requests at once, each with its own prefill's parameters: the
+ * multi-request decode that [DR] section 5 leaves open (every request of a serving batch
+ * carries its own D, hence its own codes). Request p computes
+ * Y_p = (X_p diag(1/s_p)) deq(codes_p)^T + (X_p A^T) B^T with the shared static A, B; its
+ * result equals ttq_linear_decode on request p's operands. With b <= 2 tokens per request
+ * every request runs in the same two launches (statistic fold and CUDA-core GEMV over all
+ * requests' codes); with more tokens the requests run one after another.
+ *   X      device bf16 [P, b, d];  Y  device bf16 [P, b, d_out] output
+ *   s      device fp32 [P, d];  codes  device uint32 [P, ttq_codes_words(d_out, d, q)]
+ *   scale, zero   device fp16 [P, d_out, d/g]
+ *   ws     device scratch of at least ttq_decode_batched_workspace_size(P, b, ...) bytes
+ * P = requests, 1 .. 4096 (TTQ_ERR_UNSUPPORTED otherwise). */
+TTQ_API ttq_status ttq_decode_batched_workspace_size(int32_t requests, int64_t b, int64_t d, int64_t d_out,
+                                                     const ttq_config* cfg, size_t* bytes);
+TTQ_API ttq_status ttq_linear_decode_batched(const void* X_bf16, int32_t requests, int64_t b, int64_t d,
+                                             int64_t d_out, const float* s, const uint32_t* codes,
+                                             const void* scale_f16, const void* zero_f16, const void* A_bf16,
+                                             const void* B_bf16, const ttq_config* cfg, void* Y_bf16, void* ws,
+                                             size_t ws_bytes, cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word: TTQ_OK, or
  * TTQ_ERR_TIMEOUT when a kernel gave up on a bounded wait since the last call, or
  * TTQ_ERR_CUDA when the synchronisation itself failed. */

@@ -7,7 +7,8 @@ in the library's CUDA kernels. There is no CPU fallback: when the library is mis
 or a call fails, a ``TTQError`` is raised.
 
 Functions keep the C names without the ``ttq_`` prefix:
-``act_stats``, ``requant``, ``requant_batched``, ``linear_prefill``, ``linear_decode``, ``workspace_size``,
+``act_stats``, ``requant``, ``requant_batched``, ``linear_prefill``, ``linear_decode``,
+``linear_decode_batched``, ``workspace_size``,
 ``codes_words``, ``device_status``, ``set_wait_limit_ns``. ``TTQLinear`` bundles one
 layer's weight and the per-prompt buffers (prefill, then decode reusing the codes).
 """
@@ -65,6 +66,10 @@ def load_library(path: str = LIB_PATH):
     lib.ttq_linear_prefill.restype = i32
     lib.ttq_linear_decode.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, cfgp, vp, vp, sz, vp]
     lib.ttq_linear_decode.restype = i32
+    lib.ttq_decode_batched_workspace_size.argtypes = [i32, i64, i64, i64, cfgp, ctypes.POINTER(sz)]
+    lib.ttq_decode_batched_workspace_size.restype = i32
+    lib.ttq_linear_decode_batched.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, vp, vp, cfgp, vp, vp, sz, vp]
+    lib.ttq_linear_decode_batched.restype = i32
     lib.ttq_device_status.argtypes = [vp]
     lib.ttq_device_status.restype = i32
     lib.ttq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
@@ -235,6 +240,31 @@ def linear_decode(X, s, codes, scale, zero, cfg: Config, d_out: int, A=None, B=N
         ws = alloc_workspace(b, d, d_out, cfg, dev)
     _check("ttq_linear_decode", load_library().ttq_linear_decode(
         _ptr(X, torch.bfloat16, "X"), b, d, d_out, _ptr(s, torch.float32, "s"),
+        _ptr(codes, torch.int32, "codes"), _ptr(scale, torch.float16, "scale"),
+        _ptr(zero, torch.float16, "zero"), _ptr(A, torch.bfloat16, "A"), _ptr(B, torch.bfloat16, "B"),
+        ctypes.byref(cfg), _ptr(Y, torch.bfloat16, "Y"), _ptr(ws, None, "ws"),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    return Y
+
+
+def linear_decode_batched(X, s, codes, scale, zero, cfg: Config, d_out: int, A=None, B=None, Y=None, ws=None,
+                          stream=None):
+    """Decode steps of P requests at once, each with its own prefill's s, codes, scale
+    and zero: X [P, b, d], s [P, d], codes [P, words], scale / zero [P, d_out, d/g];
+    returns Y [P, b, d_out]."""
+    import torch
+
+    P, b, d = X.shape
+    dev = X.device
+    if Y is None:
+        Y = torch.empty(P, b, d_out, dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        n = ctypes.c_size_t(0)
+        _check("ttq_decode_batched_workspace_size", load_library().ttq_decode_batched_workspace_size(
+            P, b, d, d_out, ctypes.byref(cfg), ctypes.byref(n)))
+        ws = torch.empty(max(int(n.value), 256), dtype=torch.uint8, device=dev)
+    _check("ttq_linear_decode_batched", load_library().ttq_linear_decode_batched(
+        _ptr(X, torch.bfloat16, "X"), P, b, d, d_out, _ptr(s, torch.float32, "s"),
         _ptr(codes, torch.int32, "codes"), _ptr(scale, torch.float16, "scale"),
         _ptr(zero, torch.float16, "zero"), _ptr(A, torch.bfloat16, "A"), _ptr(B, torch.bfloat16, "B"),
         ctypes.byref(cfg), _ptr(Y, torch.bfloat16, "Y"), _ptr(ws, None, "ws"),

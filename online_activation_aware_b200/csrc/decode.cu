@@ -127,8 +127,20 @@ template <int Q, int B>
 __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
     const uint32_t* __restrict__ codes, const __half* __restrict__ scale, const __half* __restrict__ zero,
     const float* xp, const float* usum, int d, int d_out, int log2g, const __nv_bfloat16* __restrict__ U,
-    const __nv_bfloat16* __restrict__ Blr, int r, __nv_bfloat16* __restrict__ Y, int nb) {
+    const __nv_bfloat16* __restrict__ Blr, int r, __nv_bfloat16* __restrict__ Y, int nb, int64_t cstride,
+    int64_t mstride, int64_t wsf) {
   extern __shared__ __align__(16) float2 meta_sm[];  // [kRowsPerCta][gpr]: (sigma, 128 + z)
+  {
+    // request blockIdx.y of a batched decode: its own codes, scale, zero, x', U and Y
+    const int64_t rq = blockIdx.y;
+    codes += rq * cstride;
+    scale += rq * mstride;
+    zero += rq * mstride;
+    xp += rq * wsf;
+    usum += rq * wsf;
+    if (U != nullptr) U += rq * nb * 64;
+    Y += rq * nb * d_out;
+  }
   constexpr int R = kRowsPerWarp;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -247,8 +259,16 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
 template <int B>
 __global__ void __launch_bounds__(256) decode_prep_kernel(const __nv_bfloat16* __restrict__ X, int nb, int d,
                                                           const float* __restrict__ s, float* __restrict__ xp,
-                                                          float* __restrict__ usum) {
+                                                          float* __restrict__ usum, int64_t wsf) {
   grid_dep_launch();  // the GEMV may start loading codes
+  {
+    // request blockIdx.y of a batched decode: its own tokens, statistic and x'
+    const int64_t rq = blockIdx.y;
+    X += rq * nb * d;
+    s += rq * d;
+    xp += rq * wsf;
+    usum += rq * wsf;
+  }
   const int lane = threadIdx.x & 31;
   const int pair = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int units = d >> 5;
@@ -284,8 +304,9 @@ cudaError_t launch_qb(const DecodeArgs& a, uint8_t* ws, cudaStream_t stream) {
   float* xp = reinterpret_cast<float*>(ws);
   float* usum = reinterpret_cast<float*>(ws + round16(static_cast<size_t>(a.d) * B * 4));
   const int units = static_cast<int>(a.d / 32);
-  decode_prep_kernel<B><<<(units * B + 7) / 8, 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(a.X), static_cast<int>(a.b), static_cast<int>(a.d), a.s, xp, usum);
+  const int64_t wsf = static_cast<int64_t>(gemv_ws_bytes(a.b, a.d) / 4);  // one request's workspace, floats
+  decode_prep_kernel<B><<<dim3((units * B + 7) / 8, a.requests), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(a.X), static_cast<int>(a.b), static_cast<int>(a.d), a.s, xp, usum, wsf);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -295,7 +316,7 @@ cudaError_t launch_qb(const DecodeArgs& a, uint8_t* ws, cudaStream_t stream) {
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  cfg.gridDim = dim3(static_cast<unsigned>((a.d_out + kRowsPerCta - 1) / kRowsPerCta));
+  cfg.gridDim = dim3(static_cast<unsigned>((a.d_out + kRowsPerCta - 1) / kRowsPerCta), static_cast<unsigned>(a.requests));
   cfg.blockDim = dim3(kGemvThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -309,7 +330,7 @@ cudaError_t launch_qb(const DecodeArgs& a, uint8_t* ws, cudaStream_t stream) {
                          static_cast<const float*>(xp), static_cast<const float*>(usum), static_cast<int>(a.d),
                          static_cast<int>(a.d_out), lg, static_cast<const __nv_bfloat16*>(a.U),
                          static_cast<const __nv_bfloat16*>(a.Blr), a.r, static_cast<__nv_bfloat16*>(a.Y),
-                         static_cast<int>(a.b));
+                         static_cast<int>(a.b), a.d_out * (a.d / 32) * Q, a.d_out * (a.d / a.g), wsf);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -12,6 +12,7 @@ namespace {
 __device__ unsigned g_ttq_error_word;
 
 constexpr int kMaxDevices = 64;
+constexpr int32_t kMaxDecodeRequests = 4096;  // batched decode: requests per call
 std::atomic<uint64_t> g_wait_ns{2000000000ull};
 cudaEvent_t g_trace[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
 bool g_trace_on = false;
@@ -300,7 +301,8 @@ ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d
     cudaError_t e = cudaSuccess;
     if (cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
     if (e == cudaSuccess) {
-      ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16};
+      ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16,
+                         1};
       e = ttq::launch_decode_gemv(da, base + L.dec_off, stream);
     }
     return cuda_status(e);
@@ -312,6 +314,92 @@ ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d
     ttq::GemmArgs ga{Xf, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g,
                      Y_bf16, gpart};
     e = ttq::launch_gemm(ga, L.plan, dev_err(di), stream);
+  }
+  return cuda_status(e);
+}
+
+// Workspace of a batched decode whose requests run on the CUDA-core GEMV (b <= 2): U for
+// all P * b rows and its K-split partials, then one GEMV slice per request.
+static size_t decode_batched_gemv_bytes(int32_t requests, int64_t b, int64_t d, int r, int num_sms) {
+  const int64_t rows = static_cast<int64_t>(requests) * b;
+  size_t bytes = 0;
+  if (r > 0)
+    bytes += round256(static_cast<size_t>(rows) * 64 * 2) + round256(ttq::lowrank_partial_bytes(rows, d, r, num_sms));
+  bytes += round256(static_cast<size_t>(requests) * ttq::decode_gemv_ws_bytes(b, d));
+  return bytes;
+}
+
+ttq_status ttq_decode_batched_workspace_size(int32_t requests, int64_t b, int64_t d, int64_t d_out,
+                                             const ttq_config* cfg, size_t* bytes) {
+  if (!bytes) return TTQ_ERR_INVALID_ARG;
+  if (requests < 1 || requests > kMaxDecodeRequests) return TTQ_ERR_UNSUPPORTED;
+  ttq_status st = check_dims(b, d, d_out);
+  if (st != TTQ_OK) return st;
+  st = check_cfg(cfg, d);
+  if (st != TTQ_OK) return st;
+  int num_sms = 148;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) == TTQ_OK) num_sms = di->num_sms;
+  if (ttq::decode_gemv_ok(b, d))
+    *bytes = decode_batched_gemv_bytes(requests, b, d, cfg->r, num_sms);
+  else
+    *bytes = ws_layout(b, d, d_out, cfg->r, cfg->q, cfg->g, num_sms).total;  // requests one after another
+  return TTQ_OK;
+}
+
+ttq_status ttq_linear_decode_batched(const void* X_bf16, int32_t requests, int64_t b, int64_t d, int64_t d_out,
+                                     const float* s, const uint32_t* codes, const void* scale_f16,
+                                     const void* zero_f16, const void* A_bf16, const void* B_bf16,
+                                     const ttq_config* cfg, void* Y_bf16, void* ws, size_t ws_bytes,
+                                     cudaStream_t stream) {
+  if (requests < 1 || requests > kMaxDecodeRequests) return TTQ_ERR_UNSUPPORTED;
+  ttq_status st = check_dims(b, d, d_out);
+  if (st != TTQ_OK) return st;
+  st = check_cfg(cfg, d);
+  if (st != TTQ_OK) return st;
+  st = check_lowrank(cfg, A_bf16, B_bf16);
+  if (st != TTQ_OK) return st;
+  if (!X_bf16 || !s || !codes || !scale_f16 || !zero_f16 || !Y_bf16) return TTQ_ERR_INVALID_ARG;
+  if (!ws) return TTQ_ERR_WORKSPACE;
+  if (!aligned16(X_bf16) || !aligned16(s) || !aligned16(codes) || !aligned16(scale_f16) ||
+      !aligned16(zero_f16) || !aligned16(Y_bf16) || !aligned16(ws))
+    return TTQ_ERR_MISALIGNED;
+  DeviceInfo* di = nullptr;
+  st = device_info(&di);
+  if (st != TTQ_OK) return st;
+  const int64_t words = static_cast<int64_t>(ttq_codes_words(d_out, d, cfg->q));
+  const int64_t metas = d_out * (d / cfg->g);
+  if (!ttq::decode_gemv_ok(b, d)) {
+    // more tokens per request: the tensor-core decode of each request in turn (the
+    // per-request strides keep every operand 16-byte aligned when b * d, b * d_out, d,
+    // the code words and d_out * d / g are multiples of 8 elements)
+    if ((b * d) % 8 || (b * d_out) % 8 || words % 4 || metas % 8) return TTQ_ERR_MISALIGNED;
+    for (int32_t p = 0; p < requests; ++p) {
+      st = ttq_linear_decode(static_cast<const __nv_bfloat16*>(X_bf16) + p * b * d, b, d, d_out, s + p * d,
+                             codes + p * words, static_cast<const __half*>(scale_f16) + p * metas,
+                             static_cast<const __half*>(zero_f16) + p * metas, A_bf16, B_bf16, cfg,
+                             static_cast<__nv_bfloat16*>(Y_bf16) + p * b * d_out, ws, ws_bytes, stream);
+      if (st != TTQ_OK) return st;
+    }
+    return TTQ_OK;
+  }
+  if (ws_bytes < decode_batched_gemv_bytes(requests, b, d, cfg->r, di->num_sms)) return TTQ_ERR_WORKSPACE;
+  auto* base = static_cast<uint8_t*>(ws);
+  const int64_t rows = static_cast<int64_t>(requests) * b;
+  void* U = nullptr;
+  cudaError_t e = cudaSuccess;
+  size_t off = 0;
+  if (cfg->r > 0) {
+    // U = X A^T for every request's tokens at once (A is shared): rows p * b .. p * b + b - 1
+    U = base;
+    float* upart = reinterpret_cast<float*>(base + round256(static_cast<size_t>(rows) * 64 * 2));
+    off = round256(static_cast<size_t>(rows) * 64 * 2) + round256(ttq::lowrank_partial_bytes(rows, d, cfg->r, di->num_sms));
+    e = ttq::launch_lowrank_u(X_bf16, rows, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
+  }
+  if (e == cudaSuccess) {
+    ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16,
+                       requests};
+    e = ttq::launch_decode_gemv(da, base + off, stream);
   }
   return cuda_status(e);
 }

@@ -68,10 +68,12 @@ struct DecodeArgs {
   int64_t b, d, d_out;
   int q, g;
   void* Y;                // bf16 [b, d_out]
+  int requests;           // batched decode: requests stacked along every per-request operand
 };
 // True when the CUDA-core GEMV handles these decode sizes (b <= 2).
 bool decode_gemv_ok(int64_t b, int64_t d);
-// Workspace bytes of launch_decode_gemv: x' (fp32, [d][B]) and its 32-input unit sums.
+// Workspace bytes of launch_decode_gemv for one request: x' (fp32, [d][B]) and its
+// 32-input unit sums (a batched decode takes `requests` such slices back to back).
 size_t decode_gemv_ws_bytes(int64_t b, int64_t d);
 // The prep kernel and the GEMV (launched as its programmatic dependent).
 cudaError_t launch_decode_gemv(const DecodeArgs& a, void* ws, cudaStream_t stream);

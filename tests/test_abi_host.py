@@ -141,6 +141,18 @@ def test_decode_argument_errors(lib):
                                  _p(a), None, 1 << 30, None) == WORKSPACE
 
 
+def test_decode_batched_argument_errors(lib):
+    a = 1 << 20
+    c = ttq.make_config(4, 32, 0.5, 0.4)
+    args = (_p(a), _p(a), _p(a), _p(a), None, None, ctypes.byref(c), _p(a), _p(a), 1 << 30, None)
+    assert lib.ttq_linear_decode_batched(_p(a), 0, 1, 128, 64, *args) == UNSUPPORTED
+    assert lib.ttq_linear_decode_batched(_p(a), 4097, 1, 128, 64, *args) == UNSUPPORTED
+    assert lib.ttq_linear_decode_batched(_p(a + 8), 2, 1, 128, 64, *args) == MISALIGNED
+    n = ctypes.c_size_t(0)
+    assert lib.ttq_decode_batched_workspace_size(4, 1, 128, 64, ctypes.byref(c), ctypes.byref(n)) == OK
+    assert n.value >= 4 * 128 * 4  # one x' slice per request
+
+
 def test_binding_refuses_cpu_tensors(lib):
     torch = pytest.importorskip("torch")
     X = torch.zeros(4, 64, dtype=torch.bfloat16)

@@ -370,6 +370,44 @@ def test_decode_parity_shapes(b, d, d_out, q, g, r):
     assert err <= Y_RTOL, err
 
 
+@pytest.mark.parametrize("P,b,d,d_out,q,g,r", [
+    (1, 1, 1024, 384, 4, 128, 0), (3, 1, 512, 300, 3, 32, 0), (8, 2, 1024, 256, 4, 64, 16),
+    (5, 2, 768, 130, 2, 32, 8), (4, 3, 512, 200, 4, 32, 16),   # b = 3: the requests one after another
+])
+def test_decode_batched_requests_match_oracle(P, b, d, d_out, q, g, r):
+    # every request carries its own prefill (own statistic, codes, scale, zero); the shared
+    # static low-rank factors come from the one weight
+    _, Wb, _, W = layer(8, d, d_out, seed=4000 + P * 7 + b)
+    A = B = None
+    Wq = W
+    if r > 0:
+        B, A, Wq = O.lowrank_split(W, r)
+    S, C, SC, Z, Xs, Ys = [], [], [], [], [], []
+    for p in range(P):
+        Xp = synthetic.bf16_values(synthetic.as_bf16(synthetic.draw_layer(64, d, 1, seed=4100 + 31 * p + b)[0]))
+        s32 = O.act_stats(Xp, 0.5, 0.4)[1]
+        oc, osc, oz = O.requant(Wq, s32, q, g)
+        xt = synthetic.bf16_values(synthetic.as_bf16(synthetic.draw_tokens(b, d, seed=4200 + 17 * p + b)))
+        S.append(s32)
+        C.append(O.pack_codes(oc, q).view(np.int32).reshape(-1))
+        SC.append(osc)
+        Z.append(oz)
+        Xs.append(xt)
+        Ys.append(O.linear(xt, s32, oc, osc, oz, g, A, B))
+    cfg = ttq.make_config(q, g, 0.5, 0.4, 2, r)
+    At = gpu(synthetic.as_bf16(A)) if A is not None else None
+    Bt = gpu(synthetic.as_bf16(B)) if B is not None else None
+    Xg = gpu(synthetic.as_bf16(np.stack(Xs)))
+    Yg = ttq.linear_decode_batched(Xg, gpu(torch.from_numpy(np.stack(S))), gpu(torch.from_numpy(np.stack(C))),
+                                   gpu(torch.from_numpy(np.stack(SC))), gpu(torch.from_numpy(np.stack(Z))), cfg,
+                                   d_out, At, Bt)
+    Yg = Yg.float().cpu().numpy()
+    assert np.isfinite(Yg).all()
+    for p in range(P):
+        err = rel_fro(Yg[p], Ys[p])
+        assert err <= Y_RTOL, (p, err)
+
+
 @pytest.mark.parametrize("b,d", [(1, 992), (2, 160), (2, 96), (3, 992), (8, 160), (7, 96)])
 def test_decode_small_hidden_parity(b, d):
     # hidden sizes with fewer 32-input units than lanes in a warp, and ragged unit counts
