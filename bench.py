@@ -483,6 +483,41 @@ def main():
     return 0
 
 
+def graph_step_us(torch, step, flush, sink, n=32):
+    """Device time of one `step` with L2 flushed before it, from two CUDA graphs replayed
+    once each: n x (flush read, step) and n x (flush read); the difference over n is the
+    step (no host launch latency inside either measurement)."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    ga, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(ga, stream=s):
+            for _ in range(n):
+                torch.sum(flush, dim=0, out=sink)
+                step(s)
+        with torch.cuda.graph(gb, stream=s):
+            for _ in range(n):
+                torch.sum(flush, dim=0, out=sink)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+
+    def run(g_):
+        ts = []
+        for _ in range(5):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g_.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    ta, tb = run(ga), run(gb)
+    del ga, gb
+    return (ta - tb) * 1e3 / n
+
+
 def requant_leg(torch, ttq, Ws, outs, d, d_out, q, g, reps=100):
     """GB/s of the re-quantization alone (the ttq_requant entry point: read W and s, write
     codes, scale and zero), back-to-back launches over the rotating weight sets (each set
@@ -550,8 +585,8 @@ def requant_batched_leg(torch, ttq, Ws, outs, d, d_out, q, g, P=4, reps=50):
 def decode_batched_leg(torch, ttq, wl, cfg, W, outs, dev, hbm_peak, P=8, b=1):
     """Decode steps of P requests with their own prefill parameters (statistic and codes
     from one weight re-quantized per request), b tokens each, in one call
-    (ttq_linear_decode_batched), each step a CUDA graph replay with L2 flushed by a read of
-    256 MB outside the events; compared with one request's step."""
+    (ttq_linear_decode_batched), L2 flushed by a read of 256 MB before each step, timed
+    as in decode_leg."""
     lin = wl.layers[0]
     d, d_out = lin.d, lin.d_out
     n = len(outs)
@@ -568,27 +603,8 @@ def decode_batched_leg(torch, ttq, wl, cfg, W, outs, dev, hbm_peak, P=8, b=1):
     for _ in range(3):
         ttq.linear_decode_batched(xt, S, codes, scale, zero, cfg, d_out, Y=Y, ws=ws)
     torch.cuda.synchronize()
-    g_ = torch.cuda.CUDAGraph()
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        with torch.cuda.graph(g_, stream=s):
-            ttq.linear_decode_batched(xt, S, codes, scale, zero, cfg, d_out, Y=Y, ws=ws, stream=s)
-    torch.cuda.current_stream().wait_stream(s)
-    torch.cuda.synchronize()
-    times = []
-    for i in range(36):
-        torch.sum(flush, dim=0, out=sink)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        g_.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        if i >= 4:
-            times.append(e0.elapsed_time(e1))
-    del g_
-    t = statistics.median(times) / 1e3
+    t = graph_step_us(torch, lambda st: ttq.linear_decode_batched(xt, S, codes, scale, zero, cfg, d_out, Y=Y, ws=ws,
+                                                                  stream=st), flush, sink) / 1e6
     by = P * decode_bytes(b, d, d_out, cfg.q, cfg.g)
     assert ttq.device_status() == 0
     return {"requests": P, "tokens_per_request": b, "us_per_step": round(t * 1e6, 2),
@@ -597,9 +613,9 @@ def decode_batched_leg(torch, ttq, wl, cfg, W, outs, dev, hbm_peak, P=8, b=1):
 
 
 def decode_leg(torch, ttq, wl, cfg, X, W, A, B, dev, hbm_peak):
-    """Decode steps reusing one prefill's codes, b tokens per step, each step a CUDA
-    graph replay timed with events; L2 is flushed between steps by a read of 256 MB
-    (outside the events)."""
+    """Decode steps reusing one prefill's codes, b tokens per step, with L2 flushed by a
+    read of 256 MB before each step; timed as the difference of two CUDA graphs (steps
+    with flushes, flushes alone)."""
     lin = wl.layers[0]
     d, d_out = lin.d, lin.d_out
     layer_ = ttq.TTQLinear(W, cfg.q, cfg.g, cfg.alpha, cfg.lambda_, cfg.p, cfg.r, A, B)
@@ -616,28 +632,7 @@ def decode_leg(torch, ttq, wl, cfg, X, W, A, B, dev, hbm_peak):
         for _ in range(3):
             layer_.decode(xt, Y=Y)
         torch.cuda.synchronize()
-        g_ = torch.cuda.CUDAGraph()
-        s = torch.cuda.Stream()
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            with torch.cuda.graph(g_, stream=s):
-                layer_.decode(xt, Y=Y, stream=s)
-        torch.cuda.current_stream().wait_stream(s)
-        torch.cuda.synchronize()
-        times = []
-        n = 64
-        for i in range(n + 4):
-            torch.sum(flush, dim=0, out=sink)
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record()
-            g_.replay()
-            e1.record()
-            torch.cuda.synchronize()
-            if i >= 4:
-                times.append(e0.elapsed_time(e1))
-        del g_
-        t = statistics.median(times) / 1e3
+        t = graph_step_us(torch, lambda st: layer_.decode(xt, Y=Y, stream=st), flush, sink) / 1e6
         by = decode_bytes(b, d, d_out, cfg.q, cfg.g)
         out[f"b{b}"] = {"us_per_step": round(t * 1e6, 2), "k_tokens_per_s": round(b / t / 1e3, 2),
                         "GBps": round(by / t / 1e9, 1), "frac_hbm": round(by / t / 1e9 / hbm_peak, 4)}
