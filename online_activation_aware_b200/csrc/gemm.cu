@@ -188,9 +188,7 @@ __device__ __forceinline__ void dequant_half(const uint32_t (&cw)[4], float sig,
                                               (((p2 >> e) & 1u) << 2)) << 16));
     }
     uint32_t o[4];
-#pragma unroll
-    for (int p = 0; p < 4; ++p)
-      o[p] = pack_bf16x2(__fmaf_rn(f[2 * p], sig, negk), __fmaf_rn(f[2 * p + 1], sig, negk));
+    dequant_pack8(f, sig, negk, o);
     const int c = half * 4 + cc;
     sts128(a_row + ((c ^ (m & 7)) << 4), o[0], o[1], o[2], o[3]);
   }

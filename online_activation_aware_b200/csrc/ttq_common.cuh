@@ -262,6 +262,24 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Eight weights (c - z) * sigma = fma(128 + c, sigma, -(128 + z) sigma) from f[k] = 128 + c_k,
+// two per packed fp32 FMA (each lane rounds like __fmaf_rn; both products are exact, so
+// the result is exact), each pair then rounded once to bf16x2.
+__device__ __forceinline__ void dequant_pack8(const float (&f)[8], float sig, float negk, uint32_t (&o)[4]) {
+  uint64_t s2, k2;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(s2) : "f"(sig));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(k2) : "f"(negk));
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(f[2 * p]), "f"(f[2 * p + 1]));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(v) : "l"(v), "l"(s2), "l"(k2));
+    float a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+    o[p] = pack_bf16x2(a, b);
+  }
+}
+
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) {
   return __uint_as_float(w & 0xFFFF0000u);
