@@ -12,6 +12,9 @@
 // tile overlaps the main loop of the next). Per stage each CTA also TMA-loads the packed
 // codes of its 128 rows and their group scale/zero.
 //
+// Warps per CTA: 0 TMA producer, 1 MMA issuer (even CTA), 2..17 dequantisers in two
+// groups that take alternate K blocks, 18..21 epilogue.
+//
 // Barriers: `full` (X' halves of both CTAs, on the even CTA), `cfull` (own codes tile),
 // `afull` (dequantised A tiles of both CTAs, on the even CTA), `empty` (stage consumed,
 // multicast to both CTAs by the MMA commit), `tfull` / `tempty` (accumulator buffers).
@@ -25,13 +28,12 @@ namespace {
 
 constexpr int kBM = 128;  // rows per CTA (256 per pair)
 constexpr int kBK = 64;
-constexpr int kNumDqWarps = 8;
+constexpr int kNumDqWarps = 16;
+constexpr int kDqGroupWarps = 8;  // dequant warps per stage (two groups take alternate stages)
 constexpr int kNumEpiWarps = 4;
 constexpr int kDqWarp0 = 2;
 constexpr int kEpiWarp0 = kDqWarp0 + kNumDqWarps;
-constexpr int kThreads = 32 * (kEpiWarp0 + kNumEpiWarps);  // 448
-constexpr int kDqThreads = 32 * kNumDqWarps;                // 256 per CTA
-constexpr int kEpiThreads = 32 * kNumEpiWarps;              // 128 per CTA
+constexpr int kThreads = 32 * (kEpiWarp0 + kNumEpiWarps);  // 704
 constexpr uint32_t kATileBytes = kBM * kBK * 2;              // 16 KB
 constexpr uint32_t kCodeTileBytes = kBM * 32;                // [128 rows x 32 B], 32 B swizzle
 constexpr uint32_t kMetaTileBytes = kBM * 16;                // [128 rows x 8 fp16 groups]
@@ -245,7 +247,9 @@ struct Pipe {
 };
 
 template <int Q, int S>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+// 22 warps: a scheduler (SM sub-partition) holds up to 6 of them in its 16 K registers, so
+// at most 80 registers per thread
+__global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
     ttq_gemm2sm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_u,
                        const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
                        const __grid_constant__ CUtensorMap tm_sc, const __grid_constant__ CUtensorMap tm_z,
@@ -286,7 +290,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(bar_full + 8 * s, 2);                 // both CTAs' expect_tx arrivals
       mbar_init(bar_cfull + 8 * s, 1);
-      mbar_init(bar_afull + 8 * s, 2 * kNumDqWarps);  // one arrival per dequant warp of the pair
+      mbar_init(bar_afull + 8 * s, 2 * kDqGroupWarps);  // one arrival per dequant warp of the pair
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -415,7 +419,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp < kEpiWarp0) {
     // ------------------------------------------------------------ dequantisers
-    const int dt = threadIdx.x - 32 * kDqWarp0;  // 0..255
+    // two groups of 8 warps take alternate items (stages), so two A tiles are being
+    // built at once: each group's 256 threads cover the 128 rows x 2 halves of an item
+    const int dtx = threadIdx.x - 32 * kDqWarp0;  // 0..511
+    const int dgroup = dtx >> 8;                   // this thread's group takes items of this parity
+    const int dt = dtx & 255;
     const int m = dt & (kBM - 1);
     const int half = dt >> 7;
     const int d = args.d;
@@ -423,7 +431,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t swz = static_cast<uint32_t>((m >> 2) & 1);  // 32-byte swizzle of row m
     Pipe p;
     ItemIter2 it;
-    for (it.begin(args); it.valid(args); it.next(args), p.advance(S)) {
+    uint32_t item = 0;
+    for (it.begin(args); it.valid(args); it.next(args), p.advance(S), ++item) {
+      if ((item & 1u) != static_cast<uint32_t>(dgroup)) continue;
       const uint32_t s = p.stage;
       // codes landed; the producer issued them only after this stage's previous MMA
       // completed, so the A tile of the stage is free as well
