@@ -36,7 +36,6 @@ constexpr int kDqWarp0 = 2;
 constexpr int kEpiWarp0 = kDqWarp0 + kNumDqWarps;
 constexpr int kThreads = 32 * (kEpiWarp0 + kNumEpiWarps);  // 448
 constexpr int kDqThreads = 32 * kNumDqWarps;                // 256
-constexpr int kEpiThreads = 32 * kNumEpiWarps;              // 128
 constexpr int kSlotBytes = 32;  // per dequant thread per K block: 16 B codes, 4 B scale, 4 B zero
 constexpr uint32_t kATileBytes = kBM * kBK * 2;  // 16 KB
 // TMA-fed codes: per stage a [128 rows x 32 B] codes tile (32-byte swizzle) and two
