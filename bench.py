@@ -505,6 +505,7 @@ def main():
         result["sweep"] = sweep_leg(torch, ttq, wl, cfg, Wb, A, B, dev, r)
         if r == 0:
             result["lowrank_r16"] = lowrank_leg(torch, ttq, wl, Xs, Ws, dev)
+            result["prefill_batched"] = prefill_batched_leg(torch, ttq, wl, cfg, Xs, Ws, dev)
     if rank == 0:
         print(json.dumps(result), flush=True)
     D.barrier()
@@ -694,6 +695,45 @@ def lowrank_leg(torch, ttq, wl, Xs, Ws, dev, r=16, K=30):
     assert ttq.device_status() == 0
     return {"r": r, "T": T, "k_tokens_per_s": round(T / t / 1e3, 2), "us_per_prompt": round(t * 1e6, 1),
             "factors": "seeded random bf16 of the SVD factors' shapes"}
+
+
+def prefill_batched_leg(torch, ttq, wl, cfg, Xs, Ws, dev, P=4, Tp=1024, K=20):
+    """P prompts of Tp tokens, each with its own statistic and codes, through one
+    ttq_linear_prefill_batched call (one read of W re-quantized for all, one grouped
+    projection) against P single-prompt prefills; rotating weight sets."""
+    d = Xs[0].shape[1]
+    d_out = Ws[0].shape[0]
+    Xb = Xs[0][: P * Tp].contiguous()
+    n = len(Ws)
+    T = [Tp] * P
+    nb = ctypes.c_size_t(0)
+    Ta = (ctypes.c_int64 * P)(*T)
+    assert ttq.load_library().ttq_prefill_batched_workspace_size(Ta, P, d, d_out, ctypes.byref(cfg),
+                                                                 ctypes.byref(nb)) == 0
+    wsb = torch.empty(int(nb.value), dtype=torch.uint8, device=dev)
+    wss = ttq.alloc_workspace(Tp, d, d_out, cfg, dev)
+    outs = [ttq.linear_prefill(Xb[:Tp], Ws[0], cfg, ws=wss) for _ in range(P)]
+
+    def timed(fn):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(K):
+            fn(i)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3 / K
+
+    tb = timed(lambda i: ttq.linear_prefill_batched(Xb, T, Ws[i % n], cfg, ws=wsb))
+    ts = timed(lambda i: [ttq.linear_prefill(Xb[p * Tp:(p + 1) * Tp], Ws[i % n], cfg, out=outs[p], ws=wss)
+                          for p in range(P)])
+    assert ttq.device_status() == 0
+    return {"prompts": P, "tokens_per_prompt": Tp, "k_tokens_per_s": round(P * Tp / tb / 1e3, 2),
+            "us_per_call": round(tb * 1e6, 1), "single_prompt_calls_us": round(ts * 1e6, 1),
+            "speedup_vs_single": round(ts / tb, 3)}
 
 
 def sweep_leg(torch, ttq, wl, cfg, Wb, A, B, dev, r):

@@ -177,6 +177,29 @@ TTQ_API ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, i
                              const ttq_config* cfg, void* Y_bf16, void* ws, size_t ws_bytes,
                              cudaStream_t stream);
 
+/* Prefill of P prompts (P = 1 .. 8) through one TTQ linear layer, each prompt with its own
+ * statistic and hence its own quantized weight (the multi-prompt case [DR] section 5
+ * leaves open): per prompt s_p = stats(X_p) and X_p diag(1/s_p); one read of W
+ * re-quantized for every prompt (as ttq_requant_batched); then, when the prompts' tokens
+ * fill 256-token tiles (more than 128 tokens in all, codes rows of 16-byte multiples,
+ * d_out > 128), one grouped tensor-core launch over every prompt's output tiles, else one
+ * projection per prompt. Prompt p's results equal ttq_linear_prefill on its own operands
+ * (same s, codes, scale, zero; Y to the same rounding).
+ *   X      device bf16 [T_0 + ... + T_{P-1}, d], the prompts' tokens one after another
+ *   T      HOST int64 [P] tokens per prompt (each >= 1)
+ *   s      device fp32 [P, d];  codes  device uint32 [P, ttq_codes_words(d_out, d, q)]
+ *   scale, zero   device fp16 [P, d_out, d/g];  Y  device bf16 [sum T, d_out]
+ *   ws     device scratch of at least ttq_prefill_batched_workspace_size(T, P, ...) bytes
+ * d_out must be a multiple of 8 and every prompt's code words and scale/zero elements a
+ * multiple of 16 bytes (TTQ_ERR_MISALIGNED otherwise). */
+TTQ_API ttq_status ttq_prefill_batched_workspace_size(const int64_t* T, int32_t prompts, int64_t d, int64_t d_out,
+                                                      const ttq_config* cfg, size_t* bytes);
+TTQ_API ttq_status ttq_linear_prefill_batched(const void* X_bf16, const int64_t* T, int32_t prompts, int64_t d,
+                                              const void* W_bf16, int64_t d_out, const void* A_bf16,
+                                              const void* B_bf16, const ttq_config* cfg, float* s,
+                                              uint32_t* codes, void* scale_f16, void* zero_f16, void* Y_bf16,
+                                              void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* Decode steps of several requests at once, each with its own prefill's parameters: the
  * multi-request decode that [DR] section 5 leaves open (every request of a serving batch
  * carries its own D, hence its own codes). Request p computes

@@ -7,8 +7,8 @@ in the library's CUDA kernels. There is no CPU fallback: when the library is mis
 or a call fails, a ``TTQError`` is raised.
 
 Functions keep the C names without the ``ttq_`` prefix:
-``act_stats``, ``requant``, ``requant_batched``, ``linear_prefill``, ``linear_decode``,
-``linear_decode_batched``, ``workspace_size``,
+``act_stats``, ``requant``, ``requant_batched``, ``linear_prefill``, ``linear_prefill_batched``,
+``linear_decode``, ``linear_decode_batched``, ``workspace_size``,
 ``codes_words``, ``device_status``, ``set_wait_limit_ns``. ``TTQLinear`` bundles one
 layer's weight and the per-prompt buffers (prefill, then decode reusing the codes).
 """
@@ -66,6 +66,12 @@ def load_library(path: str = LIB_PATH):
     lib.ttq_linear_prefill.restype = i32
     lib.ttq_linear_decode.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, cfgp, vp, vp, sz, vp]
     lib.ttq_linear_decode.restype = i32
+    i64p = ctypes.POINTER(i64)
+    lib.ttq_prefill_batched_workspace_size.argtypes = [i64p, i32, i64, i64, cfgp, ctypes.POINTER(sz)]
+    lib.ttq_prefill_batched_workspace_size.restype = i32
+    lib.ttq_linear_prefill_batched.argtypes = [vp, i64p, i32, i64, vp, i64, vp, vp, cfgp, vp, vp, vp, vp, vp, vp, sz,
+                                               vp]
+    lib.ttq_linear_prefill_batched.restype = i32
     lib.ttq_decode_batched_workspace_size.argtypes = [i32, i64, i64, i64, cfgp, ctypes.POINTER(sz)]
     lib.ttq_decode_batched_workspace_size.restype = i32
     lib.ttq_linear_decode_batched.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, vp, vp, cfgp, vp, vp, sz, vp]
@@ -245,6 +251,37 @@ def linear_decode(X, s, codes, scale, zero, cfg: Config, d_out: int, A=None, B=N
         ctypes.byref(cfg), _ptr(Y, torch.bfloat16, "Y"), _ptr(ws, None, "ws"),
         ws.numel() * ws.element_size(), _stream(stream)))
     return Y
+
+
+def linear_prefill_batched(X, T, W, cfg: Config, A=None, B=None, ws=None, stream=None):
+    """P prompts (token counts T, their tokens stacked in X [sum T, d]) through one layer,
+    each with its own statistic and codes. Returns dict(s [P, d], codes [P, words],
+    scale / zero [P, d_out, d/g], Y [sum T, d_out])."""
+    import torch
+
+    Tl = [int(t) for t in T]
+    P = len(Tl)
+    d = X.shape[1]
+    d_out = W.shape[0]
+    dev = X.device
+    Ta = (ctypes.c_int64 * P)(*Tl)
+    s = torch.empty(P, d, dtype=torch.float32, device=dev)
+    codes = torch.empty(P, codes_words(d_out, d, cfg.q), dtype=torch.int32, device=dev)
+    scale = torch.empty(P, d_out, d // cfg.g, dtype=torch.float16, device=dev)
+    zero = torch.empty(P, d_out, d // cfg.g, dtype=torch.float16, device=dev)
+    Y = torch.empty(sum(Tl), d_out, dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        n = ctypes.c_size_t(0)
+        _check("ttq_prefill_batched_workspace_size", load_library().ttq_prefill_batched_workspace_size(
+            Ta, P, d, d_out, ctypes.byref(cfg), ctypes.byref(n)))
+        ws = torch.empty(max(int(n.value), 256), dtype=torch.uint8, device=dev)
+    _check("ttq_linear_prefill_batched", load_library().ttq_linear_prefill_batched(
+        _ptr(X, torch.bfloat16, "X"), Ta, P, d, _ptr(W, torch.bfloat16, "W"), d_out,
+        _ptr(A, torch.bfloat16, "A"), _ptr(B, torch.bfloat16, "B"), ctypes.byref(cfg),
+        _ptr(s, torch.float32, "s"), _ptr(codes, torch.int32, "codes"), _ptr(scale, torch.float16, "scale"),
+        _ptr(zero, torch.float16, "zero"), _ptr(Y, torch.bfloat16, "Y"), _ptr(ws, None, "ws"),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    return {"s": s, "codes": codes, "scale": scale, "zero": zero, "Y": Y}
 
 
 def linear_decode_batched(X, s, codes, scale, zero, cfg: Config, d_out: int, A=None, B=None, Y=None, ws=None,

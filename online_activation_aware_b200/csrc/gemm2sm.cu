@@ -39,6 +39,7 @@ constexpr uint32_t kCodeTileBytes = kBM * 32;                // [128 rows x 32 B
 constexpr uint32_t kMetaTileBytes = kBM * 16;                // [128 rows x 8 fp16 groups]
 constexpr uint32_t kCStageBytes = kCodeTileBytes + 2 * kMetaTileBytes;
 constexpr int kMaxStages = 8;
+constexpr int kMaxGroups = kGemmMaxGroups;
 constexpr uint64_t kDrainNs = 2000000000ull;
 
 struct __align__(16) Tail {
@@ -191,10 +192,18 @@ struct KernelArgs2 {
   int m_tiles, n_tiles, num_tiles;  // m_tiles counts 256-row pair tiles
   int inject_stall;
   DevErr err;
+  // Prompts stacked along the token axis (grouped form; 1 for a single prompt): prompt p
+  // owns token rows seg_tok[p] .. seg_tok[p + 1] - 1 of X', U and Y, token tiles
+  // seg_tiles[p] .. seg_tiles[p + 1] - 1, and rows p * d_out .. of the codes, scale, zero.
+  int groups;
+  int seg_tiles[kMaxGroups + 1];
+  int seg_tok[kMaxGroups + 1];
 };
 
 struct TileCoord2 {
-  int m0, n0, split, kb0, nk, items;  // m0: first row of the pair tile
+  int m0, n0, split, kb0, nk, items;  // m0: first row of the pair tile (within its prompt)
+  int tend;                           // end of the tile's prompt along the token axis
+  int coff;                           // first row of the prompt's codes / scale / zero
   bool lr;
 };
 
@@ -205,7 +214,11 @@ __device__ __forceinline__ TileCoord2 tile_coord2(const KernelArgs2& a, int t) {
   const int m = rest % a.m_tiles;
   c.split = rest / a.m_tiles;
   c.m0 = m * 2 * kBM;
-  c.n0 = n * a.BN;
+  int p = 0;
+  while (p + 1 < a.groups && n >= a.seg_tiles[p + 1]) ++p;
+  c.n0 = a.seg_tok[p] + (n - a.seg_tiles[p]) * a.BN;
+  c.tend = a.seg_tok[p + 1];
+  c.coff = p * a.d_out;
   c.kb0 = c.split * a.kb_per_split;
   const int kb1 = min(a.nkb, c.kb0 + a.kb_per_split);
   c.nk = kb1 - c.kb0;
@@ -349,10 +362,11 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
           tma_load_2d_pair(sB + s * b_bytes, &tm_x, lead_full + 8 * s, kb * kBK, tok0);
           const uint32_t cst = sC + s * kCStageBytes;
           mbar_arrive_expect_tx(bar_cfull + 8 * s, kCStageBytes);
-          tma_load_2d(cst, &tm_c, bar_cfull + 8 * s, (2 * Q * kb) & ~3, row0);
+          const int crow0 = row0 + it.c.coff;  // the prompt's codes / scale / zero rows
+          tma_load_2d(cst, &tm_c, bar_cfull + 8 * s, (2 * Q * kb) & ~3, crow0);
           const int gx = ((kb * kBK) >> args.log2g) & ~7;
-          tma_load_2d(cst + kCodeTileBytes, &tm_sc, bar_cfull + 8 * s, gx, row0);
-          tma_load_2d(cst + kCodeTileBytes + kMetaTileBytes, &tm_z, bar_cfull + 8 * s, gx, row0);
+          tma_load_2d(cst + kCodeTileBytes, &tm_sc, bar_cfull + 8 * s, gx, crow0);
+          tma_load_2d(cst + kCodeTileBytes + kMetaTileBytes, &tm_z, bar_cfull + 8 * s, gx, crow0);
         }
       }
       if (aborted || *abort_flag) {
@@ -508,7 +522,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int tok = c.n0 + cc0 + j;
-            if (tok < args.T) {
+            if (tok < c.tend) {
               const float v = __uint_as_float(r[j]);
               if (args.ksplit == 1)
                 args.Y[static_cast<int64_t>(tok) * args.d_out + row] = __float2bfloat16_rn(v);
@@ -588,8 +602,9 @@ cudaError_t launch_2sm_s(int q, const CUtensorMap* m, const KernelArgs2& ka, int
 }  // namespace
 
 cudaError_t launch_gemm2sm(const GemmArgs& a, const GemmPlan& plan, const DevErr& err, int inject_stall,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, int groups, const int64_t* group_T) {
   const int BN = plan.BN;
+  if (groups < 1 || groups > kMaxGroups || (groups > 1 && plan.ksplit != 1)) return cudaErrorInvalidValue;
   const int HB = BN / 2;
   CUtensorMap m[6];  // x, u, b, codes, scale, zero
   if (!encode_tmap_2d(&m[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.Xf, a.T, a.d, a.d, 64, HB,
@@ -607,11 +622,12 @@ cudaError_t launch_gemm2sm(const GemmArgs& a, const GemmPlan& plan, const DevErr
   }
   const uint64_t wpr = static_cast<uint64_t>(a.d) * a.q / 32;
   const uint64_t gpr = static_cast<uint64_t>(a.d / a.g);
-  if (!encode_tmap_2d(&m[3], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.codes, a.d_out, wpr, wpr, 8, kBM,
+  const uint64_t crows = static_cast<uint64_t>(groups) * a.d_out;  // the prompts' codes, stacked
+  if (!encode_tmap_2d(&m[3], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.codes, crows, wpr, wpr, 8, kBM,
                       CU_TENSOR_MAP_SWIZZLE_32B) ||
-      !encode_tmap_2d(&m[4], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.scale, a.d_out, gpr, gpr, 8, kBM,
+      !encode_tmap_2d(&m[4], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.scale, crows, gpr, gpr, 8, kBM,
                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_tmap_2d(&m[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.zero, a.d_out, gpr, gpr, 8, kBM,
+      !encode_tmap_2d(&m[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.zero, crows, gpr, gpr, 8, kBM,
                       CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   int dev = 0, sms = 148;
@@ -629,8 +645,17 @@ cudaError_t launch_gemm2sm(const GemmArgs& a, const GemmPlan& plan, const DevErr
   ka.ksplit = plan.ksplit;
   ka.has_lr = a.r > 0 ? 1 : 0;
   ka.m_tiles = plan.m_tiles;
-  ka.n_tiles = plan.n_tiles;
-  ka.num_tiles = plan.m_tiles * plan.n_tiles * plan.ksplit;
+  ka.groups = groups;
+  ka.seg_tiles[0] = 0;
+  ka.seg_tok[0] = 0;
+  for (int p = 0; p < groups; ++p) {
+    const int64_t Tp = groups == 1 ? a.T : group_T[p];
+    ka.seg_tiles[p + 1] = ka.seg_tiles[p] + static_cast<int>((Tp + BN - 1) / BN);
+    ka.seg_tok[p + 1] = ka.seg_tok[p] + static_cast<int>(Tp);
+  }
+  if (ka.seg_tok[groups] != a.T) return cudaErrorInvalidValue;
+  ka.n_tiles = ka.seg_tiles[groups];
+  ka.num_tiles = plan.m_tiles * ka.n_tiles * plan.ksplit;
   ka.inject_stall = inject_stall;
   ka.err = err;
   const int pairs = sms / 2;

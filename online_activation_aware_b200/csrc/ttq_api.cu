@@ -1,6 +1,7 @@
 // C ABI of the TTQ hot path (declared in include/ttq.h): argument validation, workspace
 // layout and the launch sequence of each entry point. Every check happens before any
 // launch, so an argument error leaves the stream untouched.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 
@@ -314,6 +315,140 @@ ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d
     ttq::GemmArgs ga{Xf, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g,
                      Y_bf16, gpart};
     e = ttq::launch_gemm(ga, L.plan, dev_err(di), stream);
+  }
+  return cuda_status(e);
+}
+
+// Workspace of a batched prefill: statistic partials (largest prompt), X' and U (with its
+// K-split partials) for all prompts' tokens, and the split-K partials of the largest
+// per-prompt projection (used when the prompts cannot share one grouped launch).
+struct BatchLayout {
+  size_t stats_off, xf_off, u_off, upart_off, gpart_off, total;
+  int64_t tokens;
+  bool grouped;
+  ttq::GemmPlan plan;  // the grouped plan (tokens of all prompts), when grouped
+};
+
+static BatchLayout batch_layout(const int64_t* T, int32_t prompts, int64_t d, int64_t d_out, const ttq_config* cfg,
+                                int num_sms) {
+  BatchLayout L{};
+  size_t stats = 0, gpart = 0;
+  int64_t tokens = 0;
+  for (int32_t p = 0; p < prompts; ++p) {
+    tokens += T[p];
+    stats = std::max(stats, ttq::split_partial_bytes(T[p], d, num_sms));
+    const ttq::GemmPlan pp = ttq::gemm_plan(T[p], d, d_out, cfg->q, cfg->g, num_sms);
+    gpart = std::max(gpart, ttq::gemm_partial_bytes(pp, T[p], d_out));
+  }
+  L.tokens = tokens;
+  L.plan = ttq::gemm_plan(tokens, d, d_out, cfg->q, cfg->g, num_sms);
+  L.grouped = L.plan.pair && prompts <= ttq::kGemmMaxGroups;
+  if (L.grouped) {  // one launch over every prompt's tiles, no split-K
+    L.plan.kb_per_split = L.plan.nkb;
+    L.plan.ksplit = 1;
+    gpart = 0;
+  }
+  L.stats_off = 0;
+  L.xf_off = round256(stats);
+  L.u_off = L.xf_off + round256(static_cast<size_t>(tokens) * static_cast<size_t>(d) * 2);
+  const size_t ub = cfg->r > 0 ? round256(static_cast<size_t>(tokens) * 64 * 2) : 0;
+  L.upart_off = L.u_off + ub;
+  const size_t upb = cfg->r > 0 ? round256(ttq::lowrank_partial_bytes(tokens, d, cfg->r, num_sms)) : 0;
+  L.gpart_off = L.upart_off + upb;
+  L.total = L.gpart_off + round256(gpart);
+  return L;
+}
+
+static ttq_status check_batch(const int64_t* T, int32_t prompts, int64_t d, int64_t d_out) {
+  if (!T) return TTQ_ERR_INVALID_ARG;
+  if (prompts < 1 || prompts > ttq::kRequantMaxPrompts) return TTQ_ERR_UNSUPPORTED;
+  int64_t tokens = 0;
+  for (int32_t p = 0; p < prompts; ++p) {
+    if (T[p] < 1) return TTQ_ERR_INVALID_ARG;
+    tokens += T[p];
+  }
+  return check_dims(tokens, d, d_out);
+}
+
+ttq_status ttq_prefill_batched_workspace_size(const int64_t* T, int32_t prompts, int64_t d, int64_t d_out,
+                                              const ttq_config* cfg, size_t* bytes) {
+  if (!bytes) return TTQ_ERR_INVALID_ARG;
+  ttq_status st = check_batch(T, prompts, d, d_out);
+  if (st != TTQ_OK) return st;
+  st = check_cfg(cfg, d);
+  if (st != TTQ_OK) return st;
+  int num_sms = 148;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) == TTQ_OK) num_sms = di->num_sms;
+  *bytes = batch_layout(T, prompts, d, d_out, cfg, num_sms).total;
+  return TTQ_OK;
+}
+
+ttq_status ttq_linear_prefill_batched(const void* X_bf16, const int64_t* T, int32_t prompts, int64_t d,
+                                      const void* W_bf16, int64_t d_out, const void* A_bf16, const void* B_bf16,
+                                      const ttq_config* cfg, float* s, uint32_t* codes, void* scale_f16,
+                                      void* zero_f16, void* Y_bf16, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  ttq_status st = check_batch(T, prompts, d, d_out);
+  if (st != TTQ_OK) return st;
+  st = check_cfg(cfg, d);
+  if (st != TTQ_OK) return st;
+  st = check_lowrank(cfg, A_bf16, B_bf16);
+  if (st != TTQ_OK) return st;
+  if (!X_bf16 || !W_bf16 || !s || !codes || !scale_f16 || !zero_f16 || !Y_bf16) return TTQ_ERR_INVALID_ARG;
+  if (!ws) return TTQ_ERR_WORKSPACE;
+  if (!aligned16(X_bf16) || !aligned16(W_bf16) || !aligned16(s) || !aligned16(codes) || !aligned16(scale_f16) ||
+      !aligned16(zero_f16) || !aligned16(Y_bf16) || !aligned16(ws))
+    return TTQ_ERR_MISALIGNED;
+  const int64_t words = static_cast<int64_t>(ttq_codes_words(d_out, d, cfg->q));
+  const int64_t metas = d_out * (d / cfg->g);
+  if (d_out % 8 || words % 4 || metas % 8) return TTQ_ERR_MISALIGNED;  // every prompt's outputs 16-byte aligned
+  DeviceInfo* di = nullptr;
+  st = device_info(&di);
+  if (st != TTQ_OK) return st;
+  const BatchLayout L = batch_layout(T, prompts, d, d_out, cfg, di->num_sms);
+  if (ws_bytes < L.total) return TTQ_ERR_WORKSPACE;
+  auto* base = static_cast<uint8_t*>(ws);
+  float* spart = reinterpret_cast<float*>(base + L.stats_off);
+  auto* Xf = reinterpret_cast<__nv_bfloat16*>(base + L.xf_off);
+  void* U = cfg->r > 0 ? base + L.u_off : nullptr;
+  float* upart = cfg->r > 0 ? reinterpret_cast<float*>(base + L.upart_off) : nullptr;
+  float* gpart = reinterpret_cast<float*>(base + L.gpart_off);
+  const auto* Xb = static_cast<const __nv_bfloat16*>(X_bf16);
+  auto* Yb = static_cast<__nv_bfloat16*>(Y_bf16);
+  auto* sc = static_cast<__half*>(scale_f16);
+  auto* zr = static_cast<__half*>(zero_f16);
+  cudaError_t e = cudaSuccess;
+  // each prompt's statistic and folded activations
+  int64_t off = 0;
+  for (int32_t p = 0; p < prompts && e == cudaSuccess; ++p) {
+    e = ttq::launch_act_stats(Xb + off * d, T[p], d, d, cfg->alpha, cfg->lambda, cfg->p, s + p * d, spart,
+                              di->num_sms, stream);
+    if (e == cudaSuccess) e = ttq::launch_fold(Xb + off * d, T[p], d, d, s + p * d, Xf + off * d, stream);
+    off += T[p];
+  }
+  // the low-rank projection of every prompt's tokens at once (A is shared)
+  if (e == cudaSuccess && cfg->r > 0)
+    e = ttq::launch_lowrank_u(X_bf16, L.tokens, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
+  // one read of W re-quantized for every prompt
+  if (e == cudaSuccess)
+    e = ttq::launch_requant_batched(W_bf16, d_out, d, s, prompts, cfg->q, cfg->g, codes, scale_f16, zero_f16, stream);
+  if (e == cudaSuccess) {
+    if (L.grouped) {
+      // one grouped launch over every prompt's output tiles
+      ttq::GemmArgs ga{Xf, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, L.tokens, d, d_out, cfg->q, cfg->g,
+                       Y_bf16, nullptr};
+      e = ttq::launch_gemm2sm(ga, L.plan, dev_err(di), 0, stream, prompts, T);
+    } else {
+      off = 0;
+      for (int32_t p = 0; p < prompts && e == cudaSuccess; ++p) {
+        const ttq::GemmPlan pp = ttq::gemm_plan(T[p], d, d_out, cfg->q, cfg->g, di->num_sms);
+        ttq::GemmArgs ga{Xf + off * d, codes + p * words, sc + p * metas, zr + p * metas,
+                         U != nullptr ? static_cast<__nv_bfloat16*>(U) + off * 64 : nullptr, B_bf16, cfg->r, T[p], d,
+                         d_out, cfg->q, cfg->g, Yb + off * d_out, gpart};
+        e = ttq::launch_gemm(ga, pp, dev_err(di), stream);
+        off += T[p];
+      }
+    }
   }
   return cuda_status(e);
 }

@@ -148,9 +148,14 @@ void set_inject_stall(bool on);
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, uint32_t elem_bytes, const void* base,
                     uint64_t rows, uint64_t cols, uint64_t row_stride_elems, uint32_t box_cols,
                     uint32_t box_rows, CUtensorMapSwizzle swz);
-// The 2-SM tensor-core kernel (launched by launch_gemm_mainloop when plan.pair).
+// The 2-SM tensor-core kernel (launched by launch_gemm_mainloop when plan.pair). Grouped
+// form (groups > 1, at most kGemmMaxGroups, plan.ksplit == 1): group_T[p] tokens of prompt p
+// stacked along the token axis of Xf, U and Y (a.T their sum), each prompt with its own
+// codes / scale / zero stacked along the rows (p * d_out ..); one launch covers every
+// prompt's tiles.
+constexpr int kGemmMaxGroups = 8;
 cudaError_t launch_gemm2sm(const GemmArgs& a, const GemmPlan& plan, const DevErr& err, int inject_stall,
-                           cudaStream_t stream);
+                           cudaStream_t stream, int groups = 1, const int64_t* group_T = nullptr);
 
 // Encodes a 2-D row-major bf16 tensor map with 128-byte swizzle and a box of
 // {64 columns, box_rows rows}. Returns false when the driver refuses it.

@@ -153,6 +153,22 @@ def test_decode_batched_argument_errors(lib):
     assert n.value >= 4 * 128 * 4  # one x' slice per request
 
 
+def test_prefill_batched_argument_errors(lib):
+    a = 1 << 20
+    c = ttq.make_config(4, 32, 0.5, 0.4)
+    i64p = ctypes.c_int64 * 3
+    T = i64p(16, 32, 8)
+    tail = (_p(a), 64, None, None, ctypes.byref(c), _p(a), _p(a), _p(a), _p(a), _p(a), _p(a), 1 << 30, None)
+    assert lib.ttq_linear_prefill_batched(_p(a), T, 0, 128, *tail) == UNSUPPORTED
+    assert lib.ttq_linear_prefill_batched(_p(a), T, 9, 128, *tail) == UNSUPPORTED
+    assert lib.ttq_linear_prefill_batched(_p(a), None, 2, 128, *tail) == INVALID
+    assert lib.ttq_linear_prefill_batched(_p(a), i64p(16, 0, 8), 3, 128, *tail) == INVALID
+    assert lib.ttq_linear_prefill_batched(_p(a + 8), T, 3, 128, *tail) == MISALIGNED
+    n = ctypes.c_size_t(0)
+    assert lib.ttq_prefill_batched_workspace_size(T, 3, 128, 64, ctypes.byref(c), ctypes.byref(n)) == OK
+    assert n.value >= (16 + 32 + 8) * 128 * 2  # the folded activations of every prompt
+
+
 def test_binding_refuses_cpu_tensors(lib):
     torch = pytest.importorskip("torch")
     X = torch.zeros(4, 64, dtype=torch.bfloat16)

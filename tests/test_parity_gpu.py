@@ -278,6 +278,47 @@ def prefill_check(T, d, d_out, q, g, alpha, r, seed, rows=None):
     return out
 
 
+@pytest.mark.parametrize("Ts,d,d_out,q,g,r", [
+    ((300, 517, 256), 1024, 640, 4, 64, 0),    # grouped launch, ragged last tiles
+    ((1, 700), 768, 384, 3, 32, 16),           # grouped, a one-token prompt, low rank
+    ((16, 40), 512, 256, 2, 32, 0),            # 56 tokens: one projection per prompt
+    ((400, 200), 512, 128, 4, 128, 8),         # d_out = 128: one projection per prompt
+])
+def test_prefill_batched_matches_single_prompts(Ts, d, d_out, q, g, r):
+    # several prompts, each with its own statistic and codes, in one call; prompt p must
+    # match the oracle on its own tokens exactly as a single-prompt prefill does
+    P = len(Ts)
+    Xs, Xvs = [], []
+    for p, Tp in enumerate(Ts):
+        X = synthetic.draw_layer(Tp, d, 1, seed=5000 + 11 * p + Tp)[0]
+        Xs.append(synthetic.as_bf16(X))
+        Xvs.append(synthetic.bf16_values(Xs[-1]))
+    _, Wb, _, W = layer(8, d, d_out, seed=5100 + d)
+    A = B = At = Bt = None
+    Wq, Wqb = W, Wb
+    if r > 0:
+        B, A, Wq = O.lowrank_split(W, r)
+        At, Bt = gpu(synthetic.as_bf16(A)), gpu(synthetic.as_bf16(B))
+        Wqb = synthetic.as_bf16(Wq)
+    cfg = ttq.make_config(q, g, 0.5, 0.4, 2, r)
+    out = ttq.linear_prefill_batched(gpu(torch.cat(Xs)), Ts, gpu(Wqb), cfg, At, Bt)
+    off = 0
+    for p, Tp in enumerate(Ts):
+        s64, s32 = O.act_stats(Xvs[p], 0.5, 0.4)
+        s_gpu = out["s"][p].cpu().numpy().astype(np.float64)
+        assert np.max(np.abs(s_gpu - s64) / s64) <= S_RTOL
+        oc, osc, oz = O.requant(Wq, s32, q, g)
+        gc = O.unpack_codes(packed_np(out["codes"][p], q, d_out, d), q, d)
+        diff = np.abs(gc - oc)
+        assert diff.max() <= 1 and np.mean(diff != 0) <= 1e-3
+        Yo = O.linear(Xvs[p], s32, oc, osc, oz, g, A, B)
+        Yg = out["Y"][off:off + Tp].float().cpu().numpy()
+        assert np.isfinite(Yg).all()
+        err = rel_fro(Yg, Yo)
+        assert err <= Y_RTOL, (p, err)
+        off += Tp
+
+
 def test_prefill_single_512():
     prefill_check(128, 512, 512, 3, 32, 0.5, 0, seed=0)
 
