@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--T", type=int, default=None, help="prompt length (default: the workload's)")
     ap.add_argument("--r", type=int, default=None, help="low-rank r (default: the workload's)")
     ap.add_argument("--no-extras", action="store_true", help="skip the T sweep, decode and e2e legs")
+    ap.add_argument("--no-decoder", action="store_true", help="skip the chained decoder-stack leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline")
     return ap.parse_args()
 
@@ -506,6 +507,8 @@ def main():
         if r == 0:
             result["lowrank_r16"] = lowrank_leg(torch, ttq, wl, Xs, Ws, dev)
             result["prefill_batched"] = prefill_batched_leg(torch, ttq, wl, cfg, Xs, Ws, dev)
+        if not args.no_decoder:
+            result["decoder_stack"] = decoder_leg(torch, ttq, dev)
     if rank == 0:
         print(json.dumps(result), flush=True)
     D.barrier()
@@ -768,6 +771,62 @@ def sweep_leg(torch, ttq, wl, cfg, Wb, A, B, dev, r):
         torch.cuda.empty_cache()
     assert ttq.device_status() == 0
     return res
+
+def decoder_leg(torch, ttq, dev, K=3):
+    """The chained decoder stack (Qwen3-8B shapes: 36 layers, 4 TTQ linears each, random
+    weights): one prompt of T tokens through every layer (each layer re-quantized from its
+    own activations), then 128 decode steps reusing the codes, replayed from one captured
+    CUDA graph. Weights (14 GB) and codes stream from HBM on every pass (> L2)."""
+    from online_activation_aware_b200.decoder import TTQDecoder
+
+    wl = synthetic.WORKLOADS["qwen3_8b_stack"]
+    shape = synthetic.QWEN3_SHAPES["8B"]
+    T, steps = wl.T, wl.decode_steps
+    W = synthetic.device_decoder_weights(shape, wl.r, seed=wl.seed, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed + 1)
+    fn = (1.0 + 0.1 * torch.randn(shape["hidden"], generator=gen, device=dev)).to(torch.bfloat16)
+    x = torch.randn(T + steps, shape["hidden"], generator=gen, device=dev).to(torch.bfloat16)
+    dec = TTQDecoder(shape, W, fn, wl.q, wl.g, wl.alpha, wl.lam, r=wl.r, max_len=T + steps, device=dev)
+    for _ in range(2):
+        dec.prefill(x[:T])
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for _ in range(K):
+        e0.record()
+        dec.prefill(x[:T])
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    dec.capture_decode()
+    for i in range(4):              # warm the replay, then start over from a fresh prefill
+        dec.decode(x[T + i: T + i + 1])
+    dec.prefill(x[:T])
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(steps):
+        out = dec.decode(x[T + i: T + i + 1])
+    e1.record()
+    torch.cuda.synchronize()
+    td = e0.elapsed_time(e1)
+    ok = bool(torch.isfinite(out.float()).all())
+    tp = sorted(ts)[len(ts) // 2]
+    flops = 2.0 * T * sum(lin.d * lin.d_out + (lin.cfg.r * (lin.d + lin.d_out))
+                          for L in dec.layers for lin in L["lin"].values())
+    res = {"model": "Qwen3-8B shapes (architecture table), random-init weights", "layers": shape["layers"],
+           "T": T, "decode_steps": steps, "q": wl.q, "g": wl.g, "r": wl.r,
+           "linears_per_layer": "qkv (stacked), o, gate_up (stacked), down",
+           "prefill_ms": round(tp, 3), "prefill_k_tokens_per_s": round(T / tp, 2),
+           "prefill_linear_TFLOPs": round(flops / (tp / 1e3) / 1e12, 1),
+           "decode_ms_per_step": round(td / steps, 4), "decode_tokens_per_s": round(steps / (td / 1e3), 1),
+           "prompt_plus_decode_ms": round(tp + td, 2), "finite": ok,
+           "attention": "prompt: torch SDPA (library); decode: the library's own kernel",
+           "decode_launch": "one captured CUDA graph per step (device-held position)"}
+    del dec, W, x
+    torch.cuda.empty_cache()
+    return res
+
 
 
 if __name__ == "__main__":

@@ -220,8 +220,92 @@ TTQ_API ttq_status ttq_linear_decode_batched(const void* X_bf16, int32_t request
                                              const void* B_bf16, const ttq_config* cfg, void* Y_bf16, void* ws,
                                              size_t ws_bytes, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------------
+ * Decoder layer around the TTQ linears. The layers whose linears TTQ re-quantizes are
+ * the Qwen3 dense decoders of the architecture table on the thelatestinai.com listing of
+ * the TTQ paper (Table 15: layers, heads, KV heads, hidden size, head dim, MLP dim); the
+ * parts between the linears are the published Qwen3 layer: pre-norm RMSNorm (Zhang &
+ * Sennrich 2019), per-head RMSNorm of q and k, rotary position embedding with the
+ * half-split pairing (Su et al. 2021), grouped-query attention, SwiGLU MLP (Shazeer 2020).
+ * Arithmetic is fp32 with one bf16 rounding per stored value. The library has the
+ * decode step's attention (one token over the cache); a prompt's causal attention is
+ * left to a library kernel.
+ * --------------------------------------------------------------------------------- */
+
+/* RMSNorm over `rows` rows of n channels, with the residual add of a pre-norm layer:
+ *   when residual != NULL:  r <- bf16(r + y)  (the residual row is replaced), h = r
+ *   else:                   h = y
+ *   out = bf16(h * w / sqrt(mean(h^2) + eps))
+ *   y, residual, out   device bf16 [rows, n]; residual may be NULL; it must differ from
+ *                      y and out (TTQ_ERR_INVALID_ARG); out must not overlap y or residual
+ *   w                  device bf16 [n]
+ * n % 8 == 0, 8 <= n <= 8192; eps > 0 (an all-zero row then gives zeros). */
+TTQ_API ttq_status ttq_rmsnorm(const void* y_bf16, void* residual_bf16, const void* w_bf16, int64_t rows,
+                               int64_t n, float eps, void* out_bf16, cudaStream_t stream);
+
+/* Rotary table: table[pos][i] = (cos, sin)(pos * base^(-2i/head_dim)) for pos < positions,
+ * i < head_dim/2, computed in fp64 and stored as fp32 pairs.
+ *   table   device fp32 [positions, head_dim/2, 2] output
+ * head_dim in {64, 128, 256} (TTQ_ERR_UNSUPPORTED otherwise); base > 1. */
+TTQ_API ttq_status ttq_rope_table(int64_t positions, int64_t head_dim, double base, float* table,
+                                  cudaStream_t stream);
+
+/* The attention inputs of T tokens at positions pos0 .. pos0+T-1 from the stacked q|k|v
+ * projection: per head, q and k are RMS-normalised over head_dim (weights q_norm,
+ * k_norm) and rotated (pair (i, i + head_dim/2) by the table's angle for the position);
+ *   q   written back in place into qkv;
+ *   k   written to k_cache[pos0 + t][kv head];  v  copied to v_cache[pos0 + t][kv head].
+ *   qkv        device bf16 [T, (heads + 2 kv_heads) * head_dim]: q heads, k heads, v heads
+ *   q_norm, k_norm   device bf16 [head_dim]
+ *   rope_table device fp32 from ttq_rope_table (table_positions rows)
+ *   k_cache, v_cache device bf16 [cache_len, kv_heads, head_dim]; positions outside
+ *              pos0 .. pos0+T-1 are left untouched
+ *   pos0_dev   NULL, or a device int64 holding pos0 (then the host pos0 is ignored): the
+ *              form a captured CUDA graph replays at a new position every step. The
+ *              kernel checks pos0 + T <= min(cache_len, table_positions) itself; out of
+ *              range it writes nothing and ttq_device_status() reports TTQ_ERR_INVALID_ARG.
+ * With a host pos0, pos0 + T must fit the cache and the table (TTQ_ERR_INVALID_ARG).
+ * head_dim in {64, 128, 256}; eps > 0. */
+TTQ_API ttq_status ttq_qk_norm_rope(void* qkv_bf16, int64_t T, int64_t heads, int64_t kv_heads,
+                                    int64_t head_dim, const void* q_norm_bf16, const void* k_norm_bf16, float eps,
+                                    const float* rope_table, int64_t table_positions, int64_t pos0,
+                                    const int64_t* pos0_dev, void* k_cache_bf16, void* v_cache_bf16,
+                                    int64_t cache_len, cudaStream_t stream);
+
+/* Attention of one new token over the first L cache positions (grouped-query, causal by
+ * construction: the cache holds only earlier positions and the token's own):
+ *   out[h] = sum_p softmax_p(q_h . k_p / sqrt(head_dim)) v_p,  k, v of kv head h / (heads/kv_heads)
+ *   q        device bf16 [heads * head_dim] (the token's q heads, e.g. the first row of the
+ *            stacked projection after ttq_qk_norm_rope)
+ *   k_cache, v_cache  device bf16 [cache_len, kv_heads, head_dim]
+ *   L        = length, or *pos_dev + 1 when pos_dev (device int64, the token's position) is
+ *            given; a device-side L outside 1 .. cache_len gives zeros and
+ *            ttq_device_status() reports TTQ_ERR_INVALID_ARG
+ *   out      device bf16 [heads * head_dim]
+ *   ws       device scratch of ttq_decode_attention_workspace_size() bytes
+ * Split over positions, each split an fp32 online softmax, merged in a fixed order (the
+ * result is reproducible). head_dim in {64, 128}; heads / kv_heads in {1, 2, 4, 8}. */
+TTQ_API ttq_status ttq_decode_attention_workspace_size(int64_t heads, int64_t kv_heads, int64_t head_dim,
+                                                       int64_t cache_len, size_t* bytes);
+TTQ_API ttq_status ttq_decode_attention(const void* q_bf16, int64_t heads, int64_t kv_heads, int64_t head_dim,
+                                        const void* k_cache_bf16, const void* v_cache_bf16, int64_t cache_len,
+                                        int64_t length, const int64_t* pos_dev, void* out_bf16, void* ws,
+                                        size_t ws_bytes, cudaStream_t stream);
+
+/* *pos_dev += n on the device, in stream order (moves a captured decode step to the next
+ * position). */
+TTQ_API ttq_status ttq_position_advance(int64_t* pos_dev, int64_t n, cudaStream_t stream);
+
+/* SwiGLU gate: out[t, c] = bf16(silu(gu[t, c]) * gu[t, inter + c]), silu(u) = u/(1+e^-u).
+ *   gate_up  device bf16 [rows, 2 inter]: the gate half, then the up half (the stacked
+ *            [W_gate; W_up] projection's output);  out  device bf16 [rows, inter]
+ * inter % 8 == 0; out must not overlap gate_up. */
+TTQ_API ttq_status ttq_silu_mul(const void* gate_up_bf16, int64_t rows, int64_t inter, void* out_bf16,
+                                cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word: TTQ_OK, or
- * TTQ_ERR_TIMEOUT when a kernel gave up on a bounded wait since the last call, or
+ * TTQ_ERR_TIMEOUT when a kernel gave up on a bounded wait since the last call,
+ * TTQ_ERR_INVALID_ARG when a position read from device memory was out of range, or
  * TTQ_ERR_CUDA when the synchronisation itself failed. */
 TTQ_API ttq_status ttq_device_status(cudaStream_t stream);
 

@@ -9,8 +9,11 @@ or a call fails, a ``TTQError`` is raised.
 Functions keep the C names without the ``ttq_`` prefix:
 ``act_stats``, ``requant``, ``requant_batched``, ``linear_prefill``, ``linear_prefill_batched``,
 ``linear_decode``, ``linear_decode_batched``, ``workspace_size``,
-``codes_words``, ``device_status``, ``set_wait_limit_ns``. ``TTQLinear`` bundles one
-layer's weight and the per-prompt buffers (prefill, then decode reusing the codes).
+``codes_words``, ``device_status``, ``set_wait_limit_ns``, and the decoder-layer kernels
+``rmsnorm``, ``rope_table``, ``qk_norm_rope``, ``silu_mul``, ``decode_attention``,
+``position_advance``. ``TTQLinear`` bundles one
+layer's weight and the per-prompt buffers (prefill, then decode reusing the codes);
+``online_activation_aware_b200.decoder`` chains them into a decoder stack.
 """
 
 from __future__ import annotations
@@ -76,6 +79,20 @@ def load_library(path: str = LIB_PATH):
     lib.ttq_decode_batched_workspace_size.restype = i32
     lib.ttq_linear_decode_batched.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, vp, vp, cfgp, vp, vp, sz, vp]
     lib.ttq_linear_decode_batched.restype = i32
+    lib.ttq_rmsnorm.argtypes = [vp, vp, vp, i64, i64, f32, vp, vp]
+    lib.ttq_rmsnorm.restype = i32
+    lib.ttq_rope_table.argtypes = [i64, i64, ctypes.c_double, vp, vp]
+    lib.ttq_rope_table.restype = i32
+    lib.ttq_qk_norm_rope.argtypes = [vp, i64, i64, i64, i64, vp, vp, f32, vp, i64, i64, vp, vp, vp, i64, vp]
+    lib.ttq_qk_norm_rope.restype = i32
+    lib.ttq_decode_attention_workspace_size.argtypes = [i64, i64, i64, i64, ctypes.POINTER(sz)]
+    lib.ttq_decode_attention_workspace_size.restype = i32
+    lib.ttq_decode_attention.argtypes = [vp, i64, i64, i64, vp, vp, i64, i64, vp, vp, vp, sz, vp]
+    lib.ttq_decode_attention.restype = i32
+    lib.ttq_position_advance.argtypes = [vp, i64, vp]
+    lib.ttq_position_advance.restype = i32
+    lib.ttq_silu_mul.argtypes = [vp, i64, i64, vp, vp]
+    lib.ttq_silu_mul.restype = i32
     lib.ttq_device_status.argtypes = [vp]
     lib.ttq_device_status.restype = i32
     lib.ttq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
@@ -385,11 +402,107 @@ class TTQLinear:
             self._ws[T] = alloc_workspace(T, self.d, self.d_out, self.cfg, self.W.device)
         return self._ws[T]
 
-    def prefill(self, X, Y=None, stream=None):
+    def prefill(self, X, Y=None, ws=None, stream=None):
+        """Statistic, re-quantization and projection of one prompt X [T, d]; keeps s and the
+        codes for ``decode``. ``ws`` (optional) is a scratch buffer of at least
+        workspace_size(T, d, d_out, cfg) bytes shared with other layers."""
         out = {"s": self.s, "codes": self.codes, "scale": self.scale, "zero": self.zero, "Y": Y}
-        return linear_prefill(X, self.W, self.cfg, self.A, self.B, out=out, ws=self.workspace(X.shape[0]),
-                              stream=stream)["Y"]
+        ws = ws if ws is not None else self.workspace(X.shape[0])
+        return linear_prefill(X, self.W, self.cfg, self.A, self.B, out=out, ws=ws, stream=stream)["Y"]
 
-    def decode(self, X, Y=None, stream=None):
+    def decode(self, X, Y=None, ws=None, stream=None):
+        """Y for new tokens X [b, d] with the last prefill's s and codes."""
+        ws = ws if ws is not None else self.workspace(X.shape[0])
         return linear_decode(X, self.s, self.codes, self.scale, self.zero, self.cfg, self.d_out, self.A,
-                             self.B, Y=Y, ws=self.workspace(X.shape[0]), stream=stream)
+                             self.B, Y=Y, ws=ws, stream=stream)
+
+
+# ------------------------------------------------------------------ decoder-layer kernels
+
+
+def rmsnorm(y, w, eps: float, residual=None, out=None, stream=None):
+    """out = bf16(h w / rms(h)) per row, h = y, or h = r <- bf16(r + y) when ``residual``
+    (updated in place) is given."""
+    import torch
+
+    rows, n = y.shape
+    if out is None:
+        out = torch.empty(rows, n, dtype=torch.bfloat16, device=y.device)
+    _check("ttq_rmsnorm", load_library().ttq_rmsnorm(
+        _ptr(y, torch.bfloat16, "y"), _ptr(residual, torch.bfloat16, "residual"), _ptr(w, torch.bfloat16, "w"),
+        rows, n, ctypes.c_float(eps), _ptr(out, torch.bfloat16, "out"), _stream(stream)))
+    return out
+
+
+def rope_table(positions: int, head_dim: int, base: float, device="cuda", stream=None):
+    """fp32 [positions, head_dim/2, 2] (cos, sin) of pos * base^(-2i/head_dim)."""
+    import torch
+
+    table = torch.empty(positions, head_dim // 2, 2, dtype=torch.float32, device=device)
+    _check("ttq_rope_table", load_library().ttq_rope_table(positions, head_dim, ctypes.c_double(base),
+                                                           _ptr(table, torch.float32, "table"), _stream(stream)))
+    return table
+
+
+def qk_norm_rope(qkv, heads: int, kv_heads: int, head_dim: int, q_norm, k_norm, eps: float, table, pos0: int,
+                 k_cache, v_cache, pos0_dev=None, stream=None):
+    """q heads of the stacked projection normalised and rotated in place; k (normalised,
+    rotated) and v written to the caches at positions pos0 .. pos0 + T - 1 (pos0 read from
+    the device int64 tensor ``pos0_dev`` when given)."""
+    import torch
+
+    T = qkv.shape[0]
+    _check("ttq_qk_norm_rope", load_library().ttq_qk_norm_rope(
+        _ptr(qkv, torch.bfloat16, "qkv"), T, heads, kv_heads, head_dim, _ptr(q_norm, torch.bfloat16, "q_norm"),
+        _ptr(k_norm, torch.bfloat16, "k_norm"), ctypes.c_float(eps), _ptr(table, torch.float32, "table"),
+        table.shape[0], pos0, _ptr(pos0_dev, torch.int64, "pos0_dev"), _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], _stream(stream)))
+    return qkv
+
+
+def decode_attention_workspace_size(heads: int, kv_heads: int, head_dim: int, cache_len: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("ttq_decode_attention_workspace_size", load_library().ttq_decode_attention_workspace_size(
+        heads, kv_heads, head_dim, cache_len, ctypes.byref(n)))
+    return int(n.value)
+
+
+def decode_attention(q, heads: int, kv_heads: int, head_dim: int, k_cache, v_cache, length: int = 0, pos_dev=None,
+                     out=None, ws=None, stream=None):
+    """One token's attention over the first L cache rows (L = length, or pos_dev + 1 read
+    on the device). q [heads * head_dim] bf16 (any tensor whose first heads * head_dim
+    elements are the token's q heads); returns out [heads * head_dim] bf16."""
+    import torch
+
+    L = k_cache.shape[0]
+    if out is None:
+        out = torch.empty(heads * head_dim, dtype=torch.bfloat16, device=q.device)
+    if ws is None:
+        ws = torch.empty(decode_attention_workspace_size(heads, kv_heads, head_dim, L), dtype=torch.uint8,
+                         device=q.device)
+    _check("ttq_decode_attention", load_library().ttq_decode_attention(
+        _ptr(q, torch.bfloat16, "q"), heads, kv_heads, head_dim, _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), L, length, _ptr(pos_dev, torch.int64, "pos_dev"),
+        _ptr(out, torch.bfloat16, "out"), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)))
+    return out
+
+
+def position_advance(pos_dev, n: int = 1, stream=None):
+    """pos_dev += n on the device, in stream order."""
+    import torch
+
+    _check("ttq_position_advance", load_library().ttq_position_advance(_ptr(pos_dev, torch.int64, "pos_dev"), n,
+                                                                       _stream(stream)))
+
+
+def silu_mul(gate_up, out=None, stream=None):
+    """out = bf16(silu(gate) * up) with gate_up = [gate | up] along the channels."""
+    import torch
+
+    rows, two_i = gate_up.shape
+    inter = two_i // 2
+    if out is None:
+        out = torch.empty(rows, inter, dtype=torch.bfloat16, device=gate_up.device)
+    _check("ttq_silu_mul", load_library().ttq_silu_mul(
+        _ptr(gate_up, torch.bfloat16, "gate_up"), rows, inter, _ptr(out, torch.bfloat16, "out"), _stream(stream)))
+    return out

@@ -163,15 +163,36 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
       for (int i = 0; i < R; ++i) cb[k][i] = load_unit<Q>(crow[i] + static_cast<int64_t>(lane + 32 * k) * Q);
     }
   }
-  for (int e = threadIdx.x; e < kRowsPerCta * gpr; e += blockDim.x) {
-    const int rr = e / gpr, gi = e - rr * gpr;
-    const int mrow = blockIdx.x * kRowsPerCta + rr;
-    float2 v = make_float2(0.f, 128.f);
-    if (mrow < d_out) {
-      const int64_t o = static_cast<int64_t>(mrow) * gpr + gi;
-      v = make_float2(__half2float(scale[o]), 128.0f + __half2float(zero[o]));
+  {
+    // the CTA's rows of scale and zero are contiguous: 16-byte loads when aligned and whole
+    // (at g = 32 a row has d / 32 groups, too many for 2-byte loads one after another)
+    const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kRowsPerCta * gpr;
+    const __half* sc = scale + m0;
+    const __half* zc = zero + m0;
+    const bool whole = (blockIdx.x + 1) * kRowsPerCta <= d_out;
+    if (whole && ((reinterpret_cast<uintptr_t>(sc) | reinterpret_cast<uintptr_t>(zc)) & 15u) == 0) {
+      const int n8 = kRowsPerCta * gpr / 8;
+#pragma unroll 4
+      for (int c = threadIdx.x; c < n8; c += blockDim.x) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4*>(sc) + c);
+        const uint4 b = __ldg(reinterpret_cast<const uint4*>(zc) + c);
+        const __half* ah = reinterpret_cast<const __half*>(&a);
+        const __half* bh = reinterpret_cast<const __half*>(&b);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) meta_sm[8 * c + j] = make_float2(__half2float(ah[j]), 128.0f + __half2float(bh[j]));
+      }
+    } else {
+      for (int e = threadIdx.x; e < kRowsPerCta * gpr; e += blockDim.x) {
+        const int rr = e / gpr, gi = e - rr * gpr;
+        const int mrow = blockIdx.x * kRowsPerCta + rr;
+        float2 v = make_float2(0.f, 128.f);
+        if (mrow < d_out) {
+          const int64_t o = static_cast<int64_t>(mrow) * gpr + gi;
+          v = make_float2(__half2float(scale[o]), 128.0f + __half2float(zero[o]));
+        }
+        meta_sm[e] = v;
+      }
     }
-    meta_sm[e] = v;
   }
   grid_dep_wait();  // x' and its unit sums are written by the prep kernel
   __syncthreads();  // meta is in place

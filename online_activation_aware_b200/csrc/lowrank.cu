@@ -9,7 +9,8 @@
 // XOR-swizzled rows so that ldmatrix is conflict-free), and each of its 4 warps multiplies
 // 16 tokens by A^T with mma.sync m16n8k16 (bf16 in, fp32 accumulate). The K splits write
 // fp32 partial sums; a small dependent kernel adds them in split order (deterministic)
-// and stores U in bf16 with its row padded to 64 (columns r..63 zero).
+// and stores U in bf16 with its row padded to 64 (columns r..63 zero). For a few tokens (a
+// decode step) one block computes each output over all of d instead.
 #include "ttq_internal.h"
 
 namespace ttq {
@@ -20,6 +21,7 @@ constexpr int kLrTok = 64;      // tokens per block (4 warps x 16)
 constexpr int kLrK = 64;        // K per stage
 constexpr int kLrStages = 3;
 constexpr int kLrThreads = 128;
+constexpr int kLrSmallTokens = 8;  // up to here one block per output (no partial sums in memory)
 
 __device__ __forceinline__ void cp_async_16_zfill(uint32_t dst, const void* src, bool valid) {
   const int n = valid ? 16 : 0;
@@ -152,6 +154,44 @@ __global__ void __launch_bounds__(256) lowrank_reduce_kernel(const float* __rest
   U[e] = __float2bfloat16_rn(v);
 }
 
+// Few tokens (a decode step): one block per (token t, column j) of U, its 256 threads
+// striding over d in 8-channel chunks, fp32 sums reduced in a fixed order (warps, then
+// the 8 warp sums); U[t][j] = bf16(sum_k X[t][k] A[j][k]) for j < r and 0 for r <= j < 64.
+__global__ void __launch_bounds__(256) lowrank_small_kernel(const __nv_bfloat16* __restrict__ X, int d,
+                                                            const __nv_bfloat16* __restrict__ A, int r,
+                                                            __nv_bfloat16* __restrict__ U) {
+  __shared__ float red[8];
+  const int t = blockIdx.x >> 6, j = blockIdx.x & 63;
+  if (j >= r) {
+    if (threadIdx.x == 0) U[blockIdx.x] = __float2bfloat16_rn(0.f);
+    return;
+  }
+  const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(t) * d);
+  const uint4* ar = reinterpret_cast<const uint4*>(A + static_cast<int64_t>(j) * d);
+  const int chunks = d >> 3;
+  float acc = 0.f;
+#pragma unroll 4
+  for (int c = threadIdx.x; c < chunks; c += 256) {
+    const uint4 xv = __ldg(xr + c), av = __ldg(ar + c);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc = __fmaf_rn(__uint_as_float(xw[q] << 16), __uint_as_float(aw[q] << 16), acc);
+      acc = __fmaf_rn(__uint_as_float(xw[q] & 0xFFFF0000u), __uint_as_float(aw[q] & 0xFFFF0000u), acc);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += red[w];
+    U[blockIdx.x] = __float2bfloat16_rn(v);
+  }
+}
+
 }  // namespace
 
 int lowrank_splits(int64_t T, int64_t d, int num_sms) {
@@ -171,6 +211,12 @@ size_t lowrank_partial_bytes(int64_t T, int64_t d, int r, int num_sms) {
 
 cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A, int r, void* U, float* partial,
                              int num_sms, cudaStream_t stream) {
+  if (T <= kLrSmallTokens) {
+    lowrank_small_kernel<<<static_cast<unsigned>(T * 64), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(X), static_cast<int>(d), static_cast<const __nv_bfloat16*>(A), r,
+        static_cast<__nv_bfloat16*>(U));
+    return cudaGetLastError();
+  }
   const int ks = lowrank_splits(T, d, num_sms);
   const int64_t kst = (d + kLrK - 1) / kLrK;
   const int kc = static_cast<int>((kst + ks - 1) / ks) * kLrK;

@@ -539,6 +539,116 @@ ttq_status ttq_linear_decode_batched(const void* X_bf16, int32_t requests, int64
   return cuda_status(e);
 }
 
+// ---------------------------------------------------------------- decoder layer
+
+ttq_status ttq_rmsnorm(const void* y_bf16, void* residual_bf16, const void* w_bf16, int64_t rows, int64_t n,
+                       float eps, void* out_bf16, cudaStream_t stream) {
+  if (!y_bf16 || !w_bf16 || !out_bf16) return TTQ_ERR_INVALID_ARG;
+  if (rows < 1 || rows > (int64_t(1) << 31) - 1 || n < 8 || n > 8192 || n % 8 != 0) return TTQ_ERR_INVALID_ARG;
+  if (!std::isfinite(eps) || !(eps > 0.f)) return TTQ_ERR_INVALID_ARG;
+  if (residual_bf16 && (residual_bf16 == y_bf16 || residual_bf16 == out_bf16)) return TTQ_ERR_INVALID_ARG;
+  if (!aligned16(y_bf16) || !aligned16(w_bf16) || !aligned16(out_bf16) ||
+      (residual_bf16 && !aligned16(residual_bf16)))
+    return TTQ_ERR_MISALIGNED;
+  return cuda_status(ttq::launch_rmsnorm(y_bf16, residual_bf16, w_bf16, rows, static_cast<int>(n), eps, out_bf16,
+                                         stream));
+}
+
+ttq_status ttq_rope_table(int64_t positions, int64_t head_dim, double base, float* table, cudaStream_t stream) {
+  if (!table) return TTQ_ERR_INVALID_ARG;
+  if (positions < 1 || positions > (int64_t(1) << 24)) return TTQ_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return TTQ_ERR_UNSUPPORTED;
+  if (!std::isfinite(base) || !(base > 1.0)) return TTQ_ERR_INVALID_ARG;
+  if (!aligned16(table)) return TTQ_ERR_MISALIGNED;
+  return cuda_status(ttq::launch_rope_table(positions, static_cast<int>(head_dim), base, table, stream));
+}
+
+ttq_status ttq_qk_norm_rope(void* qkv_bf16, int64_t T, int64_t heads, int64_t kv_heads, int64_t head_dim,
+                            const void* q_norm_bf16, const void* k_norm_bf16, float eps, const float* rope_table,
+                            int64_t table_positions, int64_t pos0, const int64_t* pos0_dev, void* k_cache_bf16,
+                            void* v_cache_bf16, int64_t cache_len, cudaStream_t stream) {
+  if (!qkv_bf16 || !q_norm_bf16 || !k_norm_bf16 || !rope_table || !k_cache_bf16 || !v_cache_bf16)
+    return TTQ_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return TTQ_ERR_UNSUPPORTED;
+  if (T < 1 || heads < 1 || kv_heads < 1 || heads > 1024 || kv_heads > 1024) return TTQ_ERR_INVALID_ARG;
+  if (T > (int64_t(1) << 24) || cache_len < T || table_positions < T) return TTQ_ERR_INVALID_ARG;
+  if (!pos0_dev && (pos0 < 0 || pos0 + T > cache_len || pos0 + T > table_positions)) return TTQ_ERR_INVALID_ARG;
+  if (!std::isfinite(eps) || !(eps > 0.f)) return TTQ_ERR_INVALID_ARG;
+  if (k_cache_bf16 == v_cache_bf16) return TTQ_ERR_INVALID_ARG;
+  if (!aligned16(qkv_bf16) || !aligned16(q_norm_bf16) || !aligned16(k_norm_bf16) || !aligned16(rope_table) ||
+      !aligned16(k_cache_bf16) || !aligned16(v_cache_bf16) || (pos0_dev && (reinterpret_cast<uintptr_t>(pos0_dev) & 7)))
+    return TTQ_ERR_MISALIGNED;
+  DeviceInfo* di = nullptr;
+  ttq_status st = device_info(&di);
+  if (st != TTQ_OK) return st;
+  return cuda_status(ttq::launch_qk_norm_rope(qkv_bf16, T, static_cast<int>(heads), static_cast<int>(kv_heads),
+                                              static_cast<int>(head_dim), q_norm_bf16, k_norm_bf16, eps, rope_table,
+                                              pos0, pos0_dev, std::min(cache_len, table_positions), k_cache_bf16,
+                                              v_cache_bf16, di->err_word, stream));
+}
+
+namespace {
+ttq_status check_decode_attention(int64_t heads, int64_t kv_heads, int64_t head_dim, int64_t cache_len) {
+  if (head_dim != 64 && head_dim != 128) return TTQ_ERR_UNSUPPORTED;
+  if (heads < 1 || kv_heads < 1 || heads > 1024 || heads % kv_heads != 0) return TTQ_ERR_INVALID_ARG;
+  const int64_t G = heads / kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return TTQ_ERR_UNSUPPORTED;
+  if (cache_len < 1 || cache_len > (int64_t(1) << 30)) return TTQ_ERR_INVALID_ARG;
+  return TTQ_OK;
+}
+}  // namespace
+
+ttq_status ttq_decode_attention_workspace_size(int64_t heads, int64_t kv_heads, int64_t head_dim, int64_t cache_len,
+                                               size_t* bytes) {
+  if (!bytes) return TTQ_ERR_INVALID_ARG;
+  ttq_status st = check_decode_attention(heads, kv_heads, head_dim, cache_len);
+  if (st != TTQ_OK) return st;
+  const int splits = ttq::decode_attn_splits(cache_len, static_cast<int>(kv_heads));
+  *bytes = round256(ttq::decode_attn_partial_bytes(static_cast<int>(heads), static_cast<int>(head_dim), splits));
+  return TTQ_OK;
+}
+
+ttq_status ttq_decode_attention(const void* q_bf16, int64_t heads, int64_t kv_heads, int64_t head_dim,
+                                const void* k_cache_bf16, const void* v_cache_bf16, int64_t cache_len, int64_t length,
+                                const int64_t* pos_dev, void* out_bf16, void* ws, size_t ws_bytes,
+                                cudaStream_t stream) {
+  if (!q_bf16 || !k_cache_bf16 || !v_cache_bf16 || !out_bf16) return TTQ_ERR_INVALID_ARG;
+  ttq_status st = check_decode_attention(heads, kv_heads, head_dim, cache_len);
+  if (st != TTQ_OK) return st;
+  if (!pos_dev && (length < 1 || length > cache_len)) return TTQ_ERR_INVALID_ARG;
+  if (!ws) return TTQ_ERR_WORKSPACE;
+  const int splits = ttq::decode_attn_splits(cache_len, static_cast<int>(kv_heads));
+  if (ws_bytes < ttq::decode_attn_partial_bytes(static_cast<int>(heads), static_cast<int>(head_dim), splits))
+    return TTQ_ERR_WORKSPACE;
+  if (!aligned16(q_bf16) || !aligned16(k_cache_bf16) || !aligned16(v_cache_bf16) || !aligned16(out_bf16) ||
+      !aligned16(ws) || (pos_dev && (reinterpret_cast<uintptr_t>(pos_dev) & 7)))
+    return TTQ_ERR_MISALIGNED;
+  DeviceInfo* di = nullptr;
+  st = device_info(&di);
+  if (st != TTQ_OK) return st;
+  return cuda_status(ttq::launch_decode_attention(q_bf16, static_cast<int>(heads), static_cast<int>(kv_heads),
+                                                  static_cast<int>(head_dim), k_cache_bf16, v_cache_bf16, cache_len,
+                                                  length, pos_dev, out_bf16, static_cast<float*>(ws), splits,
+                                                  di->err_word, stream));
+}
+
+ttq_status ttq_position_advance(int64_t* pos_dev, int64_t n, cudaStream_t stream) {
+  if (!pos_dev || n < 0) return TTQ_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(pos_dev) & 7) return TTQ_ERR_MISALIGNED;
+  return cuda_status(ttq::launch_position_advance(pos_dev, n, stream));
+}
+
+ttq_status ttq_silu_mul(const void* gate_up_bf16, int64_t rows, int64_t inter, void* out_bf16, cudaStream_t stream) {
+  if (!gate_up_bf16 || !out_bf16) return TTQ_ERR_INVALID_ARG;
+  if (rows < 1 || inter < 8 || inter % 8 != 0 || rows * inter > (int64_t(1) << 40)) return TTQ_ERR_INVALID_ARG;
+  if (gate_up_bf16 == out_bf16) return TTQ_ERR_INVALID_ARG;
+  if (!aligned16(gate_up_bf16) || !aligned16(out_bf16)) return TTQ_ERR_MISALIGNED;
+  DeviceInfo* di = nullptr;
+  ttq_status st = device_info(&di);
+  if (st != TTQ_OK) return st;
+  return cuda_status(ttq::launch_silu_mul(gate_up_bf16, rows, inter, out_bf16, di->num_sms, stream));
+}
+
 ttq_status ttq_device_status(cudaStream_t stream) {
   DeviceInfo* di = nullptr;
   ttq_status st = device_info(&di);
@@ -549,7 +659,7 @@ ttq_status ttq_device_status(cudaStream_t stream) {
   if (word != 0) {
     const unsigned zero = 0;
     if (cudaMemcpyToSymbol(g_ttq_error_word, &zero, sizeof(zero)) != cudaSuccess) return TTQ_ERR_CUDA;
-    return TTQ_ERR_TIMEOUT;
+    return (word & ttq::kErrTimeout) ? TTQ_ERR_TIMEOUT : TTQ_ERR_INVALID_ARG;
   }
   return TTQ_OK;
 }

@@ -162,4 +162,35 @@ cudaError_t launch_gemm2sm(const GemmArgs& a, const GemmPlan& plan, const DevErr
 bool encode_bf16_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                       uint64_t row_stride_elems, uint32_t box_rows);
 
+// ---------------------------------------------------------------- decoder layer (decoder.cu)
+
+// r <- bf16(r + y) per row when `residual` is non-null, then out = bf16(h w / rms(h))
+// over rows of n channels (n % 8 == 0, n <= 8192).
+cudaError_t launch_rmsnorm(const void* y, void* residual, const void* w, int64_t rows, int n, float eps, void* out,
+                           cudaStream_t stream);
+// fp32 (cos, sin) pairs of pos * base^(-2i/D) for pos < positions, i < D/2.
+cudaError_t launch_rope_table(int64_t positions, int head_dim, double base, float* table, cudaStream_t stream);
+// Device error word bit: a position read from device memory was outside the cache.
+constexpr unsigned kErrRange = 2u;
+
+// Per-head RMSNorm + rotary embedding of q (in place) and k (into k_cache), v copied into
+// v_cache, for T tokens of the stacked projection at positions pos0 ... (pos0 = *pos_dev
+// when pos_dev is given, checked against `limit` on the device); head_dim in {64, 128, 256}.
+cudaError_t launch_qk_norm_rope(void* qkv, int64_t T, int heads, int kv_heads, int head_dim, const void* wq,
+                                const void* wk, float eps, const float* table, int64_t pos0, const int64_t* pos_dev,
+                                int64_t limit, void* k_cache, void* v_cache, unsigned* err, cudaStream_t stream);
+// One token's attention over the first L cache positions (L = *pos_dev + 1 when pos_dev is
+// given, else `length`): split over positions into `part` (decode_attn_partial_bytes), then
+// merged per query head into out [heads * head_dim] bf16. head_dim in {64, 128};
+// heads / kv_heads in {1, 2, 4, 8}.
+int decode_attn_splits(int64_t cache_len, int kv_heads);
+size_t decode_attn_partial_bytes(int heads, int head_dim, int splits);
+cudaError_t launch_decode_attention(const void* q, int heads, int kv_heads, int head_dim, const void* k_cache,
+                                    const void* v_cache, int64_t cache_len, int64_t length, const int64_t* pos_dev,
+                                    void* out, float* part, int splits, unsigned* err, cudaStream_t stream);
+// *pos += n on the device (one thread).
+cudaError_t launch_position_advance(int64_t* pos, int64_t n, cudaStream_t stream);
+// out = bf16(silu(gate) * up) over rows of [gate | up] (inter channels each, inter % 8 == 0).
+cudaError_t launch_silu_mul(const void* gu, int64_t rows, int64_t inter, void* out, int num_sms, cudaStream_t stream);
+
 }  // namespace ttq

@@ -123,3 +123,95 @@ WORKLOADS = {
                                alpha=0.5, lam=0.4, r=16, seed=4, decode_batches=(1,),
                                decode_steps=128, extra={"layers": 36}),
 }
+
+
+# ------------------------------------------------------------------ decoder stacks
+
+# Qwen3 dense models (Table 15 of the thelatestinai.com listing): layers, heads, KV heads,
+# hidden size, head dim, MLP dim.
+QWEN3_SHAPES = {
+    "0.6B": dict(layers=28, heads=16, kv_heads=8, hidden=1024, head_dim=128, inter=3072),
+    "1.7B": dict(layers=28, heads=16, kv_heads=8, hidden=2048, head_dim=128, inter=6144),
+    "4B": dict(layers=36, heads=32, kv_heads=8, hidden=2560, head_dim=128, inter=9728),
+    "8B": dict(layers=36, heads=32, kv_heads=8, hidden=4096, head_dim=128, inter=12288),
+    "14B": dict(layers=40, heads=40, kv_heads=8, hidden=5120, head_dim=128, inter=17408),
+    "32B": dict(layers=64, heads=64, kv_heads=8, hidden=5120, head_dim=128, inter=25600),
+}
+
+# the four TTQ linears of a decoder layer (q|k|v and gate|up each stacked into one)
+DECODER_LINEARS = ("qkv", "o", "gate_up", "down")
+
+
+def decoder_linear_parts(shape: dict, name: str):
+    """Output rows of the parts stacked in one decoder linear, and its input width."""
+    H, Hkv, D, h, I = shape["heads"], shape["kv_heads"], shape["head_dim"], shape["hidden"], shape["inter"]
+    return {"qkv": ([H * D, Hkv * D, Hkv * D], h), "o": ([h], H * D), "gate_up": ([I, I], h),
+            "down": ([h], I)}[name]
+
+
+def draw_decoder_weights(shape: dict, r: int, seed: int, layers: int | None = None):
+    """Random-init weights of a decoder stack, float64 numpy (not yet rounded), one dict
+    per layer: w_<lin> [rows, in] ~ N(0, 1/in) with the parts of a stacked linear one
+    after another; norm weights 1 + N(0, 0.1^2); with r > 0 the static low-rank factors of
+    every part, a ~ N(0, 0.02^2) [r, in] and b ~ N(0, 0.02^2) [rows, r], stacked as
+    a_<lin> [parts r, in] and the block-diagonal b_<lin> [rows, parts r] (zeros off the
+    blocks), and w_<lin> standing for the residual R."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(layers if layers is not None else shape["layers"]):
+        L = {}
+        for name in DECODER_LINEARS:
+            parts, d_in = decoder_linear_parts(shape, name)
+            L["w_" + name] = rng.normal(0.0, d_in ** -0.5, (sum(parts), d_in))
+            if r > 0:
+                L["a_" + name] = rng.normal(0.0, 0.02, (len(parts) * r, d_in))
+                b = np.zeros((sum(parts), len(parts) * r))
+                row = 0
+                for i, n in enumerate(parts):
+                    b[row: row + n, i * r: (i + 1) * r] = rng.normal(0.0, 0.02, (n, r))
+                    row += n
+                L["b_" + name] = b
+        for name, n in (("n_in", shape["hidden"]), ("n_post", shape["hidden"]), ("n_q", shape["head_dim"]),
+                        ("n_k", shape["head_dim"])):
+            L[name] = 1.0 + 0.1 * rng.normal(size=n)
+        out.append(L)
+    return out
+
+
+def draw_hidden(T: int, hidden: int, seed: int):
+    """Token embeddings entering the stack [T, hidden] ~ N(0, 1) (float64)."""
+    return np.random.default_rng(seed).normal(size=(T, hidden))
+
+
+def device_decoder_weights(shape: dict, r: int, seed: int, device="cuda", layers: int | None = None):
+    """The same recipe drawn on the device (torch's seeded CUDA generator; different numbers
+    from the numpy draw), bf16 tensors: for stacks too large to draw on the host."""
+    import torch
+
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+
+    def normal(rows, cols, std):
+        t = torch.empty(rows, cols, dtype=torch.bfloat16, device=device)
+        t.normal_(0.0, std, generator=gen)
+        return t
+
+    out = []
+    for _ in range(layers if layers is not None else shape["layers"]):
+        L = {}
+        for name in DECODER_LINEARS:
+            parts, d_in = decoder_linear_parts(shape, name)
+            L["w_" + name] = normal(sum(parts), d_in, d_in ** -0.5)
+            if r > 0:
+                L["a_" + name] = normal(len(parts) * r, d_in, 0.02)
+                b = torch.zeros(sum(parts), len(parts) * r, dtype=torch.bfloat16, device=device)
+                row = 0
+                for i, n in enumerate(parts):
+                    b[row: row + n, i * r: (i + 1) * r] = normal(n, r, 0.02)
+                    row += n
+                L["b_" + name] = b
+        for name, n in (("n_in", shape["hidden"]), ("n_post", shape["hidden"]), ("n_q", shape["head_dim"]),
+                        ("n_k", shape["head_dim"])):
+            L[name] = (1.0 + 0.1 * normal(1, n, 1.0).float()).to(torch.bfloat16).reshape(n)
+        out.append(L)
+    return out

@@ -35,6 +35,9 @@ Readings (decisions where the pages are silent; listed with reasons in the desig
   D4  q, k and v share one statistic (they read the same h), so they are one TTQ linear
       over the stacked weight [Wq; Wk; Wv]; gate and up likewise. This is exact: the
       statistic depends only on the layer input and the re-quantization is per output row.
+      With static low-rank factors, the stacked linear takes A = [A_q; A_k; A_v] and the
+      block-diagonal B = diag(B_q, B_k, B_v), whose term (X A^T) B^T gives every part its
+      own rank-r term.
 """
 
 from __future__ import annotations
@@ -131,15 +134,17 @@ class LayerState:
         self.V = None
 
 
-def ttq_linear(name, X, W, st: LayerState, q: int, g: int, alpha: float, lam: float, prefill: bool):
-    """A TTQ linear: at prefill, statistic + requant of W from this X; at decode, the
-    stored statistic and codes (the prefill's)."""
+def ttq_linear(name, X, Wl, st: LayerState, q: int, g: int, alpha: float, lam: float, prefill: bool):
+    """A TTQ linear: at prefill, statistic + requant of W (the residual R when the static
+    low-rank factors a_<name>, b_<name> are present) from this X; at decode, the stored
+    statistic and codes (the prefill's)."""
+    A, B = Wl.get("a_" + name), Wl.get("b_" + name)
     if prefill:
-        res = O.prefill(X, W, q, g, alpha, lam)
+        res = O.prefill(X, Wl["w_" + name], q, g, alpha, lam, A=A, B=B)
         st.ttq[name] = res
         return res["Y"]
     res = st.ttq[name]
-    return O.linear(X, res["s32"], res["codes"], res["scale"], res["zero"], g)
+    return O.linear(X, res["s32"], res["codes"], res["scale"], res["zero"], g, A, B)
 
 
 def decoder_layer(r, y_prev, Wl, st: LayerState, shape, pos0: int, q: int, g: int, alpha: float,
@@ -148,7 +153,8 @@ def decoder_layer(r, y_prev, Wl, st: LayerState, shape, pos0: int, q: int, g: in
 
     r is the bf16 residual stream entering the layer, y_prev the previous layer's MLP
     output still to be added (None for the first layer). Wl holds the bf16 weights
-    (w_qkv, w_o, w_gate_up, w_down, n_in, n_post, n_q, n_k). Returns a dict of every
+    (w_qkv, w_o, w_gate_up, w_down, n_in, n_post, n_q, n_k, and a_*, b_* when the linears
+    carry low-rank factors). Returns a dict of every
     intermediate, rounded to bf16 where the GPU stores it; ``r`` and ``down`` are what
     the next layer takes."""
     H, Hkv, D, I = shape["heads"], shape["kv_heads"], shape["head_dim"], shape["inter"]
@@ -157,19 +163,19 @@ def decoder_layer(r, y_prev, Wl, st: LayerState, shape, pos0: int, q: int, g: in
         r = add_residual(r, y_prev)
     out["r_in"] = r
     out["h"] = O.round_bf16(rmsnorm(r, Wl["n_in"]))
-    out["qkv"] = O.round_bf16(ttq_linear("qkv", out["h"], Wl["w_qkv"], st, q, g, alpha, lam, prefill))
+    out["qkv"] = O.round_bf16(ttq_linear("qkv", out["h"], Wl, st, q, g, alpha, lam, prefill))
     qh, kh, vh = qk_norm_rope(out["qkv"], H, Hkv, D, Wl["n_q"], Wl["n_k"], pos0)
     st.K = kh if st.K is None else np.concatenate([st.K[:pos0], kh])
     st.V = vh if st.V is None else np.concatenate([st.V[:pos0], vh])
     out["q"], out["k"], out["v"] = qh, kh, vh
     out["attn"] = O.round_bf16(attention(qh, st.K, st.V, pos0))
-    out["o"] = O.round_bf16(ttq_linear("o", out["attn"], Wl["w_o"], st, q, g, alpha, lam, prefill))
+    out["o"] = O.round_bf16(ttq_linear("o", out["attn"], Wl, st, q, g, alpha, lam, prefill))
     r = add_residual(r, out["o"])
     out["r_mid"] = r
     out["h2"] = O.round_bf16(rmsnorm(r, Wl["n_post"]))
-    out["gu"] = O.round_bf16(ttq_linear("gate_up", out["h2"], Wl["w_gate_up"], st, q, g, alpha, lam, prefill))
+    out["gu"] = O.round_bf16(ttq_linear("gate_up", out["h2"], Wl, st, q, g, alpha, lam, prefill))
     out["m"] = O.round_bf16(silu_mul(out["gu"], I))
-    out["down"] = O.round_bf16(ttq_linear("down", out["m"], Wl["w_down"], st, q, g, alpha, lam, prefill))
+    out["down"] = O.round_bf16(ttq_linear("down", out["m"], Wl, st, q, g, alpha, lam, prefill))
     out["r"] = r
     return out
 

@@ -169,6 +169,60 @@ def test_prefill_batched_argument_errors(lib):
     assert n.value >= (16 + 32 + 8) * 128 * 2  # the folded activations of every prompt
 
 
+def test_decoder_kernel_argument_errors(lib):
+    a, b, c = 1 << 20, 1 << 21, 1 << 22
+    f = ctypes.c_float
+    # rmsnorm: sizes, eps, aliasing, alignment
+    assert lib.ttq_rmsnorm(_p(a), None, _p(b), 4, 60, f(1e-6), _p(c), None) == INVALID
+    assert lib.ttq_rmsnorm(_p(a), None, _p(b), 4, 16384, f(1e-6), _p(c), None) == INVALID
+    assert lib.ttq_rmsnorm(_p(a), None, _p(b), 0, 64, f(1e-6), _p(c), None) == INVALID
+    assert lib.ttq_rmsnorm(_p(a), None, _p(b), 4, 64, f(0.0), _p(c), None) == INVALID
+    assert lib.ttq_rmsnorm(_p(a), _p(a), _p(b), 4, 64, f(1e-6), _p(c), None) == INVALID
+    assert lib.ttq_rmsnorm(_p(a), _p(c), _p(b), 4, 64, f(1e-6), _p(c), None) == INVALID
+    assert lib.ttq_rmsnorm(_p(a + 2), None, _p(b), 4, 64, f(1e-6), _p(c), None) == MISALIGNED
+    assert lib.ttq_rmsnorm(None, None, _p(b), 4, 64, f(1e-6), _p(c), None) == INVALID
+    # rotary table
+    assert lib.ttq_rope_table(16, 96, ctypes.c_double(1e6), _p(a), None) == UNSUPPORTED
+    assert lib.ttq_rope_table(0, 128, ctypes.c_double(1e6), _p(a), None) == INVALID
+    assert lib.ttq_rope_table(16, 128, ctypes.c_double(1.0), _p(a), None) == INVALID
+    assert lib.ttq_rope_table(16, 128, ctypes.c_double(1e6), _p(a + 4), None) == MISALIGNED
+    # q/k norm + rotation: head_dim, positions against the cache and the table, aliasing
+    d = 1 << 23
+    args = lambda T, D, pos0, tpos, clen, kc=b, vc=c: (_p(a), T, 8, 2, D, _p(d), _p(d), f(1e-6), _p(d), tpos, pos0,
+                                                     None, _p(kc), _p(vc), clen, None)
+    assert lib.ttq_qk_norm_rope(*args(4, 96, 0, 64, 64)) == UNSUPPORTED
+    assert lib.ttq_qk_norm_rope(*args(4, 128, 61, 64, 128)) == INVALID      # past the table
+    assert lib.ttq_qk_norm_rope(*args(4, 128, 61, 128, 64)) == INVALID      # past the cache
+    assert lib.ttq_qk_norm_rope(*args(0, 128, 0, 64, 64)) == INVALID
+    assert lib.ttq_qk_norm_rope(*args(4, 128, -1, 64, 64)) == INVALID
+    assert lib.ttq_qk_norm_rope(*args(4, 128, 0, 64, 64, kc=b, vc=b)) == INVALID
+    assert lib.ttq_qk_norm_rope(*args(4, 128, 0, 64, 64, kc=b + 8)) == MISALIGNED
+    # a device-held position is checked on the device, but its pointer alignment here
+    dev_pos = (_p(a), 4, 8, 2, 128, _p(d), _p(d), f(1e-6), _p(d), 64, 0, _p(d + 4), _p(b), _p(c), 64, None)
+    assert lib.ttq_qk_norm_rope(*dev_pos) == MISALIGNED
+    # decode attention
+    sz = ctypes.c_size_t(0)
+    assert lib.ttq_decode_attention_workspace_size(32, 8, 128, 4224, ctypes.byref(sz)) == OK
+    assert sz.value >= 32 * 32 * 130 * 4        # 32 splits (256 blocks at most), (acc, m, l) per head
+    assert lib.ttq_decode_attention_workspace_size(32, 8, 256, 4224, ctypes.byref(sz)) == UNSUPPORTED
+    assert lib.ttq_decode_attention_workspace_size(48, 8, 128, 4224, ctypes.byref(sz)) == UNSUPPORTED  # 6 per kv
+    assert lib.ttq_decode_attention_workspace_size(30, 8, 128, 4224, ctypes.byref(sz)) == INVALID
+    att = lambda L, clen, pos=None, ws=d, wsb=1 << 20: (_p(a), 32, 8, 128, _p(b), _p(c), clen, L, pos, _p(d + 256),
+                                                       _p(ws) if ws else None, wsb, None)
+    assert lib.ttq_decode_attention(*att(0, 64)) == INVALID
+    assert lib.ttq_decode_attention(*att(65, 64)) == INVALID
+    assert lib.ttq_decode_attention(*att(10, 64, ws=None)) == WORKSPACE
+    assert lib.ttq_decode_attention(*att(10, 64, wsb=16)) == WORKSPACE
+    assert lib.ttq_decode_attention(*att(10, 64, pos=_p(d + 4))) == MISALIGNED
+    assert lib.ttq_position_advance(None, 1, None) == INVALID
+    assert lib.ttq_position_advance(_p(a + 4), 1, None) == MISALIGNED
+    # SwiGLU gate
+    assert lib.ttq_silu_mul(_p(a), 4, 12, _p(b), None) == INVALID
+    assert lib.ttq_silu_mul(_p(a), 0, 16, _p(b), None) == INVALID
+    assert lib.ttq_silu_mul(_p(a), 4, 16, _p(a), None) == INVALID
+    assert lib.ttq_silu_mul(_p(a), 4, 16, _p(b + 2), None) == MISALIGNED
+
+
 def test_binding_refuses_cpu_tensors(lib):
     torch = pytest.importorskip("torch")
     X = torch.zeros(4, 64, dtype=torch.bfloat16)

@@ -158,6 +158,29 @@ def test_stacked_ttq_linear_equals_separate_linears():
         row += n
 
 
+def test_stacked_lowrank_term_equals_separate_terms():
+    # stacked A = [A_1; A_2; A_3] and block-diagonal B give each part its own rank-r term
+    rng = np.random.default_rng(7)
+    r, d = 8, 128
+    X = O.round_bf16(rng.standard_t(3, (24, d)))
+    Ws = [O.round_bf16(rng.normal(0, 0.02, (n, d))) for n in (64, 32, 32)]
+    As = [O.round_bf16(rng.normal(0, 0.02, (r, d))) for _ in Ws]
+    Bs = [O.round_bf16(rng.normal(0, 0.02, (W.shape[0], r))) for W in Ws]
+    Bst = np.zeros((128, 3 * r))
+    row = 0
+    for i, B in enumerate(Bs):
+        Bst[row: row + B.shape[0], i * r: (i + 1) * r] = B
+        row += B.shape[0]
+    st = O.prefill(X, np.concatenate(Ws), 4, 32, 0.5, 0.4, A=np.concatenate(As), B=Bst)
+    row = 0
+    for W, A, B in zip(Ws, As, Bs):
+        one = O.prefill(X, W, 4, 32, 0.5, 0.4, A=A, B=B)
+        n = W.shape[0]
+        np.testing.assert_array_equal(st["codes"][row: row + n], one["codes"])
+        np.testing.assert_allclose(st["Y"][:, row: row + n], one["Y"], rtol=1e-12, atol=1e-12)
+        row += n
+
+
 # ------------------------------------------------------------------ the layer
 
 
