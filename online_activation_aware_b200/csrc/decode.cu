@@ -5,19 +5,20 @@
 // For a weight row i and a group G of g inputs, cut into 32-input units V:
 //   sum_{k in G} x'_tk (c_ik - z) sigma
 //     = sigma * sum_{V in G} ( sum_{k in V} (128 + c_ik) x'_tk - (128 + z) sum_{k in V} x'_tk )
-// so each weight costs one byte permute (128 + c as an fp32, exact) and one FMA per token;
+// so each weight costs one byte permute (128 + c as an fp32, exact) and half of a two-wide
+// FMA (fma.rn.f32x2: pairs of inputs for one token, the token pair for two);
 // each unit is finished on its own (scale and zero of its group), so a lane may take any
 // set of units; the unit sums of x' come with x' from a small prep kernel.
 //
 // Layout of the work: one warp per 4 weight rows, the 32 lanes spanning the inputs (lane j
-// takes the rows' 32-input units j, j + 32, ...), so that each row's lanes read 512
-// contiguous bytes of codes per step (16-byte loads that bypass L1) and every x' value a
-// lane loads (16-byte loads through L1, contiguous across the warp) serves 4 weights: a
-// load's cost is its per-lane register writeback, so the reuse in registers is what keeps
-// x' traffic below the code traffic. The codes of the next kDepth units are in flight
-// while one is consumed; the 32 lanes are summed by shuffles in a fixed order. CTAs of 8 rows put about
-// 7 CTAs on each SM, all in one wave, with the rows' scale and zero staged in shared
-// memory. x' (fp32, chunk-major, see xoff) and the unit sums come from a prep kernel
+// takes the rows' 32-input units j, j + 32, ...), so that each row's lanes read contiguous
+// codes per step (16-byte loads that bypass L1) and every x' value a lane loads (16-byte
+// loads through L1, contiguous across the warp) serves 4 weights: a load's cost is its
+// per-lane register writeback, so the reuse in registers is what keeps x' traffic below
+// the code traffic (2 rows a warp measured slower at every shape of a Qwen3-8B layer).
+// The codes of the next kDepth units are in flight while one is consumed; the 32 lanes are
+// summed by shuffles in a fixed order. CTAs of 8 rows put about 7 CTAs on each SM, all in
+// one wave, with the rows' scale and zero staged in shared memory. x' (fp32, chunk-major, see xoff) and the unit sums come from a prep kernel
 // chained to the GEMV by programmatic dependent launch: the GEMV issues its first code
 // loads before waiting for x'.
 #include "ttq_internal.h"
@@ -33,6 +34,23 @@ constexpr int kRowsPerCta = kRowsPerWarp * kGemvThreads / 32;     // 8: about 7 
 
 __device__ __forceinline__ float code_plus_128f(uint32_t x, int b) {
   return __uint_as_float(__byte_perm(x, 0x43000000u, 0x7044u + (static_cast<unsigned>(b) << 8)));
+}
+
+// Packed fp32 pairs (sm_100's two-wide FMA: each lane of the pair rounds like an fp32 FMA).
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(a), "f"(b));
+  return v;
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return make_float2(a, b);
 }
 
 // The Q words holding one row's codes for one 32-input unit.
@@ -73,9 +91,13 @@ __device__ __forceinline__ void codes4(const UnitWords<Q>& u, int c4, float (&f)
     f[2] = code_plus_128f(lo, b0 + 1);
     f[3] = code_plus_128f(hi, b0 + 1);
   } else if (Q == 2) {
-    const uint32_t w = u.w[c4 >> 2] >> (8 * (c4 & 3));  // input 16v + e at bits 2e
+    // word c4 / 4 holds inputs 16j .. 16j + 15 (input 16j + e at bits 2e): masked by
+    // 0x03030303 after a shift of 2e, byte b holds input 16j + 4b + e, one byte permute
+    // per code (the masks are shared by the four c4 of a word once unrolled)
+    const uint32_t w = u.w[c4 >> 2];
+    const int b = c4 & 3;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) f[e] = __uint_as_float(0x43000000u | (((w >> (2 * e)) & 3u) << 16));
+    for (int e = 0; e < 4; ++e) f[e] = code_plus_128f((w >> (2 * e)) & 0x03030303u, b);
   } else {
     // three bit planes: bit b of input k at bit k of word b
 #pragma unroll
@@ -208,11 +230,11 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
       const int st = s0 + hb;
       if (st < nsteps) {
         const int u = lane + 32 * st;
-        float acc[R][B];
+        // two-wide accumulators: one token, pairs of inputs (even, odd); two tokens, the
+        // token pair of each input
+        uint64_t acc2[R];
 #pragma unroll
-        for (int i = 0; i < R; ++i)
-#pragma unroll
-          for (int t = 0; t < B; ++t) acc[i][t] = 0.f;
+        for (int i = 0; i < R; ++i) acc2[i] = 0ull;
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
           // x' of inputs 4 c4 .. 4 c4 + 3 of unit u for all B tokens
@@ -223,14 +245,36 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
             const float4 v = __ldg(reinterpret_cast<const float4*>(xb + 4 * i2));
             x[4 * i2] = v.x; x[4 * i2 + 1] = v.y; x[4 * i2 + 2] = v.z; x[4 * i2 + 3] = v.w;
           }
+          uint64_t xv[4];
+          if (B == 1) {
+            xv[0] = f2(x[0], x[1]);
+            xv[1] = f2(x[2], x[3]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) xv[e] = f2(x[e * B], x[e * B + 1]);
+          }
 #pragma unroll
           for (int i = 0; i < R; ++i) {
             float f[4];
             codes4<Q>(cb[hb][i], c4, f);
+            if (B == 1) {
+              acc2[i] = ffma2(f2(f[0], f[1]), xv[0], acc2[i]);
+              acc2[i] = ffma2(f2(f[2], f[3]), xv[1], acc2[i]);
+            } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
+              for (int e = 0; e < 4; ++e) acc2[i] = ffma2(f2(f[e], f[e]), xv[e], acc2[i]);
+            }
+          }
+        }
+        float acc[R][B];
 #pragma unroll
-              for (int t = 0; t < B; ++t) acc[i][t] = __fmaf_rn(f[e], x[e * B + t], acc[i][t]);
+        for (int i = 0; i < R; ++i) {
+          const float2 a = f2_unpack(acc2[i]);
+          if (B == 1) {
+            acc[i][0] = __fadd_rn(a.x, a.y);
+          } else {
+            acc[i][0] = a.x;
+            acc[i][B - 1] = a.y;
           }
         }
         if (st + kDepth < nsteps) {  // refill the slot just consumed, kDepth units ahead
@@ -267,9 +311,32 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
 #pragma unroll
       for (int t = 0; t < B; ++t)
         if (i == oi && t == ot) y = pacc[i][t];
-    for (int q = 0; q < r; ++q)
-      y = __fmaf_rn(__bfloat162float(U[static_cast<int64_t>(ot) * 64 + q]),
-                    __bfloat162float(Blr[static_cast<int64_t>(orow) * r + q]), y);
+    // the rank-r term: r % 8 == 0, the row of B and of U read as 16-byte chunks, all
+    // requested before the first FMA
+    const uint4* ur = reinterpret_cast<const uint4*>(U + static_cast<int64_t>(ot) * 64);
+    const uint4* br = reinterpret_cast<const uint4*>(Blr + static_cast<int64_t>(orow) * r);
+    for (int c0 = 0; c0 < r / 8; c0 += 4) {
+      uint4 uv[4], bv[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (c0 + c < r / 8) {
+          uv[c] = __ldg(ur + c0 + c);
+          bv[c] = __ldg(br + c0 + c);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (c0 + c < r / 8) {
+          const uint32_t uw[4] = {uv[c].x, uv[c].y, uv[c].z, uv[c].w};
+          const uint32_t bw[4] = {bv[c].x, bv[c].y, bv[c].z, bv[c].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            y = __fmaf_rn(__uint_as_float(uw[k] << 16), __uint_as_float(bw[k] << 16), y);
+            y = __fmaf_rn(__uint_as_float(uw[k] & 0xFFFF0000u), __uint_as_float(bw[k] & 0xFFFF0000u), y);
+          }
+        }
+      }
+    }
     Y[static_cast<int64_t>(ot) * d_out + orow] = __float2bfloat16_rn(y);
   }
 }

@@ -10,7 +10,7 @@
 //   qk_norm_rope_kernel one warp per (token, head) of the stacked q|k|v projection
 //   silu_mul_kernel     out = bf16(silu(gate) * up), grid-stride over 8-channel chunks
 //   decode_attn_*       one new token's grouped-query attention over the cache, split over
-//                       positions and merged (flash-decoding form), fp32 online softmax
+//                       positions and merged (flash-decoding form), fp32 softmax
 #include <algorithm>
 #include <cmath>
 
@@ -247,164 +247,150 @@ __global__ void __launch_bounds__(256) silu_mul_kernel(const __nv_bfloat16* __re
 // ---------------------------------------------------------------- decode attention
 //
 // One new token's attention over the key/value cache (split over positions, then
-// combined): block (kv head kh, split sp) of 8 warps takes positions
-// [sp * per, (sp + 1) * per) of the L valid ones, per = ceil(L / splits); each warp walks
-// positions in rounds of kDecUnroll, lane l holding channels [E l, E l + E) of k and v and
-// of the G query heads that read kv head kh (h = kh G + g). Per head it keeps the running
-// maximum m, the sum l of e^(score - m) and the e^(score - m)-weighted sum of v (fp32); the
-// warps' triples are merged in shared memory and written to `part`
-// [kv_heads][splits][G][D + 2] (acc[D], m, l). decode_attn_combine_kernel merges the
-// splits of one query head and rounds the output to bf16.
-constexpr int kDecWarps = 8;
-constexpr int kDecUnroll = 4;
+// combined). Block (kv head kh, split sp) of 256 threads takes positions
+// [sp * per, (sp + 1) * per) of the L valid ones, per = ceil(L / splits), in chunks of 256:
+//   scores   thread i: s_g = q_g . k_p for position p = chunk start + i and the G query heads
+//            h = kh G + g that read kv head kh (q pre-scaled by 1/sqrt(D), broadcast from
+//            shared memory; k read as 16-byte chunks of its row);
+//   softmax  per head the chunk's maximum and sum (one warp per head, fixed order), the
+//            running maximum m, the rescale e^(m_old - m), weights e^(s - m) in place;
+//   values   lane l holds channels [E l, E l + E) (coalesced v rows), warp w the positions
+//            i = w (mod 8) of the chunk: acc_g += w_g,p v_p.
+// The 8 warps' accumulators are added in a fixed order and written with (m, l) to `part`
+// [kv_heads][splits][G][D + 2]; decode_attn_combine_kernel merges the splits per query head.
+constexpr int kDecThreads = 256;
+constexpr int kDecChunk = 256;
 
 template <int E, int G>
-__global__ void __launch_bounds__(kDecWarps * 32) decode_attn_partial_kernel(
+__global__ void __launch_bounds__(kDecThreads) decode_attn_partial_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_cache,
     const __nv_bfloat16* __restrict__ v_cache, int kv_heads, int64_t cache_len, int64_t length,
     const int64_t* __restrict__ pos_dev, int splits, float scale, float* __restrict__ part,
     unsigned* __restrict__ err) {
   using V = typename LaneVec<E>::T;
   constexpr int D = 32 * E;
-  __shared__ float sm[kDecWarps][G][D + 2];
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
+  constexpr int kWarps = kDecThreads / 32;
+  __shared__ __align__(16) float qs[G][D];
+  __shared__ float sc[G][kDecChunk];
+  __shared__ float sm_acc[kWarps][G][D];
+  __shared__ float m_sh[G], l_sh[G], c_sh[G];
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
   const int kh = blockIdx.x;
   const int sp = blockIdx.y;
   int64_t L = pos_dev ? *pos_dev + 1 : length;
   if (L < 1 || L > cache_len) {
-    if (kh == 0 && sp == 0 && threadIdx.x == 0) atomicOr(err, kErrRange);
+    if (kh == 0 && sp == 0 && tid == 0) atomicOr(err, kErrRange);
     L = 0;
   }
   const int64_t per = (L + splits - 1) / splits;
   const int64_t p0 = static_cast<int64_t>(sp) * per;
   const int64_t p1 = min(L, p0 + per);
-  float qf[G][E];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    float t[E];
-    lane_unpack<E>(*reinterpret_cast<const V*>(q + static_cast<int64_t>(kh * G + g) * D + lane * E), t);
-#pragma unroll
-    for (int e = 0; e < E; ++e) qf[g][e] = __fmul_rn(t[e], scale);
+  for (int i = tid; i < G * D; i += kDecThreads)
+    qs[i / D][i % D] = __fmul_rn(__bfloat162float(q[static_cast<int64_t>(kh * G) * D + i]), scale);
+  if (tid < G) {
+    m_sh[tid] = -INFINITY;
+    l_sh[tid] = 0.f;
   }
-  float m[G], l[G], acc[G][E];
+  float acc[G][E];
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m[g] = -INFINITY;
-    l[g] = 0.f;
+  for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[g][e] = 0.f;
-  }
   const int64_t row = static_cast<int64_t>(kv_heads) * D;
-  const __nv_bfloat16* kb = k_cache + kh * D + lane * E;
-  const __nv_bfloat16* vb = v_cache + kh * D + lane * E;
-  constexpr int kStep = kDecWarps * kDecUnroll;
-  // the next round's rows are requested while this round is computed (p1 > p0 here, so the
-  // clamped row index stays inside the valid range)
-  V kn[kDecUnroll], vn[kDecUnroll];
-  if (p1 > p0) {
+  __syncthreads();
+  for (int64_t c0 = p0; c0 < p1; c0 += kDecChunk) {
+    const int n = static_cast<int>(min(static_cast<int64_t>(kDecChunk), p1 - c0));
+    // scores of position c0 + tid
+    if (tid < n) {
+      const uint4* kr = reinterpret_cast<const uint4*>(k_cache + (c0 + tid) * row + kh * D);
+      float s[G];
 #pragma unroll
-    for (int u = 0; u < kDecUnroll; ++u) {
-      const int64_t p = min(p0 + warp * kDecUnroll + u, p1 - 1);
-      kn[u] = *reinterpret_cast<const V*>(kb + p * row);
-      vn[u] = *reinterpret_cast<const V*>(vb + p * row);
+      for (int g = 0; g < G; ++g) s[g] = 0.f;
+#pragma unroll 4
+      for (int c = 0; c < D / 8; ++c) {
+        float kf[8];
+        unpack8(__ldg(kr + c), kf);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float4 qa = *reinterpret_cast<const float4*>(&qs[g][8 * c]);
+          const float4 qb = *reinterpret_cast<const float4*>(&qs[g][8 * c + 4]);
+          s[g] = __fmaf_rn(qa.x, kf[0], s[g]);
+          s[g] = __fmaf_rn(qa.y, kf[1], s[g]);
+          s[g] = __fmaf_rn(qa.z, kf[2], s[g]);
+          s[g] = __fmaf_rn(qa.w, kf[3], s[g]);
+          s[g] = __fmaf_rn(qb.x, kf[4], s[g]);
+          s[g] = __fmaf_rn(qb.y, kf[5], s[g]);
+          s[g] = __fmaf_rn(qb.z, kf[6], s[g]);
+          s[g] = __fmaf_rn(qb.w, kf[7], s[g]);
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) sc[g][tid] = s[g];
     }
-  }
-  for (int64_t base = p0 + warp * kDecUnroll; base < p1; base += kStep) {
-    V kr[kDecUnroll], vr[kDecUnroll];
+    __syncthreads();
+    // per head (warp g): the chunk's maximum, the new running maximum, weights in place
+    if (warp < G) {
+      const int g = warp;
+      float mx = -INFINITY;
+      for (int i = lane; i < n; i += 32) mx = fmaxf(mx, sc[g][i]);
 #pragma unroll
-    for (int u = 0; u < kDecUnroll; ++u) {
-      kr[u] = kn[u];
-      vr[u] = vn[u];
-    }
-    if (base + kStep < p1) {
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float m_old = m_sh[g];
+      const float m_new = fmaxf(m_old, mx);
+      float sum = 0.f;
+      for (int i = lane; i < n; i += 32) {
+        const float w = expf(sc[g][i] - m_new);
+        sc[g][i] = w;
+        sum += w;
+      }
 #pragma unroll
-      for (int u = 0; u < kDecUnroll; ++u) {
-        const int64_t p = min(base + kStep + u, p1 - 1);  // clamped: rows past p1 are read but not used
-        kn[u] = *reinterpret_cast<const V*>(kb + p * row);
-        vn[u] = *reinterpret_cast<const V*>(vb + p * row);
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      if (lane == 0) {
+        const float c = expf(m_old - m_new);  // m_old = -inf on the first chunk: c = 0
+        c_sh[g] = c;
+        l_sh[g] = __fmaf_rn(l_sh[g], c, sum);
+        m_sh[g] = m_new;
       }
     }
-    // the round's kDecUnroll x G scores, reduced across the warp together
-    float sc[kDecUnroll][G];
-#pragma unroll
-    for (int u = 0; u < kDecUnroll; ++u) {
-      float kf[E];
-      lane_unpack<E>(kr[u], kf);
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float dot = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) dot = __fmaf_rn(qf[g][e], kf[e], dot);
-        sc[u][g] = dot;
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-      for (int u = 0; u < kDecUnroll; ++u)
-#pragma unroll
-        for (int g = 0; g < G; ++g) sc[u][g] += __shfl_xor_sync(0xffffffffu, sc[u][g], off);
-    // one online-softmax update per head for the whole round
-    const int nvalid = static_cast<int>(min(static_cast<int64_t>(kDecUnroll), p1 - base));
-    float vf[kDecUnroll][E];
-#pragma unroll
-    for (int u = 0; u < kDecUnroll; ++u) lane_unpack<E>(vr[u], vf[u]);
+    __syncthreads();
+    // values: lane's channels, warp's positions
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      float mn = m[g];
+      const float c = c_sh[g];
 #pragma unroll
-      for (int u = 0; u < kDecUnroll; ++u)
-        if (u < nvalid) mn = fmaxf(mn, sc[u][g]);
-      const float c = expf(m[g] - mn);  // m = -inf before the first position: c = 0
-      float w[kDecUnroll];
-      float wsum = 0.f;
-#pragma unroll
-      for (int u = 0; u < kDecUnroll; ++u) {
-        w[u] = u < nvalid ? expf(sc[u][g] - mn) : 0.f;
-        wsum = __fadd_rn(wsum, w[u]);
-      }
-      l[g] = __fmaf_rn(l[g], c, wsum);
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        float a = __fmul_rn(acc[g][e], c);
-#pragma unroll
-        for (int u = 0; u < kDecUnroll; ++u) a = __fmaf_rn(w[u], vf[u][e], a);
-        acc[g][e] = a;
-      }
-      m[g] = mn;
+      for (int e = 0; e < E; ++e) acc[g][e] = __fmul_rn(acc[g][e], c);
     }
+    const __nv_bfloat16* vb = v_cache + kh * D + lane * E;
+#pragma unroll 4
+    for (int i = warp; i < n; i += kWarps) {
+      float vf[E];
+      lane_unpack<E>(*reinterpret_cast<const V*>(vb + (c0 + i) * row), vf);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float w = sc[g][i];
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[g][e] = __fmaf_rn(w, vf[e], acc[g][e]);
+      }
+    }
+    __syncthreads();  // sc is rewritten by the next chunk
   }
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
+  for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int e = 0; e < E; ++e) sm[warp][g][lane * E + e] = acc[g][e];
-    if (lane == 0) {
-      sm[warp][g][D] = m[g];
-      sm[warp][g][D + 1] = l[g];
-    }
-  }
+    for (int e = 0; e < E; ++e) sm_acc[warp][g][lane * E + e] = acc[g][e];
   __syncthreads();
   float* out = part + (static_cast<int64_t>(kh) * splits + sp) * G * (D + 2);
-  for (int i = threadIdx.x; i < G * D; i += kDecWarps * 32) {
-    const int g = i / D;
-    const int j = i - g * D;
-    float M = -INFINITY;
+  for (int i = tid; i < G * D; i += kDecThreads) {
+    const int g = i / D, j = i % D;
+    float a = 0.f;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sm[w][g][D]);
-    float a = 0.f, s = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) {
-        const float f = expf(sm[w][g][D] - M);  // a warp with no positions has m = -inf: f = 0
-        a = __fmaf_rn(sm[w][g][j], f, a);
-        s = __fmaf_rn(sm[w][g][D + 1], f, s);
-      }
-    }
+    for (int w = 0; w < kWarps; ++w) a += sm_acc[w][g][j];
     out[g * (D + 2) + j] = a;
     if (j == 0) {
-      out[g * (D + 2) + D] = M;
-      out[g * (D + 2) + D + 1] = s;
+      out[g * (D + 2) + D] = m_sh[g];     // -inf and 0 when the split holds no position
+      out[g * (D + 2) + D + 1] = l_sh[g];
     }
   }
 }
@@ -496,8 +482,8 @@ static cudaError_t decode_attn_partial(dim3 grid, cudaStream_t stream, const __n
                                        const __nv_bfloat16* kc, const __nv_bfloat16* vc, int kv_heads,
                                        int64_t cache_len, int64_t length, const int64_t* pos_dev, int splits,
                                        float scale, float* part, unsigned* err) {
-  decode_attn_partial_kernel<E, G><<<grid, kDecWarps * 32, 0, stream>>>(q, kc, vc, kv_heads, cache_len, length,
-                                                                        pos_dev, splits, scale, part, err);
+  decode_attn_partial_kernel<E, G><<<grid, kDecThreads, 0, stream>>>(q, kc, vc, kv_heads, cache_len, length,
+                                                                      pos_dev, splits, scale, part, err);
   return cudaGetLastError();
 }
 
