@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--r", type=int, default=None, help="low-rank r (default: the workload's)")
     ap.add_argument("--no-extras", action="store_true", help="skip the T sweep, decode and e2e legs")
     ap.add_argument("--no-decoder", action="store_true", help="skip the chained decoder-stack leg")
+    ap.add_argument("--probe", choices=["decode_gemv_oproj"], default=None,
+                    help="run one small fixed case for a profiler capture and exit (no timing)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline")
     return ap.parse_args()
 
@@ -290,8 +292,39 @@ def run_reference(args, wl, T):
 # ------------------------------------------------------------------ GPU legs
 
 
+def probe_decode_gemv_oproj():
+    """The o-projection shape of a Qwen3-8B layer under decode: 36 TTQ linears of
+    4096 x 4096 (q = 2, g = 32, r = 16, seeded random bf16 W, A, B; codes 36 x 6.3 MB > L2),
+    one prefill of 256 tokens each, then three rounds of one-token decode over all 36."""
+    import torch
+    import online_activation_aware_b200 as ttq
+
+    torch.manual_seed(0)
+    d, n, T = 4096, 4096, 256
+    lins = []
+    for _ in range(36):
+        W = (torch.randn(n, d, device="cuda") * 0.02).bfloat16()
+        A = (torch.randn(16, d, device="cuda") * 0.02).bfloat16()
+        B = (torch.randn(n, 16, device="cuda") * 0.02).bfloat16()
+        lins.append(ttq.TTQLinear(W, 2, 32, 0.5, 0.4, 2, 16, A, B))
+    X = torch.randn(T, d, device="cuda").bfloat16()
+    for lin in lins:
+        lin.prefill(X)
+    x = torch.randn(1, d, device="cuda").bfloat16()
+    Y = torch.empty(1, n, device="cuda", dtype=torch.bfloat16)
+    ws = ttq.alloc_workspace(T, d, n, lins[0].cfg)
+    for _ in range(3):
+        for lin in lins:
+            lin.decode(x, Y=Y, ws=ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"probe": "decode_gemv_oproj", "mean_abs_y": float(Y.float().abs().mean())}))
+    return 0
+
+
 def main():
     args = parse()
+    if args.probe == "decode_gemv_oproj":
+        return probe_decode_gemv_oproj()
     wl = synthetic.WORKLOADS[args.workload]
     T = args.T or wl.T
     r = wl.r if args.r is None else args.r
