@@ -227,3 +227,32 @@ def test_layer_decode_reuses_prefill_codes_and_cache():
     np.testing.assert_array_equal(out["qkv"], qkv)
     _, kh, _ = DO.qk_norm_rope(qkv, 2, 1, 32, Wl["n_q"], Wl["n_k"], 8)
     np.testing.assert_array_equal(st.K[8:], kh)
+
+
+# ------------------------------------------------------------------ the synthetic stack (host logic)
+
+
+def test_decoder_weights_layout_follows_the_architecture_table():
+    from online_activation_aware_b200 import synthetic
+
+    sh = synthetic.QWEN3_SHAPES["8B"]          # Table 15: 36 layers, 32 / 8 heads, 4096, 128, 12288
+    assert (sh["layers"], sh["heads"], sh["kv_heads"], sh["hidden"], sh["head_dim"], sh["inter"]) == \
+        (36, 32, 8, 4096, 128, 12288)
+    assert synthetic.decoder_linear_parts(sh, "qkv") == ([4096, 1024, 1024], 4096)
+    assert synthetic.decoder_linear_parts(sh, "o") == ([4096], 4096)
+    assert synthetic.decoder_linear_parts(sh, "gate_up") == ([12288, 12288], 4096)
+    assert synthetic.decoder_linear_parts(sh, "down") == ([4096], 12288)
+    small = dict(layers=1, heads=4, kv_heads=2, hidden=128, head_dim=32, inter=96)
+    L = synthetic.draw_decoder_weights(small, 8, seed=3)[0]
+    assert L["w_qkv"].shape == (4 * 32 + 2 * 2 * 32, 128) and L["a_qkv"].shape == (24, 128)
+    b = L["b_qkv"]
+    assert b.shape == (256, 24)
+    # block diagonal: part i's rows use only columns i r .. (i + 1) r
+    for i, (r0, r1) in enumerate(((0, 128), (128, 192), (192, 256))):
+        blk = np.zeros_like(b[r0:r1], dtype=bool)
+        blk[:, i * 8:(i + 1) * 8] = True
+        assert np.all(b[r0:r1][~blk] == 0) and np.all(b[r0:r1][blk] != 0)
+    assert L["b_gate_up"].shape == (192, 16) and L["a_down"].shape == (8, 96)
+    # the same seed draws the same numbers
+    L2 = synthetic.draw_decoder_weights(small, 8, seed=3)[0]
+    assert all(np.array_equal(L[k], L2[k]) for k in L)
