@@ -236,8 +236,9 @@ TTQ_API ttq_status ttq_linear_decode_batched(const void* X_bf16, int32_t request
  *   when residual != NULL:  r <- bf16(r + y)  (the residual row is replaced), h = r
  *   else:                   h = y
  *   out = bf16(h * w / sqrt(mean(h^2) + eps))
- *   y, residual, out   device bf16 [rows, n]; residual may be NULL; it must differ from
- *                      y and out (TTQ_ERR_INVALID_ARG); out must not overlap y or residual
+ *   y, residual, out   device bf16 [rows, n]; residual may be NULL; the three must be
+ *                      distinct buffers (equal pointers: TTQ_ERR_INVALID_ARG) that do not
+ *                      overlap
  *   w                  device bf16 [n]
  * n % 8 == 0, 8 <= n <= 8192; eps > 0 (an all-zero row then gives zeros). */
 TTQ_API ttq_status ttq_rmsnorm(const void* y_bf16, void* residual_bf16, const void* w_bf16, int64_t rows,

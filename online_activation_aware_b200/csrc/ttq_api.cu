@@ -546,7 +546,8 @@ ttq_status ttq_rmsnorm(const void* y_bf16, void* residual_bf16, const void* w_bf
   if (!y_bf16 || !w_bf16 || !out_bf16) return TTQ_ERR_INVALID_ARG;
   if (rows < 1 || rows > (int64_t(1) << 31) - 1 || n < 8 || n > 8192 || n % 8 != 0) return TTQ_ERR_INVALID_ARG;
   if (!std::isfinite(eps) || !(eps > 0.f)) return TTQ_ERR_INVALID_ARG;
-  if (residual_bf16 && (residual_bf16 == y_bf16 || residual_bf16 == out_bf16)) return TTQ_ERR_INVALID_ARG;
+  if (out_bf16 == y_bf16 || (residual_bf16 && (residual_bf16 == y_bf16 || residual_bf16 == out_bf16)))
+    return TTQ_ERR_INVALID_ARG;
   if (!aligned16(y_bf16) || !aligned16(w_bf16) || !aligned16(out_bf16) ||
       (residual_bf16 && !aligned16(residual_bf16)))
     return TTQ_ERR_MISALIGNED;

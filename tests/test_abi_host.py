@@ -179,6 +179,7 @@ def test_decoder_kernel_argument_errors(lib):
     assert lib.ttq_rmsnorm(_p(a), None, _p(b), 4, 64, f(0.0), _p(c), None) == INVALID
     assert lib.ttq_rmsnorm(_p(a), _p(a), _p(b), 4, 64, f(1e-6), _p(c), None) == INVALID
     assert lib.ttq_rmsnorm(_p(a), _p(c), _p(b), 4, 64, f(1e-6), _p(c), None) == INVALID
+    assert lib.ttq_rmsnorm(_p(a), None, _p(b), 4, 64, f(1e-6), _p(a), None) == INVALID
     assert lib.ttq_rmsnorm(_p(a + 2), None, _p(b), 4, 64, f(1e-6), _p(c), None) == MISALIGNED
     assert lib.ttq_rmsnorm(None, None, _p(b), 4, 64, f(1e-6), _p(c), None) == INVALID
     # rotary table
