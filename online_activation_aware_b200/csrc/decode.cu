@@ -17,10 +17,10 @@
 // per-lane register writeback, so the reuse in registers is what keeps x' traffic below
 // the code traffic (2 rows a warp measured slower at every shape of a Qwen3-8B layer).
 // The codes of the next kDepth units are in flight while one is consumed; the 32 lanes are
-// summed by shuffles in a fixed order. CTAs of 8 rows put about 7 CTAs on each SM, all in
-// one wave, with the rows' scale and zero staged in shared memory. x' (fp32, chunk-major, see xoff) and the unit sums come from a prep kernel
-// chained to the GEMV by programmatic dependent launch: the GEMV issues its first code
-// loads before waiting for x'.
+// summed by shuffles in a fixed order. CTAs of 8 rows (up to 8 on an SM at 128 registers a
+// thread) stage the rows' scale and zero in shared memory. x' (fp32, chunk-major, see xoff)
+// and the unit sums come from a prep kernel chained to the GEMV by programmatic dependent
+// launch: the GEMV issues its first code loads before waiting for x'.
 #include "ttq_internal.h"
 
 namespace ttq {
@@ -30,7 +30,7 @@ namespace {
 constexpr int kRowsPerWarp = 4;
 constexpr int kDepth = 4;  // 32-input units of codes in flight per lane (for each of its rows)
 constexpr int kGemvThreads = 64;                                  // 2 warps
-constexpr int kRowsPerCta = kRowsPerWarp * kGemvThreads / 32;     // 8: about 7 CTAs per SM, one wave
+constexpr int kRowsPerCta = kRowsPerWarp * kGemvThreads / 32;     // 8
 
 __device__ __forceinline__ float code_plus_128f(uint32_t x, int b) {
   return __uint_as_float(__byte_perm(x, 0x43000000u, 0x7044u + (static_cast<unsigned>(b) << 8)));
