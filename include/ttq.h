@@ -107,9 +107,12 @@ TTQ_API ttq_status ttq_act_stats(const void* X_bf16, int64_t T, int64_t d, int64
  * the partial sums live in a fixed scratch array in the library's device memory (1 MiB
  * of fp32 partial sums plus 1 KiB of counters, held on every GPU that loads the library
  * until the process exits). Limits: d <= 65536 channels, else TTQ_ERR_TOO_LARGE and
- * nothing is launched; the row split of the reduction shrinks so that it fits.
+ * nothing is launched (at most about 600 blocks of 256 channels are launched, so the
+ * partial sums of any d up to that limit fit in the array).
  * The first call on a device looks up the scratch array's device address (with that
- * device current); make that first call before any stream capture. Every call on a
+ * device current); make that first call before any stream capture. The address is cached
+ * per CUDA context: the first call in a new context (after cudaDeviceReset, or under a
+ * caller's own driver-API context) looks it up again. Every call on a
  * device shares the one array and overwrites it (its counters are cleared by each
  * call): calls whose kernels overlap on the GPU (other streams, other host threads)
  * race and must be serialised by the caller. */

@@ -3,7 +3,7 @@
 // counters) lives in one fixed array in the library's own device memory instead of a
 // caller workspace. Host code reaches the array only through the device address that
 // cudaGetSymbolAddress returns (the symbol itself is a host-side stand-in, not a device
-// pointer), looked up once per device with that device current.
+// pointer), looked up with the device current on the first call in each CUDA context.
 #include <mutex>
 
 #include "ttq.h"
@@ -19,20 +19,32 @@ constexpr int64_t kScratchBytes = kPartialFloats * 4 + kCounterBytes;
 static __device__ __align__(256) unsigned char g_act_stats_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
+struct ScratchAddr {
+  unsigned long long ctx_id = 0;  // context the address belongs to (0: not looked up yet)
+  void* addr = nullptr;
+};
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+ScratchAddr g_scratch[kMaxDevices];
 
-// Device address of the scratch array on the current device (looked up on first use).
+// Device address of the scratch array in the context current on this thread, looked up
+// with cudaGetSymbolAddress on the first call in that context and cached per device
+// ordinal together with the context's id. A module's symbols get new addresses when its
+// context is rebuilt (cudaDeviceReset) and differ in a caller's own driver-API context,
+// so a change of context id triggers a fresh lookup instead of reusing a dead address.
 ttq_status scratch_on_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TTQ_ERR_CUDA;
+  unsigned long long ctx = 0;
+  if (!ttq::current_context_id(&ctx)) return TTQ_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
+  ScratchAddr& e = g_scratch[dev];
+  if (e.ctx_id != ctx || e.addr == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_act_stats_scratch) != cudaSuccess || p == nullptr) return TTQ_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    e.addr = p;
+    e.ctx_id = ctx;
   }
-  *out = g_scratch_addr[dev];
+  *out = e.addr;
   return TTQ_OK;
 }
 

@@ -355,6 +355,10 @@ cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t
                                     int64_t max_partial_floats, unsigned* counters,
                                     cudaStream_t stream) {
   StatsPlan pl = stats_plan(T, d);
+  // stats_plan launches at most about 592 + col_blocks blocks (nsplit <= ceil(592 /
+  // col_blocks)), so nsplit * d <= (592 + col_blocks) * 256 floats: 217,088 for d = 65,536,
+  // below the 262,144 of the allocation-free entry point's array. The branch below only
+  // guards callers with a smaller array.
   if (static_cast<int64_t>(pl.nsplit) * d > max_partial_floats) {
     int64_t ns = max_partial_floats / d;
     if (ns < 1) ns = 1;

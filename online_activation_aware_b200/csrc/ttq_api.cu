@@ -4,9 +4,44 @@
 #include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <mutex>
 
 #include "ttq.h"
 #include "ttq_internal.h"
+
+namespace ttq {
+
+namespace {
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename F>
+F driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<F>(p);
+}
+}  // namespace
+
+bool current_context_id(unsigned long long* id) {
+  static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return false;
+  if (ctx == nullptr) {
+    // no context bound to this thread yet: make the runtime bind the current device's
+    // primary context
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return false;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  }
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+}  // namespace ttq
 
 namespace {
 
@@ -23,26 +58,37 @@ inline cudaError_t trace(int i, cudaStream_t stream) {
 }
 
 struct DeviceInfo {
-  bool init = false;
+  unsigned long long ctx_id = 0;  // context the cached addresses belong to (0: none yet)
   unsigned* err_word = nullptr;
   int num_sms = 148;
 };
 DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+thread_local DeviceInfo t_dev;  // this host thread's copy of the entry it last looked up
 
+// Per-device facts of the current context: the device address of the error word (module
+// symbols move when a context is rebuilt, e.g. after cudaDeviceReset, or differ in a
+// caller's own driver-API context, so the cache is keyed on the context's id) and the SM
+// count. The table is shared by every host thread and guarded by a mutex; the caller gets
+// a pointer to its own thread's copy.
 ttq_status device_info(DeviceInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TTQ_ERR_CUDA;
+  unsigned long long ctx = 0;
+  if (!ttq::current_context_id(&ctx)) return TTQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
   DeviceInfo& di = g_dev[dev];
-  if (!di.init) {
+  if (di.ctx_id != ctx) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_ttq_error_word) != cudaSuccess) return TTQ_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, g_ttq_error_word) != cudaSuccess || p == nullptr) return TTQ_ERR_CUDA;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return TTQ_ERR_CUDA;
     di.err_word = static_cast<unsigned*>(p);
     di.num_sms = sms;
-    di.init = true;
+    di.ctx_id = ctx;
   }
-  *out = &di;
+  t_dev = di;
+  *out = &t_dev;
   return TTQ_OK;
 }
 

@@ -10,6 +10,11 @@
 
 namespace ttq {
 
+// Identifier (cuCtxGetId) of the CUDA context current on this host thread; when none is,
+// the current device's primary context is bound first. False when the driver refuses.
+// Device addresses of module symbols are per context, so caches of them key on this.
+bool current_context_id(unsigned long long* id);
+
 // ---------------------------------------------------------------- act_stats / fold
 
 // Column-split plan of the statistics kernels: blocks of 256 columns, T split in
