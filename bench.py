@@ -30,6 +30,7 @@ sys.path.insert(0, ROOT)
 
 from online_activation_aware_b200 import dist as D  # noqa: E402
 from online_activation_aware_b200 import synthetic  # noqa: E402
+from online_activation_aware_b200.lowrank_setup import lowrank_factors  # noqa: E402
 
 METRIC = "TTQ linear k tokens/s (stats+requant+GEMM), 5120→8192 4-bit; requant GB/s"
 FALLBACK_HBM_GBS = 6650.0
@@ -47,8 +48,6 @@ def parse():
     ap.add_argument("--r", type=int, default=None, help="low-rank r (default: the workload's)")
     ap.add_argument("--no-extras", action="store_true", help="skip the T sweep, decode and e2e legs")
     ap.add_argument("--no-decoder", action="store_true", help="skip the chained decoder-stack leg")
-    ap.add_argument("--probe", choices=["decode_gemv_oproj"], default=None,
-                    help="run one small fixed case for a profiler capture and exit (no timing)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline")
     return ap.parse_args()
 
@@ -78,6 +77,25 @@ def fold_bytes(T, d):
 
 def gemm_flops(T, d, d_out, r):
     return 2.0 * T * d * d_out + (2.0 * T * r * d_out if r else 0.0)
+
+
+def input_sets(T, d, d_out):
+    """Number of input buffer sets the timed steps rotate over, so that no step finds its
+    operands in the 126 MB L2, and the bytes of one set."""
+    import math
+
+    set_bytes = (T * d + d_out * d) * 2
+    return min(6, max(2, int(math.ceil(3 * 126e6 / set_bytes)) + 1)), set_bytes
+
+
+def bench_config(wl, T, r, world):
+    """The workload description both arms print (identical for the same arguments)."""
+    lin = wl.layers[0]
+    nsets, set_bytes = input_sets(T, lin.d, lin.d_out)
+    return {"workload": f"{wl.name} {lin.d}->{lin.d_out} q={wl.q} g={wl.g} T={T}", "T": T, "d": lin.d,
+            "d_out": lin.d_out, "q": wl.q, "g": wl.g, "alpha": wl.alpha, "lambda": wl.lam, "p": wl.p, "r": r,
+            "parallelism": f"replicas{world}",
+            "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.0f} MB (> 126 MB L2)"}
 
 
 def whole_job_ktoks(T, steps, world, t_max_ms):
@@ -148,6 +166,84 @@ class ClockSampler:
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "power_w_max": max(pw) if pw else None, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+class NvmlClockSampler:
+    """Samples the SM clock, power and clock-event reasons every ~2 ms through NVML
+    (read-only queries) on a background thread, so that even a timed region of a few
+    milliseconds gets samples. Falls back to the nvidia-smi sampler when NVML is absent."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, gpu_id: str, period_s: float = 0.002):
+        self.gpu_id = gpu_id
+        self.period = period_s
+        self.samples = []
+        self._stop = threading.Event()
+        self._fallback = None
+
+    def start(self):
+        try:
+            import pynvml as N
+
+            N.nvmlInit()
+            self.N = N
+            self.h = N.nvmlDeviceGetHandleByUUID(self.gpu_id)
+            self.max_mhz = float(N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM))
+            self.bits = [(name, getattr(N, attr, 0)) for name, attr in self.REASONS]
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception:
+            self._fallback = ClockSampler(self.gpu_id)
+            self._fallback.start()
+
+    def _run(self):
+        N, h = self.N, self.h
+        while not self._stop.is_set():
+            try:
+                t = time.perf_counter()
+                sm = float(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM))
+                rs = int(N.nvmlDeviceGetCurrentClocksEventReasons(h))
+                pw = N.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((t, sm, rs, pw))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def window(self, t0, t1):
+        self.t0, self.t1 = t0, t1
+        if self._fallback is not None:
+            self._fallback.window(t0, t1)
+
+    def stop(self):
+        if self._fallback is not None:
+            out = self._fallback.stop()
+            out["source"] = "nvidia-smi"
+            return out
+        self._stop.set()
+        self._t.join(timeout=2)
+        t0, t1 = getattr(self, "t0", -1e30), getattr(self, "t1", 1e30)
+        inside = [x for x in self.samples if t0 <= x[0] <= t1]
+        out = {"source": "nvml", "period_ms": self.period * 1e3, "samples": len(inside)}
+        if not inside:
+            # the region was shorter than one period: the nearest sample on each side
+            before = [x for x in self.samples if x[0] < t0][-1:]
+            after = [x for x in self.samples if x[0] > t1][:1]
+            inside = before + after
+            out["window"] = "no sample inside the timed region; the nearest one on each side"
+        sm = [x[1] for x in inside]
+        reasons = sorted({name for x in inside for name, bit in self.bits if bit and (x[2] & bit)})
+        out.update({"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                    "power_w_max": max((x[3] for x in inside), default=None), "reasons": reasons})
+        try:
+            self.N.nvmlShutdown()
+        except Exception:
+            pass
+        return out
 
 
 def gpu_uuid(torch, dev):
@@ -250,7 +346,7 @@ def cpu_baseline(Xv, Wv, wl, budget_s):
             "seconds": round(time.perf_counter() - t_start, 2)}
 
 
-def run_reference(args, wl, T):
+def run_reference(args, wl, T, r):
     rank, world, _ = D.env()
     if rank != 0:
         return 0
@@ -276,10 +372,8 @@ def run_reference(args, wl, T):
     out = {"metric": METRIC, "value": round(value, 6), "unit": "k tokens/s", "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic", "impl": "reference",
-           "config": {"workload": f"{wl.name} {lin.d}->{lin.d_out} q={wl.q} g={wl.g} T={T}", "T": T,
-                      "d": lin.d, "d_out": lin.d_out, "q": wl.q, "g": wl.g, "alpha": wl.alpha, "lambda": wl.lam,
-                      "r": 0},
+           "data": "synthetic", "impl": "reference", "extrapolated": True,
+           "config": bench_config(wl, T, r, args.gpus),
            "cpu_baseline": {"value": round(value, 6), "unit": "k tokens/s", "cores": cores, "kind": "oracle",
                             "sample": f"each step: {T_tok} tokens x {rows} output rows, extrapolated to "
                                       f"{T} tokens x {lin.d_out} rows; median over {args.steps} steps"},
@@ -292,44 +386,13 @@ def run_reference(args, wl, T):
 # ------------------------------------------------------------------ GPU legs
 
 
-def probe_decode_gemv_oproj():
-    """The o-projection shape of a Qwen3-8B layer under decode: 36 TTQ linears of
-    4096 x 4096 (q = 2, g = 32, r = 16, seeded random bf16 W, A, B; codes 36 x 6.3 MB > L2),
-    one prefill of 256 tokens each, then three rounds of one-token decode over all 36."""
-    import torch
-    import online_activation_aware_b200 as ttq
-
-    torch.manual_seed(0)
-    d, n, T = 4096, 4096, 256
-    lins = []
-    for _ in range(36):
-        W = (torch.randn(n, d, device="cuda") * 0.02).bfloat16()
-        A = (torch.randn(16, d, device="cuda") * 0.02).bfloat16()
-        B = (torch.randn(n, 16, device="cuda") * 0.02).bfloat16()
-        lins.append(ttq.TTQLinear(W, 2, 32, 0.5, 0.4, 2, 16, A, B))
-    X = torch.randn(T, d, device="cuda").bfloat16()
-    for lin in lins:
-        lin.prefill(X)
-    x = torch.randn(1, d, device="cuda").bfloat16()
-    Y = torch.empty(1, n, device="cuda", dtype=torch.bfloat16)
-    ws = ttq.alloc_workspace(T, d, n, lins[0].cfg)
-    for _ in range(3):
-        for lin in lins:
-            lin.decode(x, Y=Y, ws=ws)
-    torch.cuda.synchronize()
-    print(json.dumps({"probe": "decode_gemv_oproj", "mean_abs_y": float(Y.float().abs().mean())}))
-    return 0
-
-
 def main():
     args = parse()
-    if args.probe == "decode_gemv_oproj":
-        return probe_decode_gemv_oproj()
     wl = synthetic.WORKLOADS[args.workload]
     T = args.T or wl.T
     r = wl.r if args.r is None else args.r
     if args.impl == "reference":
-        return run_reference(args, wl, T)
+        return run_reference(args, wl, T, r)
 
     import numpy as np
     import torch
@@ -351,12 +414,10 @@ def main():
     Xb, Wb = host_inputs(wl, T, D.rank_seed(wl.seed, rank))
     A = B = None
     if r > 0:
-        Bh, Ah, Rh = ttq.lowrank_factors(Wb, r)
+        Bh, Ah, Rh = lowrank_factors(Wb, r)
         A, B = Ah.to(dev), Bh.to(dev)
         Wb = Rh
-    set_bytes = (T * d + d_out * d) * 2
-    nsets = max(2, int(np.ceil(3 * 126e6 / set_bytes)) + 1)
-    nsets = min(nsets, 6)
+    nsets, set_bytes = input_sets(T, d, d_out)
     Xs = [Xb.to(dev) for _ in range(nsets)]
     Ws = [Wb.to(dev) for _ in range(nsets)]
     outs = [{"s": torch.empty(d, dtype=torch.float32, device=dev),
@@ -380,9 +441,9 @@ def main():
     # between two kernels would stop the next one from starting early as a programmatic
     # dependent)
     K = args.steps
-    sampler = ClockSampler(gpu_uuid(torch, dev))
+    sampler = NvmlClockSampler(gpu_uuid(torch, dev))
     sampler.start()
-    time.sleep(0.3)
+    time.sleep(0.05)
     D.barrier()
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
@@ -458,9 +519,7 @@ def main():
         "metric": METRIC, "value": round(value, 3), "unit": "k tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(t_max_ms / K, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{wl.name} {d}->{d_out} q={q} g={g} T={T}", "T": T, "d": d, "d_out": d_out,
-                   "q": q, "g": g, "alpha": wl.alpha, "lambda": wl.lam, "r": r, "parallelism": f"replicas{world}",
-                   "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.0f} MB (> 126 MB L2)"},
+        "config": bench_config(wl, T, r, world),
         "requant_gbs": requant_leg(torch, ttq, Ws, outs, d, d_out, q, g),
         "requant_batched": requant_batched_leg(torch, ttq, Ws, outs, d, d_out, q, g),
         "roofline": roof,
@@ -537,6 +596,14 @@ def main():
         result["decode"] = decode_leg(torch, ttq, wl, cfg, Xs[0], Ws[0], A, B, dev, hbm_peak)
         result["decode_batched"] = decode_batched_leg(torch, ttq, wl, cfg, Ws[0], outs, dev, hbm_peak)
         result["sweep"] = sweep_leg(torch, ttq, wl, cfg, Wb, A, B, dev, r)
+        if r == 0:
+            result["rho_sweep"] = rho_sweep_leg(torch, ttq, wl, cfg, Wb, dev, hbm_peak)
+        sets = {"single_512": workload_set_leg(torch, ttq, "single_512", dev, hbm_peak, tc_peak),
+                "opt125m_set": workload_set_leg(torch, ttq, "opt125m_set", dev, hbm_peak, tc_peak)}
+        for g_ in synthetic.WORKLOADS["qwen3_1p7b_set"].g_sweep:
+            sets[f"qwen3_1p7b_set_g{g_}"] = workload_set_leg(torch, ttq, "qwen3_1p7b_set", dev, hbm_peak, tc_peak,
+                                                             g=g_)
+        result["workloads"] = sets
         if r == 0:
             result["lowrank_r16"] = lowrank_leg(torch, ttq, wl, Xs, Ws, dev)
             result["prefill_batched"] = prefill_batched_leg(torch, ttq, wl, cfg, Xs, Ws, dev)
@@ -804,6 +871,107 @@ def sweep_leg(torch, ttq, wl, cfg, Wb, A, B, dev, r):
         torch.cuda.empty_cache()
     assert ttq.device_status() == 0
     return res
+
+def rho_sweep_leg(torch, ttq, wl, cfg, Wb, dev, hbm_peak, Ts=(128, 1024, 4096, 16384), reps=20):
+    """The overhead ratio across prompt lengths: per T, the stage split of the prefill from
+    the library's stage events (median over `reps` prompts, rotating buffer sets larger
+    than L2), rho = (statistic + fold and re-quantization) / projection, next to the
+    pages' count rho_model = 1/d' + 3/T (gist.science French summary, section 2A:
+    O(dT + 3d'd) extra against O(d'dT)). The trend holds when rho / rho_model stays within
+    a constant band wherever the projection runs at its tensor-core rate."""
+    lin = wl.layers[0]
+    d, d_out = lin.d, lin.d_out
+    res = {}
+    for T in Ts:
+        Xb = synthetic.as_bf16(synthetic.draw_layer(T, d, 8, seed=600 + T)[0])
+        nsets = 3 if T <= 4096 else 2
+        Xs = [Xb.to(dev) for _ in range(nsets)]
+        Ws = [Wb.to(dev) for _ in range(nsets)]
+        ws = ttq.alloc_workspace(T, d, d_out, cfg, dev)
+        outs = [ttq.linear_prefill(Xs[i], Ws[i], cfg, ws=ws) for i in range(nsets)]
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(reps)]
+        for i in range(reps):
+            ttq.set_trace_events(evs[i])
+            k = i % nsets
+            ttq.linear_prefill(Xs[k], Ws[k], cfg, out=outs[k], ws=ws)
+        torch.cuda.synchronize()
+        ttq.set_trace_events(None)
+        med = lambda a, b: statistics.median(e[a].elapsed_time(e[b]) for e in evs) * 1e3  # noqa: E731
+        t_stats, t_req, t_gemm = med(0, 1), med(2, 3), med(3, 5)
+        rho = (t_stats + t_req) / t_gemm
+        rho_model = 1.0 / d_out + 3.0 / T
+        res[f"T{T}"] = {"stats_us": round(t_stats, 2), "fold_requant_us": round(t_req, 2),
+                        "gemm_us": round(t_gemm, 2), "rho": round(rho, 5), "rho_model": round(rho_model, 6),
+                        "rho_over_model": round(rho / rho_model, 2), "rho_T": round(rho * T, 1)}
+        del Xs, Ws, outs, ws
+        torch.cuda.empty_cache()
+    ratios = [v["rho_over_model"] for k, v in res.items() if int(k[1:]) >= 1024]
+    res["band_T_ge_1024"] = round(max(ratios) / min(ratios), 3) if ratios else None
+    res["rho_decreasing"] = all(res[f"T{a}"]["rho"] > res[f"T{b}"]["rho"] for a, b in zip(Ts, Ts[1:]))
+    assert ttq.device_status() == 0
+    return res
+
+
+def set_roofline_us(layers, T, hbm_peak, tc_peak):
+    """Lower bound of one prompt through a set of TTQ linears, stage by stage (the stages
+    of a linear depend on each other): statistic 2 B per X element; fold and
+    re-quantization 4 B per X element plus 2 + q/8 + 4/g B per weight; low-rank U = X A^T
+    2 B per X element; projection the larger of 2 T d d' (+ 2 T r (d + d')) flops at the
+    tensor peak and its bytes (X' 2 B per element, codes and scale/zero q/8 + 4/g B per
+    weight, Y 2 B per element) at the HBM peak. Peaks in GB/s and TFLOP/s."""
+    t = 0.0
+    for d, d_out, q, g, r in layers:
+        hb = 2 * T * d + 4 * T * d + (2 + q / 8 + 4 / g) * d * d_out + (2 * T * d if r else 0)
+        t += hb / (hbm_peak * 1e3)
+        fl = 2.0 * T * d * d_out + 2.0 * T * r * (d + d_out)
+        gb = 2 * T * d + (q / 8 + 4 / g) * d * d_out + 2 * T * d_out
+        t += max(fl / (tc_peak * 1e6), gb / (hbm_peak * 1e3))
+    return t
+
+
+def workload_set_leg(torch, ttq, name, dev, hbm_peak, tc_peak, g=None, n=8):
+    """One prompt of T tokens through every linear of a workload's layer set (each linear
+    with its own seeded X and W, not chained; statistic, re-quantization and projection
+    per linear), L2 flushed before each prompt, timed as the difference of two CUDA graphs
+    (n x (flush, set) and n x flush). With r > 0 the static factors are the top-r fp64 SVD
+    of each weight (set-up, untimed) and the residual is re-quantized."""
+    wl = synthetic.WORKLOADS[name]
+    g = g or wl.g
+    T = wl.T
+    Ls = []
+    need = 0
+    for i, lin in enumerate(wl.layers):
+        X, W = synthetic.draw_layer(T, lin.d, lin.d_out, wl.layer_seed(i))
+        Xb, Wb = synthetic.as_bf16(X), synthetic.as_bf16(W)
+        A = B = None
+        if wl.r > 0:
+            B, A, Wb = lowrank_factors(Wb, wl.r, device=dev)
+        cfg = ttq.make_config(wl.q, g, wl.alpha, wl.lam, wl.p, wl.r)
+        need = max(need, ttq.workspace_size(T, lin.d, lin.d_out, cfg))
+        Ls.append({"X": Xb.to(dev), "W": Wb.to(dev), "A": A, "B": B, "cfg": cfg, "out": None})
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    for L in Ls:
+        L["out"] = ttq.linear_prefill(L["X"], L["W"], L["cfg"], L["A"], L["B"], ws=ws)
+    torch.cuda.synchronize()
+
+    def step(st):
+        for L in Ls:
+            ttq.linear_prefill(L["X"], L["W"], L["cfg"], L["A"], L["B"], out=L["out"], ws=ws, stream=st)
+
+    flush = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    t_us = graph_step_us(torch, step, flush, sink, n=n)
+    assert ttq.device_status() == 0
+    roof = set_roofline_us([(lin.d, lin.d_out, wl.q, g, wl.r) for lin in wl.layers], T, hbm_peak, tc_peak)
+    flops = sum(2.0 * T * lin.d * lin.d_out for lin in wl.layers)
+    del Ls, ws, flush
+    torch.cuda.empty_cache()
+    return {"linears": [f"{lin.name} {lin.d}->{lin.d_out}" for lin in wl.layers], "T": T, "q": wl.q, "g": g,
+            "alpha": wl.alpha, "r": wl.r, "us_per_prompt": round(t_us, 2), "k_tokens_per_s": round(T / t_us * 1e3, 2),
+            "projection_TFLOPs": round(flops / (t_us * 1e-6) / 1e12, 1), "roofline_us": round(roof, 2),
+            "frac_of_roofline": round(roof / t_us, 4), "l2": "flushed (256 MB read) before each prompt"}
+
 
 def decoder_leg(torch, ttq, dev, K=3):
     """The chained decoder stack (Qwen3-8B shapes: 36 layers, 4 TTQ linears each, random

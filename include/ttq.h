@@ -86,6 +86,16 @@ TTQ_API size_t ttq_codes_words(int64_t d_out, int64_t d, int32_t q);
 TTQ_API ttq_status ttq_workspace_size(int64_t T, int64_t d, int64_t d_out, const ttq_config* cfg,
                               size_t* bytes);
 
+/* Where the folded activations sit in the workspace of ttq_linear_prefill (and of
+ * ttq_linear_decode with T = b rows when b > 2). Once such a call has run (in stream
+ * order), bytes [*offset, *offset + 2*T*d) of its workspace hold X diag(1/s) as bf16
+ * [T, d] row-major, x'_tj = RN_bf16(x_tj * RN_fp32(1/s_j)): the pre-scaling of the
+ * activations that [DR] section 5 suggests fusing, which the projection multiplies. They
+ * stay there until the workspace is used again. Same arguments and errors as
+ * ttq_workspace_size (d_out >= 1). For inspection and tests. */
+TTQ_API ttq_status ttq_workspace_folded_offset(int64_t T, int64_t d, int64_t d_out, const ttq_config* cfg,
+                                               size_t* offset);
+
 /* Online activation statistics ([DR] section 2 online diagonal D of each prompt;
  * [GDE] section 2 D_ii from the norms of the input rows).
  *   X      device bf16 [T, ld_x] (first d columns used), ld_x >= d, ld_x % 8 == 0

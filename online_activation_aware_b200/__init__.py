@@ -57,6 +57,8 @@ def load_library(path: str = LIB_PATH):
     lib.ttq_codes_words.restype = sz
     lib.ttq_workspace_size.argtypes = [i64, i64, i64, cfgp, ctypes.POINTER(sz)]
     lib.ttq_workspace_size.restype = i32
+    lib.ttq_workspace_folded_offset.argtypes = [i64, i64, i64, cfgp, ctypes.POINTER(sz)]
+    lib.ttq_workspace_folded_offset.restype = i32
     lib.ttq_act_stats.argtypes = [vp, i64, i64, i64, f32, f32, i32, vp, vp, sz, vp]
     lib.ttq_act_stats.restype = i32
     lib.ttq_act_stats_noalloc.argtypes = [vp, i64, i64, i64, f32, f32, i32, vp, vp]
@@ -157,6 +159,15 @@ def workspace_size(T: int, d: int, d_out: int, cfg: Config | None = None) -> int
     _check("ttq_workspace_size",
            load_library().ttq_workspace_size(T, d, d_out, ctypes.byref(cfg) if cfg is not None else None,
                                              ctypes.byref(n)))
+    return int(n.value)
+
+
+def workspace_folded_offset(T: int, d: int, d_out: int, cfg: Config) -> int:
+    """Byte offset of the folded activations X diag(1/s) (bf16 [T, d]) in the workspace of
+    a prefill (or of a decode of more than 2 rows) with these sizes."""
+    n = ctypes.c_size_t(0)
+    _check("ttq_workspace_folded_offset",
+           load_library().ttq_workspace_folded_offset(T, d, d_out, ctypes.byref(cfg), ctypes.byref(n)))
     return int(n.value)
 
 
@@ -355,25 +366,6 @@ def set_trace_events(events):
     arr = (ctypes.c_void_p * len(handles))(*handles)
     set_trace_events._keep = (arr, events)
     _check("ttq_set_trace_events", lib.ttq_set_trace_events(arr, len(handles)))
-
-
-def lowrank_factors(W, r: int):
-    """Host set-up of the static low-rank side path (untimed, once per weight).
-
-    Returns bf16 CPU tensors (B [d_out, r], A [r, d], R [d_out, d]) with B = U_r S_r^(1/2),
-    A = S_r^(1/2) V_r^T from the fp64 SVD of W, and R = W - B A rounded to bf16, the
-    residual that is re-quantized per prompt (paper-daily.com deep reading of TTQ,
-    section 2: W_hat = W_q + BA with SVD-initialised factors, r = 16).
-    """
-    import torch
-
-    Wd = W.detach().to("cpu", torch.float64)
-    U, S, Vh = torch.linalg.svd(Wd, full_matrices=False)
-    root = S[:r].sqrt()
-    Bf = (U[:, :r] * root[None, :]).to(torch.bfloat16)
-    Af = (root[:, None] * Vh[:r, :]).to(torch.bfloat16)
-    R = (Wd - Bf.to(torch.float64) @ Af.to(torch.float64)).to(torch.bfloat16)
-    return Bf.contiguous(), Af.contiguous(), R.contiguous()
 
 
 class TTQLinear:

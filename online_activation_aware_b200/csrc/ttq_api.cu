@@ -203,6 +203,20 @@ ttq_status ttq_workspace_size(int64_t T, int64_t d, int64_t d_out, const ttq_con
   return TTQ_OK;
 }
 
+ttq_status ttq_workspace_folded_offset(int64_t T, int64_t d, int64_t d_out, const ttq_config* cfg,
+                                       size_t* offset) {
+  if (!offset || !cfg) return TTQ_ERR_INVALID_ARG;
+  ttq_status st = check_dims(T, d, d_out);
+  if (st != TTQ_OK) return st;
+  st = check_cfg(cfg, d);
+  if (st != TTQ_OK) return st;
+  int num_sms = 148;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) == TTQ_OK) num_sms = di->num_sms;
+  *offset = ws_layout(T, d, d_out, cfg->r, cfg->q, cfg->g, num_sms).xf_off;
+  return TTQ_OK;
+}
+
 ttq_status ttq_act_stats(const void* X_bf16, int64_t T, int64_t d, int64_t ld_x, float alpha,
                          float lambda, int32_t p, float* s, void* ws, size_t ws_bytes,
                          cudaStream_t stream) {

@@ -244,6 +244,22 @@ def dequant_original(codes, scale, zero, g: int, s) -> np.ndarray:
 # --------------------------------------------------------------------------------------
 
 
+def fold(X, s) -> np.ndarray:
+    """The folded activations X' = RN_bf16(x_tj / s_j) the projection multiplies: the
+    D^(-1/2) of W_hat = Q[W D^(1/2)] D^(-1/2) applied to the activations instead of the
+    weight ([DR §2]; [DR §5] names a kernel that fuses this pre-scaling), stored in bf16.
+
+    X [T, d] holds bf16 values, s fp32 values. The quotient is formed in fp64 and rounded
+    once to bf16. That equals rounding the exact quotient: for a bf16 midpoint m, x - m s
+    is zero or at least 2^-33 |m s| (x has 8 significant bits, m 9 and s 24), far above
+    the 2^-53 relative error of the fp64 division, so that division never moves a
+    quotient onto or across a midpoint.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    return round_bf16(X / np.asarray(s, dtype=np.float64)[None, :])
+
+
+
 def linear(X, s, codes, scale, zero, g: int, A=None, B=None) -> np.ndarray:
     """Y = (X diag(1/s)) w'^T  (+ (X A^T) B^T when low-rank factors are given), fp64.
 
@@ -283,6 +299,9 @@ def overhead_counts(T: int, d: int, d_out: int):
 
 
 def activation_loss(W, W_hat, X) -> float:
-    """L = ||(W - W_hat) X^T||_F^2 for X [T, d] ([DR §2] activation-weighted loss)."""
+    """L = ||(W - W_hat) X^T||_F^2 for W, W_hat [d', d] and X [T, d] ([DR §2] the
+    activation-weighted loss that AWQ-style scaling targets; the pages write it with X as
+    [d, T], channels by tokens, which is the transpose of the layout here). The sum runs
+    over every output channel and token (no mean over T)."""
     E = np.asarray(W, dtype=np.float64) - np.asarray(W_hat, dtype=np.float64)
     return float(np.sum((np.asarray(X, dtype=np.float64) @ E.T) ** 2))

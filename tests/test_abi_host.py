@@ -66,6 +66,22 @@ def test_workspace_size_components(lib):
     assert ttq.workspace_size(4096, 5120, 8192, cfg_r) >= ws_full + 4096 * 64 * 2
 
 
+def test_folded_offset_inside_workspace(lib):
+    # the folded activations (bf16 [T, d]) fit inside the workspace at a 16-byte aligned offset
+    for T, d, d_out, r in ((4096, 5120, 8192, 0), (17, 256, 96, 16), (3, 1024, 300, 8)):
+        cfg = ttq.make_config(4, 32, 0.5, 0.4, r=r)
+        off = ttq.workspace_folded_offset(T, d, d_out, cfg)
+        assert off % 16 == 0
+        assert off + 2 * T * d <= ttq.workspace_size(T, d, d_out, cfg)
+    n = ctypes.c_size_t(0)
+    cfg = ttq.make_config(4, 32, 0.5, 0.4)
+    assert lib.ttq_workspace_folded_offset(16, 64, 8, None, ctypes.byref(n)) == INVALID
+    assert lib.ttq_workspace_folded_offset(16, 64, 8, ctypes.byref(cfg), None) == INVALID
+    assert lib.ttq_workspace_folded_offset(16, 64, 0, ctypes.byref(cfg), ctypes.byref(n)) == INVALID
+    assert lib.ttq_workspace_folded_offset(16, 64, 8, ctypes.byref(ttq.make_config(5, 32, 0.5, 0.4)),
+                                           ctypes.byref(n)) == UNSUPPORTED
+
+
 def _p(v):
     return ctypes.c_void_p(v)
 

@@ -320,3 +320,62 @@ def test_ttq_lowers_activation_loss_against_rtn():
         What = O.dequant_original(out["codes"], out["scale"], out["zero"], 32, out["s32"])
         losses[name] = O.activation_loss(W, What, X)
     assert losses["ttq"] < losses["rtn"]
+
+
+# ---------------------------------------------------------------- activation-weighted loss
+
+
+def test_activation_loss_golden():
+    # hand-worked cases: a transposed operand, a dropped square, a missing cross term or a
+    # mean instead of a sum each gives one of the recorded wrong values instead
+    for case in _load("activation_loss_examples.json")["cases"]:
+        L = O.activation_loss(np.array(case["W"]), np.array(case["W_hat"]), np.array(case["X"]))
+        assert L == case["loss"], case
+        for wrong in case.get("wrong_readings", {}).values():
+            assert wrong != case["loss"]
+
+
+def test_activation_loss_equals_per_token_output_error():
+    # L sums, over tokens, the squared output error of the layer: ||W x_t - W_hat x_t||^2
+    rng = np.random.default_rng(91)
+    W, Wh = rng.standard_normal((5, 7)), rng.standard_normal((5, 7))
+    X = rng.standard_normal((4, 7))
+    want = sum(float(np.sum((W @ X[t] - Wh @ X[t]) ** 2)) for t in range(4))
+    assert abs(O.activation_loss(W, Wh, X) - want) <= 1e-12 * want
+
+
+# ---------------------------------------------------------------- fold
+
+
+def test_fold_exact_rational():
+    # X' = RN_bf16(x / s): against the nearest bf16 value to the exact rational quotient,
+    # found among its two neighbours, ties to the even significand
+    rng = np.random.default_rng(92)
+    x = O.round_bf16(rng.standard_normal(400) * np.exp(rng.uniform(-6, 6, 400)))
+    s = rng.uniform(0.05, 20.0, 400).astype(np.float32)
+    got = O.fold(x[None, :], s)[0]
+    for xi, si, gi in zip(x, s, got):
+        fq = Fraction(float(xi)) / Fraction(float(si))
+        if fq == 0:
+            assert gi == 0
+            continue
+        _, e = np.frexp(float(fq))
+        q = Fraction(2) ** (int(e) - 8)
+        lo = (fq / q).__floor__() * q
+        hi = lo + q
+        if fq - lo < hi - fq:
+            want = lo
+        elif hi - fq < fq - lo:
+            want = hi
+        else:
+            want = lo if (lo / q) % 2 == 0 else hi
+        assert Fraction(float(gi)) == want, (xi, si)
+
+
+def test_fold_hand_values():
+    # 1/3 = 1.0101010101...b x 2^-2: the ninth significant bit and those after it are more
+    # than half an ulp, so it rounds up to 1.0101011b x 2^-2 = 0.333984375; 6/4 = 1.5 is exact;
+    # 1 / 1.0078125 lies between 0.9921875 and 0.99609375, nearer the former
+    X = np.array([[1.0, 6.0, 1.0]])
+    s = np.array([3.0, 4.0, 1.0078125], dtype=np.float32)
+    np.testing.assert_array_equal(O.fold(X, s), [[0.333984375, 1.5, 0.9921875]])
