@@ -521,6 +521,7 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": bench_config(wl, T, r, world),
         "requant_gbs": requant_leg(torch, ttq, Ws, outs, d, d_out, q, g),
+        "act_stats_standalone": act_stats_leg(torch, ttq, Xs, outs, wl, hbm_peak),
         "requant_batched": requant_batched_leg(torch, ttq, Ws, outs, d, d_out, q, g),
         "roofline": roof,
         "kernels": kern,
@@ -673,6 +674,31 @@ def requant_leg(torch, ttq, Ws, outs, d, d_out, q, g, reps=100):
     torch.cuda.synchronize()
     sec = e0.elapsed_time(e1) / 1e3 / reps
     return round(requant_bytes(d, d_out, q, g) / sec / 1e9, 1)
+
+
+def act_stats_leg(torch, ttq, Xs, outs, wl, hbm_peak, reps=200):
+    """GB/s of the statistic alone (the ttq_act_stats entry point: read X, write s),
+    back-to-back launches over the rotating activation sets (larger than L2 together with
+    the weights), CUDA events around the loop."""
+    n = len(Xs)
+    T, d = Xs[0].shape
+
+    def one(i):
+        ttq.act_stats(Xs[i % n], wl.alpha, wl.lam, wl.p, s=outs[i % n]["s"])
+
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(reps):
+        one(i)
+    e1.record()
+    torch.cuda.synchronize()
+    sec = e0.elapsed_time(e1) / 1e3 / reps
+    gbs = stats_bytes(T, d) / sec / 1e9
+    return {"us": round(sec * 1e6, 2), "GBps": round(gbs, 1), "frac": round(gbs / hbm_peak, 4)}
 
 
 def requant_batched_leg(torch, ttq, Ws, outs, d, d_out, q, g, P=4, reps=50):

@@ -81,8 +81,8 @@ TTQ_API size_t ttq_codes_words(int64_t d_out, int64_t d, int32_t q);
  * T = b rows; and ttq_act_stats with d_out = 0) needs for these sizes. For the prefill
  * and decode it holds the folded activations X diag(1/s) in bf16, the low-rank
  * projection X A^T, split-K partial products and the decode GEMV's operands; for
- * ttq_act_stats (d_out = 0) the partial column sums of the statistic. Contents need
- * not be initialised and are not preserved. */
+ * ttq_act_stats (d_out = 0) nothing (0 bytes). Contents need not be initialised and are
+ * not preserved. */
 TTQ_API ttq_status ttq_workspace_size(int64_t T, int64_t d, int64_t d_out, const ttq_config* cfg,
                               size_t* bytes);
 
@@ -100,7 +100,10 @@ TTQ_API ttq_status ttq_workspace_folded_offset(int64_t T, int64_t d, int64_t d_o
  * [GDE] section 2 D_ii from the norms of the input rows).
  *   X      device bf16 [T, ld_x] (first d columns used), ld_x >= d, ld_x % 8 == 0
  *   s      device fp32 [d] output: s_j = (mean_t |x_tj|^p + lambda)^(alpha/p)
- *   ws     device scratch of at least ttq_workspace_size(T, d, 0, ...) bytes
+ *   ws     scratch of ttq_workspace_size(T, d, 0, ...) bytes, which is 0: the reduction
+ *          runs on chip (the row splits of each 256-channel strip form one thread-block
+ *          cluster and add their partial sums in shared memory), so ws may be NULL and
+ *          ws_bytes is ignored; a non-NULL ws must be 16-byte aligned
  * The column sums accumulate in fp32 in a fixed order, so results are deterministic. */
 TTQ_API ttq_status ttq_act_stats(const void* X_bf16, int64_t T, int64_t d, int64_t ld_x, float alpha,
                          float lambda, int32_t p, float* s, void* ws, size_t ws_bytes,

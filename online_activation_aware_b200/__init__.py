@@ -184,11 +184,11 @@ def act_stats(X, alpha: float, lam: float, p: int = 2, s=None, ws=None, stream=N
     T, d = X.shape
     if s is None:
         s = torch.empty(d, dtype=torch.float32, device=X.device)
-    if ws is None:
+    if ws is None and workspace_size(T, d, 0) > 0:
         ws = alloc_workspace(T, d, 0, None, X.device)
     _check("ttq_act_stats", load_library().ttq_act_stats(
         _ptr(X, torch.bfloat16, "X"), T, d, X.stride(0), alpha, lam, p, _ptr(s, torch.float32, "s"),
-        _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)))
+        _ptr(ws, None, "ws"), 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
     return s
 
 

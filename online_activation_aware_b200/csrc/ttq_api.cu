@@ -143,7 +143,7 @@ struct WsLayout {
 WsLayout ws_layout(int64_t T, int64_t d, int64_t d_out, int r, int q, int g, int num_sms) {
   WsLayout L{};
   L.stats_off = 0;
-  L.stats_bytes = round256(ttq::split_partial_bytes(T, d, num_sms));  // per-split partial sums
+  L.stats_bytes = 0;  // the statistic reduces on chip
   L.xf_off = L.stats_off + L.stats_bytes;
   L.xf_bytes = d_out > 0 ? round256(static_cast<size_t>(T) * static_cast<size_t>(d) * 2) : 0;
   L.u_off = L.xf_off + L.xf_bytes;
@@ -226,14 +226,12 @@ ttq_status ttq_act_stats(const void* X_bf16, int64_t T, int64_t d, int64_t ld_x,
   st = check_stats_args(alpha, lambda, p);
   if (st != TTQ_OK) return st;
   if (!X_bf16 || !s) return TTQ_ERR_INVALID_ARG;
-  if (!ws) return TTQ_ERR_WORKSPACE;
-  if (!aligned16(X_bf16) || !aligned16(s) || !aligned16(ws)) return TTQ_ERR_MISALIGNED;
+  if (!aligned16(X_bf16) || !aligned16(s) || (ws && !aligned16(ws))) return TTQ_ERR_MISALIGNED;
+  (void)ws_bytes;  // the statistic reduces on chip and needs no workspace
   DeviceInfo* di = nullptr;
-  const int num_sms = device_info(&di) == TTQ_OK ? di->num_sms : 148;
-  if (ws_bytes < ws_layout(T, d, 0, 0, 4, 128, num_sms).total) return TTQ_ERR_WORKSPACE;
-  if (!di) return TTQ_ERR_CUDA;
-  float* partial = static_cast<float*>(ws);
-  return cuda_status(ttq::launch_act_stats(X_bf16, T, d, ld_x, alpha, lambda, p, s, partial, num_sms, stream));
+  ttq_status dst = device_info(&di);
+  if (dst != TTQ_OK) return dst;
+  return cuda_status(ttq::launch_act_stats(X_bf16, T, d, ld_x, alpha, lambda, p, s, di->num_sms, dev_err(di), stream));
 }
 
 ttq_status ttq_requant(const void* W_bf16, int64_t d_out, int64_t d, const float* s, int32_t q,
@@ -299,7 +297,6 @@ ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const vo
   const WsLayout L = ws_layout(T, d, d_out, cfg->r, cfg->q, cfg->g, di->num_sms);
   if (ws_bytes < L.total) return TTQ_ERR_WORKSPACE;
   auto* base = static_cast<uint8_t*>(ws);
-  float* spart = reinterpret_cast<float*>(base + L.stats_off);
   void* Xf = base + L.xf_off;
   void* U = cfg->r > 0 ? base + L.u_off : nullptr;
   float* upart = cfg->r > 0 ? reinterpret_cast<float*>(base + L.u_off + round256(static_cast<size_t>(T) * 64 * 2))
@@ -310,7 +307,7 @@ ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const vo
   // W -> projection
   cudaError_t e = trace(0, stream);
   if (e == cudaSuccess)
-    e = ttq::launch_act_stats(X_bf16, T, d, d, cfg->alpha, cfg->lambda, cfg->p, s, spart, di->num_sms, stream);
+    e = ttq::launch_act_stats(X_bf16, T, d, d, cfg->alpha, cfg->lambda, cfg->p, s, di->num_sms, dev_err(di), stream);
   if (e == cudaSuccess) e = trace(1, stream);
   if (e == cudaSuccess && cfg->r > 0)
     e = ttq::launch_lowrank_u(X_bf16, T, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
@@ -396,7 +393,6 @@ static BatchLayout batch_layout(const int64_t* T, int32_t prompts, int64_t d, in
   int64_t tokens = 0;
   for (int32_t p = 0; p < prompts; ++p) {
     tokens += T[p];
-    stats = std::max(stats, ttq::split_partial_bytes(T[p], d, num_sms));
     const ttq::GemmPlan pp = ttq::gemm_plan(T[p], d, d_out, cfg->q, cfg->g, num_sms);
     gpart = std::max(gpart, ttq::gemm_partial_bytes(pp, T[p], d_out));
   }
@@ -468,7 +464,6 @@ ttq_status ttq_linear_prefill_batched(const void* X_bf16, const int64_t* T, int3
   const BatchLayout L = batch_layout(T, prompts, d, d_out, cfg, di->num_sms);
   if (ws_bytes < L.total) return TTQ_ERR_WORKSPACE;
   auto* base = static_cast<uint8_t*>(ws);
-  float* spart = reinterpret_cast<float*>(base + L.stats_off);
   auto* Xf = reinterpret_cast<__nv_bfloat16*>(base + L.xf_off);
   void* U = cfg->r > 0 ? base + L.u_off : nullptr;
   float* upart = cfg->r > 0 ? reinterpret_cast<float*>(base + L.upart_off) : nullptr;
@@ -481,8 +476,8 @@ ttq_status ttq_linear_prefill_batched(const void* X_bf16, const int64_t* T, int3
   // each prompt's statistic and folded activations
   int64_t off = 0;
   for (int32_t p = 0; p < prompts && e == cudaSuccess; ++p) {
-    e = ttq::launch_act_stats(Xb + off * d, T[p], d, d, cfg->alpha, cfg->lambda, cfg->p, s + p * d, spart,
-                              di->num_sms, stream);
+    e = ttq::launch_act_stats(Xb + off * d, T[p], d, d, cfg->alpha, cfg->lambda, cfg->p, s + p * d, di->num_sms,
+                              dev_err(di), stream);
     if (e == cudaSuccess) e = ttq::launch_fold(Xb + off * d, T[p], d, d, s + p * d, Xf + off * d, stream);
     off += T[p];
   }

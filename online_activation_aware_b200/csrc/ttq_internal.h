@@ -27,16 +27,18 @@ struct StatsPlan {
 // Plan of the single-kernel statistic with arrival counters (launch_act_stats_capped).
 StatsPlan stats_plan(int64_t T, int64_t d);
 
-// Row split of the statistic over `num_sms` SMs: blocks of 256 columns x rows_per_split
-// rows, chosen to balance the rows each SM reduces. The partial sums take
-// split_partial_bytes() of workspace.
-StatsPlan split_plan(int64_t T, int64_t d, int num_sms);
-size_t split_partial_bytes(int64_t T, int64_t d, int num_sms);
+// Row split of the single-launch statistic: blocks of 256 columns x rows_per_split rows,
+// about two blocks per SM, the nsplit <= kStatsMaxSplit blocks of a column strip forming
+// one thread-block cluster.
+constexpr int kStatsMaxSplit = 16;
+StatsPlan cluster_plan(int64_t T, int64_t d, int num_sms);
 
-// s = (mean_t |x|^p + lambda)^(alpha/p): per-split partial sums into `partial` (workspace),
-// then a finishing kernel (programmatic dependent launch) that adds them in a fixed order.
+// s = (mean_t |x|^p + lambda)^(alpha/p) in one launch with no scratch memory (the row
+// splits of a strip reduce through distributed shared memory); launched with programmatic
+// stream serialization and lets the next kernel launch at once.
+// X streams through a TMA ring in shared memory (every wait bounded by err.wait_ns).
 cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d, int64_t ld_x, float alpha, float lambda, int p,
-                             float* s, float* partial, int num_sms, cudaStream_t stream);
+                             float* s, int num_sms, const DevErr& err, cudaStream_t stream);
 
 // Same statistic, with at most `max_partial_floats` fp32 partial sums: the row split is
 // reduced until nsplit * d fits (used where the scratch has a fixed size).

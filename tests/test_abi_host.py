@@ -57,8 +57,8 @@ def test_workspace_size_components(lib):
     cfg = ttq.make_config(4, 128, 0.5, 0.4)
     ws_stats = ttq.workspace_size(4096, 5120, 0)
     ws_full = ttq.workspace_size(4096, 5120, 8192, cfg)
-    # the statistic alone keeps its partial column sums in the workspace
-    assert ws_stats >= 5120 * 4
+    # the statistic alone reduces on chip and needs no workspace
+    assert ws_stats == 0
     # the prefill's fused statistic + fold reduces on chip; the folded activations alone
     # are T * d bf16
     assert ws_full >= 4096 * 5120 * 2
@@ -113,9 +113,8 @@ def test_act_stats_argument_errors(lib):
     assert lib.ttq_act_stats(_p(a), 8, 64, 64, f(0.5), f(0.0), 2, _p(a), _p(a), 1 << 20, None) == INVALID
     assert lib.ttq_act_stats(_p(a), 8, 64, 32, f(0.5), f(0.4), 2, _p(a), _p(a), 1 << 20, None) == INVALID
     assert lib.ttq_act_stats(_p(a), 8, 60, 64, f(0.5), f(0.4), 2, _p(a), _p(a), 1 << 20, None) == INVALID
-    assert lib.ttq_act_stats(_p(a), 8, 64, 64, f(0.5), f(0.4), 2, _p(a), None, 1 << 20, None) == WORKSPACE
     assert lib.ttq_act_stats(_p(a + 4), 8, 64, 64, f(0.5), f(0.4), 2, _p(a), _p(a), 1 << 20, None) == MISALIGNED
-    assert lib.ttq_act_stats(_p(a), 8, 64, 64, f(0.5), f(0.4), 2, _p(a), _p(a), 16, None) == WORKSPACE
+    assert lib.ttq_act_stats(_p(a), 8, 64, 64, f(0.5), f(0.4), 2, _p(a), _p(a + 4), 16, None) == MISALIGNED
     assert lib.ttq_act_stats(_p(a), 0, 64, 64, f(0.5), f(0.4), 2, _p(a), _p(a), 1 << 20, None) == INVALID
 
 

@@ -268,7 +268,7 @@ def test_gemm_parity_with_oracle_codes(T, d, d_out, q, g, r):
     Yg = gpu_linear_with_oracle_codes(Xb, s32, oc, osc, oz, A, B, q, g, r, d_out)
     Yo = O.linear(X, s32, oc, osc, oz, g, A, B)
     assert np.isfinite(Yg).all()
-    check_y(Yg, Yo, err)
+    check_y(Yg, Yo)
 
 
 # ------------------------------------------------------------------ full prefill
@@ -301,7 +301,7 @@ def prefill_check(T, d, d_out, q, g, alpha, r, seed, rows=None, p=2):
     Ao = A
     Yo = O.linear(X, s32, oc, osc, oz, g, Ao, B[rows] if B is not None else None)
     Yg = out["Y"].float().cpu().numpy()[:, rows]
-    check_y(Yg, Yo, err)
+    check_y(Yg, Yo)
     return out
 
 
@@ -341,7 +341,7 @@ def test_prefill_batched_matches_single_prompts(Ts, d, d_out, q, g, r):
         Yo = O.linear(Xvs[p], s32, oc, osc, oz, g, A, B)
         Yg = out["Y"][off:off + Tp].float().cpu().numpy()
         assert np.isfinite(Yg).all()
-        check_y(Yg, Yo, (p, err))
+        check_y(Yg, Yo, p)
         off += Tp
 
 
@@ -424,7 +424,7 @@ def test_decode_qwen3_32b_qproj(b):
     xtb = synthetic.as_bf16(xt)
     Yg = gpu_linear_with_oracle_codes(xtb, s32, oc, osc, oz, None, None, q, g, 0, d_out)
     Yo = O.linear(synthetic.bf16_values(xtb), s32, oc, osc, oz, g)
-    check_y(Yg, Yo, err)
+    check_y(Yg, Yo)
 
 
 def test_prefill_then_decode_reuses_codes():
@@ -456,7 +456,7 @@ def test_decode_few_tokens_parity(b, q, g, r, d_out):
     Yg = gpu_linear_with_oracle_codes(xt, s32, oc, osc, oz, A, B, q, g, r, d_out)
     Yo = O.linear(synthetic.bf16_values(xt), s32, oc, osc, oz, g, A, B)
     assert np.isfinite(Yg).all()
-    check_y(Yg, Yo, err)
+    check_y(Yg, Yo)
 
 
 @pytest.mark.parametrize("b,d,d_out,q,g,r", [
@@ -476,7 +476,7 @@ def test_decode_parity_shapes(b, d, d_out, q, g, r):
     Yg = gpu_linear_with_oracle_codes(xt, s32, oc, osc, oz, A, B, q, g, r, d_out)
     Yo = O.linear(synthetic.bf16_values(xt), s32, oc, osc, oz, g, A, B)
     assert np.isfinite(Yg).all()
-    check_y(Yg, Yo, err)
+    check_y(Yg, Yo)
 
 
 @pytest.mark.parametrize("P,b,d,d_out,q,g,r", [
@@ -513,7 +513,7 @@ def test_decode_batched_requests_match_oracle(P, b, d, d_out, q, g, r):
     Yg = Yg.float().cpu().numpy()
     assert np.isfinite(Yg).all()
     for p in range(P):
-        check_y(Yg[p], Ys[p], (p, err))
+        check_y(Yg[p], Ys[p], p)
 
 
 @pytest.mark.parametrize("b,d", [(1, 992), (2, 160), (2, 96), (3, 992), (8, 160), (7, 96)])
@@ -524,7 +524,7 @@ def test_decode_small_hidden_parity(b, d):
     xt = synthetic.as_bf16(synthetic.draw_tokens(b, d, seed=9 + b))
     Yg = gpu_linear_with_oracle_codes(xt, s32, oc, osc, oz, None, None, q, g, 0, d_out)
     Yo = O.linear(synthetic.bf16_values(xt), s32, oc, osc, oz, g)
-    check_y(Yg, Yo, err)
+    check_y(Yg, Yo)
 
 
 @pytest.mark.parametrize("b", [1, 8])
@@ -560,7 +560,7 @@ def test_decode_far_zero_points(g, b):
     xt = synthetic.as_bf16(synthetic.draw_tokens(b, d, seed=12))
     Yg = gpu_linear_with_oracle_codes(xt, s32, oc, osc, oz, None, None, q, g, 0, d_out)
     Yo = O.linear(synthetic.bf16_values(xt), s32, oc, osc, oz, g)
-    check_y(Yg, Yo, err)
+    check_y(Yg, Yo)
 
 
 # ------------------------------------------------------------------ fold (X diag(1/s) in bf16)
