@@ -477,13 +477,18 @@ def main():
     value = whole_job_ktoks(T, K, world, t_max_ms)
 
     plan_split = stage_ms["reduce"] > 0.002
-    # kernels of ours per step: statistic partial sums, statistic finish, (low-rank X A^T
-    # partial products and their reduction), fold + requant, tensor-core GEMM, (split-K
-    # reduce)
-    launches_per_step = 4 + (2 if r > 0 else 0) + (1 if plan_split else 0)
+    # kernels of ours per step: statistic, (low-rank X A^T partial products and their
+    # reduction), fold + requant, tensor-core GEMM, (split-K reduce)
+    launches_per_step = 3 + (2 if r > 0 else 0) + (1 if plan_split else 0)
+    flush = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)  # 256 MB read flushes L2
+    sink = torch.empty((), dtype=torch.float32, device=dev)
 
+    # the statistic's kernel timed on its own (graph difference, L2 flushed): the traced
+    # stage adds the gap that the event between two launches opens
+    stats_sa = act_stats_leg(torch, ttq, Xs, outs, wl, hbm_peak, flush, sink)
     kern = {
-        "stats": {"ms": stage_ms["stats"], "bound": "hbm", "bytes": stats_bytes(T, d)},
+        "stats": {"ms": stats_sa["us"] / 1e3, "bound": "hbm", "bytes": stats_bytes(T, d),
+                  "method": "ttq_act_stats alone, graph difference, L2 flushed"},
         "fold_requant": {"ms": stage_ms["fold_requant"], "bound": "hbm",
                          "bytes": fold_bytes(T, d) + requant_bytes(d, d_out, q, g)},
         **({"lowrank_u": {"ms": stage_ms["lowrank_u"], "bound": "hbm", "bytes": T * d * 2 + r * d * 2 + T * 128}}
@@ -509,7 +514,7 @@ def main():
                 "algorithmic": f"2*T*d*d_out flops per launch = {dk['flops']:.4g}",
                 "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"}
     else:
-        roof = {"kernel": {"fold_requant": "requant_kernel", "stats": "stats_partial_kernel",
+        roof = {"kernel": {"fold_requant": "requant_kernel", "stats": "stats_tma_kernel",
                            "lowrank_u": "lowrank_u_kernel"}[dom],
                 "bound": "hbm", "achieved": dk["GBps"], "peak": hbm_peak, "unit": "GB/s", "frac": dk["frac"],
                 "traffic": profiled_traffic(dom, wkey), "algorithmic": f"{dk['bytes']} bytes per launch",
@@ -520,8 +525,8 @@ def main():
         "warmup": args.warmup, "ms_per_step": round(t_max_ms / K, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": bench_config(wl, T, r, world),
-        "requant_gbs": requant_leg(torch, ttq, Ws, outs, d, d_out, q, g),
-        "act_stats_standalone": act_stats_leg(torch, ttq, Xs, outs, wl, hbm_peak),
+        "requant_gbs": requant_leg(torch, ttq, Ws, outs, d, d_out, q, g, flush, sink),
+        "stage_trace_ms": {k_: round(v, 5) for k_, v in stage_ms.items()},
         "requant_batched": requant_batched_leg(torch, ttq, Ws, outs, d, d_out, q, g),
         "roofline": roof,
         "kernels": kern,
@@ -652,53 +657,46 @@ def graph_step_us(torch, step, flush, sink, n=32):
     return (ta - tb) * 1e3 / n
 
 
-def requant_leg(torch, ttq, Ws, outs, d, d_out, q, g, reps=100):
+def requant_leg(torch, ttq, Ws, outs, d, d_out, q, g, flush, sink):
     """GB/s of the re-quantization alone (the ttq_requant entry point: read W and s, write
-    codes, scale and zero), back-to-back launches over the rotating weight sets (each set
-    larger than L2 together with the others), CUDA events around the loop."""
+    codes, scale and zero) with L2 flushed before each launch, device time from the
+    difference of two CUDA graphs (no host launch latency)."""
     n = len(Ws)
+    ctr = [0]
 
-    def one(i):
+    def one(st):
+        i = ctr[0]
+        ctr[0] += 1
         o = outs[i % n]
-        ttq.requant(Ws[i % n], o["s"], q, g, codes=o["codes"], scale=o["scale"], zero=o["zero"])
+        ttq.requant(Ws[i % n], o["s"], q, g, codes=o["codes"], scale=o["scale"], zero=o["zero"], stream=st)
 
-    for i in range(3):
-        one(i)
+    for _ in range(3):
+        one(torch.cuda.current_stream())
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(reps):
-        one(i)
-    e1.record()
-    torch.cuda.synchronize()
-    sec = e0.elapsed_time(e1) / 1e3 / reps
-    return round(requant_bytes(d, d_out, q, g) / sec / 1e9, 1)
+    us = graph_step_us(torch, one, flush, sink)
+    return round(requant_bytes(d, d_out, q, g) / (us * 1e-6) / 1e9, 1)
 
 
-def act_stats_leg(torch, ttq, Xs, outs, wl, hbm_peak, reps=200):
-    """GB/s of the statistic alone (the ttq_act_stats entry point: read X, write s),
-    back-to-back launches over the rotating activation sets (larger than L2 together with
-    the weights), CUDA events around the loop."""
+def act_stats_leg(torch, ttq, Xs, outs, wl, hbm_peak, flush, sink):
+    """The statistic alone (the ttq_act_stats entry point: read X, write s) with L2 flushed
+    before each launch, device time from the difference of two CUDA graphs (launches with
+    flushes, flushes alone), so host launch latency does not enter."""
     n = len(Xs)
     T, d = Xs[0].shape
+    ctr = [0]
 
-    def one(i):
-        ttq.act_stats(Xs[i % n], wl.alpha, wl.lam, wl.p, s=outs[i % n]["s"])
+    def one(st):
+        i = ctr[0]
+        ctr[0] += 1
+        ttq.act_stats(Xs[i % n], wl.alpha, wl.lam, wl.p, s=outs[i % n]["s"], stream=st)
 
-    for i in range(3):
-        one(i)
+    for _ in range(3):
+        one(torch.cuda.current_stream())
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(reps):
-        one(i)
-    e1.record()
-    torch.cuda.synchronize()
-    sec = e0.elapsed_time(e1) / 1e3 / reps
-    gbs = stats_bytes(T, d) / sec / 1e9
-    return {"us": round(sec * 1e6, 2), "GBps": round(gbs, 1), "frac": round(gbs / hbm_peak, 4)}
+    us = graph_step_us(torch, one, flush, sink)
+    gbs = stats_bytes(T, d) / (us * 1e-6) / 1e9
+    return {"us": round(us, 2), "GBps": round(gbs, 1), "frac": round(gbs / hbm_peak, 4),
+            "method": "graph difference, L2 flushed before each launch"}
 
 
 def requant_batched_leg(torch, ttq, Ws, outs, d, d_out, q, g, P=4, reps=50):
