@@ -87,7 +87,7 @@ TTQ_API ttq_status ttq_workspace_size(int64_t T, int64_t d, int64_t d_out, const
                               size_t* bytes);
 
 /* Where the folded activations sit in the workspace of ttq_linear_prefill (and of
- * ttq_linear_decode with T = b rows when b > 8). Once such a call has run (in stream
+ * ttq_linear_decode with T = b rows when b > 2). Once such a call has run (in stream
  * order), bytes [*offset, *offset + 2*T*d) of its workspace hold X diag(1/s) as bf16
  * [T, d] row-major, x'_tj = RN_bf16(x_tj * RN_fp32(1/s_j)): the pre-scaling of the
  * activations that [DR] section 5 suggests fusing, which the projection multiplies. They
@@ -220,7 +220,7 @@ TTQ_API ttq_status ttq_linear_prefill_batched(const void* X_bf16, const int64_t*
  * multi-request decode that [DR] section 5 leaves open (every request of a serving batch
  * carries its own D, hence its own codes). Request p computes
  * Y_p = (X_p diag(1/s_p)) deq(codes_p)^T + (X_p A^T) B^T with the shared static A, B; its
- * result equals ttq_linear_decode on request p's operands. With b <= 8 tokens per request
+ * result equals ttq_linear_decode on request p's operands. With b <= 2 tokens per request
  * every request runs in the same two launches (statistic fold and CUDA-core GEMV over all
  * requests' codes); with more tokens the requests run one after another.
  *   X      device bf16 [P, b, d];  Y  device bf16 [P, b, d_out] output

@@ -1,25 +1,24 @@
-// Decode steps with few tokens (b <= 8): the projection as a CUDA-core GEMV that streams
+// Decode steps with few tokens (b <= 2): the projection as a CUDA-core GEMV that streams
 // the prefill's packed codes once (paper-daily.com deep reading of TTQ, section 6:
 // quantisation parameters are computed at prefill and reused at decode).
 //
 // For a weight row i and a group G of g inputs, cut into 32-input units V:
 //   sum_{k in G} x'_tk (c_ik - z) sigma
 //     = sigma * sum_{V in G} ( sum_{k in V} (128 + c_ik) x'_tk - (128 + z) sum_{k in V} x'_tk )
-// so each weight costs one byte permute (128 + c as an fp32, exact) and B/2 two-wide FMAs
-// (fma.rn.f32x2: pairs of inputs for one token; token pairs of each input for B = 2, 4, 8
-// tokens, b rounded up to the block and the missing tokens zero);
+// so each weight costs one byte permute (128 + c as an fp32, exact) and half of a two-wide
+// FMA (fma.rn.f32x2: pairs of inputs for one token, the token pair for two);
 // each unit is finished on its own (scale and zero of its group), so a lane may take any
 // set of units; the unit sums of x' come with x' from a small prep kernel.
 //
-// Layout of the work: one warp per 4 weight rows (2 at B = 8), the 32 lanes spanning the inputs (lane j
+// Layout of the work: one warp per 4 weight rows, the 32 lanes spanning the inputs (lane j
 // takes the rows' 32-input units j, j + 32, ...), so that each row's lanes read contiguous
 // codes per step (16-byte loads that bypass L1) and every x' value a lane loads (16-byte
 // loads through L1, contiguous across the warp) serves 4 weights: a load's cost is its
 // per-lane register writeback, so the reuse in registers is what keeps x' traffic below
 // the code traffic (2 rows a warp measured slower at every shape of a Qwen3-8B layer).
 // The codes of the next kDepth units are in flight while one is consumed; the 32 lanes are
-// summed by shuffles in a fixed order. CTAs of 2 warps (up to 8 on an SM at 128 registers a
-// thread) stage their rows' scale and zero in shared memory. x' (fp32, chunk-major, see xoff)
+// summed by shuffles in a fixed order. CTAs of 8 rows (up to 8 on an SM at 128 registers a
+// thread) stage the rows' scale and zero in shared memory. x' (fp32, chunk-major, see xoff)
 // and the unit sums come from a prep kernel chained to the GEMV by programmatic dependent
 // launch: the GEMV issues its first code loads before waiting for x'.
 #include "ttq_internal.h"
@@ -28,17 +27,10 @@ namespace ttq {
 
 namespace {
 
-constexpr int kGemvThreads = 64;  // 2 warps
-
-// Rows a warp takes and units of codes in flight per lane, by token block B: four rows share
-// every x' load up to B = 4; at B = 8 two rows (the accumulators of 4 rows x 8 tokens and
-// the x' of 8 tokens would not fit the register budget next to the codes in flight).
-template <int B>
-struct GemvShape {
-  static constexpr int R = B <= 4 ? 4 : 2;
-  static constexpr int kDepth = B <= 2 ? 4 : (B == 4 ? 3 : 4);
-  static constexpr int kRowsPerCta = R * kGemvThreads / 32;
-};
+constexpr int kRowsPerWarp = 4;
+constexpr int kDepth = 4;  // 32-input units of codes in flight per lane (for each of its rows)
+constexpr int kGemvThreads = 64;                                  // 2 warps
+constexpr int kRowsPerCta = kRowsPerWarp * kGemvThreads / 32;     // 8
 
 __device__ __forceinline__ float code_plus_128f(uint32_t x, int b) {
   return __uint_as_float(__byte_perm(x, 0x43000000u, 0x7044u + (static_cast<unsigned>(b) << 8)));
@@ -171,10 +163,7 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
     if (U != nullptr) U += rq * nb * 64;
     Y += rq * nb * d_out;
   }
-  constexpr int R = GemvShape<B>::R;
-  constexpr int kDepth = GemvShape<B>::kDepth;
-  constexpr int kRowsPerCta = GemvShape<B>::kRowsPerCta;
-  constexpr int BP = B == 1 ? 1 : B / 2;  // two-wide accumulators per row
+  constexpr int R = kRowsPerWarp;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int upr = d >> 5;                            // 32-input units per row
@@ -241,13 +230,11 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
       const int st = s0 + hb;
       if (st < nsteps) {
         const int u = lane + 32 * st;
-        // two-wide accumulators: one token, pairs of inputs (even, odd); B >= 2 tokens,
-        // the token pairs of each input
-        uint64_t acc2[R][BP];
+        // two-wide accumulators: one token, pairs of inputs (even, odd); two tokens, the
+        // token pair of each input
+        uint64_t acc2[R];
 #pragma unroll
-        for (int i = 0; i < R; ++i)
-#pragma unroll
-          for (int tp = 0; tp < BP; ++tp) acc2[i][tp] = 0ull;
+        for (int i = 0; i < R; ++i) acc2[i] = 0ull;
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
           // x' of inputs 4 c4 .. 4 c4 + 3 of unit u for all B tokens
@@ -258,46 +245,36 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
             const float4 v = __ldg(reinterpret_cast<const float4*>(xb + 4 * i2));
             x[4 * i2] = v.x; x[4 * i2 + 1] = v.y; x[4 * i2 + 2] = v.z; x[4 * i2 + 3] = v.w;
           }
-          uint64_t xv[4][BP];
+          uint64_t xv[4];
           if (B == 1) {
-            xv[0][0] = f2(x[0], x[1]);
-            xv[1][0] = f2(x[2], x[3]);
+            xv[0] = f2(x[0], x[1]);
+            xv[1] = f2(x[2], x[3]);
           } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-#pragma unroll
-              for (int tp = 0; tp < BP; ++tp) xv[e][tp] = f2(x[e * B + 2 * tp], x[e * B + 2 * tp + 1]);
+            for (int e = 0; e < 4; ++e) xv[e] = f2(x[e * B], x[e * B + 1]);
           }
 #pragma unroll
           for (int i = 0; i < R; ++i) {
             float f[4];
             codes4<Q>(cb[hb][i], c4, f);
             if (B == 1) {
-              acc2[i][0] = ffma2(f2(f[0], f[1]), xv[0][0], acc2[i][0]);
-              acc2[i][0] = ffma2(f2(f[2], f[3]), xv[1][0], acc2[i][0]);
+              acc2[i] = ffma2(f2(f[0], f[1]), xv[0], acc2[i]);
+              acc2[i] = ffma2(f2(f[2], f[3]), xv[1], acc2[i]);
             } else {
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const uint64_t ff = f2(f[e], f[e]);
-#pragma unroll
-                for (int tp = 0; tp < BP; ++tp) acc2[i][tp] = ffma2(ff, xv[e][tp], acc2[i][tp]);
-              }
+              for (int e = 0; e < 4; ++e) acc2[i] = ffma2(f2(f[e], f[e]), xv[e], acc2[i]);
             }
           }
         }
         float acc[R][B];
 #pragma unroll
         for (int i = 0; i < R; ++i) {
+          const float2 a = f2_unpack(acc2[i]);
           if (B == 1) {
-            const float2 a = f2_unpack(acc2[i][0]);
             acc[i][0] = __fadd_rn(a.x, a.y);
           } else {
-#pragma unroll
-            for (int tp = 0; tp < BP; ++tp) {
-              const float2 a = f2_unpack(acc2[i][tp]);
-              acc[i][2 * tp] = a.x;
-              acc[i][2 * tp + 1] = a.y;
-            }
+            acc[i][0] = a.x;
+            acc[i][B - 1] = a.y;
           }
         }
         if (st + kDepth < nsteps) {  // refill the slot just consumed, kDepth units ahead
@@ -398,8 +375,7 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __nv_bfloat16* _
   if (lane == 0) usum[static_cast<int64_t>(v) * B + t] = sum;
 }
 
-// Token block of the GEMV: b rounded up to 1, 2, 4 or 8 (rows past b are zero in x').
-int gemv_tokens(int64_t b) { return b <= 1 ? 1 : (b <= 2 ? 2 : (b <= 4 ? 4 : 8)); }
+int gemv_tokens(int64_t b) { return b <= 1 ? 1 : 2; }
 
 size_t round16(size_t v) { return (v + 15) & ~static_cast<size_t>(15); }
 
@@ -422,7 +398,6 @@ cudaError_t launch_qb(const DecodeArgs& a, uint8_t* ws, cudaStream_t stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  constexpr int kRowsPerCta = GemvShape<B>::kRowsPerCta;
   const size_t smem = static_cast<size_t>(kRowsPerCta) * (a.d / a.g) * sizeof(float2);
   if (smem > 48 * 1024) {
     e = cudaFuncSetAttribute(decode_gemv_kernel<Q, B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -450,12 +425,8 @@ cudaError_t launch_qb(const DecodeArgs& a, uint8_t* ws, cudaStream_t stream) {
 
 template <int Q>
 cudaError_t launch_q(const DecodeArgs& a, uint8_t* ws, cudaStream_t stream) {
-  switch (gemv_tokens(a.b)) {
-    case 1: return launch_qb<Q, 1>(a, ws, stream);
-    case 2: return launch_qb<Q, 2>(a, ws, stream);
-    case 4: return launch_qb<Q, 4>(a, ws, stream);
-    default: return launch_qb<Q, 8>(a, ws, stream);
-  }
+  if (gemv_tokens(a.b) == 1) return launch_qb<Q, 1>(a, ws, stream);
+  return launch_qb<Q, 2>(a, ws, stream);
 }
 
 }  // namespace

@@ -135,7 +135,7 @@ struct WsLayout {
   size_t xf_off, xf_bytes;
   size_t u_off, u_bytes;
   size_t part_off, part_bytes;
-  size_t dec_off, dec_bytes;  // CUDA-core decode (b <= 8): x' and its unit sums
+  size_t dec_off, dec_bytes;  // CUDA-core decode (b <= 2): x' and its unit sums
   size_t total;
   ttq::GemmPlan plan;
 };
@@ -508,7 +508,7 @@ ttq_status ttq_linear_prefill_batched(const void* X_bf16, const int64_t* T, int3
   return cuda_status(e);
 }
 
-// Workspace of a batched decode whose requests run on the CUDA-core GEMV (b <= 8): U for
+// Workspace of a batched decode whose requests run on the CUDA-core GEMV (b <= 2): U for
 // all P * b rows and its K-split partials, then one GEMV slice per request.
 static size_t decode_batched_gemv_bytes(int32_t requests, int64_t b, int64_t d, int r, int num_sms) {
   const int64_t rows = static_cast<int64_t>(requests) * b;

@@ -62,7 +62,7 @@ cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A,
 
 // ---------------------------------------------------------------- decode
 
-constexpr int kGemvMaxTokens = 8;  // larger decode batches run on the tensor cores
+constexpr int kGemvMaxTokens = 2;  // larger decode batches run on the tensor cores
 struct DecodeArgs {
   const void* X;          // bf16 [b, d] new tokens (not folded)
   const float* s;         // fp32 [d] the prefill's statistic
@@ -77,7 +77,7 @@ struct DecodeArgs {
   void* Y;                // bf16 [b, d_out]
   int requests;           // batched decode: requests stacked along every per-request operand
 };
-// True when the CUDA-core GEMV handles these decode sizes (b <= 8).
+// True when the CUDA-core GEMV handles these decode sizes (b <= 2).
 bool decode_gemv_ok(int64_t b, int64_t d);
 // Workspace bytes of launch_decode_gemv for one request: x' (fp32, [d][B]) and its
 // 32-input unit sums (a batched decode takes `requests` such slices back to back).

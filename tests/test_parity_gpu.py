@@ -605,9 +605,9 @@ def test_prefill_fold_matches_oracle(T, d, d_out, q, g, r):
     fold_check(read_folded(ws, T, d, d_out, cfg), X, out["s"].cpu().numpy())
 
 
-@pytest.mark.parametrize("b,d", [(9, 512), (64, 5120), (17, 800)])
+@pytest.mark.parametrize("b,d", [(3, 512), (64, 5120), (17, 800)])
 def test_decode_fold_matches_oracle(b, d):
-    # decode batches above eight rows fold in their own kernel ahead of the tensor-core GEMM
+    # decode batches above two rows fold in their own kernel ahead of the tensor-core GEMM
     d_out, q, g = 256, 4, 32
     Xb, X, s32, oc, osc, oz, A, B = oracle_inputs(64, d, d_out, q, g, 0, seed=b + d)
     xt = synthetic.as_bf16(synthetic.draw_tokens(b, d, seed=b))
