@@ -1046,7 +1046,7 @@ def decoder_leg(torch, ttq, dev, K=3):
            "prefill_linear_TFLOPs": round(flops / (tp / 1e3) / 1e12, 1),
            "decode_ms_per_step": round(td / steps, 4), "decode_tokens_per_s": round(steps / (td / 1e3), 1),
            "prompt_plus_decode_ms": round(tp + td, 2), "finite": ok,
-           "attention": "prompt: torch SDPA (library); decode: the library's own kernel",
+           "attention": "the library's own kernels: prompt on the tensor cores, decode split over positions",
            "decode_launch": "one captured CUDA graph per step (device-held position)"}
     del dec, W, x
     torch.cuda.empty_cache()

@@ -244,8 +244,8 @@ TTQ_API ttq_status ttq_linear_decode_batched(const void* X_bf16, int32_t request
  * Sennrich 2019), per-head RMSNorm of q and k, rotary position embedding with the
  * half-split pairing (Su et al. 2021), grouped-query attention, SwiGLU MLP (Shazeer 2020).
  * Arithmetic is fp32 with one bf16 rounding per stored value. The library has the
- * decode step's attention (one token over the cache); a prompt's causal attention is
- * left to a library kernel.
+ * prompt's causal attention (tensor cores) and the decode step's attention (one token
+ * over the cache).
  * --------------------------------------------------------------------------------- */
 
 /* RMSNorm over `rows` rows of n channels, with the residual add of a pre-norm layer:
@@ -308,6 +308,21 @@ TTQ_API ttq_status ttq_decode_attention(const void* q_bf16, int64_t heads, int64
                                         const void* k_cache_bf16, const void* v_cache_bf16, int64_t cache_len,
                                         int64_t length, const int64_t* pos_dev, void* out_bf16, void* ws,
                                         size_t ws_bytes, cudaStream_t stream);
+
+/* Causal grouped-query attention of a prompt at positions 0 .. T-1 on the tensor cores:
+ *   out[t, h] = sum_{p <= t} softmax_p(q_t,h . k_p / sqrt(head_dim)) v_p   (k, v of kv head
+ *   h / (heads / kv_heads)), with q from the stacked projection and k, v from the caches
+ *   qkv        device bf16 [T, (heads + 2 kv_heads) * head_dim], the q heads first (as left by
+ *              ttq_qk_norm_rope, which also wrote positions 0 .. T-1 of the caches)
+ *   k_cache, v_cache  device bf16 [cache_len, kv_heads, head_dim], cache_len >= T
+ *   out        device bf16 [T, heads * head_dim], distinct from qkv
+ * One CTA per (tile of 128 queries, head) walks the key tiles up to its diagonal: S = Q K^T
+ * and O += P V on tcgen05 with fp32 accumulators in tensor memory, an fp32 online softmax
+ * (running row maximum and sum), P rounded to bf16 for the second product.
+ * head_dim 128 (TTQ_ERR_UNSUPPORTED otherwise); heads % kv_heads == 0; T <= 2^24. */
+TTQ_API ttq_status ttq_prompt_attention(const void* qkv_bf16, int64_t T, int64_t heads, int64_t kv_heads,
+                                        int64_t head_dim, const void* k_cache_bf16, const void* v_cache_bf16,
+                                        int64_t cache_len, void* out_bf16, cudaStream_t stream);
 
 /* *pos_dev += n on the device, in stream order (moves a captured decode step to the next
  * position). */

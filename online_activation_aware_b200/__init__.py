@@ -10,8 +10,8 @@ Functions keep the C names without the ``ttq_`` prefix:
 ``act_stats``, ``requant``, ``requant_batched``, ``linear_prefill``, ``linear_prefill_batched``,
 ``linear_decode``, ``linear_decode_batched``, ``workspace_size``,
 ``codes_words``, ``device_status``, ``set_wait_limit_ns``, and the decoder-layer kernels
-``rmsnorm``, ``rope_table``, ``qk_norm_rope``, ``silu_mul``, ``decode_attention``,
-``position_advance``. ``TTQLinear`` bundles one
+``rmsnorm``, ``rope_table``, ``qk_norm_rope``, ``silu_mul``, ``prompt_attention``,
+``decode_attention``, ``position_advance``. ``TTQLinear`` bundles one
 layer's weight and the per-prompt buffers (prefill, then decode reusing the codes);
 ``online_activation_aware_b200.decoder`` chains them into a decoder stack.
 """
@@ -91,6 +91,8 @@ def load_library(path: str = LIB_PATH):
     lib.ttq_decode_attention_workspace_size.restype = i32
     lib.ttq_decode_attention.argtypes = [vp, i64, i64, i64, vp, vp, i64, i64, vp, vp, vp, sz, vp]
     lib.ttq_decode_attention.restype = i32
+    lib.ttq_prompt_attention.argtypes = [vp, i64, i64, i64, i64, vp, vp, i64, vp, vp]
+    lib.ttq_prompt_attention.restype = i32
     lib.ttq_position_advance.argtypes = [vp, i64, vp]
     lib.ttq_position_advance.restype = i32
     lib.ttq_silu_mul.argtypes = [vp, i64, i64, vp, vp]
@@ -476,6 +478,22 @@ def decode_attention(q, heads: int, kv_heads: int, head_dim: int, k_cache, v_cac
         _ptr(q, torch.bfloat16, "q"), heads, kv_heads, head_dim, _ptr(k_cache, torch.bfloat16, "k_cache"),
         _ptr(v_cache, torch.bfloat16, "v_cache"), L, length, _ptr(pos_dev, torch.int64, "pos_dev"),
         _ptr(out, torch.bfloat16, "out"), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)))
+    return out
+
+
+def prompt_attention(qkv, heads: int, kv_heads: int, head_dim: int, k_cache, v_cache, out=None, stream=None):
+    """Causal grouped-query attention of a prompt at positions 0 .. T-1 (q from the stacked
+    projection qkv [T, ...], k and v from the caches' first T positions); returns
+    out [T, heads * head_dim] bf16."""
+    import torch
+
+    T = qkv.shape[0]
+    if out is None:
+        out = torch.empty(T, heads * head_dim, dtype=torch.bfloat16, device=qkv.device)
+    _check("ttq_prompt_attention", load_library().ttq_prompt_attention(
+        _ptr(qkv, torch.bfloat16, "qkv"), T, heads, kv_heads, head_dim, _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], _ptr(out, torch.bfloat16, "out"),
+        _stream(stream)))
     return out
 
 

@@ -655,6 +655,22 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, uint32_t elem_byte
   return r == CUDA_SUCCESS;
 }
 
+// 3-D tensor map (innermost first): dims {n0, n1, n2} with byte strides {s1, s2} of dims 1
+// and 2, a {b0, b1, b2} box, bf16 elements, 128-byte swizzle, zero fill outside.
+bool encode_bf16_tmap_3d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1, uint64_t n2, uint64_t s1,
+                         uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[3] = {n0, n1, n2};
+  cuuint64_t gstride[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int q, int g, int num_sms) {
   GemmPlan p{};
   int BN = 16;

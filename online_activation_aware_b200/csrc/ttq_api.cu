@@ -688,6 +688,24 @@ ttq_status ttq_decode_attention(const void* q_bf16, int64_t heads, int64_t kv_he
                                                   di->err_word, stream));
 }
 
+ttq_status ttq_prompt_attention(const void* qkv_bf16, int64_t T, int64_t heads, int64_t kv_heads, int64_t head_dim,
+                                const void* k_cache_bf16, const void* v_cache_bf16, int64_t cache_len, void* out_bf16,
+                                cudaStream_t stream) {
+  if (!qkv_bf16 || !k_cache_bf16 || !v_cache_bf16 || !out_bf16) return TTQ_ERR_INVALID_ARG;
+  if (head_dim != 128) return TTQ_ERR_UNSUPPORTED;
+  if (heads < 1 || kv_heads < 1 || heads > 1024 || heads % kv_heads != 0) return TTQ_ERR_INVALID_ARG;
+  if (T < 1 || T > (int64_t(1) << 24) || cache_len < T) return TTQ_ERR_INVALID_ARG;
+  if (out_bf16 == qkv_bf16 || k_cache_bf16 == v_cache_bf16) return TTQ_ERR_INVALID_ARG;
+  if (!aligned16(qkv_bf16) || !aligned16(k_cache_bf16) || !aligned16(v_cache_bf16) || !aligned16(out_bf16))
+    return TTQ_ERR_MISALIGNED;
+  DeviceInfo* di = nullptr;
+  ttq_status st = device_info(&di);
+  if (st != TTQ_OK) return st;
+  return cuda_status(ttq::launch_prompt_attention(qkv_bf16, T, static_cast<int>(heads), static_cast<int>(kv_heads),
+                                                  static_cast<int>(head_dim), k_cache_bf16, v_cache_bf16, out_bf16,
+                                                  dev_err(di), stream));
+}
+
 ttq_status ttq_position_advance(int64_t* pos_dev, int64_t n, cudaStream_t stream) {
   if (!pos_dev || n < 0) return TTQ_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(pos_dev) & 7) return TTQ_ERR_MISALIGNED;

@@ -164,6 +164,11 @@ constexpr int kGemmMaxGroups = 8;
 cudaError_t launch_gemm2sm(const GemmArgs& a, const GemmPlan& plan, const DevErr& err, int inject_stall,
                            cudaStream_t stream, int groups = 1, const int64_t* group_T = nullptr);
 
+// 3-D bf16 tensor map (dims innermost first, byte strides of dims 1 and 2), 128-byte
+// swizzle, zero fill outside the tensor.
+bool encode_bf16_tmap_3d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1, uint64_t n2, uint64_t s1,
+                         uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2);
+
 // Encodes a 2-D row-major bf16 tensor map with 128-byte swizzle and a box of
 // {64 columns, box_rows rows}. Returns false when the driver refuses it.
 bool encode_bf16_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
@@ -195,6 +200,12 @@ size_t decode_attn_partial_bytes(int heads, int head_dim, int splits);
 cudaError_t launch_decode_attention(const void* q, int heads, int kv_heads, int head_dim, const void* k_cache,
                                     const void* v_cache, int64_t cache_len, int64_t length, const int64_t* pos_dev,
                                     void* out, float* part, int splits, unsigned* err, cudaStream_t stream);
+// Causal grouped-query attention of a prompt at positions 0 .. T-1 on the tensor cores:
+// q from the stacked projection (after ttq_qk_norm_rope), k and v from the caches' first T
+// positions, out [T, heads * head_dim] bf16. head_dim 128.
+cudaError_t launch_prompt_attention(const void* qkv, int64_t T, int heads, int kv_heads, int head_dim,
+                                    const void* k_cache, const void* v_cache, void* out, const DevErr& err,
+                                    cudaStream_t stream);
 // *pos += n on the device (one thread).
 cudaError_t launch_position_advance(int64_t* pos, int64_t n, cudaStream_t stream);
 // out = bf16(silu(gate) * up) over rows of [gate | up] (inter channels each, inter % 8 == 0).

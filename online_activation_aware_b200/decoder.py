@@ -10,9 +10,8 @@ statistic serves all three and stacking the rows changes no result), Wo, the sta
 A = [A_1; A_2; ...] and the block-diagonal B, which gives every part its own term.
 
 Between the linears run the library's kernels (``rmsnorm`` with the residual add,
-``qk_norm_rope`` with the key/value cache write, ``silu_mul``, and at decode
-``decode_attention``); the prompt's causal attention is torch's
-``scaled_dot_product_attention``, a library kernel like a cuBLAS GEMM. A decode step reads
+``qk_norm_rope`` with the key/value cache write, ``silu_mul``, the prompt's causal
+``prompt_attention`` on the tensor cores, and at decode ``decode_attention``). A decode step reads
 its position from device memory and advances it on the device, so one captured CUDA graph
 replays every step (``capture_decode``). There is no CPU path: every call raises when the
 library is missing.
@@ -21,7 +20,6 @@ library is missing.
 from __future__ import annotations
 
 import torch
-import torch.nn.functional as F
 
 import online_activation_aware_b200 as ttq
 
@@ -85,11 +83,7 @@ class TTQDecoder:
             # one token at the device-held position, over the cache up to and including it
             return ttq.decode_attention(qkv, H, self.Hkv, D, self.k_cache[li], self.v_cache[li], pos_dev=self.pos,
                                         ws=self.attn_ws).view(1, H * D)
-        qv = qkv[:, : H * D].view(T, H, D).transpose(0, 1).unsqueeze(0)
-        kv = self.k_cache[li, :T].transpose(0, 1).unsqueeze(0)
-        vv = self.v_cache[li, :T].transpose(0, 1).unsqueeze(0)
-        o = F.scaled_dot_product_attention(qv, kv, vv, is_causal=True, enable_gqa=True)
-        return o[0].transpose(0, 1).reshape(T, H * D)
+        return ttq.prompt_attention(qkv, H, self.Hkv, D, self.k_cache[li], self.v_cache[li])
 
     def _run(self, x, prefill: bool, trace=None):
         T = x.shape[0]

@@ -11,8 +11,8 @@ Bars:
   TTQ linears in the stack   as in the single-layer tests: s within 1e-5, codes bit-exact
       given the GPU's s, Y within 5e-3 relative Frobenius of the oracle's fp64 product,
       and every output row within 3e-2 of the RMS row norm;
-  attention (a library kernel: bf16 probabilities, fp32 accumulation)   8e-3 relative
-      Frobenius against the oracle's fp64 softmax.
+  prompt attention (the library's tensor-core kernel: bf16 probabilities, fp32 scores,
+      softmax and accumulation)   8e-3 relative Frobenius against the oracle's fp64 softmax.
 """
 
 import numpy as np
@@ -341,3 +341,54 @@ def test_captured_decode_step_equals_eager_steps():
     for a, b in zip(eager, graphed):
         assert torch.equal(a, b)
     assert int(dec.pos.item()) == T + steps
+
+
+# ------------------------------------------------------------------ prompt attention (tensor cores)
+
+
+def _attn_inputs(T, H, Hkv, D, seed, extra=0):
+    rng = np.random.default_rng(seed)
+    qkv = bf16(rng.normal(size=(T, (H + 2 * Hkv) * D)))
+    kc = bf16(rng.normal(size=(T + extra, Hkv, D)))
+    vc = bf16(rng.normal(size=(T + extra, Hkv, D)))
+    return qkv, kc, vc
+
+
+@pytest.mark.parametrize("T,H,Hkv", [(128, 8, 2), (1, 8, 8), (200, 4, 4), (257, 16, 2), (700, 32, 8), (1000, 2, 1)])
+def test_prompt_attention_parity(T, H, Hkv):
+    # every query row against the oracle's fp64 causal softmax attention; the probabilities
+    # enter the second product in bf16, hence the attention bar; each row within 4x of it
+    D = 128
+    qkv, kc, vc = _attn_inputs(T, H, Hkv, D, seed=T + H)
+    out = ttq.prompt_attention(qkv, H, Hkv, D, kc, vc)
+    torch.cuda.synchronize()
+    q = vals(qkv)[:, : H * D].reshape(T, H, D)
+    a64 = DO.attention(q, vals(kc[:T]), vals(vc[:T]), 0)
+    got = vals(out)
+    assert np.isfinite(got).all()
+    assert rel_fro(got, a64) <= ATTN_RTOL, rel_fro(got, a64)
+    row = np.linalg.norm(got - a64, axis=1) / np.linalg.norm(a64, axis=1)
+    assert row.max() <= 4 * ATTN_RTOL, float(row.max())
+
+
+def test_prompt_attention_full_size_sampled_rows_and_cache_padding():
+    # the Qwen3-8B shape (32 query heads, 8 key/value heads of 128) at a 4096-token prompt,
+    # caches longer than the prompt (their later rows hold values that must not be read):
+    # 64 sampled query rows, all heads, against the oracle; the same call twice gives the
+    # same bits
+    T, H, Hkv, D = 4096, 32, 8, 128
+    qkv, kc, vc = _attn_inputs(T, H, Hkv, D, seed=11, extra=64)
+    kc[T:] = 30.0
+    vc[T:] = -30.0
+    out = ttq.prompt_attention(qkv, H, Hkv, D, kc, vc)
+    out2 = ttq.prompt_attention(qkv, H, Hkv, D, kc, vc)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+    q = vals(qkv)[:, : H * D].reshape(T, H, D)
+    K, V = vals(kc), vals(vc)
+    rows = np.unique(np.concatenate([[0, 127, 128, T - 1], np.random.default_rng(12).choice(T, 60, replace=False)]))
+    got = vals(out)
+    for t in rows:
+        a64 = DO.attention(q[t: t + 1], K[: t + 1], V[: t + 1], t)
+        err = np.linalg.norm(got[t] - a64[0]) / np.linalg.norm(a64[0])
+        assert err <= 4 * ATTN_RTOL, (int(t), float(err))
