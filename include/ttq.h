@@ -319,7 +319,7 @@ TTQ_API ttq_status ttq_decode_attention(const void* q_bf16, int64_t heads, int64
  * One CTA per (tile of 128 queries, head) walks the key tiles up to its diagonal: S = Q K^T
  * and O += P V on tcgen05 with fp32 accumulators in tensor memory, an fp32 online softmax
  * (running row maximum and sum), P rounded to bf16 for the second product.
- * head_dim 128 (TTQ_ERR_UNSUPPORTED otherwise); heads % kv_heads == 0; T <= 2^24. */
+ * head_dim 64 or 128 (TTQ_ERR_UNSUPPORTED otherwise); heads % kv_heads == 0; T <= 2^24. */
 TTQ_API ttq_status ttq_prompt_attention(const void* qkv_bf16, int64_t T, int64_t heads, int64_t kv_heads,
                                         int64_t head_dim, const void* k_cache_bf16, const void* v_cache_bf16,
                                         int64_t cache_len, void* out_bf16, cudaStream_t stream);

@@ -32,11 +32,10 @@ namespace ttq {
 namespace {
 
 constexpr int kAttnTile = 128;        // queries per CTA, positions per key tile
-constexpr int kHeadDim = 128;
 constexpr int kAttnThreads = 192;     // 6 warps
 constexpr uint32_t kBoxBytes = kAttnTile * 64 * 2;        // 128 rows x 64 channels, bf16
-constexpr uint32_t kTileBytes = 2 * kBoxBytes;            // 128 rows x 128 channels
-constexpr uint32_t kTmemCols = 512;                       // S0, S1, O (128 columns each)
+constexpr uint32_t kPBytes = 2 * kBoxBytes;               // P: 128 queries x 128 positions
+constexpr uint32_t kTmemCols = 512;                       // S0, S1, O
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 
 struct AttnBars {
@@ -53,13 +52,18 @@ struct AttnBars {
   int abort_flag;
 };
 
-// smem: Q | K0 | K1 | V0 | V1 | P, each 32 KB and 1024-byte aligned, then the barriers
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTileBytes;
-constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;
-constexpr uint32_t kOffP = kOffV + 2 * kTileBytes;
-constexpr uint32_t kOffBars = kOffP + kTileBytes;
-constexpr size_t kAttnSmem = kOffBars + sizeof(AttnBars) + 1024;  // + alignment slack
+// smem: Q | K0 | K1 | V0 | V1 | P (1024-byte aligned; Q, K, V tiles of 128 rows x D
+// channels as D / 64 boxes), then the barriers
+template <int D>
+struct AttnLayout {
+  static constexpr uint32_t kTileBytes = (D / 64) * kBoxBytes;
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffK = kOffQ + kTileBytes;
+  static constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;
+  static constexpr uint32_t kOffP = kOffV + 2 * kTileBytes;
+  static constexpr uint32_t kOffBars = kOffP + kPBytes;
+  static constexpr size_t kSmem = kOffBars + sizeof(AttnBars) + 1024;  // + alignment slack
+};
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
                                             int z) {
@@ -127,13 +131,17 @@ struct AttnArgs {
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v ? 1 : 0) != 0; }
 
+template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     prompt_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+  using L = AttnLayout<D>;
+  constexpr uint32_t kTileBytes = L::kTileBytes, kOffQ = L::kOffQ, kOffK = L::kOffK, kOffV = L::kOffV,
+                     kOffP = L::kOffP;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  AttnBars* bars = reinterpret_cast<AttnBars*>(smem_raw + (base - raw) + kOffBars);
+  AttnBars* bars = reinterpret_cast<AttnBars*>(smem_raw + (base - raw) + L::kOffBars);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int h = blockIdx.x;
@@ -185,8 +193,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       mbar_arrive_expect_tx(b_q, kTileBytes);
-      tma_load_2d(base + kOffQ, &tm_q, b_q, h * kHeadDim, q0);
-      tma_load_2d(base + kOffQ + kBoxBytes, &tm_q, b_q, h * kHeadDim + 64, q0);
+#pragma unroll
+      for (int bx = 0; bx < D / 64; ++bx) tma_load_2d(base + kOffQ + bx * kBoxBytes, &tm_q, b_q, h * D + 64 * bx, q0);
       int j = 0;
       for (; j < nkv; ++j) {
         const int st = j & 1;
@@ -195,11 +203,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t ks = base + kOffK + st * kTileBytes;
         const uint32_t vs = base + kOffV + st * kTileBytes;
         mbar_arrive_expect_tx(b_kf + 8 * st, kTileBytes);
-        tma_load_3d(ks, &tm_k, b_kf + 8 * st, 0, hk, p0);
-        tma_load_3d(ks + kBoxBytes, &tm_k, b_kf + 8 * st, 64, hk, p0);
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx) tma_load_3d(ks + bx * kBoxBytes, &tm_k, b_kf + 8 * st, 64 * bx, hk, p0);
         mbar_arrive_expect_tx(b_vf + 8 * st, kTileBytes);
-        tma_load_3d(vs, &tm_v, b_vf + 8 * st, 0, hk, p0);
-        tma_load_3d(vs + kBoxBytes, &tm_v, b_vf + 8 * st, 64, hk, p0);
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx) tma_load_3d(vs + bx * kBoxBytes, &tm_v, b_vf + 8 * st, 64 * bx, hk, p0);
       }
       if (*abort_flag) {
         // every copy this CTA started lands before its shared memory is released
@@ -213,7 +221,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     const uint32_t idesc_s = idesc_bf16_f32(kAttnTile, kAttnTile);
-    const uint32_t idesc_pv = idesc_bf16_f32(kAttnTile, kHeadDim) | (1u << 16);  // B (V) MN-major
+    const uint32_t idesc_pv = idesc_bf16_f32(kAttnTile, D) | (1u << 16);  // B (V) MN-major
     bool ok = warp_all(mbar_wait(b_q, 0, err, abort_flag));
     // S_j = Q K_j^T into accumulator j & 1 (K = head_dim in steps of 16: 4 per 64-channel box)
     auto issue_s = [&](int j) -> bool {
@@ -225,7 +233,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t d = tmem + (st ? kColS1 : kColS0);
         const uint32_t ks = base + kOffK + st * kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
           umma_bf16(d, sw128_kmajor_desc(base + kOffQ + off), sw128_kmajor_desc(ks + off), idesc_s, kk > 0 ? 1u : 0u);
         }
@@ -313,7 +321,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
         if (__any_sync(0xffffffffu, corr != 1.f ? 1 : 0)) {
 #pragma unroll 1
-          for (int cc = 0; cc < kHeadDim / 32; ++cc) {
+          for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
             tmem_ld_32x32b_x32(tl + kColO + 32 * cc, o);
             tmem_ld_wait();
@@ -355,9 +363,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_after();
       const float inv = __fdiv_rn(1.f, l);
       const int t = q0 + r;
-      __nv_bfloat16* orow = a.out + static_cast<int64_t>(t) * a.ld_out + h * kHeadDim;
+      __nv_bfloat16* orow = a.out + static_cast<int64_t>(t) * a.ld_out + h * D;
 #pragma unroll 1
-      for (int cc = 0; cc < kHeadDim / 32; ++cc) {
+      for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
         tmem_ld_32x32b_x32(tl + kColO + 32 * cc, o);
         tmem_ld_wait();
@@ -385,10 +393,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
 }  // namespace
 
+namespace {
+
+template <int D>
+cudaError_t launch_attention_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
+                               int heads, cudaStream_t stream) {
+  constexpr size_t smem = AttnLayout<D>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(prompt_attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(heads), static_cast<unsigned>(a.n_q));
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, prompt_attention_kernel<D>, tq, tk, tv, a);
+}
+
+}  // namespace
+
 cudaError_t launch_prompt_attention(const void* qkv, int64_t T, int heads, int kv_heads, int head_dim,
                                     const void* k_cache, const void* v_cache, void* out, const DevErr& err,
                                     cudaStream_t stream) {
-  if (head_dim != kHeadDim || heads % kv_heads != 0 || T < 1) return cudaErrorInvalidValue;
+  if ((head_dim != 64 && head_dim != 128) || heads % kv_heads != 0 || T < 1) return cudaErrorInvalidValue;
   const uint64_t ncols = static_cast<uint64_t>(heads + 2 * kv_heads) * head_dim;
   CUtensorMap tq, tk, tv;
   // q: the first heads * head_dim channels of each row of the stacked projection
@@ -406,20 +438,8 @@ cudaError_t launch_prompt_attention(const void* qkv, int64_t T, int heads, int k
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(head_dim)));
   a.out = static_cast<__nv_bfloat16*>(out);
   a.err = err;
-  cudaError_t e = cudaFuncSetAttribute(prompt_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kAttnSmem));
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(heads), static_cast<unsigned>(a.n_q));
-  cfg.blockDim = dim3(kAttnThreads);
-  cfg.dynamicSmemBytes = kAttnSmem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, prompt_attention_kernel, tq, tk, tv, a);
+  return head_dim == 64 ? launch_attention_d<64>(tq, tk, tv, a, heads, stream)
+                        : launch_attention_d<128>(tq, tk, tv, a, heads, stream);
 }
 
 }  // namespace ttq

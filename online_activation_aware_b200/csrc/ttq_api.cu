@@ -692,7 +692,7 @@ ttq_status ttq_prompt_attention(const void* qkv_bf16, int64_t T, int64_t heads, 
                                 const void* k_cache_bf16, const void* v_cache_bf16, int64_t cache_len, void* out_bf16,
                                 cudaStream_t stream) {
   if (!qkv_bf16 || !k_cache_bf16 || !v_cache_bf16 || !out_bf16) return TTQ_ERR_INVALID_ARG;
-  if (head_dim != 128) return TTQ_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return TTQ_ERR_UNSUPPORTED;
   if (heads < 1 || kv_heads < 1 || heads > 1024 || heads % kv_heads != 0) return TTQ_ERR_INVALID_ARG;
   if (T < 1 || T > (int64_t(1) << 24) || cache_len < T) return TTQ_ERR_INVALID_ARG;
   if (out_bf16 == qkv_bf16 || k_cache_bf16 == v_cache_bf16) return TTQ_ERR_INVALID_ARG;

@@ -202,7 +202,7 @@ cudaError_t launch_decode_attention(const void* q, int heads, int kv_heads, int 
                                     void* out, float* part, int splits, unsigned* err, cudaStream_t stream);
 // Causal grouped-query attention of a prompt at positions 0 .. T-1 on the tensor cores:
 // q from the stacked projection (after ttq_qk_norm_rope), k and v from the caches' first T
-// positions, out [T, heads * head_dim] bf16. head_dim 128.
+// positions, out [T, heads * head_dim] bf16. head_dim 64 or 128.
 cudaError_t launch_prompt_attention(const void* qkv, int64_t T, int heads, int kv_heads, int head_dim,
                                     const void* k_cache, const void* v_cache, void* out, const DevErr& err,
                                     cudaStream_t stream);

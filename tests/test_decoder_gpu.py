@@ -354,11 +354,11 @@ def _attn_inputs(T, H, Hkv, D, seed, extra=0):
     return qkv, kc, vc
 
 
-@pytest.mark.parametrize("T,H,Hkv", [(128, 8, 2), (1, 8, 8), (200, 4, 4), (257, 16, 2), (700, 32, 8), (1000, 2, 1)])
-def test_prompt_attention_parity(T, H, Hkv):
+@pytest.mark.parametrize("T,H,Hkv,D", [(128, 8, 2, 128), (1, 8, 8, 128), (200, 4, 4, 128), (257, 16, 2, 128),
+                                       (700, 32, 8, 128), (1000, 2, 1, 128), (96, 8, 2, 64), (300, 4, 2, 64)])
+def test_prompt_attention_parity(T, H, Hkv, D):
     # every query row against the oracle's fp64 causal softmax attention; the probabilities
     # enter the second product in bf16, hence the attention bar; each row within 4x of it
-    D = 128
     qkv, kc, vc = _attn_inputs(T, H, Hkv, D, seed=T + H)
     out = ttq.prompt_attention(qkv, H, Hkv, D, kc, vc)
     torch.cuda.synchronize()
