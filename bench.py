@@ -695,8 +695,24 @@ def act_stats_leg(torch, ttq, Xs, outs, wl, hbm_peak, flush, sink):
     torch.cuda.synchronize()
     us = graph_step_us(torch, one, flush, sink)
     gbs = stats_bytes(T, d) / (us * 1e-6) / 1e9
+    # the same kernel over prompts of 1/4, 1 and 4 times T tokens: a fixed cost per launch
+    # plus a streaming rate (the least-squares line through time against bytes)
+    pts = []
+    for f in (0.25, 1.0, 4.0):
+        Tf = int(T * f)
+        Xf = Xs[0] if Tf == T else torch.randn(Tf, d, device=Xs[0].device).to(torch.bfloat16)
+        sf = torch.empty(d, dtype=torch.float32, device=Xs[0].device)
+        u = graph_step_us(torch, lambda st: ttq.act_stats(Xf, wl.alpha, wl.lam, wl.p, s=sf, stream=st), flush, sink)
+        pts.append((stats_bytes(Tf, d), u))
+        del Xf
+    n = len(pts)
+    mb = sum(b for b, _ in pts) / n
+    mu = sum(u for _, u in pts) / n
+    slope = sum((b - mb) * (u - mu) for b, u in pts) / sum((b - mb) ** 2 for b, _ in pts)  # us per byte
     return {"us": round(us, 2), "GBps": round(gbs, 1), "frac": round(gbs / hbm_peak, 4),
-            "method": "graph difference, L2 flushed before each launch"}
+            "method": "graph difference, L2 flushed before each launch",
+            "size_sweep_us": {f"{b / 1e6:.0f}MB": round(u, 2) for b, u in pts},
+            "streaming_GBps": round(1e-3 / slope, 1), "fixed_us": round(mu - slope * mb, 2)}
 
 
 def requant_batched_leg(torch, ttq, Ws, outs, d, d_out, q, g, P=4, reps=50):
@@ -1024,6 +1040,17 @@ def decoder_leg(torch, ttq, dev, K=3):
         e1.record()
         torch.cuda.synchronize()
         ts.append(e0.elapsed_time(e1))
+    # the prompt attention alone (layer 0's caches after the prefill), as the difference of
+    # two CUDA graphs: causal flops 4 * D * H * T (T + 1) / 2
+    H, Hkv, D = shape["heads"], shape["kv_heads"], shape["head_dim"]
+    qkv0 = torch.randn(T, (H + 2 * Hkv) * D, generator=gen, device=dev).to(torch.bfloat16)
+    aout = torch.empty(T, H * D, dtype=torch.bfloat16, device=dev)
+    flush = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    t_attn = graph_step_us(torch, lambda st: ttq.prompt_attention(qkv0, H, Hkv, D, dec.k_cache[0], dec.v_cache[0],
+                                                                   out=aout, stream=st), flush, sink, n=8)
+    attn_flops = 4.0 * D * H * T * (T + 1) / 2
+    del qkv0, aout, flush
     dec.capture_decode()
     for i in range(4):              # warm the replay, then start over from a fresh prefill
         dec.decode(x[T + i: T + i + 1])
@@ -1047,6 +1074,7 @@ def decoder_leg(torch, ttq, dev, K=3):
            "decode_ms_per_step": round(td / steps, 4), "decode_tokens_per_s": round(steps / (td / 1e3), 1),
            "prompt_plus_decode_ms": round(tp + td, 2), "finite": ok,
            "attention": "the library's own kernels: prompt on the tensor cores, decode split over positions",
+           "prompt_attention_us": round(t_attn, 1), "prompt_attention_TFLOPs": round(attn_flops / (t_attn * 1e-6) / 1e12, 1),
            "decode_launch": "one captured CUDA graph per step (device-held position)"}
     del dec, W, x
     torch.cuda.empty_cache()
