@@ -912,13 +912,14 @@ def sweep_leg(torch, ttq, wl, cfg, Wb, A, B, dev, r):
     assert ttq.device_status() == 0
     return res
 
-def rho_sweep_leg(torch, ttq, wl, cfg, Wb, dev, hbm_peak, Ts=(128, 1024, 4096, 16384), reps=20):
+def rho_sweep_leg(torch, ttq, wl, cfg, Wb, dev, hbm_peak, Ts=(128, 1024, 2048, 4096, 8192, 16384), reps=20):
     """The overhead ratio across prompt lengths: per T, the stage split of the prefill from
     the library's stage events (median over `reps` prompts, rotating buffer sets larger
     than L2), rho = (statistic + fold and re-quantization) / projection, next to the
     pages' count rho_model = 1/d' + 3/T (gist.science French summary, section 2A:
-    O(dT + 3d'd) extra against O(d'dT)). The trend holds when rho / rho_model stays within
-    a constant band wherever the projection runs at its tensor-core rate."""
+    O(dT + 3d'd) extra against O(d'dT)). The count's structure, as times: the overhead is a
+    constant (requant) plus a term linear in T (statistic, fold), the projection is
+    proportional to T (checked from T = 2048, where it runs at its tensor-core rate)."""
     lin = wl.layers[0]
     d, d_out = lin.d, lin.d_out
     res = {}
@@ -946,8 +947,20 @@ def rho_sweep_leg(torch, ttq, wl, cfg, Wb, dev, hbm_peak, Ts=(128, 1024, 4096, 1
                         "rho_over_model": round(rho / rho_model, 2), "rho_T": round(rho * T, 1)}
         del Xs, Ws, outs, ws
         torch.cuda.empty_cache()
-    ratios = [v["rho_over_model"] for k, v in res.items() if int(k[1:]) >= 1024]
-    res["band_T_ge_1024"] = round(max(ratios) / min(ratios), 3) if ratios else None
+    # the count's structure as times (T >= 2048, the projection at its tensor-core rate):
+    # overhead = a + b T, projection time per token constant, rho falling
+    import numpy as np
+
+    big = [T for T in Ts if T >= 2048]
+    y = np.array([res[f"T{T}"]["stats_us"] + res[f"T{T}"]["fold_requant_us"] for T in big])
+    x = np.array(big, dtype=np.float64)
+    A = np.stack([np.ones_like(x), x], axis=1) / y[:, None]
+    (a_, b_), *_ = np.linalg.lstsq(A, np.ones_like(y), rcond=None)
+    per_tok = [res[f"T{T}"]["gemm_us"] / T for T in big]
+    res["overhead_fit"] = {"constant_us": round(float(a_), 2), "per_token_ns": round(float(b_) * 1e3, 3),
+                           "max_rel_residual": round(float(np.max(np.abs(a_ + b_ * x - y) / y)), 4),
+                           "projection_per_token_spread": round(max(per_tok) / min(per_tok), 3),
+                           "T": big}
     res["rho_decreasing"] = all(res[f"T{a}"]["rho"] > res[f"T{b}"]["rho"] for a, b in zip(Ts, Ts[1:]))
     assert ttq.device_status() == 0
     return res
