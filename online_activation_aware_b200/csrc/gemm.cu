@@ -195,8 +195,8 @@ __device__ __forceinline__ void dequant_half(const uint32_t (&cw)[4], float sig,
 
 // TQ: codes, scale and zero arrive by TMA in each stage (rows of 16-byte multiples);
 // otherwise each dequantiser streams its own row through a private cp.async ring.
-template <int Q, int S, int RING, bool TQ>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int Q, int S, int RING, bool TQ, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB)
     ttq_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_u,
                     const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
                     const __grid_constant__ CUtensorMap tm_sc, const __grid_constant__ CUtensorMap tm_z,
@@ -597,9 +597,9 @@ struct Maps {
   CUtensorMap x, u, b, c, sc, z;
 };
 
-template <int Q, int S, int RING, bool TQ>
+template <int Q, int S, int RING, bool TQ, int MINB = 1>
 cudaError_t launch_q(const Maps& mp, const KernelArgs& ka, int grid, size_t smem, cudaStream_t stream) {
-  auto kern = ttq_gemm_kernel<Q, S, RING, TQ>;
+  auto kern = ttq_gemm_kernel<Q, S, RING, TQ, MINB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -685,10 +685,13 @@ GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int q, int g, int num_sm
   p.n_tiles = static_cast<int>((T + BN - 1) / BN);
   p.nkb = static_cast<int>((d + kBK - 1) / kBK);
   p.smem_bytes = 0;
-  // One persistent CTA (or CTA pair) per SM (pair of SMs). Split K only when the tiles
-  // cannot fill one wave, and then just enough to fill it: every split adds an fp32
+  // 16-token tiles (decode of a few tokens, very short prompts) run two CTAs per SM when
+  // the codes come by TMA (4 stages of 26 KB each fit twice in shared memory)
+  p.ctas_per_sm = (!p.pair && BN == 16 && tma_codes_ok(d, q, g)) ? 2 : 1;
+  // One persistent CTA (or CTA pair) per SM slot (pair of SMs). Split K only when the
+  // tiles cannot fill one wave, and then just enough to fill it: every split adds an fp32
   // partial write and read of Y.
-  const int64_t slots = p.pair ? num_sms / 2 : num_sms;
+  const int64_t slots = p.pair ? num_sms / 2 : static_cast<int64_t>(num_sms) * p.ctas_per_sm;
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
   int best = 1;
   if (tiles < slots) {
@@ -761,7 +764,18 @@ cudaError_t launch_gemm_mainloop(const GemmArgs& a, const GemmPlan& plan, const 
   ka.num_tiles = plan.m_tiles * plan.n_tiles * plan.ksplit;
   ka.inject_stall = g_inject_stall ? 1 : 0;
   ka.err = err;
-  const int grid = ka.num_tiles < sms ? ka.num_tiles : sms;
+  const int slots = sms * plan.ctas_per_sm;
+  const int grid = ka.num_tiles < slots ? ka.num_tiles : slots;
+  if (plan.ctas_per_sm == 2) {
+    // 16-token tiles, two CTAs per SM (4 stages each, at most 72 registers a thread): two
+    // independent pipelines per SM for the latency-bound hand-off of short K loops
+    const size_t smem2 = smem_bytes_for(plan.BN, 4, 4, true);
+    switch (a.q) {
+      case 2: return launch_q<2, 4, 4, true, 2>(mp, ka, grid, smem2, stream);
+      case 3: return launch_q<3, 4, 4, true, 2>(mp, ka, grid, smem2, stream);
+      default: return launch_q<4, 4, 4, true, 2>(mp, ka, grid, smem2, stream);
+    }
+  }
   const int S = plan_stages(plan.BN, tq);
   const int R = plan_ring(plan.BN);
   const size_t smem = smem_bytes_for(plan.BN, S, R, tq);

@@ -117,6 +117,7 @@ struct GemmPlan {
   int nkb;          // K blocks of 64: ceil(d / 64)
   int ksplit;       // split-K factor (1 = direct bf16 epilogue)
   int kb_per_split;
+  int ctas_per_sm;  // single-CTA kernel: 2 for 16-token tiles with TMA-loaded codes, else 1
   size_t smem_bytes;
 };
 GemmPlan gemm_plan(int64_t T, int64_t d, int64_t d_out, int q, int g, int num_sms);
