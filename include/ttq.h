@@ -337,8 +337,9 @@ TTQ_API ttq_status ttq_silu_mul(const void* gate_up_bf16, int64_t rows, int64_t 
 
 /* Synchronises `stream`, then reads and clears the device error word: TTQ_OK, or
  * TTQ_ERR_TIMEOUT when a kernel gave up on a bounded wait since the last call,
- * TTQ_ERR_INVALID_ARG when a position read from device memory was out of range, or
- * TTQ_ERR_CUDA when the synchronisation itself failed. */
+ * TTQ_ERR_INVALID_ARG when a position read from device memory was out of range or a
+ * kernel found its shared-memory allocation too small for its layout (it then did no
+ * work), or TTQ_ERR_CUDA when the synchronisation itself failed. */
 TTQ_API ttq_status ttq_device_status(cudaStream_t stream);
 
 /* Sets the limit, in nanoseconds, after which a kernel waiting on an mbarrier gives up

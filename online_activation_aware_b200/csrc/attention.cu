@@ -31,12 +31,9 @@ namespace ttq {
 
 namespace {
 
-constexpr int kAttnTile = 128;        // queries per CTA, positions per key tile
+constexpr int kAttnTile = 128;        // queries per CTA
 constexpr int kAttnThreads = 192;     // 6 warps
-constexpr uint32_t kBoxBytes = kAttnTile * 64 * 2;        // 128 rows x 64 channels, bf16
-constexpr uint32_t kPBytes = 2 * kBoxBytes;               // P: 128 queries x 128 positions
-constexpr uint32_t kTmemCols = 512;                       // S0, S1, O
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+constexpr uint32_t kRowBox = 128 * 128;                  // 128 rows x 128 B (64 bf16): a Q or P box
 
 struct AttnBars {
   uint64_t q_full;
@@ -52,17 +49,29 @@ struct AttnBars {
   int abort_flag;
 };
 
-// smem: Q | K0 | K1 | V0 | V1 | P (1024-byte aligned; Q, K, V tiles of 128 rows x D
-// channels as D / 64 boxes), then the barriers
-template <int D>
+// D channels, key tiles of BK positions. smem: Q | K0 | K1 | V0 | V1 | P (1024-byte
+// aligned; Q as D / 64 boxes of 128 rows x 64 channels, K and V as D / 64 boxes of BK rows,
+// P as BK / 64 boxes of 128 rows x 64 positions), then the barriers. Tensor memory: S0, S1
+// (BK columns each), O (D columns). Two CTAs share an SM when both fit twice.
+template <int D, int BK>
 struct AttnLayout {
-  static constexpr uint32_t kTileBytes = (D / 64) * kBoxBytes;
+  static constexpr uint32_t kKVBox = BK * 128;
+  static constexpr uint32_t kQBytes = (D / 64) * kRowBox;
+  static constexpr uint32_t kKVBytes = (D / 64) * kKVBox;
+  static constexpr uint32_t kPBytes = (BK / 64) * kRowBox;
   static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffK = kOffQ + kTileBytes;
-  static constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;
-  static constexpr uint32_t kOffP = kOffV + 2 * kTileBytes;
+  static constexpr uint32_t kOffK = kOffQ + kQBytes;
+  static constexpr uint32_t kOffV = kOffK + 2 * kKVBytes;
+  static constexpr uint32_t kOffP = kOffV + 2 * kKVBytes;
   static constexpr uint32_t kOffBars = kOffP + kPBytes;
-  static constexpr size_t kSmem = kOffBars + sizeof(AttnBars) + 1024;  // + alignment slack
+  // + up to 896 bytes to align the base to 1024 (the dynamic base is 128-byte aligned; the
+  // kernel checks its layout fits before it touches shared memory)
+  static constexpr size_t kSmem = kOffBars + sizeof(AttnBars) + 896;
+  static constexpr uint32_t kColS0 = 0, kColS1 = BK, kColO = 2 * BK;
+  static constexpr uint32_t kTmemCols = (2 * BK + D) <= 256 ? 256u : 512u;
+  // two CTAs per SM when their shared memory (plus the 1 KB each reserves) fits the SM's
+  // 228 KB and their tensor memory its 512 columns
+  static constexpr int kMinBlocks = (2 * (kSmem + 1024) <= 228 * 1024 && 2 * kTmemCols <= 512) ? 2 : 1;
 };
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
@@ -131,16 +140,23 @@ struct AttnArgs {
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v ? 1 : 0) != 0; }
 
-template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+template <int D, int BK>
+__global__ void __launch_bounds__(kAttnThreads, AttnLayout<D, BK>::kMinBlocks)
     prompt_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
-  using L = AttnLayout<D>;
-  constexpr uint32_t kTileBytes = L::kTileBytes, kOffQ = L::kOffQ, kOffK = L::kOffK, kOffV = L::kOffV,
-                     kOffP = L::kOffP;
+  using L = AttnLayout<D, BK>;
+  constexpr uint32_t kOffQ = L::kOffQ, kOffK = L::kOffK, kOffV = L::kOffV, kOffP = L::kOffP;
+  constexpr uint32_t kKVBox = L::kKVBox, kKVBytes = L::kKVBytes;
+  constexpr uint32_t kColS0 = L::kColS0, kColS1 = L::kColS1, kColO = L::kColO;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
+  if ((base - raw) + L::kOffBars + sizeof(AttnBars) > L::kSmem) {
+    // the allocation cannot hold the aligned layout: report and leave before any barrier,
+    // copy or tensor-memory allocation
+    if (threadIdx.x == 0) atomicOr(a.err.word, kErrLayout);
+    return;
+  }
   AttnBars* bars = reinterpret_cast<AttnBars*>(smem_raw + (base - raw) + L::kOffBars);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -148,7 +164,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int qt = a.n_q - 1 - static_cast<int>(blockIdx.y);  // the longest rows first
   const int hk = h / a.G;
   const int q0 = qt * kAttnTile;
-  const int nkv = qt + 1;                                   // key tiles up to the diagonal
+  // key tiles up to the diagonal (and not past the prompt)
+  const int nkv = min((q0 + kAttnTile + BK - 1) / BK, (a.T + BK - 1) / BK);
   volatile int* abort_flag = &bars->abort_flag;
   const DevErr err = a.err;
   const uint32_t b_q = smem_addr(&bars->q_full);
@@ -179,7 +196,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     prefetch_tensormap(&tm_v);
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(&bars->tmem_base), kTmemCols);
+    tmem_alloc(smem_addr(&bars->tmem_base), L::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -192,22 +209,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(b_q, kTileBytes);
+      mbar_arrive_expect_tx(b_q, L::kQBytes);
 #pragma unroll
-      for (int bx = 0; bx < D / 64; ++bx) tma_load_2d(base + kOffQ + bx * kBoxBytes, &tm_q, b_q, h * D + 64 * bx, q0);
+      for (int bx = 0; bx < D / 64; ++bx) tma_load_2d(base + kOffQ + bx * kRowBox, &tm_q, b_q, h * D + 64 * bx, q0);
       int j = 0;
       for (; j < nkv; ++j) {
         const int st = j & 1;
         if (j >= 2 && !mbar_wait(b_ke + 8 * st, ((j >> 1) - 1) & 1, err, abort_flag)) break;
-        const int p0 = j * kAttnTile;
-        const uint32_t ks = base + kOffK + st * kTileBytes;
-        const uint32_t vs = base + kOffV + st * kTileBytes;
-        mbar_arrive_expect_tx(b_kf + 8 * st, kTileBytes);
+        const int p0 = j * BK;
+        const uint32_t ks = base + kOffK + st * kKVBytes;
+        const uint32_t vs = base + kOffV + st * kKVBytes;
+        mbar_arrive_expect_tx(b_kf + 8 * st, kKVBytes);
 #pragma unroll
-        for (int bx = 0; bx < D / 64; ++bx) tma_load_3d(ks + bx * kBoxBytes, &tm_k, b_kf + 8 * st, 64 * bx, hk, p0);
-        mbar_arrive_expect_tx(b_vf + 8 * st, kTileBytes);
+        for (int bx = 0; bx < D / 64; ++bx) tma_load_3d(ks + bx * kKVBox, &tm_k, b_kf + 8 * st, 64 * bx, hk, p0);
+        mbar_arrive_expect_tx(b_vf + 8 * st, kKVBytes);
 #pragma unroll
-        for (int bx = 0; bx < D / 64; ++bx) tma_load_3d(vs + bx * kBoxBytes, &tm_v, b_vf + 8 * st, 64 * bx, hk, p0);
+        for (int bx = 0; bx < D / 64; ++bx) tma_load_3d(vs + bx * kKVBox, &tm_v, b_vf + 8 * st, 64 * bx, hk, p0);
       }
       if (*abort_flag) {
         // every copy this CTA started lands before its shared memory is released
@@ -220,7 +237,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t idesc_s = idesc_bf16_f32(kAttnTile, kAttnTile);
+    const uint32_t idesc_s = idesc_bf16_f32(kAttnTile, BK);
     const uint32_t idesc_pv = idesc_bf16_f32(kAttnTile, D) | (1u << 16);  // B (V) MN-major
     bool ok = warp_all(mbar_wait(b_q, 0, err, abort_flag));
     // S_j = Q K_j^T into accumulator j & 1 (K = head_dim in steps of 16: 4 per 64-channel box)
@@ -231,11 +248,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_after();
       if (elect_one()) {
         const uint32_t d = tmem + (st ? kColS1 : kColS0);
-        const uint32_t ks = base + kOffK + st * kTileBytes;
+        const uint32_t ks = base + kOffK + st * kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          umma_bf16(d, sw128_kmajor_desc(base + kOffQ + off), sw128_kmajor_desc(ks + off), idesc_s, kk > 0 ? 1u : 0u);
+          const uint32_t qo = (kk >> 2) * kRowBox + (kk & 3) * 32;
+          const uint32_t ko = (kk >> 2) * kKVBox + (kk & 3) * 32;
+          umma_bf16(d, sw128_kmajor_desc(base + kOffQ + qo), sw128_kmajor_desc(ks + ko), idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(b_sf + 8 * st);
       }
@@ -253,13 +271,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       tc_fence_after();
       if (elect_one()) {
-        // O += P_j V_j: K = the tile's 128 positions in steps of 16 (P: 4 per 64-position box;
-        // V: 16 positions = two 8-row groups of 1024 B)
-        const uint32_t vs = base + kOffV + st * kTileBytes;
+        // O += P_j V_j: K = the tile's BK positions in steps of 16 (P: 4 per 64-position box;
+        // V: 16 positions = two 8-row groups of 1024 B, the next 64 channels one box on)
+        const uint32_t vs = base + kOffV + st * kKVBytes;
 #pragma unroll
-        for (int kk = 0; kk < kAttnTile / 16; ++kk) {
-          const uint32_t pa = base + kOffP + (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          umma_bf16(tmem + kColO, sw128_kmajor_desc(pa), sw128_mnmajor_desc(vs + kk * 2048, kBoxBytes), idesc_pv,
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint32_t pa = base + kOffP + (kk >> 2) * kRowBox + (kk & 3) * 32;
+          umma_bf16(tmem + kColO, sw128_kmajor_desc(pa), sw128_mnmajor_desc(vs + kk * 2048, kKVBox), idesc_pv,
                     (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(b_ke + 8 * st);  // K_j and V_j may be overwritten once these are done
@@ -286,27 +304,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         break;
       }
       tc_fence_after();
-      uint32_t sr[kAttnTile];
+      uint32_t sr[BK];
       {
-        uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-        uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        uint32_t (&s2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
-        uint32_t (&s3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
         const uint32_t sc = tl + (st ? kColS1 : kColS0);
-        tmem_ld_32x32b_x32(sc, s0);
-        tmem_ld_32x32b_x32(sc + 32, s1);
-        tmem_ld_32x32b_x32(sc + 64, s2);
-        tmem_ld_32x32b_x32(sc + 96, s3);
+#pragma unroll
+        for (int c32 = 0; c32 < BK / 32; ++c32)
+          tmem_ld_32x32b_x32(sc + 32 * c32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c32]));
         tmem_ld_wait();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(b_sfree + 8 * st);  // the accumulator may take S_{j+2}
-      // scaled scores (log2 units); on the diagonal tile keys after the query are masked
-      const int lim = j == qt ? r : kAttnTile - 1;
+      // scaled scores (log2 units); keys after the query (the diagonal tiles) are masked:
+      // key j * BK + k is visible to row q0 + r when k <= q0 + r - j * BK
+      const int lim = min(BK - 1, q0 + r - j * BK);
       float mx = m;
 #pragma unroll
-      for (int k = 0; k < kAttnTile; ++k) {
+      for (int k = 0; k < BK; ++k) {
         const float sv = k <= lim ? __fmul_rn(__uint_as_float(sr[k]), c) : -FLT_MAX;
         sr[k] = __float_as_uint(sv);
         mx = fmaxf(mx, sv);
@@ -338,7 +352,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float rs = 0.f;
       const uint32_t prow = base + kOffP + r * 128;
 #pragma unroll
-      for (int k8 = 0; k8 < kAttnTile / 8; ++k8) {
+      for (int k8 = 0; k8 < BK / 8; ++k8) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -347,7 +361,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           w[e] = pack_bf16x2(p0, p1);
           rs = __fadd_rn(rs, __fadd_rn(bf16lo_to_f32(w[e]), bf16hi_to_f32(w[e])));
         }
-        const uint32_t addr = prow + (k8 >> 3) * kBoxBytes + (((k8 & 7) ^ (r & 7)) << 4);
+        const uint32_t addr = prow + (k8 >> 3) * kRowBox + (((k8 & 7) ^ (r & 7)) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]),
                      "r"(w[3])
                      : "memory");
@@ -387,7 +401,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 
@@ -395,12 +409,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
 namespace {
 
-template <int D>
+template <int D, int BK>
 cudaError_t launch_attention_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
                                int heads, cudaStream_t stream) {
-  constexpr size_t smem = AttnLayout<D>::kSmem;
-  cudaError_t e = cudaFuncSetAttribute(prompt_attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  constexpr size_t smem = AttnLayout<D, BK>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(prompt_attention_kernel<D, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
+  if (e == cudaSuccess)  // all of the SM's unified memory as shared memory, for two CTAs
+    e = cudaFuncSetAttribute(prompt_attention_kernel<D, BK>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(heads), static_cast<unsigned>(a.n_q));
@@ -412,8 +428,15 @@ cudaError_t launch_attention_d(const CUtensorMap& tq, const CUtensorMap& tk, con
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, prompt_attention_kernel<D>, tq, tk, tv, a);
+  return cudaLaunchKernelEx(&cfg, prompt_attention_kernel<D, BK>, tq, tk, tv, a);
 }
+
+// Key tiles of 64 positions: with the two-stage K/V ring and the P tile, a CTA takes 112 KB of
+// shared memory (D = 128) and 256 tensor-memory columns, so two CTAs share each SM and one's
+// products run while the other's softmax works.
+constexpr int kKeyTile = 64;
+static_assert(AttnLayout<128, kKeyTile>::kMinBlocks == 2 && AttnLayout<64, kKeyTile>::kMinBlocks == 2,
+              "two CTAs per SM");
 
 }  // namespace
 
@@ -427,8 +450,8 @@ cudaError_t launch_prompt_attention(const void* qkv, int64_t T, int heads, int k
   if (!encode_bf16_tmap(&tq, qkv, static_cast<uint64_t>(T), ncols, ncols, kAttnTile)) return cudaErrorInvalidValue;
   // caches [position, kv head, channel], of which positions 0 .. T-1 (later ones read as zero)
   const uint64_t s1 = static_cast<uint64_t>(head_dim) * 2, s2 = static_cast<uint64_t>(kv_heads) * head_dim * 2;
-  if (!encode_bf16_tmap_3d(&tk, k_cache, head_dim, kv_heads, static_cast<uint64_t>(T), s1, s2, 64, 1, kAttnTile) ||
-      !encode_bf16_tmap_3d(&tv, v_cache, head_dim, kv_heads, static_cast<uint64_t>(T), s1, s2, 64, 1, kAttnTile))
+  if (!encode_bf16_tmap_3d(&tk, k_cache, head_dim, kv_heads, static_cast<uint64_t>(T), s1, s2, 64, 1, kKeyTile) ||
+      !encode_bf16_tmap_3d(&tv, v_cache, head_dim, kv_heads, static_cast<uint64_t>(T), s1, s2, 64, 1, kKeyTile))
     return cudaErrorInvalidValue;
   AttnArgs a;
   a.T = static_cast<int>(T);
@@ -438,8 +461,8 @@ cudaError_t launch_prompt_attention(const void* qkv, int64_t T, int heads, int k
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(head_dim)));
   a.out = static_cast<__nv_bfloat16*>(out);
   a.err = err;
-  return head_dim == 64 ? launch_attention_d<64>(tq, tk, tv, a, heads, stream)
-                        : launch_attention_d<128>(tq, tk, tv, a, heads, stream);
+  return head_dim == 64 ? launch_attention_d<64, kKeyTile>(tq, tk, tv, a, heads, stream)
+                        : launch_attention_d<128, kKeyTile>(tq, tk, tv, a, heads, stream);
 }
 
 }  // namespace ttq

@@ -183,8 +183,10 @@ cudaError_t launch_rmsnorm(const void* y, void* residual, const void* w, int64_t
                            cudaStream_t stream);
 // fp32 (cos, sin) pairs of pos * base^(-2i/D) for pos < positions, i < D/2.
 cudaError_t launch_rope_table(int64_t positions, int head_dim, double base, float* table, cudaStream_t stream);
-// Device error word bit: a position read from device memory was outside the cache.
+// Device error word bits: a position read from device memory was outside the cache; a
+// kernel's shared-memory layout did not fit its allocation (it returned without work).
 constexpr unsigned kErrRange = 2u;
+constexpr unsigned kErrLayout = 4u;
 
 // Per-head RMSNorm + rotary embedding of q (in place) and k (into k_cache), v copied into
 // v_cache, for T tokens of the stacked projection at positions pos0 ... (pos0 = *pos_dev
