@@ -81,3 +81,97 @@ def test_whole_job_throughput_formula():
 
     # two ranks, 4096 tokens each per step, 10 steps, slowest rank 20 ms
     assert bench.whole_job_ktoks(4096, 10, 2, 20.0) == pytest.approx(2 * 4096 * 10 / 0.02 / 1e3)
+
+
+# ------------------------------------------------------------------ one linear split by output rows
+
+
+class _OracleBlock:
+    """A rank's block of a TTQ linear computed by the CPU oracle (stands in for the CUDA
+    layer in these CPU tests): prefill keeps s and the codes, decode reuses them."""
+
+    def __init__(self, W_block, q, g, alpha, lam):
+        self.W, self.q, self.g, self.alpha, self.lam = W_block, q, g, alpha, lam
+
+    def prefill(self, X):
+        from oracle import ttq_oracle as O
+
+        out = O.prefill(X.numpy(), self.W, self.q, self.g, self.alpha, self.lam)
+        self.s32, self.codes, self.scale, self.zero = out["s32"], out["codes"], out["scale"], out["zero"]
+        return torch.from_numpy(out["Y"])
+
+    def decode(self, X):
+        from oracle import ttq_oracle as O
+
+        return torch.from_numpy(O.linear(X.numpy(), self.s32, self.codes, self.scale, self.zero, self.g))
+
+
+def _split_worker(rank, world, port, q_):
+    os.environ.update({"RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    try:
+        import numpy as np
+
+        from online_activation_aware_b200 import synthetic
+        from online_activation_aware_b200.tensor_parallel import ColumnParallelTTQLinear, shard_rows
+
+        assert D.init("gloo", timeout_s=60) == world
+        T, d, d_out, q, g = 48, 256, 96, 4, 64
+        X, W = synthetic.draw_layer(T, d, d_out, seed=17)
+        Xv = synthetic.bf16_values(synthetic.as_bf16(X))
+        Wv = synthetic.bf16_values(synthetic.as_bf16(W))
+        lo, hi = shard_rows(d_out, rank, world)
+        layer = ColumnParallelTTQLinear(local=_OracleBlock(Wv[lo:hi], q, g, 0.5, 0.4))
+        Y = layer.prefill(torch.from_numpy(Xv)).numpy()
+        xt = synthetic.bf16_values(synthetic.as_bf16(synthetic.draw_tokens(3, d, seed=18)))
+        Yd = layer.decode(torch.from_numpy(xt)).numpy()
+        blk = layer.local
+        q_.put((rank, Y, Yd, blk.s32, blk.codes, lo, hi))
+        D.barrier()
+        D.finalize()
+    except Exception as e:
+        q_.put((rank, "error", repr(e)))
+
+
+def test_column_split_two_gloo_ranks_matches_whole_layer():
+    # each rank re-quantizes its 48 of 96 rows from its own (identical) statistic; the
+    # gathered Y and decode rows equal the whole layer's, and each rank's codes are the
+    # whole layer's codes of its rows
+    import numpy as np
+
+    from online_activation_aware_b200 import synthetic
+    from oracle import ttq_oracle as O
+
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q_ = ctx.Queue()
+    procs = [ctx.Process(target=_split_worker, args=(r, world, port, q_)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = sorted([q_.get(timeout=180) for _ in range(world)], key=lambda o: o[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for o in out:
+        assert not (isinstance(o[1], str) and o[1] == "error"), o
+    X, W = synthetic.draw_layer(48, 256, 96, seed=17)
+    Xv = synthetic.bf16_values(synthetic.as_bf16(X))
+    Wv = synthetic.bf16_values(synthetic.as_bf16(W))
+    full = O.prefill(Xv, Wv, 4, 64, 0.5, 0.4)
+    xt = synthetic.bf16_values(synthetic.as_bf16(synthetic.draw_tokens(3, 256, seed=18)))
+    Yd_full = O.linear(xt, full["s32"], full["codes"], full["scale"], full["zero"], 64)
+    for rank, Y, Yd, s32, codes, lo, hi in out:
+        np.testing.assert_allclose(Y, full["Y"], rtol=1e-12, atol=1e-12 * np.abs(full["Y"]).max())
+        np.testing.assert_allclose(Yd, Yd_full, rtol=1e-12, atol=1e-12 * np.abs(Yd_full).max())
+        np.testing.assert_array_equal(s32, full["s32"])
+        np.testing.assert_array_equal(codes, full["codes"][lo:hi])
+
+
+def test_shard_rows_blocks():
+    from online_activation_aware_b200.tensor_parallel import shard_rows
+
+    assert [shard_rows(8192, r, 4) for r in range(4)] == [(0, 2048), (2048, 4096), (4096, 6144), (6144, 8192)]
+    for d_out, world in ((100, 2), (96, 5), (8, 2)):
+        with pytest.raises(ValueError):
+            shard_rows(d_out, 0, world)
