@@ -17,7 +17,8 @@
 //             causal mask on the diagonal tile, new row maximum, P = exp2(s - m) rounded to
 //             bf16 into shared memory as the A operand of the second product, the running sum
 //             from the same rounded values, and the rescaling of O in tensor memory by
-//             exp2(m_old - m_new) before the next product lands; at the end O / l in bf16.
+//             exp2(m_old - m_new) before the next product lands, only when some row's
+//             maximum has risen by more than 2^8; at the end O / l in bf16.
 // The probabilities are rounded to bf16 for the tensor cores (the sum uses the rounded
 // values, so the normalisation matches them); scores, maxima, sums and O stay fp32.
 // Every mbarrier wait is bounded: a CTA that gives up records TTQ_ERR_TIMEOUT, drains the
@@ -33,6 +34,7 @@ namespace {
 
 constexpr int kAttnTile = 128;        // queries per CTA
 constexpr int kAttnThreads = 192;     // 6 warps
+constexpr float kRescaleSlack = 8.0f;  // log2 units a row maximum may rise before O is rescaled
 constexpr uint32_t kRowBox = 128 * 128;                  // 128 rows x 128 B (64 bf16): a Q or P box
 
 struct AttnBars {
@@ -318,13 +320,20 @@ __global__ void __launch_bounds__(kAttnThreads, AttnLayout<D, BK>::kMinBlocks)
       // scaled scores (log2 units); keys after the query (the diagonal tiles) are masked:
       // key j * BK + k is visible to row q0 + r when k <= q0 + r - j * BK
       const int lim = min(BK - 1, q0 + r - j * BK);
-      float mx = m;
+      // the row maximum as four interleaved chains (a 64-deep chain would set the latency)
+      float mx4[4] = {m, -FLT_MAX, -FLT_MAX, -FLT_MAX};
 #pragma unroll
       for (int k = 0; k < BK; ++k) {
         const float sv = k <= lim ? __fmul_rn(__uint_as_float(sr[k]), c) : -FLT_MAX;
         sr[k] = __float_as_uint(sv);
-        mx = fmaxf(mx, sv);
+        mx4[k & 3] = fmaxf(mx4[k & 3], sv);
       }
+      float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      // the row keeps its reference maximum until the tile's maximum exceeds it by more
+      // than kRescaleSlack (log2 units): P = exp2(s - m) then stays below 2^kRescaleSlack
+      // (exact in range for bf16, and l sums the same values), and O is rescaled in tensor
+      // memory only when some row of the warp moves its reference
+      if (mx <= m + kRescaleSlack) mx = m;
       const float corr = exp2_approx(__fsub_rn(m, mx));
       if (j > 0) {
         // P_{j-1} V_{j-1} has landed: O may be rescaled and the P buffer rewritten
@@ -349,7 +358,7 @@ __global__ void __launch_bounds__(kAttnThreads, AttnLayout<D, BK>::kMinBlocks)
       // P = exp2(s - m) rounded to bf16 into the swizzled K-major A tile (row r, positions in
       // 16-byte chunks of 8: chunk k8 of box k8 / 8 at slot (k8 % 8) ^ (r % 8)); the row sum
       // adds the rounded values
-      float rs = 0.f;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};  // the row sum as four chains, added in a fixed order
       const uint32_t prow = base + kOffP + r * 128;
 #pragma unroll
       for (int k8 = 0; k8 < BK / 8; ++k8) {
@@ -359,13 +368,14 @@ __global__ void __launch_bounds__(kAttnThreads, AttnLayout<D, BK>::kMinBlocks)
           const float p0 = exp2_approx(__fsub_rn(__uint_as_float(sr[8 * k8 + 2 * e]), mx));
           const float p1 = exp2_approx(__fsub_rn(__uint_as_float(sr[8 * k8 + 2 * e + 1]), mx));
           w[e] = pack_bf16x2(p0, p1);
-          rs = __fadd_rn(rs, __fadd_rn(bf16lo_to_f32(w[e]), bf16hi_to_f32(w[e])));
+          rs4[e] = __fadd_rn(rs4[e], __fadd_rn(bf16lo_to_f32(w[e]), bf16hi_to_f32(w[e])));
         }
         const uint32_t addr = prow + (k8 >> 3) * kRowBox + (((k8 & 7) ^ (r & 7)) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]),
                      "r"(w[3])
                      : "memory");
       }
+      const float rs = __fadd_rn(__fadd_rn(rs4[0], rs4[1]), __fadd_rn(rs4[2], rs4[3]));
       l = __fmaf_rn(l, corr, rs);
       m = mx;
       fence_proxy_async_smem();  // the tensor cores read P through the async proxy
