@@ -139,9 +139,9 @@ __global__ void __launch_bounds__(256) act_stats_kernel(const __nv_bfloat16* __r
 //   - the order of every sum is fixed (lanes' rows in row order, warps in warp order,
 //     splits in cluster rank order), so s is deterministic;
 //   - the kernel is launched as a programmatic dependent (its launch overlaps the tail
-//     of the kernel ahead, which it waits for before it reads X) and lets the next kernel
-//     of the stream launch at once: that kernel's set-up and first loads overlap this
-//     pass over X.
+//     of the kernel ahead, which it waits for before it reads X), and once that wait is
+//     over lets the next kernel of the stream launch: that kernel's set-up and first loads
+//     overlap this pass over X.
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -180,8 +180,7 @@ __global__ void __launch_bounds__(256) stats_cluster_kernel(const __nv_bfloat16*
                                                             float* __restrict__ s) {
   __shared__ float red[kRowWarps][kColsPerBlock];
   __shared__ float colsum[kColsPerBlock];
-  grid_dep_launch();
-  grid_dep_wait();  // X (and s) may be written by the kernel ahead in the stream
+  pdl_enter();  // X (and s) may be written by the kernel ahead in the stream
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int col0 = blockIdx.x * kColsPerBlock + lane * 8;
@@ -262,8 +261,7 @@ __global__ void __launch_bounds__(288) stats_tma_kernel(const __grid_constant__ 
                                                         float lambda, float* __restrict__ s, DevErr err) {
   extern __shared__ uint8_t smem_raw[];
   StatsSmem* sm = reinterpret_cast<StatsSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  grid_dep_launch();
-  grid_dep_wait();  // X (and s) may be written by the kernel ahead in the stream
+  pdl_enter();  // X (and s) may be written by the kernel ahead in the stream
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;

@@ -204,8 +204,7 @@ __global__ void __launch_bounds__(kAttnThreads, AttnLayout<D, BK>::kMinBlocks)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  grid_dep_launch();
-  grid_dep_wait();  // q, k and v are written by the kernel ahead in the stream
+  pdl_enter();  // q, k and v are written by the kernel ahead in the stream
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {

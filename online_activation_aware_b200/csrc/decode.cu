@@ -216,7 +216,8 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
       }
     }
   }
-  grid_dep_wait();  // x' and its unit sums are written by the prep kernel
+  grid_dep_wait();    // x' and its unit sums are written by the prep kernel
+  grid_dep_launch();  // the next kernel of the stream may begin launching
   __syncthreads();  // meta is in place
 
   float pacc[R][B];
@@ -348,7 +349,7 @@ template <int B>
 __global__ void __launch_bounds__(256) decode_prep_kernel(const __nv_bfloat16* __restrict__ X, int nb, int d,
                                                           const float* __restrict__ s, float* __restrict__ xp,
                                                           float* __restrict__ usum, int64_t wsf) {
-  grid_dep_launch();  // the GEMV may start loading codes
+  pdl_enter();  // X is written by the kernel ahead; then the GEMV may start loading codes
   {
     // request blockIdx.y of a batched decode: its own tokens, statistic and x'
     const int64_t rq = blockIdx.y;
@@ -393,9 +394,9 @@ cudaError_t launch_qb(const DecodeArgs& a, uint8_t* ws, cudaStream_t stream) {
   float* usum = reinterpret_cast<float*>(ws + round16(static_cast<size_t>(a.d) * B * 4));
   const int units = static_cast<int>(a.d / 32);
   const int64_t wsf = static_cast<int64_t>(gemv_ws_bytes(a.b, a.d) / 4);  // one request's workspace, floats
-  decode_prep_kernel<B><<<dim3((units * B + 7) / 8, a.requests), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(a.X), static_cast<int>(a.b), static_cast<int>(a.d), a.s, xp, usum, wsf);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(decode_prep_kernel<B>, dim3((units * B + 7) / 8, a.requests), dim3(256), 0, stream,
+                             static_cast<const __nv_bfloat16*>(a.X), static_cast<int>(a.b), static_cast<int>(a.d), a.s,
+                             xp, usum, wsf);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   const size_t smem = static_cast<size_t>(kRowsPerCta) * (a.d / a.g) * sizeof(float2);

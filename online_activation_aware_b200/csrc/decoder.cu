@@ -64,6 +64,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const __nv_bfloat
                                                               __nv_bfloat16* __restrict__ residual,
                                                               const __nv_bfloat16* __restrict__ w,
                                                               __nv_bfloat16* __restrict__ out, int n, float eps) {
+  pdl_enter();
   __shared__ float red[kNormThreads / 32];
   const int64_t row = blockIdx.x;
   const int nchunks = n >> 3;
@@ -167,6 +168,7 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(__nv_bfloat16* __rest
                                                           __nv_bfloat16* __restrict__ k_cache,
                                                           __nv_bfloat16* __restrict__ v_cache,
                                                           unsigned* __restrict__ err) {
+  pdl_enter();
   using V = typename LaneVec<E>::T;
   constexpr int D = 32 * E;
   const int lane = threadIdx.x & 31;
@@ -227,6 +229,7 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(__nv_bfloat16* __rest
 // out[t, c] = bf16(silu(gu[t, c]) * gu[t, I + c]), silu(u) = u / (1 + e^-u).
 __global__ void __launch_bounds__(256) silu_mul_kernel(const __nv_bfloat16* __restrict__ gu, int64_t rows,
                                                       int64_t inter, __nv_bfloat16* __restrict__ out) {
+  pdl_enter();
   const int64_t per_row = inter >> 3;
   const int64_t total = rows * per_row;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
@@ -267,6 +270,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_partial_kernel(
     const __nv_bfloat16* __restrict__ v_cache, int kv_heads, int64_t cache_len, int64_t length,
     const int64_t* __restrict__ pos_dev, int splits, float scale, float* __restrict__ part,
     unsigned* __restrict__ err) {
+  pdl_enter();
   using V = typename LaneVec<E>::T;
   constexpr int D = 32 * E;
   constexpr int kWarps = kDecThreads / 32;
@@ -407,6 +411,7 @@ __global__ void __launch_bounds__(256) decode_attn_combine_kernel(const float* _
   __shared__ float red[8];
   __shared__ float Msh, Lsh;
   grid_dep_wait();
+  grid_dep_launch();
   const int h = blockIdx.x;
   const int kh = h / G;
   const int g = h - kh * G;
@@ -462,7 +467,10 @@ __global__ void __launch_bounds__(256) decode_attn_combine_kernel(const float* _
   }
 }
 
-__global__ void position_advance_kernel(int64_t* pos, int64_t n) { *pos += n; }
+__global__ void position_advance_kernel(int64_t* pos, int64_t n) {
+  pdl_enter();
+  *pos += n;
+}
 
 }  // namespace
 
@@ -482,9 +490,8 @@ static cudaError_t decode_attn_partial(dim3 grid, cudaStream_t stream, const __n
                                        const __nv_bfloat16* kc, const __nv_bfloat16* vc, int kv_heads,
                                        int64_t cache_len, int64_t length, const int64_t* pos_dev, int splits,
                                        float scale, float* part, unsigned* err) {
-  decode_attn_partial_kernel<E, G><<<grid, kDecThreads, 0, stream>>>(q, kc, vc, kv_heads, cache_len, length,
-                                                                      pos_dev, splits, scale, part, err);
-  return cudaGetLastError();
+  return launch_pdl(decode_attn_partial_kernel<E, G>, grid, dim3(kDecThreads), 0, stream, q, kc, vc, kv_heads,
+                    cache_len, length, pos_dev, splits, scale, part, err);
 }
 
 cudaError_t launch_decode_attention(const void* q, int heads, int kv_heads, int head_dim, const void* k_cache,
@@ -510,8 +517,7 @@ cudaError_t launch_decode_attention(const void* q, int heads, int kv_heads, int 
 }
 
 cudaError_t launch_position_advance(int64_t* pos, int64_t n, cudaStream_t stream) {
-  position_advance_kernel<<<1, 1, 0, stream>>>(pos, n);
-  return cudaGetLastError();
+  return launch_pdl(position_advance_kernel, dim3(1), dim3(1), 0, stream, pos, n);
 }
 
 namespace {
@@ -525,13 +531,9 @@ cudaError_t launch_rmsnorm(const void* y, void* residual, const void* w, int64_t
   auto ww = static_cast<const __nv_bfloat16*>(w);
   auto oo = static_cast<__nv_bfloat16*>(out);
   const dim3 grid(static_cast<unsigned>(rows));
-  if (cpt <= 1)
-    rmsnorm_kernel<1><<<grid, kNormThreads, 0, stream>>>(yy, rr, ww, oo, n, eps);
-  else if (cpt <= 2)
-    rmsnorm_kernel<2><<<grid, kNormThreads, 0, stream>>>(yy, rr, ww, oo, n, eps);
-  else
-    rmsnorm_kernel<4><<<grid, kNormThreads, 0, stream>>>(yy, rr, ww, oo, n, eps);
-  return cudaGetLastError();
+  if (cpt <= 1) return launch_pdl(rmsnorm_kernel<1>, grid, dim3(kNormThreads), 0, stream, yy, rr, ww, oo, n, eps);
+  if (cpt <= 2) return launch_pdl(rmsnorm_kernel<2>, grid, dim3(kNormThreads), 0, stream, yy, rr, ww, oo, n, eps);
+  return launch_pdl(rmsnorm_kernel<4>, grid, dim3(kNormThreads), 0, stream, yy, rr, ww, oo, n, eps);
 }
 
 cudaError_t launch_rope_table(int64_t positions, int head_dim, double base, float* table, cudaStream_t stream) {
@@ -555,26 +557,24 @@ cudaError_t launch_qk_norm_rope(void* qkv, int64_t T, int heads, int kv_heads, i
   auto vc = static_cast<__nv_bfloat16*>(v_cache);
   switch (head_dim) {
     case 64:
-      qk_norm_rope_kernel<2><<<grid, 256, 0, stream>>>(q, T, heads, kv_heads, a, b, eps, tb, pos0, pos_dev, limit, kc, vc, err);
-      break;
+      return launch_pdl(qk_norm_rope_kernel<2>, grid, dim3(256), 0, stream, q, T, heads, kv_heads, a, b, eps, tb, pos0,
+                        pos_dev, limit, kc, vc, err);
     case 128:
-      qk_norm_rope_kernel<4><<<grid, 256, 0, stream>>>(q, T, heads, kv_heads, a, b, eps, tb, pos0, pos_dev, limit, kc, vc, err);
-      break;
+      return launch_pdl(qk_norm_rope_kernel<4>, grid, dim3(256), 0, stream, q, T, heads, kv_heads, a, b, eps, tb, pos0,
+                        pos_dev, limit, kc, vc, err);
     case 256:
-      qk_norm_rope_kernel<8><<<grid, 256, 0, stream>>>(q, T, heads, kv_heads, a, b, eps, tb, pos0, pos_dev, limit, kc, vc, err);
-      break;
+      return launch_pdl(qk_norm_rope_kernel<8>, grid, dim3(256), 0, stream, q, T, heads, kv_heads, a, b, eps, tb, pos0,
+                        pos_dev, limit, kc, vc, err);
     default:
       return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_silu_mul(const void* gu, int64_t rows, int64_t inter, void* out, int num_sms, cudaStream_t stream) {
   const int64_t total = rows * (inter / 8);
   const int64_t blocks = std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(num_sms) * 8);
-  silu_mul_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(gu), rows,
-                                                                      inter, static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError();
+  return launch_pdl(silu_mul_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+                    static_cast<const __nv_bfloat16*>(gu), rows, inter, static_cast<__nv_bfloat16*>(out));
 }
 
 }  // namespace ttq

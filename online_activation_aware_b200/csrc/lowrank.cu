@@ -53,6 +53,7 @@ template <int NT>
 __global__ void __launch_bounds__(kLrThreads) lowrank_partial_kernel(const __nv_bfloat16* __restrict__ X, int T,
                                                                      int d, const __nv_bfloat16* __restrict__ A,
                                                                      int kc, float* __restrict__ part) {
+  pdl_enter();
   constexpr int R = NT * 8;
   constexpr uint32_t kXBytes = kLrTok * kLrK * 2;  // 8 KB
   constexpr uint32_t kABytes = R * kLrK * 2;
@@ -145,6 +146,7 @@ __global__ void __launch_bounds__(kLrThreads) lowrank_partial_kernel(const __nv_
 __global__ void __launch_bounds__(256) lowrank_reduce_kernel(const float* __restrict__ part, int T, int r, int ks,
                                                              __nv_bfloat16* __restrict__ U) {
   grid_dep_wait();
+  grid_dep_launch();
   const int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;  // t * 64 + j
   if (e >= static_cast<int64_t>(T) * 64) return;
   const int t = static_cast<int>(e >> 6), j = static_cast<int>(e & 63);
@@ -160,6 +162,7 @@ __global__ void __launch_bounds__(256) lowrank_reduce_kernel(const float* __rest
 __global__ void __launch_bounds__(256) lowrank_small_kernel(const __nv_bfloat16* __restrict__ X, int d,
                                                             const __nv_bfloat16* __restrict__ A, int r,
                                                             __nv_bfloat16* __restrict__ U) {
+  pdl_enter();
   __shared__ float red[8];
   const int t = blockIdx.x >> 6, j = blockIdx.x & 63;
   if (j >= r) {
@@ -212,10 +215,9 @@ size_t lowrank_partial_bytes(int64_t T, int64_t d, int r, int num_sms) {
 cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A, int r, void* U, float* partial,
                              int num_sms, cudaStream_t stream) {
   if (T <= kLrSmallTokens) {
-    lowrank_small_kernel<<<static_cast<unsigned>(T * 64), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(X), static_cast<int>(d), static_cast<const __nv_bfloat16*>(A), r,
-        static_cast<__nv_bfloat16*>(U));
-    return cudaGetLastError();
+    return launch_pdl(lowrank_small_kernel, dim3(static_cast<unsigned>(T * 64)), dim3(256), 0, stream,
+                      static_cast<const __nv_bfloat16*>(X), static_cast<int>(d), static_cast<const __nv_bfloat16*>(A),
+                      r, static_cast<__nv_bfloat16*>(U));
   }
   const int ks = lowrank_splits(T, d, num_sms);
   const int64_t kst = (d + kLrK - 1) / kLrK;
@@ -225,17 +227,18 @@ cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A,
   const auto* Xb = static_cast<const __nv_bfloat16*>(X);
   const auto* Ab = static_cast<const __nv_bfloat16*>(A);
   const int Ti = static_cast<int>(T), di = static_cast<int>(d);
+  cudaError_t e;
+  const dim3 blk(kLrThreads);
   switch (r / 8) {
-    case 1: lowrank_partial_kernel<1><<<grid, kLrThreads, 0, stream>>>(Xb, Ti, di, Ab, kc, partial); break;
-    case 2: lowrank_partial_kernel<2><<<grid, kLrThreads, 0, stream>>>(Xb, Ti, di, Ab, kc, partial); break;
-    case 3: lowrank_partial_kernel<3><<<grid, kLrThreads, 0, stream>>>(Xb, Ti, di, Ab, kc, partial); break;
-    case 4: lowrank_partial_kernel<4><<<grid, kLrThreads, 0, stream>>>(Xb, Ti, di, Ab, kc, partial); break;
-    case 5: lowrank_partial_kernel<5><<<grid, kLrThreads, 0, stream>>>(Xb, Ti, di, Ab, kc, partial); break;
-    case 6: lowrank_partial_kernel<6><<<grid, kLrThreads, 0, stream>>>(Xb, Ti, di, Ab, kc, partial); break;
-    case 7: lowrank_partial_kernel<7><<<grid, kLrThreads, 0, stream>>>(Xb, Ti, di, Ab, kc, partial); break;
-    default: lowrank_partial_kernel<8><<<grid, kLrThreads, 0, stream>>>(Xb, Ti, di, Ab, kc, partial); break;
+    case 1: e = launch_pdl(lowrank_partial_kernel<1>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
+    case 2: e = launch_pdl(lowrank_partial_kernel<2>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
+    case 3: e = launch_pdl(lowrank_partial_kernel<3>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
+    case 4: e = launch_pdl(lowrank_partial_kernel<4>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
+    case 5: e = launch_pdl(lowrank_partial_kernel<5>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
+    case 6: e = launch_pdl(lowrank_partial_kernel<6>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
+    case 7: e = launch_pdl(lowrank_partial_kernel<7>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
+    default: e = launch_pdl(lowrank_partial_kernel<8>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
   }
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>((T * 64 + 255) / 256));

@@ -234,6 +234,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
+// First statement of a kernel launched as a programmatic dependent (launch_pdl): waits until
+// the kernel ahead in the stream has completed and its writes are visible, before any
+// global memory is touched, then lets the next kernel of the stream begin launching. Every
+// kernel of a chain doing this keeps the chain fully ordered while each launch overlaps the
+// tail of the kernel before it.
+__device__ __forceinline__ void pdl_enter() {
+  grid_dep_wait();
+  grid_dep_launch();
+}
+
 // ------------------------------------------------------------------ L2 eviction hints
 
 // Cache policy that marks the lines an access touches as the first to evict from L2:

@@ -6,9 +6,30 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "ttq_common.cuh"
 
 namespace ttq {
+
+// Launches `kernel` with programmatic stream serialization: it may start launching while the
+// kernel ahead in the stream finishes, so it must begin with pdl_enter() (or wait with
+// grid_dep_wait() before it reads anything that kernel writes).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Identifier (cuCtxGetId) of the CUDA context current on this host thread; when none is,
 // the current device's primary context is bound first. False when the driver refuses.
@@ -35,7 +56,8 @@ StatsPlan cluster_plan(int64_t T, int64_t d, int num_sms);
 
 // s = (mean_t |x|^p + lambda)^(alpha/p) in one launch with no scratch memory (the row
 // splits of a strip reduce through distributed shared memory); launched with programmatic
-// stream serialization and lets the next kernel launch at once.
+// stream serialization: it waits for the kernel ahead before it reads X, then lets the
+// next kernel launch.
 // X streams through a TMA ring in shared memory (every wait bounded by err.wait_ns).
 cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d, int64_t ld_x, float alpha, float lambda, int p,
                              float* s, int num_sms, const DevErr& err, cudaStream_t stream);
