@@ -505,8 +505,9 @@ def main():
             v["frac"] = round(v["TFLOPs"] / tc_peak, 4)
         v["ms"] = round(v["ms"], 5)
     # the GEMM's stage time comes from steps run right after the timed region: against the
-    # sustained bf16 peak when that region was long or ran under the power cap, else the burst
-    long_run = t_max_ms >= 500.0 or "sw_power_cap" in (clocks.get("reasons") or [])
+    # sustained bf16 peak when the SM clock fell under the power cap there, else the burst
+    sm, smax = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    long_run = bool(sm and smax and sm < 0.95 * smax)  # the clock fell (power cap) in the timed region
     tc_ref = tc_sust if long_run else tc_peak
     kern["gemm"]["frac"] = round(kern["gemm"]["TFLOPs"] / tc_ref, 4)
     dom = max(kern, key=lambda k_: kern[k_]["ms"])
@@ -518,7 +519,7 @@ def main():
                 "frac_of_burst": round(dk["TFLOPs"] / tc_peak, 4),
                 "traffic": profiled_traffic("ttq_gemm2sm_kernel" if T > 128 else "ttq_gemm_kernel", wkey),
                 "algorithmic": f"2*T*d*d_out flops per launch = {dk['flops']:.4g}",
-                "peak_source": f"{peak_src} bf16 {'sustained (long, power-capped run)' if long_run else 'burst'} "
+                "peak_source": f"{peak_src} bf16 {'sustained (power-capped clock)' if long_run else 'burst'} "
                                "(MEASURED_PEAKS.json)"}
     else:
         roof = {"kernel": {"fold_requant": "requant_kernel", "stats": "stats_tma_kernel",

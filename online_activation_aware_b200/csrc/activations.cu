@@ -348,6 +348,7 @@ __global__ void __launch_bounds__(256) fold_kernel(const __nv_bfloat16* __restri
                                                    const float* __restrict__ s,
                                                    int64_t rows_per_split,
                                                    __nv_bfloat16* __restrict__ Xf) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int col0 = blockIdx.x * kColsPerBlock + lane * 8;
@@ -521,10 +522,8 @@ cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const
   const int64_t rps = (T + ns - 1) / ns;
   ns = (T + rps - 1) / rps;
   dim3 grid(col_blocks, static_cast<unsigned>(ns));
-  fold_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T,
-                                        static_cast<int>(d), ld_x, s, rps,
-                                        static_cast<__nv_bfloat16*>(Xf));
-  return cudaGetLastError();
+  return launch_pdl(fold_kernel, grid, dim3(256), 0, stream, static_cast<const __nv_bfloat16*>(X), T,
+                    static_cast<int>(d), ld_x, s, rps, static_cast<__nv_bfloat16*>(Xf));
 }
 
 }  // namespace ttq

@@ -263,6 +263,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   // launched as a programmatic dependent: the set-up above overlaps the end of the kernel
   // that writes X' (and the codes); no global memory is touched before this wait
   grid_dep_wait();
+  grid_dep_launch();  // the split-K reduction (or the next kernel) may begin launching
   const uint32_t tmem = tail->tmem_base;
 
   if (warp == 0) {
@@ -546,6 +547,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ partial,
                                                             int ksplit, int64_t n,
                                                             __nv_bfloat16* __restrict__ Y) {
+  pdl_enter();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += stride) {
     float acc = partial[e];
@@ -801,9 +803,8 @@ cudaError_t launch_gemm_reduce(const GemmArgs& a, const GemmPlan& plan, cudaStre
   const int64_t n = a.T * a.d_out;
   int64_t blocks = (n + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  splitk_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      a.partial, plan.ksplit, n, static_cast<__nv_bfloat16*>(a.Y));
-  return cudaGetLastError();
+  return launch_pdl(splitk_reduce_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+                    static_cast<const float*>(a.partial), plan.ksplit, n, static_cast<__nv_bfloat16*>(a.Y));
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, const GemmPlan& plan, const DevErr& err,

@@ -334,6 +334,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
   // launched as a programmatic dependent: the set-up above overlaps the end of the kernel
   // that writes X' and the codes; no global memory is touched before this wait
   grid_dep_wait();
+  grid_dep_launch();  // the next kernel of the stream may begin launching
   const uint32_t tmem = tail->tmem_base;
 
   if (warp == 0) {
