@@ -437,6 +437,27 @@ def main():
     torch.cuda.synchronize()
     assert ttq.device_status() == 0
 
+    # stage split: a separate run of the same steps with the library's stage events (each
+    # stage then starts only when the one before it has finished), right after the warm-up
+    # and before the timed region, with its own clock samples: the GEMM's roofline comes
+    # from it
+    Ks = max(3, min(K, 50))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(Ks)]
+    tsampler = NvmlClockSampler(gpu_uuid(torch, dev))
+    tsampler.start()
+    time.sleep(0.02)
+    tw0 = time.perf_counter()
+    for i in range(Ks):
+        ttq.set_trace_events(evs[i])
+        step(i)
+    torch.cuda.synchronize()
+    tsampler.window(tw0, time.perf_counter())
+    trace_clocks = tsampler.stop()
+    ttq.set_trace_events(None)
+    stage_names = ["stats", "lowrank_u", "fold_requant", "gemm", "reduce"]
+    stage_ms = {n: statistics.median(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(Ks))
+                for j, n in enumerate(stage_names)}
+
     # timed region: K prefill steps back to back (no stage events inside it: an event
     # between two kernels would stop the next one from starting early as a programmatic
     # dependent)
@@ -462,18 +483,6 @@ def main():
     t_ms = start.elapsed_time(end)
     t_max_ms = D.max_over_ranks(t_ms, dev)
 
-    # stage split: a separate run of the same steps with the library's stage events
-    # (each stage then starts only when the one before it has finished)
-    Ks = max(3, min(K, 50))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(Ks)]
-    for i in range(Ks):
-        ttq.set_trace_events(evs[i])
-        step(i)
-    torch.cuda.synchronize()
-    ttq.set_trace_events(None)
-    stage_names = ["stats", "lowrank_u", "fold_requant", "gemm", "reduce"]
-    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(Ks))
-                for j, n in enumerate(stage_names)}
     value = whole_job_ktoks(T, K, world, t_max_ms)
 
     plan_split = stage_ms["reduce"] > 0.002
@@ -504,10 +513,10 @@ def main():
             v["TFLOPs"] = round(v["flops"] / sec / 1e12, 1)
             v["frac"] = round(v["TFLOPs"] / tc_peak, 4)
         v["ms"] = round(v["ms"], 5)
-    # the GEMM's stage time comes from steps run right after the timed region: against the
-    # sustained bf16 peak when the SM clock fell under the power cap there, else the burst
-    sm, smax = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
-    long_run = bool(sm and smax and sm < 0.95 * smax)  # the clock fell (power cap) in the timed region
+    # the GEMM's stage time comes from the traced steps: against the sustained bf16 peak
+    # when the SM clock fell under the power cap there, else the burst
+    sm, smax = trace_clocks.get("sm_mhz"), trace_clocks.get("sm_max_mhz")
+    long_run = bool(sm and smax and sm < 0.95 * smax)  # the clock fell (power cap) during the traced steps
     tc_ref = tc_sust if long_run else tc_peak
     kern["gemm"]["frac"] = round(kern["gemm"]["TFLOPs"] / tc_ref, 4)
     dom = max(kern, key=lambda k_: kern[k_]["ms"])
@@ -535,6 +544,7 @@ def main():
         "config": bench_config(wl, T, r, world),
         "requant_gbs": requant_leg(torch, ttq, Ws, outs, d, d_out, q, g, flush, sink),
         "stage_trace_ms": {k_: round(v, 5) for k_, v in stage_ms.items()},
+        "stage_trace_clocks": trace_clocks,
         "act_stats_standalone": stats_sa,
         "requant_batched": requant_batched_leg(torch, ttq, Ws, outs, d, d_out, q, g),
         "roofline": roof,
