@@ -55,12 +55,6 @@ __device__ __forceinline__ void accum8(float (&acc)[8], const uint4& v) {
   }
 }
 
-__device__ __forceinline__ float finalize_scale(float colsum, float T, float alpha_over_p,
-                                                float lambda) {
-  const float m = __fdiv_rn(colsum, T);  // mean over the prompt's tokens
-  return powf(__fadd_rn(m, lambda), alpha_over_p);
-}
-
 // grid: (col_blocks, nsplit); block: 256 threads. Each block reduces its rows for 256
 // columns into partial[split, col]; the last block of a column strip (in arrival order,
 // counted in `counters`) sums the strip's partials in split order and writes s. The

@@ -6,11 +6,18 @@
 // A skinny product (r <= 64 outputs per token) bound by the single read of X. Block
 // (token block of 64, K split ks) streams its [64 x Kc] slice of X and the matching
 // [r x Kc] slice of A through a 3-stage cp.async ring in shared memory (16-byte chunks,
-// XOR-swizzled rows so that ldmatrix is conflict-free), and each of its 4 warps multiplies
-// 16 tokens by A^T with mma.sync m16n8k16 (bf16 in, fp32 accumulate). The K splits write
+// XOR-swizzled rows so that ldmatrix is conflict-free), and each of its first 4 warps
+// multiplies 16 tokens by A^T with mma.sync m16n8k16 (bf16 in, fp32 accumulate). The K splits write
 // fp32 partial sums; a small dependent kernel adds them in split order (deterministic)
 // and stores U in bf16 with its row padded to 64 (columns r..63 zero). For a few tokens (a
 // decode step) one block computes each output over all of d instead.
+//
+// A prefill also needs the statistic s of the same X (paper-daily.com deep reading, section
+// 2: s from the prompt's per-channel |x|^p means). With P = 1 or 2 the partial kernel sums
+// |x|^p over its 64 tokens for every channel of each stage while the stage sits in shared
+// memory (for r >= 32 in 4 more warps of its own), and the dependent kernel adds those
+// rows in token-block order and finishes s: one read of X serves both, where a separate
+// statistic kernel would read it once more.
 #include "ttq_internal.h"
 
 namespace ttq {
@@ -48,16 +55,25 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
 // byte offset of 16-byte chunk c (0..7) of row `row` in a [rows x 64] bf16 tile
 __device__ __forceinline__ uint32_t swz(int row, int c) { return static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4)); }
 
-// grid: (token blocks, K splits); NT = r / 8 output tiles of 8 ranks.
-template <int NT>
-__global__ void __launch_bounds__(kLrThreads) lowrank_partial_kernel(const __nv_bfloat16* __restrict__ X, int T,
+// Threads of a block: with the statistic and r >= 32 four more warps take the statistic
+// (the multiplying warps are busier there); otherwise the 4 warps do both.
+template <int NT, int P>
+constexpr int lr_threads() { return (P != 0 && NT >= 4) ? 2 * kLrThreads : kLrThreads; }
+
+// grid: (token blocks, K splits); NT = r / 8 output tiles of 8 ranks; P = 0 (U only) or the
+// statistic's exponent, whose per-block column sums go to spart[token block][channel].
+template <int NT, int P>
+__global__ void __launch_bounds__(lr_threads<NT, P>()) lowrank_partial_kernel(const __nv_bfloat16* __restrict__ X, int T,
                                                                      int d, const __nv_bfloat16* __restrict__ A,
-                                                                     int kc, float* __restrict__ part) {
+                                                                     int kc, float* __restrict__ part,
+                                                                     float* __restrict__ spart) {
   pdl_enter();
   constexpr int R = NT * 8;
   constexpr uint32_t kXBytes = kLrTok * kLrK * 2;  // 8 KB
   constexpr uint32_t kABytes = R * kLrK * 2;
-  __shared__ __align__(128) uint8_t sm[kLrStages * (kXBytes + kABytes)];
+  extern __shared__ __align__(128) uint8_t sm[];  // kLrStages x (X tile, A tile)
+  constexpr int kThreads = lr_threads<NT, P>();
+  constexpr bool kSplit = kThreads > kLrThreads;  // warps 4..7 take the statistic
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
@@ -73,14 +89,14 @@ __global__ void __launch_bounds__(kLrThreads) lowrank_partial_kernel(const __nv_
       const uint32_t xs = sbase + slot * (kXBytes + kABytes);
       const uint32_t as = xs + kXBytes;
 #pragma unroll
-      for (int i = 0; i < (kLrTok * 8) / kLrThreads; ++i) {  // X: 64 rows x 8 chunks
-        const int e = tid + i * kLrThreads;
+      for (int i = 0; i < (kLrTok * 8) / kThreads; ++i) {  // X: 64 rows x 8 chunks
+        const int e = tid + i * kThreads;
         const int row = e >> 3, c = e & 7;
         const int t = min(t0 + row, T - 1);
         const int k = kb + c * 8;
         cp_async_16_zfill(xs + swz(row, c), X + static_cast<int64_t>(t) * d + (k < d ? k : 0), k < d);
       }
-      for (int e = tid; e < R * 8; e += kLrThreads) {  // A: R rows x 8 chunks
+      for (int e = tid; e < R * 8; e += kThreads) {  // A: R rows x 8 chunks
         const int row = e >> 3, c = e & 7;
         const int k = kb + c * 8;
         cp_async_16_zfill(as + swz(row, c), A + static_cast<int64_t>(row) * d + (k < d ? k : 0), k < d);
@@ -105,7 +121,7 @@ __global__ void __launch_bounds__(kLrThreads) lowrank_partial_kernel(const __nv_
     const uint32_t xs = sbase + slot * (kXBytes + kABytes);
     const uint32_t as = xs + kXBytes;
 #pragma unroll
-    for (int kk = 0; kk < kLrK / 16; ++kk) {
+    for (int kk = 0; kk < kLrK / 16 && (!kSplit || warp < 4); ++kk) {
       // A fragment: this warp's 16 tokens x 16 k (matrices: rows 0-7 / 8-15, k 0-7 / 8-15)
       uint32_t af[4];
       {
@@ -124,10 +140,44 @@ __global__ void __launch_bounds__(kLrThreads) lowrank_partial_kernel(const __nv_
         mma_bf16_16816(acc[n], af, bf[0], bf[1]);
       }
     }
+    if (P != 0 && (!kSplit || warp >= 4)) {
+      // sum of |x|^p over the block's tokens for the stage's 64 channels: lane (pair cp,
+      // quarter qr) takes channels 2cp, 2cp + 1 of rows 8 (i / 2) + 2 qr + i % 2, i = 0..15
+      // (under the row swizzle a warp's four quarters then read 32 different banks); rows
+      // past T (loaded as copies of the last token) are left out, and the quarters meet
+      // by two shuffles
+      const int cp = (warp & 3) * 8 + (lane & 7), qr = lane >> 3;
+      const int nrows = min(kLrTok, T - t0);
+      const uint8_t* xt = sm + slot * (kXBytes + kABytes) + (cp & 3) * 4;
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int row = 8 * (i >> 1) + 2 * qr + (i & 1);
+        if (row < nrows) {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(xt + swz(row, cp >> 2));
+          const float a = bf16lo_to_f32(w), b = bf16hi_to_f32(w);
+          if constexpr (P == 2) {
+            s0 = __fmaf_rn(a, a, s0);
+            s1 = __fmaf_rn(b, b, s1);
+          } else {
+            s0 = __fadd_rn(s0, fabsf(a));
+            s1 = __fadd_rn(s1, fabsf(b));
+          }
+        }
+      }
+      s0 = __fadd_rn(s0, __shfl_xor_sync(0xffffffffu, s0, 8));
+      s1 = __fadd_rn(s1, __shfl_xor_sync(0xffffffffu, s1, 8));
+      s0 = __fadd_rn(s0, __shfl_xor_sync(0xffffffffu, s0, 16));
+      s1 = __fadd_rn(s1, __shfl_xor_sync(0xffffffffu, s1, 16));
+      const int k = k0 + st * kLrK + 2 * cp;
+      if (qr == 0 && k < d)
+        *reinterpret_cast<float2*>(spart + static_cast<int64_t>(blockIdx.x) * d + k) = make_float2(s0, s1);
+    }
   }
   cp_async_wait<0>();
 
   // partial[ks][t][rank]: rows groupID and groupID + 8 of the warp's 16 tokens
+  if (kSplit && warp >= 4) return;
   const int g = lane >> 2, tig = lane & 3;
   float* pbase = part + static_cast<int64_t>(blockIdx.y) * T * R;
 #pragma unroll
@@ -142,17 +192,44 @@ __global__ void __launch_bounds__(kLrThreads) lowrank_partial_kernel(const __nv_
   }
 }
 
-// U[t][j] = bf16(sum over splits of part[ks][t][j]) for j < r, 0 for r <= j < 64.
+// U[t][j] = bf16(sum over splits of part[ks][t][j]) for j < r, 0 for r <= j < 64, in the
+// first ceil(T / 4) blocks. With P != 0 the blocks after them finish the statistic: block
+// c takes channels 32c .. 32c + 31, its warp w sums the token-block rows w, w + 8, ... of
+// spart in order, and warp 0 adds the 8 warp sums in order and writes s.
+template <int P>
 __global__ void __launch_bounds__(256) lowrank_reduce_kernel(const float* __restrict__ part, int T, int r, int ks,
-                                                             __nv_bfloat16* __restrict__ U) {
+                                                             __nv_bfloat16* __restrict__ U,
+                                                             const float* __restrict__ spart, int d,
+                                                             float alpha_over_p, float lambda, float* __restrict__ s) {
   grid_dep_wait();
   grid_dep_launch();
+  const int nu = (T + 3) >> 2;  // blocks of U (256 outputs each)
+  if constexpr (P != 0) {
+    if (static_cast<int>(blockIdx.x) >= nu) {
+      __shared__ float ws[8][32];
+      const int col = (static_cast<int>(blockIdx.x) - nu) * 32 + (threadIdx.x & 31);
+      const int w = threadIdx.x >> 5;
+      const int ntb = (T + kLrTok - 1) / kLrTok;
+      float v = 0.f;
+      if (col < d)
+        for (int tb = w; tb < ntb; tb += 8) v = __fadd_rn(v, spart[static_cast<int64_t>(tb) * d + col]);
+      ws[w][threadIdx.x & 31] = v;
+      __syncthreads();
+      if (w == 0 && col < d) {
+        float tot = ws[0][threadIdx.x];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) tot = __fadd_rn(tot, ws[i][threadIdx.x]);
+        s[col] = finalize_scale(tot, static_cast<float>(T), alpha_over_p, lambda);
+      }
+      return;
+    }
+  }
   const int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;  // t * 64 + j
   if (e >= static_cast<int64_t>(T) * 64) return;
   const int t = static_cast<int>(e >> 6), j = static_cast<int>(e & 63);
   float v = 0.f;
   if (j < r)
-    for (int s = 0; s < ks; ++s) v = __fadd_rn(v, part[(static_cast<int64_t>(s) * T + t) * r + j]);
+    for (int sp = 0; sp < ks; ++sp) v = __fadd_rn(v, part[(static_cast<int64_t>(sp) * T + t) * r + j]);
   U[e] = __float2bfloat16_rn(v);
 }
 
@@ -212,6 +289,62 @@ size_t lowrank_partial_bytes(int64_t T, int64_t d, int r, int num_sms) {
          sizeof(float);
 }
 
+int lowrank_small_tokens() { return kLrSmallTokens; }
+
+size_t lowrank_stats_bytes(int64_t T, int64_t d) {
+  return static_cast<size_t>((T + kLrTok - 1) / kLrTok) * static_cast<size_t>(d) * sizeof(float);
+}
+
+namespace {
+
+template <int NT, int P>
+cudaError_t launch_partial_nt(dim3 grid, const __nv_bfloat16* Xb, int T, int d, const __nv_bfloat16* Ab, int kc,
+                              float* partial, float* spart, cudaStream_t stream) {
+  constexpr size_t smem = static_cast<size_t>(kLrStages) * (kLrTok + NT * 8) * kLrK * 2;
+  const cudaError_t e =
+      cudaFuncSetAttribute(lowrank_partial_kernel<NT, P>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(lowrank_partial_kernel<NT, P>, grid, dim3(lr_threads<NT, P>()), smem, stream, Xb, T, d, Ab, kc, partial,
+                    spart);
+}
+
+template <int P>
+cudaError_t launch_partial(int nt, dim3 grid, const __nv_bfloat16* Xb, int T, int d, const __nv_bfloat16* Ab,
+                           int kc, float* partial, float* spart, cudaStream_t stream) {
+  switch (nt) {
+    case 1: return launch_partial_nt<1, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
+    case 2: return launch_partial_nt<2, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
+    case 3: return launch_partial_nt<3, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
+    case 4: return launch_partial_nt<4, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
+    case 5: return launch_partial_nt<5, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
+    case 6: return launch_partial_nt<6, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
+    case 7: return launch_partial_nt<7, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
+    default: return launch_partial_nt<8, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
+  }
+}
+
+// The partial kernel and its reduce; P = 0 for U alone, else also the statistic with
+// exponent P into s.
+template <int P>
+cudaError_t launch_tiled(const void* X, int64_t T, int64_t d, const void* A, int r, void* U, float* partial,
+                         float* spart, float alpha_over_p, float lambda, float* s, int num_sms, cudaStream_t stream) {
+  const int ks = lowrank_splits(T, d, num_sms);
+  const int64_t kst = (d + kLrK - 1) / kLrK;
+  const int kc = static_cast<int>((kst + ks - 1) / ks) * kLrK;
+  const int ksr = static_cast<int>((d + kc - 1) / kc);  // splits that hold any K
+  const dim3 grid(static_cast<unsigned>((T + kLrTok - 1) / kLrTok), static_cast<unsigned>(ksr));
+  const int Ti = static_cast<int>(T), di = static_cast<int>(d);
+  cudaError_t e = launch_partial<P>(r / 8, grid, static_cast<const __nv_bfloat16*>(X), Ti, di,
+                                    static_cast<const __nv_bfloat16*>(A), kc, partial, spart, stream);
+  if (e != cudaSuccess) return e;
+  const int64_t nblk = (T + 3) / 4 + (P != 0 ? (d + 31) / 32 : 0);
+  return launch_pdl(lowrank_reduce_kernel<P>, dim3(static_cast<unsigned>(nblk)), dim3(256), 0, stream,
+                    static_cast<const float*>(partial), Ti, r, ksr, static_cast<__nv_bfloat16*>(U),
+                    static_cast<const float*>(spart), di, alpha_over_p, lambda, s);
+}
+
+}  // namespace
+
 cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A, int r, void* U, float* partial,
                              int num_sms, cudaStream_t stream) {
   if (T <= kLrSmallTokens) {
@@ -219,38 +352,16 @@ cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A,
                       static_cast<const __nv_bfloat16*>(X), static_cast<int>(d), static_cast<const __nv_bfloat16*>(A),
                       r, static_cast<__nv_bfloat16*>(U));
   }
-  const int ks = lowrank_splits(T, d, num_sms);
-  const int64_t kst = (d + kLrK - 1) / kLrK;
-  const int kc = static_cast<int>((kst + ks - 1) / ks) * kLrK;
-  const int ksr = static_cast<int>((d + kc - 1) / kc);  // splits that hold any K
-  const dim3 grid(static_cast<unsigned>((T + kLrTok - 1) / kLrTok), static_cast<unsigned>(ksr));
-  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
-  const auto* Ab = static_cast<const __nv_bfloat16*>(A);
-  const int Ti = static_cast<int>(T), di = static_cast<int>(d);
-  cudaError_t e;
-  const dim3 blk(kLrThreads);
-  switch (r / 8) {
-    case 1: e = launch_pdl(lowrank_partial_kernel<1>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
-    case 2: e = launch_pdl(lowrank_partial_kernel<2>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
-    case 3: e = launch_pdl(lowrank_partial_kernel<3>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
-    case 4: e = launch_pdl(lowrank_partial_kernel<4>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
-    case 5: e = launch_pdl(lowrank_partial_kernel<5>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
-    case 6: e = launch_pdl(lowrank_partial_kernel<6>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
-    case 7: e = launch_pdl(lowrank_partial_kernel<7>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
-    default: e = launch_pdl(lowrank_partial_kernel<8>, grid, blk, 0, stream, Xb, Ti, di, Ab, kc, partial); break;
-  }
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((T * 64 + 255) / 256));
-  cfg.blockDim = dim3(256);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, lowrank_reduce_kernel, static_cast<const float*>(partial), Ti, r, ksr,
-                            static_cast<__nv_bfloat16*>(U));
+  return launch_tiled<0>(X, T, d, A, r, U, partial, nullptr, 0.f, 0.f, nullptr, num_sms, stream);
+}
+
+cudaError_t launch_lowrank_u_stats(const void* X, int64_t T, int64_t d, const void* A, int r, void* U,
+                                   float* partial, float* stats_part, float alpha, float lambda, int p, float* s,
+                                   int num_sms, cudaStream_t stream) {
+  if (T <= kLrSmallTokens || (p != 1 && p != 2)) return cudaErrorInvalidValue;
+  const float ap = alpha / static_cast<float>(p);
+  return p == 2 ? launch_tiled<2>(X, T, d, A, r, U, partial, stats_part, ap, lambda, s, num_sms, stream)
+                : launch_tiled<1>(X, T, d, A, r, U, partial, stats_part, ap, lambda, s, num_sms, stream);
 }
 
 }  // namespace ttq

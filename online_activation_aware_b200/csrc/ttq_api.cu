@@ -143,7 +143,11 @@ struct WsLayout {
 WsLayout ws_layout(int64_t T, int64_t d, int64_t d_out, int r, int q, int g, int num_sms) {
   WsLayout L{};
   L.stats_off = 0;
-  L.stats_bytes = 0;  // the statistic reduces on chip
+  // the statistic reduces on chip, except when it rides on the low-rank pass over X
+  // (r > 0): then its per-token-block column sums take [ceil(T / 64), d] fp32
+  L.stats_bytes = (d_out > 0 && r > 0 && T > ttq::lowrank_small_tokens())
+                      ? round256(ttq::lowrank_stats_bytes(T, d))
+                      : 0;
   L.xf_off = L.stats_off + L.stats_bytes;
   L.xf_bytes = d_out > 0 ? round256(static_cast<size_t>(T) * static_cast<size_t>(d) * 2) : 0;
   L.u_off = L.xf_off + L.xf_bytes;
@@ -303,13 +307,18 @@ ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const vo
                             : nullptr;
   float* gpart = L.part_bytes ? reinterpret_cast<float*>(base + L.part_off) : nullptr;
 
-  // statistic (partial sums, then s) -> (X A^T) -> fold of X fused with the requant of
-  // W -> projection
+  // statistic -> (X A^T) -> fold of X fused with the requant of W -> projection; with a
+  // low-rank side path the statistic comes out of the same pass over X as X A^T
+  const bool stats_in_lowrank = L.stats_bytes > 0;
   cudaError_t e = trace(0, stream);
-  if (e == cudaSuccess)
+  if (e == cudaSuccess && !stats_in_lowrank)
     e = ttq::launch_act_stats(X_bf16, T, d, d, cfg->alpha, cfg->lambda, cfg->p, s, di->num_sms, dev_err(di), stream);
   if (e == cudaSuccess) e = trace(1, stream);
-  if (e == cudaSuccess && cfg->r > 0)
+  if (e == cudaSuccess && stats_in_lowrank)
+    e = ttq::launch_lowrank_u_stats(X_bf16, T, d, A_bf16, cfg->r, U, upart,
+                                    reinterpret_cast<float*>(base + L.stats_off), cfg->alpha, cfg->lambda, cfg->p, s,
+                                    di->num_sms, stream);
+  else if (e == cudaSuccess && cfg->r > 0)
     e = ttq::launch_lowrank_u(X_bf16, T, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
   if (e == cudaSuccess) e = trace(2, stream);
   if (e == cudaSuccess)

@@ -73,6 +73,13 @@ cudaError_t launch_act_stats_capped(const void* X, int64_t T, int64_t d, int64_t
 cudaError_t launch_fold(const void* X, int64_t T, int64_t d, int64_t ld_x, const float* s,
                         void* Xf, cudaStream_t stream);
 
+// s_j from the column sum of |x_tj|^p over the prompt's T tokens (every statistic kernel
+// finishes with this one step, so their results agree whenever their sums do).
+__device__ __forceinline__ float finalize_scale(float colsum, float T, float alpha_over_p, float lambda) {
+  const float m = __fdiv_rn(colsum, T);  // mean over the prompt's tokens
+  return powf(__fadd_rn(m, lambda), alpha_over_p);
+}
+
 // U[t, :] = X[t, :] A^T in fp32 accumulation (tensor cores, K split over blocks, the
 // splits added in a fixed order by a dependent kernel), stored bf16 with row stride 64
 // (columns r..63 zero). Requires r % 8 == 0, r <= 64; `partial` holds
@@ -81,6 +88,17 @@ int lowrank_splits(int64_t T, int64_t d, int num_sms);
 size_t lowrank_partial_bytes(int64_t T, int64_t d, int r, int num_sms);
 cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A, int r, void* U, float* partial,
                              int num_sms, cudaStream_t stream);
+
+// The same pass over X also yielding the statistic s (p in {1, 2}): each block sums |x|^p
+// over its 64 tokens for the channels of its K slice (fp32, fixed order) into `stats_part`
+// ([ceil(T / 64), d] fp32, lowrank_stats_bytes() of workspace), and the dependent kernel
+// that adds the K splits of U also adds those rows in token-block order and writes s.
+// Only for T > lowrank_small_tokens() (fewer tokens take one block per output of U).
+int lowrank_small_tokens();
+size_t lowrank_stats_bytes(int64_t T, int64_t d);
+cudaError_t launch_lowrank_u_stats(const void* X, int64_t T, int64_t d, const void* A, int r, void* U,
+                                   float* partial, float* stats_part, float alpha, float lambda, int p, float* s,
+                                   int num_sms, cudaStream_t stream);
 
 // ---------------------------------------------------------------- decode
 

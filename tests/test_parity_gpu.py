@@ -355,6 +355,30 @@ def test_prefill_p1_statistic(T, d, d_out, q, g, r):
     prefill_check(T, d, d_out, q, g, 0.5, r, seed=T + d + 1, rows=rows, p=1)
 
 
+@pytest.mark.parametrize("T,d,d_out,r,p", [
+    (8, 256, 128, 8, 2),        # the last token count with the separate statistic kernel
+    (9, 256, 128, 8, 2),        # the first with the statistic in the low-rank pass; 9 of 64 rows
+    (65, 1088, 256, 24, 1),     # one token in the second block; K not a multiple of 64
+    (300, 512, 384, 16, 2), (2048, 768, 512, 16, 1),
+    (4100, 5120, 8192, 64, 2),  # the 32B query projection's width, ragged last token block
+])
+def test_statistic_from_lowrank_pass(T, d, d_out, r, p):
+    # with a rank-r side path the prefill takes s from the same pass over X as X A^T: s
+    # against the oracle, and against the separate statistic kernel (two fp32 sums in
+    # different orders), then codes and Y as for every prefill
+    rows = None if d_out <= 1024 else np.unique(np.concatenate([[0, d_out - 1],
+                                                                np.random.default_rng(T).choice(d_out, 62, replace=False)]))
+    prefill_check(T, d, d_out, 4, 128 if d % 128 == 0 else 32, 0.5, r, seed=T + 7 * d + r, rows=rows, p=p)
+    Xb, Wb = layer(T, d, d_out, T + 7 * d + r)[:2]
+    s_sep = ttq.act_stats(gpu(Xb), 0.5, 0.4, p).cpu().numpy().astype(np.float64)
+    At = gpu(synthetic.as_bf16(np.zeros((r, d))))
+    Bt = gpu(synthetic.as_bf16(np.zeros((d_out, r))))
+    s_fused = ttq.linear_prefill(gpu(Xb), gpu(Wb), ttq.make_config(4, 32, 0.5, 0.4, p, r), At, Bt)["s"]
+    s_fused = s_fused.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(s_fused - s_sep) / s_sep) <= 2e-6
+    assert ttq.device_status() == 0
+
+
 def test_decode_after_p1_prefill_matches_oracle():
     # decode steps reuse the p = 1 prefill's s and codes (the decode does not see p)
     T, d, d_out, q, g = 256, 1024, 384, 4, 64
