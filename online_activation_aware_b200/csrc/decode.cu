@@ -20,7 +20,8 @@
 // summed by shuffles in a fixed order. CTAs of 8 rows (up to 8 on an SM at 128 registers a
 // thread) stage the rows' scale and zero in shared memory. x' (fp32, chunk-major, see xoff)
 // and the unit sums come from a prep kernel chained to the GEMV by programmatic dependent
-// launch: the GEMV issues its first code loads before waiting for x'.
+// launch: the GEMV issues its first code loads before waiting for x'. For two tokens the
+// CTA's codes come instead by bulk copies into shared memory (fewer registers a thread).
 #include "ttq_internal.h"
 
 namespace ttq {
@@ -109,6 +110,31 @@ __device__ __forceinline__ void codes4(const UnitWords<Q>& u, int c4, float (&f)
   }
 }
 
+// One row's codes of one unit from shared memory (BULK form).
+template <int Q>
+__device__ __forceinline__ UnitWords<Q> lds_unit(const uint32_t* p) {
+  UnitWords<Q> u;
+  if (Q == 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p);
+    u.w[0] = v.x; u.w[1] = v.y; u.w[2] = v.z; u.w[3] = v.w;
+  } else if (Q == 2) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    u.w[0] = v.x; u.w[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < Q; ++i) u.w[i] = p[i];
+  }
+  return u;
+}
+
+// Bulk copy (no multicast) of `bytes` from global memory into this CTA's shared memory,
+// counted in bytes on the barrier at `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 // B floats of x' (or of the unit sums) for one input, token-minor.
 template <int B>
 struct TokVec {
@@ -145,13 +171,18 @@ __host__ __device__ __forceinline__ int64_t xoff(int c, int u, int units, int B)
 // register writeback, so reuse in registers is what cuts it). The codes of the next
 // kDepth units are in flight while one is consumed (at d = 5120 a lane's five units are
 // nearly all requested at once).
-template <int Q, int B>
+// BULK: instead, one thread copies the CTA's rows of codes (contiguous in memory) into
+// shared memory with bulk copies, in np pieces along the inputs, each counted on a barrier
+// of its own, before x' is ready; the lanes read their units from there as the pieces land.
+template <int Q, int B, bool BULK>
 __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
     const uint32_t* __restrict__ codes, const __half* __restrict__ scale, const __half* __restrict__ zero,
     const float* xp, const float* usum, int d, int d_out, int log2g, const __nv_bfloat16* __restrict__ U,
     const __nv_bfloat16* __restrict__ Blr, int r, __nv_bfloat16* __restrict__ Y, int nb, int64_t cstride,
-    int64_t mstride, int64_t wsf) {
-  extern __shared__ __align__(16) float2 meta_sm[];  // [kRowsPerCta][gpr]: (sigma, 128 + z)
+    int64_t mstride, int64_t wsf, int np, DevErr err) {
+  // [kRowsPerCta][gpr] (sigma, 128 + z); BULK: then the codes [kRowsPerCta][d q / 32] words,
+  // np barriers and an abort flag
+  extern __shared__ __align__(16) float2 meta_sm[];
   {
     // request blockIdx.y of a batched decode: its own codes, scale, zero, x', U and Y
     const int64_t rq = blockIdx.y;
@@ -174,15 +205,36 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
 #pragma unroll
   for (int i = 0; i < R; ++i) crow[i] = codes + static_cast<int64_t>(row0 + i < d_out ? row0 + i : 0) * upr * Q;
   const int nsteps = (upr - lane + 31) >> 5;         // units of this lane: lane, lane + 32, ...
+  uint32_t* code_sm = reinterpret_cast<uint32_t*>(meta_sm + kRowsPerCta * gpr);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(code_sm + kRowsPerCta * upr * Q);
+  volatile int* abort_sm = reinterpret_cast<volatile int*>(bars + np);
+  const int pu = upr / (np > 0 ? np : 1);  // units per piece (BULK)
 
-  // the first kDepth units' codes, and the CTA's scale/zero into shared memory, before x'
-  // is ready
-  UnitWords<Q> cb[kDepth][R];
+  // the first kDepth units' codes (BULK: all of the CTA's codes), and the CTA's scale/zero
+  // into shared memory, before x' is ready
+  UnitWords<Q> cb[BULK ? 1 : kDepth][R];
+  if (BULK) {
+    if (threadIdx.x == 0) {
+      for (int pc = 0; pc < np; ++pc) mbar_init(smem_addr(bars + pc), 1);
+      *abort_sm = 0;
+      fence_mbar_init();
+      const int nrows = min(kRowsPerCta, d_out - static_cast<int>(blockIdx.x) * kRowsPerCta);
+      const uint32_t pbytes = static_cast<uint32_t>(pu * Q * 4);
+      const uint32_t* src0 = codes + static_cast<int64_t>(blockIdx.x) * kRowsPerCta * upr * Q;
+      for (int pc = 0; pc < np; ++pc) {
+        mbar_arrive_expect_tx(smem_addr(bars + pc), static_cast<uint32_t>(nrows) * pbytes);
+        for (int i = 0; i < nrows; ++i)
+          bulk_load(smem_addr(code_sm + (i * upr + pc * pu) * Q), src0 + (static_cast<int64_t>(i) * upr + pc * pu) * Q,
+                    pbytes, smem_addr(bars + pc));
+      }
+    }
+  } else {
 #pragma unroll
-  for (int k = 0; k < kDepth; ++k) {
-    if (k < nsteps) {
+    for (int k = 0; k < kDepth; ++k) {
+      if (k < nsteps) {
 #pragma unroll
-      for (int i = 0; i < R; ++i) cb[k][i] = load_unit<Q>(crow[i] + static_cast<int64_t>(lane + 32 * k) * Q);
+        for (int i = 0; i < R; ++i) cb[k][i] = load_unit<Q>(crow[i] + static_cast<int64_t>(lane + 32 * k) * Q);
+      }
     }
   }
   {
@@ -225,10 +277,22 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
   for (int i = 0; i < R; ++i)
 #pragma unroll
     for (int t = 0; t < B; ++t) pacc[i][t] = 0.f;
-  for (int s0 = 0; s0 < nsteps; s0 += kDepth) {
+  int landed = 0;  // BULK: pieces known to have landed
+  bool ok = true;
+  const int wsteps = (upr + 31) >> 5;  // steps of the warp (of lane 0): the loop is warp-uniform
+  for (int s0 = 0; ok && s0 < wsteps; s0 += kDepth) {
 #pragma unroll
     for (int hb = 0; hb < kDepth; ++hb) {
       const int st = s0 + hb;
+      if (BULK) {
+        // the pieces holding this step's units of every lane of the warp (warp-uniform)
+        const int need = min(np - 1, (32 * st + 31) / pu);
+        while (ok && landed <= need) {
+          ok = __all_sync(0xffffffffu, mbar_wait(smem_addr(bars + landed), 0, err, abort_sm) ? 1 : 0);
+          ++landed;
+        }
+        if (!ok) break;
+      }
       if (st < nsteps) {
         const int u = lane + 32 * st;
         // two-wide accumulators: one token, pairs of inputs (even, odd); two tokens, the
@@ -257,7 +321,10 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
 #pragma unroll
           for (int i = 0; i < R; ++i) {
             float f[4];
-            codes4<Q>(cb[hb][i], c4, f);
+            if (BULK)
+              codes4<Q>(lds_unit<Q>(code_sm + ((R * warp + i) * upr + u) * Q), c4, f);
+            else
+              codes4<Q>(cb[hb][i], c4, f);
             if (B == 1) {
               acc2[i] = ffma2(f2(f[0], f[1]), xv[0], acc2[i]);
               acc2[i] = ffma2(f2(f[2], f[3]), xv[1], acc2[i]);
@@ -278,7 +345,7 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
             acc[i][B - 1] = a.y;
           }
         }
-        if (st + kDepth < nsteps) {  // refill the slot just consumed, kDepth units ahead
+        if (!BULK && st + kDepth < nsteps) {  // refill the slot just consumed, kDepth units ahead
 #pragma unroll
           for (int i = 0; i < R; ++i)
             cb[hb][i] = load_unit<Q>(crow[i] + static_cast<int64_t>(u + 32 * kDepth) * Q);
@@ -294,6 +361,18 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
         }
       }
     }
+  }
+  if (BULK) {
+    // after a failed wait, let every copy land before the shared memory is released
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_sm) {
+      for (int pc = 0; pc < np; ++pc) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(smem_addr(bars + pc), 0) && globaltimer_ns() - t0 < 2000000000ull) {
+        }
+      }
+    }
+    if (*abort_sm) return;
   }
   // the warp's 32 lanes in a fixed order (butterfly: every lane ends with the same sums)
 #pragma unroll
@@ -398,13 +477,30 @@ cudaError_t launch_qb(const DecodeArgs& a, uint8_t* ws, cudaStream_t stream) {
                              static_cast<const __nv_bfloat16*>(a.X), static_cast<int>(a.b), static_cast<int>(a.d), a.s,
                              xp, usum, wsf);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  const size_t smem = static_cast<size_t>(kRowsPerCta) * (a.d / a.g) * sizeof(float2);
+  // two tokens: codes by bulk copies when every row and every piece of a row is a whole
+  // number of 16-byte blocks and the CTA's codes fit in shared memory beside its
+  // scale/zero (at 5120 -> 8192, q = 4: 18.5 us a step against 19.9 us with the codes in
+  // registers; for one token the register form is faster, 12.2 against 14.9 us)
+  const size_t meta_bytes = static_cast<size_t>(kRowsPerCta) * (a.d / a.g) * sizeof(float2);
+  const int64_t upr = a.d / 32;
+  int np = 0;
+  if (B == 2 && (a.d * Q) % 128 == 0 && (reinterpret_cast<uintptr_t>(a.codes) & 15u) == 0) {
+    for (int n : {4, 2, 1}) {
+      if (upr % n == 0 && ((upr / n) * Q) % 4 == 0 && (n == 1 || upr / n >= 32)) {
+        np = n;
+        break;
+      }
+    }
+  }
+  const size_t bulk_smem = meta_bytes + static_cast<size_t>(kRowsPerCta) * upr * Q * 4 + 8 * 4 + 16;
+  if (bulk_smem > 200 * 1024) np = 0;
+  const size_t smem = np > 0 ? bulk_smem : meta_bytes;
+  auto kern = np > 0 ? decode_gemv_kernel<Q, B, true> : decode_gemv_kernel<Q, B, false>;
   if (smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(decode_gemv_kernel<Q, B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>((a.d_out + kRowsPerCta - 1) / kRowsPerCta), static_cast<unsigned>(a.requests));
   cfg.blockDim = dim3(kGemvThreads);
   cfg.dynamicSmemBytes = smem;
@@ -414,12 +510,12 @@ cudaError_t launch_qb(const DecodeArgs& a, uint8_t* ws, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, decode_gemv_kernel<Q, B>, static_cast<const uint32_t*>(a.codes),
+  e = cudaLaunchKernelEx(&cfg, kern, static_cast<const uint32_t*>(a.codes),
                          static_cast<const __half*>(a.scale), static_cast<const __half*>(a.zero),
                          static_cast<const float*>(xp), static_cast<const float*>(usum), static_cast<int>(a.d),
                          static_cast<int>(a.d_out), lg, static_cast<const __nv_bfloat16*>(a.U),
                          static_cast<const __nv_bfloat16*>(a.Blr), a.r, static_cast<__nv_bfloat16*>(a.Y),
-                         static_cast<int>(a.b), a.d_out * (a.d / 32) * Q, a.d_out * (a.d / a.g), wsf);
+                         static_cast<int>(a.b), a.d_out * (a.d / 32) * Q, a.d_out * (a.d / a.g), wsf, np, a.err);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -369,7 +369,7 @@ ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d
     if (cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
     if (e == cudaSuccess) {
       ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16,
-                         1};
+                         1, dev_err(di)};
       e = ttq::launch_decode_gemv(da, base + L.dec_off, stream);
     }
     return cuda_status(e);
@@ -597,7 +597,7 @@ ttq_status ttq_linear_decode_batched(const void* X_bf16, int32_t requests, int64
   }
   if (e == cudaSuccess) {
     ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16,
-                       requests};
+                       requests, dev_err(di)};
     e = ttq::launch_decode_gemv(da, base + off, stream);
   }
   return cuda_status(e);

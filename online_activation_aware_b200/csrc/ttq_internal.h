@@ -116,6 +116,7 @@ struct DecodeArgs {
   int q, g;
   void* Y;                // bf16 [b, d_out]
   int requests;           // batched decode: requests stacked along every per-request operand
+  DevErr err;             // device error word and wait limit
 };
 // True when the CUDA-core GEMV handles these decode sizes (b <= 2).
 bool decode_gemv_ok(int64_t b, int64_t d);
