@@ -441,7 +441,7 @@ def main():
     # stage then starts only when the one before it has finished), right after the warm-up
     # and before the timed region, with its own clock samples: the GEMM's roofline comes
     # from it
-    Ks = max(3, min(K, 50))
+    Ks = max(3, min(args.steps, 50))
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(Ks)]
     tsampler = NvmlClockSampler(gpu_uuid(torch, dev))
     tsampler.start()

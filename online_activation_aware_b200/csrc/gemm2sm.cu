@@ -130,6 +130,39 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, const 
   }
 }
 
+// A bounded wait for the single-thread roles (TMA producer, MMA issuer) that lets the
+// hardware suspend the thread until the phase completes (suspend-time hint) instead of
+// polling: their polls would take issue slots from the dequantising warps that share
+// their schedulers (the projection at 5120 -> 8192, T = 4096 ran 287 -> 271 us).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_suspend(uint32_t bar, uint32_t parity, const DevErr& err,
+                                                  volatile int* abort_flag) {
+  constexpr uint32_t kHintNs = 2000;
+  if (mbar_try_wait_hint(bar, parity, kHintNs)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait_hint(bar, parity, kHintNs)) return true;
+    if ((it & 7u) == 7u) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > err.wait_ns) {
+        atomicOr(err.word, kErrTimeout);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
@@ -346,7 +379,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
       for (it.begin(args); it.valid(args); it.next(args), p.advance(S)) {
         const uint32_t s = p.stage;
         if (p.count >= static_cast<uint32_t>(S) &&
-            !mbar_wait(bar_empty + 8 * s, p.phase ^ 1u, err, abort_flag)) {
+            !mbar_wait_suspend(bar_empty + 8 * s, p.phase ^ 1u, err, abort_flag)) {
           aborted = true;
           break;
         }
@@ -406,8 +439,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
         const uint32_t dacc = tmem + b * static_cast<uint32_t>(BN);
         for (int j = 0; j < c.items; ++j, p.advance(S)) {
           const uint32_t s = p.stage;
-          const bool ready = mbar_wait(bar_full + 8 * s, p.phase, err, abort_flag) &&
-                             mbar_wait(bar_afull + 8 * s, p.phase, err, abort_flag);
+          const bool ready = mbar_wait_suspend(bar_full + 8 * s, p.phase, err, abort_flag) &&
+                             mbar_wait_suspend(bar_afull + 8 * s, p.phase, err, abort_flag);
           if (!__all_sync(0xffffffffu, ready ? 1 : 0)) {
             ok = false;
             break;
