@@ -5,9 +5,10 @@
 //
 // A skinny product (r <= 64 outputs per token) bound by the single read of X. Block
 // (token block of 64, K split ks) streams its [64 x Kc] slice of X and the matching
-// [r x Kc] slice of A through a 3-stage cp.async ring in shared memory (16-byte chunks,
-// XOR-swizzled rows so that ldmatrix is conflict-free), and each of its first 4 warps
-// multiplies 16 tokens by A^T with mma.sync m16n8k16 (bf16 in, fp32 accumulate). The K splits write
+// [r x Kc] slice of A by TMA through a 4-stage ring in shared memory (128-byte swizzle, so
+// that ldmatrix is conflict-free; a producer warp issues the copies and the consumer
+// warps hand stages back on mbarriers), and each of its first 4 warps multiplies 16
+// tokens by A^T with mma.sync m16n8k16 (bf16 in, fp32 accumulate). The K splits write
 // fp32 partial sums; a small dependent kernel adds them in split order (deterministic)
 // and stores U in bf16 with its row padded to 64 (columns r..63 zero). For a few tokens (a
 // decode step) one block computes each output over all of d instead.
@@ -26,14 +27,9 @@ namespace {
 
 constexpr int kLrTok = 64;      // tokens per block (4 warps x 16)
 constexpr int kLrK = 64;        // K per stage
-constexpr int kLrStages = 3;
-constexpr int kLrThreads = 128;
+constexpr int kLrStages = 4;
+constexpr int kLrThreads = 128;  // the multiplying warps
 constexpr int kLrSmallTokens = 8;  // up to here one block per output (no partial sums in memory)
-
-__device__ __forceinline__ void cp_async_16_zfill(uint32_t dst, const void* src, bool valid) {
-  const int n = valid ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
-}
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -52,28 +48,59 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// byte offset of 16-byte chunk c (0..7) of row `row` in a [rows x 64] bf16 tile
+// byte offset of 16-byte chunk c (0..7) of row `row` in a [rows x 64] bf16 tile as the
+// 128-byte TMA swizzle lays it out (tile base 1024-byte aligned)
 __device__ __forceinline__ uint32_t swz(int row, int c) { return static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4)); }
 
-// Threads of a block: with the statistic and r >= 32 four more warps take the statistic
-// (the multiplying warps are busier there); otherwise the 4 warps do both.
+// Consumer warps of a block: with the statistic and r >= 32 four more warps take the
+// statistic (the multiplying warps are busier there); otherwise the 4 warps do both.
 template <int NT, int P>
-constexpr int lr_threads() { return (P != 0 && NT >= 4) ? 2 * kLrThreads : kLrThreads; }
+constexpr int lr_consumer_warps() { return (P != 0 && NT >= 4) ? 8 : 4; }
+template <int NT, int P>
+constexpr int lr_threads() { return 32 * (lr_consumer_warps<NT, P>() + 1); }  // + the TMA producer warp
+
+// Shared memory of a block: kLrStages x (X tile [64 x 64], A tile [R x 64]), 1024-byte
+// aligned tiles, then the stage barriers and an abort flag.
+template <int NT>
+constexpr uint32_t lr_stage_bytes() { return kLrTok * kLrK * 2 + NT * 8 * kLrK * 2; }
+template <int NT>
+constexpr size_t lr_smem_bytes() { return 1024 + kLrStages * lr_stage_bytes<NT>() + 2 * kLrStages * 8 + 16; }
+
+// Waits (bounded by a fixed two seconds) for the copies of a stage to land before the
+// block's shared memory is released after an abort.
+__device__ __forceinline__ void lr_drain(uint32_t bar, uint32_t parity, const DevErr& err) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > 2000000000ull) {
+      atomicOr(err.word, kErrTimeout);
+      return;
+    }
+  }
+}
 
 // grid: (token blocks, K splits); NT = r / 8 output tiles of 8 ranks; P = 0 (U only) or the
 // statistic's exponent, whose per-block column sums go to spart[token block][channel].
+// The last warp streams the block's X tiles [64 tokens x 64 channels] and A tiles
+// [r x 64] by TMA (128-byte swizzle; rows past T and channels past d read as zero) into a
+// ring of kLrStages stages (`full` barriers count the bytes); each consumer warp hands a
+// stage back on its `empty` barrier when it is done with it, so the warps never meet at a
+// block barrier.
 template <int NT, int P>
-__global__ void __launch_bounds__(lr_threads<NT, P>()) lowrank_partial_kernel(const __nv_bfloat16* __restrict__ X, int T,
-                                                                     int d, const __nv_bfloat16* __restrict__ A,
-                                                                     int kc, float* __restrict__ part,
-                                                                     float* __restrict__ spart) {
-  pdl_enter();
+__global__ void __launch_bounds__(lr_threads<NT, P>(), 1) lowrank_partial_kernel(
+    const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a, int T, int d, int kc,
+    float* __restrict__ part, float* __restrict__ spart, const DevErr err) {
   constexpr int R = NT * 8;
   constexpr uint32_t kXBytes = kLrTok * kLrK * 2;  // 8 KB
-  constexpr uint32_t kABytes = R * kLrK * 2;
-  extern __shared__ __align__(128) uint8_t sm[];  // kLrStages x (X tile, A tile)
-  constexpr int kThreads = lr_threads<NT, P>();
-  constexpr bool kSplit = kThreads > kLrThreads;  // warps 4..7 take the statistic
+  constexpr uint32_t kStage = lr_stage_bytes<NT>();
+  constexpr int kCons = lr_consumer_warps<NT, P>();
+  constexpr bool kSplit = kCons > 4;  // warps 4..7 take the statistic
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw);  // the same stages through a generic pointer
+  const uint32_t bar_full = sbase + kLrStages * kStage;
+  const uint32_t bar_empty = bar_full + 8 * kLrStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + kLrStages * kStage + 16 * kLrStages);
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
@@ -81,29 +108,41 @@ __global__ void __launch_bounds__(lr_threads<NT, P>()) lowrank_partial_kernel(co
   const int k0 = blockIdx.y * kc;
   const int k1 = min(d, k0 + kc);
   const int nst = (k1 - k0 + kLrK - 1) / kLrK;
-  const uint32_t sbase = smem_addr(sm);
 
-  auto issue = [&](int st, int slot) {
-    if (st < nst) {
-      const int kb = k0 + st * kLrK;
-      const uint32_t xs = sbase + slot * (kXBytes + kABytes);
-      const uint32_t as = xs + kXBytes;
-#pragma unroll
-      for (int i = 0; i < (kLrTok * 8) / kThreads; ++i) {  // X: 64 rows x 8 chunks
-        const int e = tid + i * kThreads;
-        const int row = e >> 3, c = e & 7;
-        const int t = min(t0 + row, T - 1);
-        const int k = kb + c * 8;
-        cp_async_16_zfill(xs + swz(row, c), X + static_cast<int64_t>(t) * d + (k < d ? k : 0), k < d);
+  if (tid == 0) {
+    for (int s = 0; s < kLrStages; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, kCons);  // one arrival per consumer warp
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&tm_x);
+    prefetch_tensormap(&tm_a);
+  }
+  __syncthreads();
+  pdl_enter();  // X (and A) are read only after the kernel ahead has finished
+
+  if (warp == kCons) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int st = 0; st < nst; ++st) {
+        const int s = st % kLrStages;
+        if (st >= kLrStages && !mbar_wait(bar_empty + 8 * s, ((st / kLrStages) - 1) & 1, err, abort_flag)) break;
+        const uint32_t xs = sbase + s * kStage;
+        mbar_arrive_expect_tx(bar_full + 8 * s, kStage);
+        tma_load_2d(xs, &tm_x, bar_full + 8 * s, k0 + st * kLrK, t0);
+        tma_load_2d(xs + kXBytes, &tm_a, bar_full + 8 * s, k0 + st * kLrK, 0);
+        ++issued;
       }
-      for (int e = tid; e < R * 8; e += kThreads) {  // A: R rows x 8 chunks
-        const int row = e >> 3, c = e & 7;
-        const int k = kb + c * 8;
-        cp_async_16_zfill(as + swz(row, c), A + static_cast<int64_t>(row) * d + (k < d ? k : 0), k < d);
+      if (*abort_flag) {
+        // every copy this block started lands before its shared memory is released
+        for (int st = issued > kLrStages ? issued - kLrStages : 0; st < issued; ++st)
+          lr_drain(bar_full + 8 * (st % kLrStages), (st / kLrStages) & 1, err);
       }
     }
-    cp_async_commit();
-  };
+    return;
+  }
 
   float acc[NT][4];
 #pragma unroll
@@ -111,14 +150,10 @@ __global__ void __launch_bounds__(lr_threads<NT, P>()) lowrank_partial_kernel(co
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[n][j] = 0.f;
 
-#pragma unroll
-  for (int i = 0; i < kLrStages - 1; ++i) issue(i, i);
   for (int st = 0; st < nst; ++st) {
-    cp_async_wait<kLrStages - 2>();
-    __syncthreads();  // stage st is in place for every thread; the slot refilled next is free
-    issue(st + kLrStages - 1, (st + kLrStages - 1) % kLrStages);
-    const int slot = st % kLrStages;
-    const uint32_t xs = sbase + slot * (kXBytes + kABytes);
+    const int s = st % kLrStages;
+    if (!__all_sync(0xffffffffu, mbar_wait(bar_full + 8 * s, (st / kLrStages) & 1, err, abort_flag) ? 1 : 0)) break;
+    const uint32_t xs = sbase + s * kStage;
     const uint32_t as = xs + kXBytes;
 #pragma unroll
     for (int kk = 0; kk < kLrK / 16 && (!kSplit || warp < 4); ++kk) {
@@ -143,26 +178,22 @@ __global__ void __launch_bounds__(lr_threads<NT, P>()) lowrank_partial_kernel(co
     if (P != 0 && (!kSplit || warp >= 4)) {
       // sum of |x|^p over the block's tokens for the stage's 64 channels: lane (pair cp,
       // quarter qr) takes channels 2cp, 2cp + 1 of rows 8 (i / 2) + 2 qr + i % 2, i = 0..15
-      // (under the row swizzle a warp's four quarters then read 32 different banks); rows
-      // past T (loaded as copies of the last token) are left out, and the quarters meet
-      // by two shuffles
+      // (under the row swizzle a warp's four quarters then read 32 different banks; rows
+      // past T are zero), and the quarters meet by two shuffles
       const int cp = (warp & 3) * 8 + (lane & 7), qr = lane >> 3;
-      const int nrows = min(kLrTok, T - t0);
-      const uint8_t* xt = sm + slot * (kXBytes + kABytes) + (cp & 3) * 4;
+      const uint8_t* xt = sgen + s * kStage + (cp & 3) * 4;
       float s0 = 0.f, s1 = 0.f;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int row = 8 * (i >> 1) + 2 * qr + (i & 1);
-        if (row < nrows) {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(xt + swz(row, cp >> 2));
-          const float a = bf16lo_to_f32(w), b = bf16hi_to_f32(w);
-          if constexpr (P == 2) {
-            s0 = __fmaf_rn(a, a, s0);
-            s1 = __fmaf_rn(b, b, s1);
-          } else {
-            s0 = __fadd_rn(s0, fabsf(a));
-            s1 = __fadd_rn(s1, fabsf(b));
-          }
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(xt + swz(row, cp >> 2));
+        const float a = bf16lo_to_f32(w), b = bf16hi_to_f32(w);
+        if constexpr (P == 2) {
+          s0 = __fmaf_rn(a, a, s0);
+          s1 = __fmaf_rn(b, b, s1);
+        } else {
+          s0 = __fadd_rn(s0, fabsf(a));
+          s1 = __fadd_rn(s1, fabsf(b));
         }
       }
       s0 = __fadd_rn(s0, __shfl_xor_sync(0xffffffffu, s0, 8));
@@ -173,11 +204,13 @@ __global__ void __launch_bounds__(lr_threads<NT, P>()) lowrank_partial_kernel(co
       if (qr == 0 && k < d)
         *reinterpret_cast<float2*>(spart + static_cast<int64_t>(blockIdx.x) * d + k) = make_float2(s0, s1);
     }
+    __syncwarp();  // the warp's reads of the stage are done before its one arrival
+    if (lane == 0) mbar_arrive(bar_empty + 8 * s);
   }
-  cp_async_wait<0>();
 
   // partial[ks][t][rank]: rows groupID and groupID + 8 of the warp's 16 tokens
   if (kSplit && warp >= 4) return;
+  if (*abort_flag) return;
   const int g = lane >> 2, tig = lane & 3;
   float* pbase = part + static_cast<int64_t>(blockIdx.y) * T * R;
 #pragma unroll
@@ -298,28 +331,28 @@ size_t lowrank_stats_bytes(int64_t T, int64_t d) {
 namespace {
 
 template <int NT, int P>
-cudaError_t launch_partial_nt(dim3 grid, const __nv_bfloat16* Xb, int T, int d, const __nv_bfloat16* Ab, int kc,
-                              float* partial, float* spart, cudaStream_t stream) {
-  constexpr size_t smem = static_cast<size_t>(kLrStages) * (kLrTok + NT * 8) * kLrK * 2;
+cudaError_t launch_partial_nt(dim3 grid, const CUtensorMap& mx, const CUtensorMap& ma, int T, int d, int kc,
+                              float* partial, float* spart, const DevErr& err, cudaStream_t stream) {
+  constexpr size_t smem = lr_smem_bytes<NT>();
   const cudaError_t e =
       cudaFuncSetAttribute(lowrank_partial_kernel<NT, P>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  return launch_pdl(lowrank_partial_kernel<NT, P>, grid, dim3(lr_threads<NT, P>()), smem, stream, Xb, T, d, Ab, kc, partial,
-                    spart);
+  return launch_pdl(lowrank_partial_kernel<NT, P>, grid, dim3(lr_threads<NT, P>()), smem, stream, mx, ma, T, d, kc,
+                    partial, spart, err);
 }
 
 template <int P>
-cudaError_t launch_partial(int nt, dim3 grid, const __nv_bfloat16* Xb, int T, int d, const __nv_bfloat16* Ab,
-                           int kc, float* partial, float* spart, cudaStream_t stream) {
+cudaError_t launch_partial(int nt, dim3 grid, const CUtensorMap& mx, const CUtensorMap& ma, int T, int d, int kc,
+                           float* partial, float* spart, const DevErr& err, cudaStream_t stream) {
   switch (nt) {
-    case 1: return launch_partial_nt<1, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
-    case 2: return launch_partial_nt<2, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
-    case 3: return launch_partial_nt<3, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
-    case 4: return launch_partial_nt<4, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
-    case 5: return launch_partial_nt<5, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
-    case 6: return launch_partial_nt<6, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
-    case 7: return launch_partial_nt<7, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
-    default: return launch_partial_nt<8, P>(grid, Xb, T, d, Ab, kc, partial, spart, stream);
+    case 1: return launch_partial_nt<1, P>(grid, mx, ma, T, d, kc, partial, spart, err, stream);
+    case 2: return launch_partial_nt<2, P>(grid, mx, ma, T, d, kc, partial, spart, err, stream);
+    case 3: return launch_partial_nt<3, P>(grid, mx, ma, T, d, kc, partial, spart, err, stream);
+    case 4: return launch_partial_nt<4, P>(grid, mx, ma, T, d, kc, partial, spart, err, stream);
+    case 5: return launch_partial_nt<5, P>(grid, mx, ma, T, d, kc, partial, spart, err, stream);
+    case 6: return launch_partial_nt<6, P>(grid, mx, ma, T, d, kc, partial, spart, err, stream);
+    case 7: return launch_partial_nt<7, P>(grid, mx, ma, T, d, kc, partial, spart, err, stream);
+    default: return launch_partial_nt<8, P>(grid, mx, ma, T, d, kc, partial, spart, err, stream);
   }
 }
 
@@ -327,15 +360,23 @@ cudaError_t launch_partial(int nt, dim3 grid, const __nv_bfloat16* Xb, int T, in
 // exponent P into s.
 template <int P>
 cudaError_t launch_tiled(const void* X, int64_t T, int64_t d, const void* A, int r, void* U, float* partial,
-                         float* spart, float alpha_over_p, float lambda, float* s, int num_sms, cudaStream_t stream) {
+                         float* spart, float alpha_over_p, float lambda, float* s, int num_sms, const DevErr& err,
+                         cudaStream_t stream) {
+  // X [T, d] and A [r, d] as tensor maps with 64-channel boxes (128 bytes, 128-byte swizzle):
+  // 64 token rows of X, all r rows of A
+  CUtensorMap mx, ma;
+  if (!encode_tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, static_cast<uint64_t>(T), static_cast<uint64_t>(d),
+                      static_cast<uint64_t>(d), kLrK, kLrTok, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, static_cast<uint64_t>(r), static_cast<uint64_t>(d),
+                      static_cast<uint64_t>(d), kLrK, static_cast<uint32_t>(r), CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   const int ks = lowrank_splits(T, d, num_sms);
   const int64_t kst = (d + kLrK - 1) / kLrK;
   const int kc = static_cast<int>((kst + ks - 1) / ks) * kLrK;
   const int ksr = static_cast<int>((d + kc - 1) / kc);  // splits that hold any K
   const dim3 grid(static_cast<unsigned>((T + kLrTok - 1) / kLrTok), static_cast<unsigned>(ksr));
   const int Ti = static_cast<int>(T), di = static_cast<int>(d);
-  cudaError_t e = launch_partial<P>(r / 8, grid, static_cast<const __nv_bfloat16*>(X), Ti, di,
-                                    static_cast<const __nv_bfloat16*>(A), kc, partial, spart, stream);
+  cudaError_t e = launch_partial<P>(r / 8, grid, mx, ma, Ti, di, kc, partial, spart, err, stream);
   if (e != cudaSuccess) return e;
   const int64_t nblk = (T + 3) / 4 + (P != 0 ? (d + 31) / 32 : 0);
   return launch_pdl(lowrank_reduce_kernel<P>, dim3(static_cast<unsigned>(nblk)), dim3(256), 0, stream,
@@ -346,22 +387,22 @@ cudaError_t launch_tiled(const void* X, int64_t T, int64_t d, const void* A, int
 }  // namespace
 
 cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A, int r, void* U, float* partial,
-                             int num_sms, cudaStream_t stream) {
+                             int num_sms, const DevErr& err, cudaStream_t stream) {
   if (T <= kLrSmallTokens) {
     return launch_pdl(lowrank_small_kernel, dim3(static_cast<unsigned>(T * 64)), dim3(256), 0, stream,
                       static_cast<const __nv_bfloat16*>(X), static_cast<int>(d), static_cast<const __nv_bfloat16*>(A),
                       r, static_cast<__nv_bfloat16*>(U));
   }
-  return launch_tiled<0>(X, T, d, A, r, U, partial, nullptr, 0.f, 0.f, nullptr, num_sms, stream);
+  return launch_tiled<0>(X, T, d, A, r, U, partial, nullptr, 0.f, 0.f, nullptr, num_sms, err, stream);
 }
 
 cudaError_t launch_lowrank_u_stats(const void* X, int64_t T, int64_t d, const void* A, int r, void* U,
                                    float* partial, float* stats_part, float alpha, float lambda, int p, float* s,
-                                   int num_sms, cudaStream_t stream) {
+                                   int num_sms, const DevErr& err, cudaStream_t stream) {
   if (T <= kLrSmallTokens || (p != 1 && p != 2)) return cudaErrorInvalidValue;
   const float ap = alpha / static_cast<float>(p);
-  return p == 2 ? launch_tiled<2>(X, T, d, A, r, U, partial, stats_part, ap, lambda, s, num_sms, stream)
-                : launch_tiled<1>(X, T, d, A, r, U, partial, stats_part, ap, lambda, s, num_sms, stream);
+  return p == 2 ? launch_tiled<2>(X, T, d, A, r, U, partial, stats_part, ap, lambda, s, num_sms, err, stream)
+                : launch_tiled<1>(X, T, d, A, r, U, partial, stats_part, ap, lambda, s, num_sms, err, stream);
 }
 
 }  // namespace ttq

@@ -317,9 +317,9 @@ ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const vo
   if (e == cudaSuccess && stats_in_lowrank)
     e = ttq::launch_lowrank_u_stats(X_bf16, T, d, A_bf16, cfg->r, U, upart,
                                     reinterpret_cast<float*>(base + L.stats_off), cfg->alpha, cfg->lambda, cfg->p, s,
-                                    di->num_sms, stream);
+                                    di->num_sms, dev_err(di), stream);
   else if (e == cudaSuccess && cfg->r > 0)
-    e = ttq::launch_lowrank_u(X_bf16, T, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
+    e = ttq::launch_lowrank_u(X_bf16, T, d, A_bf16, cfg->r, U, upart, di->num_sms, dev_err(di), stream);
   if (e == cudaSuccess) e = trace(2, stream);
   if (e == cudaSuccess)
     e = ttq::launch_fold_requant(X_bf16, T, Xf, W_bf16, d_out, d, s, cfg->q, cfg->g, codes, scale_f16, zero_f16,
@@ -366,7 +366,7 @@ ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d
   if (L.dec_bytes > 0) {
     // few tokens: the CUDA-core GEMV streams the codes once
     cudaError_t e = cudaSuccess;
-    if (cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
+    if (cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, upart, di->num_sms, dev_err(di), stream);
     if (e == cudaSuccess) {
       ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16,
                          1, dev_err(di)};
@@ -376,7 +376,7 @@ ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d
   }
   cudaError_t e = ttq::launch_fold(X_bf16, b, d, d, s, Xf, stream);
   if (e == cudaSuccess && cfg->r > 0)
-    e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
+    e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, upart, di->num_sms, dev_err(di), stream);
   if (e == cudaSuccess) {
     ttq::GemmArgs ga{Xf, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g,
                      Y_bf16, gpart};
@@ -492,7 +492,7 @@ ttq_status ttq_linear_prefill_batched(const void* X_bf16, const int64_t* T, int3
   }
   // the low-rank projection of every prompt's tokens at once (A is shared)
   if (e == cudaSuccess && cfg->r > 0)
-    e = ttq::launch_lowrank_u(X_bf16, L.tokens, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
+    e = ttq::launch_lowrank_u(X_bf16, L.tokens, d, A_bf16, cfg->r, U, upart, di->num_sms, dev_err(di), stream);
   // one read of W re-quantized for every prompt
   if (e == cudaSuccess)
     e = ttq::launch_requant_batched(W_bf16, d_out, d, s, prompts, cfg->q, cfg->g, codes, scale_f16, zero_f16, stream);
@@ -593,7 +593,7 @@ ttq_status ttq_linear_decode_batched(const void* X_bf16, int32_t requests, int64
     U = base;
     float* upart = reinterpret_cast<float*>(base + round256(static_cast<size_t>(rows) * 64 * 2));
     off = round256(static_cast<size_t>(rows) * 64 * 2) + round256(ttq::lowrank_partial_bytes(rows, d, cfg->r, di->num_sms));
-    e = ttq::launch_lowrank_u(X_bf16, rows, d, A_bf16, cfg->r, U, upart, di->num_sms, stream);
+    e = ttq::launch_lowrank_u(X_bf16, rows, d, A_bf16, cfg->r, U, upart, di->num_sms, dev_err(di), stream);
   }
   if (e == cudaSuccess) {
     ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16,

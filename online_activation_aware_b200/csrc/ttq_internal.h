@@ -87,7 +87,7 @@ __device__ __forceinline__ float finalize_scale(float colsum, float T, float alp
 int lowrank_splits(int64_t T, int64_t d, int num_sms);
 size_t lowrank_partial_bytes(int64_t T, int64_t d, int r, int num_sms);
 cudaError_t launch_lowrank_u(const void* X, int64_t T, int64_t d, const void* A, int r, void* U, float* partial,
-                             int num_sms, cudaStream_t stream);
+                             int num_sms, const DevErr& err, cudaStream_t stream);
 
 // The same pass over X also yielding the statistic s (p in {1, 2}): each block sums |x|^p
 // over its 64 tokens for the channels of its K slice (fp32, fixed order) into `stats_part`
@@ -98,7 +98,7 @@ int lowrank_small_tokens();
 size_t lowrank_stats_bytes(int64_t T, int64_t d);
 cudaError_t launch_lowrank_u_stats(const void* X, int64_t T, int64_t d, const void* A, int r, void* U,
                                    float* partial, float* stats_part, float alpha, float lambda, int p, float* s,
-                                   int num_sms, cudaStream_t stream);
+                                   int num_sms, const DevErr& err, cudaStream_t stream);
 
 // ---------------------------------------------------------------- decode
 
