@@ -28,7 +28,6 @@ namespace {
 constexpr int kLrTok = 64;      // tokens per block (4 warps x 16)
 constexpr int kLrK = 64;        // K per stage
 constexpr int kLrStages = 4;
-constexpr int kLrThreads = 128;  // the multiplying warps
 constexpr int kLrSmallTokens = 8;  // up to here one block per output (no partial sums in memory)
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4]) {
