@@ -423,19 +423,59 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(
 
 // x'[k][t] = bf16(x[t][k] * (1 / s_k)) as fp32 (rows t >= nb zero), the same rounding as
 // the prefill's fold, in the chunk-major layout of xoff, and usum[v][t] = sum of x' over
-// the 32-input unit v. One warp per (unit, token).
+// the 32-input unit v. One warp per (unit, token), in the first `prep_blocks` blocks.
+// With a low-rank side path (A non-null) nb * 64 more blocks form U = X A^T (row stride
+// 64): block (t, j) strides its 256 threads over d in 8-input chunks, fp32 sums reduced in
+// a fixed order (warps, then the 8 warp sums); U[t][j] = 0 for r <= j < 64.
 template <int B>
 __global__ void __launch_bounds__(256) decode_prep_kernel(const __nv_bfloat16* __restrict__ X, int nb, int d,
                                                           const float* __restrict__ s, float* __restrict__ xp,
-                                                          float* __restrict__ usum, int64_t wsf) {
+                                                          float* __restrict__ usum, int64_t wsf, int prep_blocks,
+                                                          const __nv_bfloat16* __restrict__ A, int r,
+                                                          __nv_bfloat16* __restrict__ U) {
   pdl_enter();  // X is written by the kernel ahead; then the GEMV may start loading codes
   {
-    // request blockIdx.y of a batched decode: its own tokens, statistic and x'
+    // request blockIdx.y of a batched decode: its own tokens, statistic, x' and U
     const int64_t rq = blockIdx.y;
     X += rq * nb * d;
     s += rq * d;
     xp += rq * wsf;
     usum += rq * wsf;
+    if (U != nullptr) U += rq * nb * 64;
+  }
+  if (static_cast<int>(blockIdx.x) >= prep_blocks) {
+    __shared__ float red[8];
+    const int o = static_cast<int>(blockIdx.x) - prep_blocks;  // t * 64 + j
+    const int t = o >> 6, j = o & 63;
+    if (j >= r) {
+      if (threadIdx.x == 0) U[o] = __float2bfloat16_rn(0.f);
+      return;
+    }
+    const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(t) * d);
+    const uint4* ar = reinterpret_cast<const uint4*>(A + static_cast<int64_t>(j) * d);
+    const int chunks = d >> 3;
+    float acc = 0.f;
+#pragma unroll 4
+    for (int c = threadIdx.x; c < chunks; c += 256) {
+      const uint4 xv = __ldg(xr + c), av = __ldg(ar + c);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc = __fmaf_rn(__uint_as_float(xw[q] << 16), __uint_as_float(aw[q] << 16), acc);
+        acc = __fmaf_rn(__uint_as_float(xw[q] & 0xFFFF0000u), __uint_as_float(aw[q] & 0xFFFF0000u), acc);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) v += red[w];
+      U[o] = __float2bfloat16_rn(v);
+    }
+    return;
   }
   const int lane = threadIdx.x & 31;
   const int pair = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -473,9 +513,14 @@ cudaError_t launch_qb(const DecodeArgs& a, uint8_t* ws, cudaStream_t stream) {
   float* usum = reinterpret_cast<float*>(ws + round16(static_cast<size_t>(a.d) * B * 4));
   const int units = static_cast<int>(a.d / 32);
   const int64_t wsf = static_cast<int64_t>(gemv_ws_bytes(a.b, a.d) / 4);  // one request's workspace, floats
-  cudaError_t e = launch_pdl(decode_prep_kernel<B>, dim3((units * B + 7) / 8, a.requests), dim3(256), 0, stream,
+  // the prep blocks, then (low-rank side path) one block per output of U
+  const int prep_blocks = (units * B + 7) / 8;
+  const bool lr = a.A != nullptr && a.r > 0;
+  const int u_blocks = lr ? static_cast<int>(a.b) * 64 : 0;
+  cudaError_t e = launch_pdl(decode_prep_kernel<B>, dim3(prep_blocks + u_blocks, a.requests), dim3(256), 0, stream,
                              static_cast<const __nv_bfloat16*>(a.X), static_cast<int>(a.b), static_cast<int>(a.d), a.s,
-                             xp, usum, wsf);
+                             xp, usum, wsf, prep_blocks, static_cast<const __nv_bfloat16*>(lr ? a.A : nullptr),
+                             lr ? a.r : 0, static_cast<__nv_bfloat16*>(lr ? const_cast<void*>(a.U) : nullptr));
   if (e != cudaSuccess) return e;
   // two tokens: codes by bulk copies when every row and every piece of a row is a whole
   // number of 16-byte blocks and the CTA's codes fit in shared memory beside its

@@ -364,15 +364,12 @@ ttq_status ttq_linear_decode(const void* X_bf16, int64_t b, int64_t d, int64_t d
                             : nullptr;
   float* gpart = L.part_bytes ? reinterpret_cast<float*>(base + L.part_off) : nullptr;
   if (L.dec_bytes > 0) {
-    // few tokens: the CUDA-core GEMV streams the codes once
-    cudaError_t e = cudaSuccess;
-    if (cfg->r > 0) e = ttq::launch_lowrank_u(X_bf16, b, d, A_bf16, cfg->r, U, upart, di->num_sms, dev_err(di), stream);
-    if (e == cudaSuccess) {
-      ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16,
-                         1, dev_err(di)};
-      e = ttq::launch_decode_gemv(da, base + L.dec_off, stream);
-    }
-    return cuda_status(e);
+    // few tokens: the CUDA-core GEMV streams the codes once; its prep kernel also forms
+    // U = X A^T for the low-rank side path
+    ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16,
+                       1, dev_err(di)};
+    da.A = cfg->r > 0 ? A_bf16 : nullptr;
+    return cuda_status(ttq::launch_decode_gemv(da, base + L.dec_off, stream));
   }
   cudaError_t e = ttq::launch_fold(X_bf16, b, d, d, s, Xf, stream);
   if (e == cudaSuccess && cfg->r > 0)
@@ -586,21 +583,17 @@ ttq_status ttq_linear_decode_batched(const void* X_bf16, int32_t requests, int64
   auto* base = static_cast<uint8_t*>(ws);
   const int64_t rows = static_cast<int64_t>(requests) * b;
   void* U = nullptr;
-  cudaError_t e = cudaSuccess;
   size_t off = 0;
   if (cfg->r > 0) {
-    // U = X A^T for every request's tokens at once (A is shared): rows p * b .. p * b + b - 1
+    // U = X A^T of request p's tokens in rows p * b .. p * b + b - 1, formed by the GEMV's
+    // prep kernel (A is shared)
     U = base;
-    float* upart = reinterpret_cast<float*>(base + round256(static_cast<size_t>(rows) * 64 * 2));
     off = round256(static_cast<size_t>(rows) * 64 * 2) + round256(ttq::lowrank_partial_bytes(rows, d, cfg->r, di->num_sms));
-    e = ttq::launch_lowrank_u(X_bf16, rows, d, A_bf16, cfg->r, U, upart, di->num_sms, dev_err(di), stream);
   }
-  if (e == cudaSuccess) {
-    ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16,
-                       requests, dev_err(di)};
-    e = ttq::launch_decode_gemv(da, base + off, stream);
-  }
-  return cuda_status(e);
+  ttq::DecodeArgs da{X_bf16, s, codes, scale_f16, zero_f16, U, B_bf16, cfg->r, b, d, d_out, cfg->q, cfg->g, Y_bf16,
+                     requests, dev_err(di)};
+  da.A = cfg->r > 0 ? A_bf16 : nullptr;
+  return cuda_status(ttq::launch_decode_gemv(da, base + off, stream));
 }
 
 // ---------------------------------------------------------------- decoder layer

@@ -117,6 +117,7 @@ struct DecodeArgs {
   void* Y;                // bf16 [b, d_out]
   int requests;           // batched decode: requests stacked along every per-request operand
   DevErr err;             // device error word and wait limit
+  const void* A = nullptr;  // bf16 [r, d]: when set, the prep kernel also forms U (b <= 8)
 };
 // True when the CUDA-core GEMV handles these decode sizes (b <= 2).
 bool decode_gemv_ok(int64_t b, int64_t d);
