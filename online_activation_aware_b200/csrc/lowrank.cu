@@ -85,7 +85,7 @@ __device__ __forceinline__ void lr_drain(uint32_t bar, uint32_t parity, const De
 // stage back on its `empty` barrier when it is done with it, so the warps never meet at a
 // block barrier.
 template <int NT, int P>
-__global__ void __launch_bounds__(lr_threads<NT, P>(), 1) lowrank_partial_kernel(
+__global__ void __launch_bounds__(lr_threads<NT, P>(), 2) lowrank_partial_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a, int T, int d, int kc,
     float* __restrict__ part, float* __restrict__ spart, const DevErr err) {
   constexpr int R = NT * 8;
@@ -333,8 +333,11 @@ template <int NT, int P>
 cudaError_t launch_partial_nt(dim3 grid, const CUtensorMap& mx, const CUtensorMap& ma, int T, int d, int kc,
                               float* partial, float* spart, const DevErr& err, cudaStream_t stream) {
   constexpr size_t smem = lr_smem_bytes<NT>();
-  const cudaError_t e =
+  cudaError_t e =
       cudaFuncSetAttribute(lowrank_partial_kernel<NT, P>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  // all of the SM's unified memory as shared memory, so that two or three blocks fit
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(lowrank_partial_kernel<NT, P>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   return launch_pdl(lowrank_partial_kernel<NT, P>, grid, dim3(lr_threads<NT, P>()), smem, stream, mx, ma, T, d, kc,
                     partial, spart, err);
