@@ -3,14 +3,15 @@
 // thelatestinai.com listing of the TTQ paper, Table 15: 32 query heads, 8 key/value heads of
 // head dim 128 for Qwen3-8B). For query row t and head h (key/value head h / (H / Hkv)):
 //   out[t, h] = sum_{p <= t} softmax_p(q_t . k_p / sqrt(D)) v_p,
-// computed flash-style: one CTA per (tile of 128 queries, head) walks the key tiles of 128
-// positions up to its diagonal, keeping a running row maximum m and sum l in fp32.
+// computed flash-style: one CTA per (tile of 128 queries, head) walks the key tiles of BK
+// positions (64: two CTAs then share an SM) up to its diagonal, keeping a running row
+// maximum m and sum l in fp32.
 //
 // Roles (6 warps):
 //   warp 0    TMA: the Q tile once, then K and V tiles of the head's key/value head into a
-//             two-stage ring (128-byte swizzled boxes of 128 positions x 64 channels);
+//             two-stage ring (128-byte swizzled boxes of BK positions x 64 channels);
 //   warp 1    owns the tensor memory and issues tcgen05.mma: S_j = Q K_j^T into one of two
-//             128-column fp32 accumulators (issued one tile ahead, so S_{j+1} runs while the
+//             BK-column fp32 accumulators (issued one tile ahead, so S_{j+1} runs while the
 //             softmax works on S_j), and O += P_j V_j into a third; V is read as an MN-major
 //             operand straight from its [position, channel] tile;
 //   warps 2-5 softmax, one query row per thread (tensor-memory lane quadrant w % 4): scale,
