@@ -309,7 +309,9 @@ __global__ void __launch_bounds__(256) lowrank_small_kernel(const __nv_bfloat16*
 int lowrank_splits(int64_t T, int64_t d, int num_sms) {
   const int64_t tb = (T + kLrTok - 1) / kLrTok;
   const int64_t kst = (d + kLrK - 1) / kLrK;  // stages of K in all
-  int64_t ks = (2 * static_cast<int64_t>(num_sms) + tb - 1) / tb;  // about two blocks per SM
+  // at most two blocks per SM, so that the grid is one wave (a partial second wave of a
+  // few blocks would double the pass)
+  int64_t ks = (2 * static_cast<int64_t>(num_sms)) / tb;
   if (ks > kst) ks = kst;
   if (ks < 1) ks = 1;
   return static_cast<int>(ks);
