@@ -492,6 +492,7 @@ def test_decode_few_tokens_parity(b, q, g, r, d_out):
     (5, 256, 128 * 300, 4, 128, 0),  # many row blocks
     (2, 5120, 1024, 4, 128, 16),  # the Qwen3-32B hidden size with low rank
     (3, 5120, 520, 3, 64, 0),     # 3-bit bit planes, 10 slices of 10 units per row
+    (1, 4096, 512, 2, 32, 24),    # one token: U formed in the GEMV's prep launch, odd 8-rank tiles
 ])
 def test_decode_parity_shapes(b, d, d_out, q, g, r):
     # b <= 8 runs on the CUDA-core GEMV (one lane per weight row), larger b on the tensor cores
