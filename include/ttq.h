@@ -174,7 +174,11 @@ TTQ_API ttq_status ttq_requant_batched(const void* W_bf16, int64_t d_out, int64_
  *   s, codes, scale, zero   outputs as in ttq_act_stats / ttq_requant, kept by the
  *          caller for the decode steps that follow
  *   Y      device bf16 [T, d_out] output
- *   ws     device scratch of at least ttq_workspace_size(T, d, d_out, cfg) bytes */
+ *   ws     device scratch of at least ttq_workspace_size(T, d, d_out, cfg) bytes
+ * With r > 0 and T > 8 the statistic comes out of the same pass over X as X A^T: per
+ * 64-token block and channel the sum of |x|^p, then the blocks added in order. It is
+ * deterministic, and it equals ttq_act_stats's s up to the fp32 rounding of a different
+ * summation order (a few units in the last place). */
 TTQ_API ttq_status ttq_linear_prefill(const void* X_bf16, int64_t T, int64_t d, const void* W_bf16,
                               int64_t d_out, const void* A_bf16, const void* B_bf16,
                               const ttq_config* cfg, float* s, uint32_t* codes, void* scale_f16,
