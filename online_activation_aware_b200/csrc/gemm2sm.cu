@@ -547,12 +547,30 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
       tc_fence_after();
       const int row = c.m0 + static_cast<int>(rank) * kBM + quarter * 32 + lane;
       const bool rok = row < args.d_out;
+      // rows in pairs (an even d_out keeps every pair inside Y and 4-byte aligned)
+      const bool pair_rows = (args.d_out & 1) == 0;
       const uint32_t taddr = lane_base + b * static_cast<uint32_t>(BN);
       for (int cc0 = 0; cc0 < BN; cc0 += 16) {
         uint32_t r[16];
         tmem_ld_32x32b_x16(taddr + cc0, r);
         tmem_ld_wait();
-        if (rok) {
+        if (args.ksplit == 1 && pair_rows) {
+          // lanes 2i and 2i + 1 hold rows `row` and `row + 1`: the even lane stores both rows
+          // of the even tokens, the odd lane those of the odd tokens (one 4-byte bf16 pair
+          // each, 128 contiguous bytes per warp store), after one exchange per token pair
+          const bool odd = (lane & 1) != 0;
+          const int row0 = row & ~1;
+#pragma unroll
+          for (int j = 0; j < 16; j += 2) {
+            const float keep = __uint_as_float(odd ? r[j + 1] : r[j]);
+            const float give = __uint_as_float(odd ? r[j] : r[j + 1]);
+            const float got = __shfl_xor_sync(0xffffffffu, give, 1);
+            const int tok = c.n0 + cc0 + j + (odd ? 1 : 0);
+            if (tok < c.tend && row0 < args.d_out)
+              *reinterpret_cast<uint32_t*>(args.Y + static_cast<int64_t>(tok) * args.d_out + row0) =
+                  odd ? pack_bf16x2(got, keep) : pack_bf16x2(keep, got);
+          }
+        } else if (rok) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int tok = c.n0 + cc0 + j;
