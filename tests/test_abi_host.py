@@ -63,7 +63,11 @@ def test_workspace_size_components(lib):
     # are T * d bf16
     assert ws_full >= 4096 * 5120 * 2
     cfg_r = ttq.make_config(4, 128, 0.5, 0.4, r=16)
-    assert ttq.workspace_size(4096, 5120, 8192, cfg_r) >= ws_full + 4096 * 64 * 2
+    # with a low-rank side path: U (bf16 [T, 64]) and the statistic's per-64-token-block
+    # column sums of the fused pass (fp32 [T / 64, d])
+    assert ttq.workspace_size(4096, 5120, 8192, cfg_r) >= ws_full + 4096 * 64 * 2 + (4096 // 64) * 5120 * 4
+    # a decode of one or two tokens forms U in its prep launch: no block sums there
+    assert ttq.workspace_size(2, 5120, 8192, cfg_r) < (4096 // 64) * 5120 * 4
 
 
 def test_folded_offset_inside_workspace(lib):
