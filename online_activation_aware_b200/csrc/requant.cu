@@ -430,16 +430,10 @@ struct RqArgs {
 
 template <int Q, int G, int MODE>
 cudaError_t launch_qg(dim3 grid, const RqArgs& args, bool pdl, cudaStream_t stream) {
-  static bool attr_set[64] = {};  // per instantiation and device (set for the largest batch)
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  // set on every launch (it belongs to the current context; for the largest batch)
+  cudaError_t e = cudaFuncSetAttribute(requant_kernel<Q, G, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(rq_smem_bytes(MODE, MODE == kRqBatch ? kRequantMaxPrompts : 1)));
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(requant_kernel<Q, G, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(rq_smem_bytes(MODE, MODE == kRqBatch ? kRequantMaxPrompts : 1)));
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3((kRqWarps + (MODE == kRqFold ? kFoldWarps : 0)) * 32);
